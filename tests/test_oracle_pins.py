@@ -1,0 +1,329 @@
+"""Pins for the CPU oracle: each check ties the oracle to something other
+than itself -- values the pages print, closed forms, special cases that
+reduce to a library routine, invariants of the mathematics and finite
+differences.  CPU only."""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+from scipy.stats import norm
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- codebook
+
+@pytest.mark.parametrize("p", [1e-9, 0.001, 0.03, 0.2, 0.5, 0.5585, 0.75, 0.9677083, 0.999])
+def test_norm_ppf_matches_library(p):
+    assert oracle.norm_ppf(p) == pytest.approx(norm.ppf(p), rel=1e-12, abs=1e-15)
+
+
+def test_nf4_codebook_shape():
+    c64, c32 = oracle.nf4_codebook()
+    assert np.all(np.diff(c64) > 0) and np.all(np.diff(c32) > 0)
+    assert c32[0] == -1.0 and c32[7] == 0.0 and c32[15] == 1.0
+    assert (c32 < 0).sum() == 7 and (c32 > 0).sum() == 8
+    assert np.array_equal(c32, c64.astype(np.float32))
+
+
+def test_nf4_levels_are_equispaced_normal_quantiles():
+    """Mapped back through the normal CDF, the unnormalised levels sit at
+    probabilities spaced evenly from the offset down to 1/2: 8 steps on the
+    positive side, 7 on the negative side (levels follow a normal law)."""
+    c64, _ = oracle.nf4_codebook()
+    delta = 0.5 * ((1 - 1 / 30) + (1 - 1 / 32))
+    z = norm.ppf(delta)
+    pos = norm.cdf(c64[8:] * z)[::-1]          # from the top level down
+    neg = norm.cdf(-c64[:7] * z)               # from the bottom level up
+    assert pos[0] == pytest.approx(delta, abs=1e-13)
+    assert neg[0] == pytest.approx(delta, abs=1e-13)
+    assert np.allclose(np.diff(pos), (0.5 - delta) / 8, atol=1e-13)
+    assert np.allclose(np.diff(neg), (0.5 - delta) / 7, atol=1e-13)
+    assert pos[-1] + (0.5 - delta) / 8 == pytest.approx(0.5, abs=1e-13)
+
+
+# ------------------------------------------------------- the pages' example
+
+def test_toy_two_bit_example():
+    g = _golden("toy_2bit.json")
+    levels = np.array([float(Fraction(s)) for s in g["levels"]])
+    for case in g["cases"]:
+        codes, scales, w_hat = oracle.quantize_levels(np.array(case["block"], np.float32), 64, levels)
+        assert scales[0] == case["scale"]
+        d = case["decimals"]
+        assert round(w_hat[case["index"]], d) == case["reconstructed"]
+        if "abs_error" in case:
+            err = abs(w_hat[case["index"]] - case["block"][case["index"]])
+            assert round(err, d) == case["abs_error"]
+
+
+# ------------------------------------------------------------- NF4 format
+
+def test_nibble_order_low_first():
+    """First logical value in the low nibble, next in the high nibble
+    ("QLoRA Fine-Tuning", NF4 representation)."""
+    _, c32 = oracle.nf4_codebook()
+    w = oracle.quantize_nf4(c32.reshape(1, 16), B=16, C=4)
+    assert list(w.codes) == [0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE]
+
+
+def test_zero_block_rule():
+    W = synth.weight(synth.workload("fp32_single_256"), 0)
+    w, s = oracle.quantize_nf4(W, 64, 256, return_s=True)
+    b = 5
+    assert s[b] == 0.0
+    assert np.all(w.codes[b * 32:(b + 1) * 32] == 0x77)
+    Wh = oracle.dequantize(w).reshape(-1)
+    assert np.all(Wh[b * 64:(b + 1) * 64] == 0.0)
+    # its scale code still follows the double-quant formula (not 128 unless mu == 0)
+    assert w.qcodes[b] != 128 and s.min() == 0.0
+
+
+def test_exact_round_trip_with_common_power_of_two_scale():
+    _, c32 = oracle.nf4_codebook()
+    rng = np.random.default_rng(1)
+    B, C, nb = 64, 4, 37                         # partial last group (37 = 9*4 + 1)
+    sc = np.float32(2.0 ** -5)
+    k = rng.integers(0, 16, size=(nb, B))
+    k[:, 0] = rng.choice([0, 15], size=nb)       # every block reaches |c| = 1
+    W = (c32[k] * sc).astype(np.float32).reshape(1, -1)
+    w, s = oracle.quantize_nf4(W, B, C, return_s=True)
+    assert np.all(s == sc) and w.mu == sc
+    assert np.all(w.t == 0) and np.all(w.qcodes == 128)
+    assert np.array_equal(oracle.dequantize(w).view(np.uint32), W.view(np.uint32))
+
+
+def test_double_quant_special_codes_and_error_bound():
+    W = synth.normal(77, (64, 1024), std=0.02)
+    w, s = oracle.quantize_nf4(W, 64, 256, return_s=True)
+    mu = np.float32(w.mu)
+    assert mu == pytest.approx(np.mean(s.astype(np.float64)), rel=1e-6)
+    for g in range(w.t.size):
+        blk = np.arange(g * 256, min(s.size, (g + 1) * 256))
+        d = (s[blk] - mu).astype(np.float32)
+        j = int(np.argmax(np.abs(d)))
+        assert w.t[g] == np.abs(d[j])
+        # the block with the largest deviation takes an end code
+        assert w.qcodes[blk[j]] == (255 if d[j] > 0 else 1)
+        # decoded scales are within half a code step of the exact ones
+        sh = np.array([oracle.decode_scale(w.qcodes[b], w.t[g], mu) for b in blk], np.float64)
+        assert np.all(np.abs(sh - s[blk]) <= w.t[g] / 254.0 * (1 + 1e-5) + 4e-7 * np.abs(s[blk]))
+    # a block whose scale equals mu gets the centre code
+    W2 = np.concatenate([np.full(64, 1.0, np.float32), np.full(64, 3.0, np.float32),
+                         np.full(64, 2.0, np.float32)]).reshape(1, -1)
+    w2 = oracle.quantize_nf4(W2, 64, 4)
+    assert w2.mu == 2.0 and list(w2.qcodes) == [1, 255, 128]
+    assert oracle.decode_scale(1, w2.t[0], w2.mu) == 1.0
+    assert oracle.decode_scale(255, w2.t[0], w2.mu) == 3.0
+
+
+def test_decode_scale_clamps_at_zero():
+    assert oracle.decode_scale(1, 5.0, 1.0) == 0.0
+    assert oracle.decode_scale(128, 5.0, 1.0) == 1.0
+
+
+def test_payload_bytes_and_bits_per_weight():
+    g = _golden("payload_and_counts.json")
+    for (O, I, B, C) in [(256, 256, 64, 256), (7, 33, 64, 256), (3, 50, 16, 3)]:
+        W = synth.normal(5, (O, I), std=0.02)
+        w = oracle.quantize_nf4(W, B, C)
+        N = O * I
+        actual = w.codes.size + w.qcodes.size + 4 * w.t.size + 4
+        assert actual == oracle.nf4_payload_bytes(N, B, C)
+        assert w.codes.size == -(-N // 2)
+    N = 4096 * 12288
+    assert round(8 * oracle.nf4_payload_bytes(N, 64, 256) / N, 2) == g["dq_bits_per_weight_2dp"]
+    assert 8 * oracle.legacy_payload_bytes(N, 64) / N == g["legacy_bits_per_weight"]
+
+
+def test_qwen3_packed_numel_and_adapter_count():
+    g = _golden("payload_and_counts.json")
+    q = g["qwen3_0.6b"]
+    H, L = q["hidden"], q["layers"]
+    shapes = [(q["q_out"], H), (q["kv_out"], H), (q["kv_out"], H), (H, q["o_in"]),
+              (q["intermediate"], H), (q["intermediate"], H), (H, q["intermediate"])]
+    logical = L * sum(o * i for o, i in shapes)
+    packed = 0
+    for o, i in shapes[:2]:  # packing count checked on real quantizer output for two shapes
+        w = oracle.quantize_nf4(np.zeros((o, i), np.float32), 64, 256)
+        assert w.codes.size * 2 == o * i
+    packed = logical // 2
+    assert g["numel_fp32_model"] - g["numel_4bit_model"] == packed
+    wl = synth.workload("qwen3_0.6b_attn_qv")
+    assert wl.r == q["lora_rank"]
+    per_layer = sum(sum(a.size for a in synth.adapters(wl, li)) for li in range(len(wl.linears)))
+    assert L * per_layer == g["trainable_params"]
+
+
+def test_odd_n_partial_block_and_empty():
+    W = synth.normal(9, (1, 101), std=1.0)
+    w = oracle.quantize_nf4(W, 64, 256)
+    assert w.codes.size == 51 and (w.codes[-1] >> 4) == 0
+    assert w.qcodes.size == 2 and w.t.size == 1
+    e = oracle.quantize_nf4(np.zeros((0, 64), np.float32), 64, 256)
+    assert e.codes.size == 0 and e.mu == 0.0
+
+
+def test_nonfinite_rejected():
+    W = np.ones((2, 64), np.float32)
+    W[1, 3] = np.inf
+    with pytest.raises(FloatingPointError):
+        oracle.quantize_nf4(W, 64, 256)
+    W[1, 3] = np.nan
+    with pytest.raises(FloatingPointError):
+        oracle.quantize_affine(W, 4, 64)
+
+
+def test_nearest_code_with_ties_to_lower_index():
+    c64, c32 = oracle.nf4_codebook()
+    rng = np.random.default_rng(3)
+    x = rng.uniform(-1, 1, 4000).astype(np.float32)
+    x[0], x[1] = 1.0, -1.0
+    W = x.reshape(1, -1)
+    w = oracle.quantize_nf4(W, W.size, 1)
+    codes = np.empty(W.size, np.int64)
+    codes[0::2] = w.codes & 15
+    codes[1::2] = w.codes >> 4
+    dist = np.abs(x.astype(np.float64)[:, None] - c32.astype(np.float64)[None, :])
+    assert np.array_equal(codes, np.argmin(dist, axis=1))  # argmin keeps the first minimum
+
+
+# ---------------------------------------------------------------- affine
+
+def test_affine_grid_round_trip_and_constant_group():
+    k = np.arange(16, dtype=np.float32)
+    W = np.concatenate([k * np.float32(2.0 ** -4), np.full(16, 0.375, np.float32)]).reshape(1, -1)
+    w = oracle.quantize_affine(W, 4, 16)
+    assert w.scale[0] == 2.0 ** -4 and w.bias[0] == 0.0
+    assert w.scale[1] == 0.0 and w.bias[1] == np.float32(0.375)
+    assert list(w.codes[:8]) == [0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE]
+    assert np.all(w.codes[8:] == 0)
+    assert np.array_equal(oracle.dequantize(w), W)
+    w8 = oracle.quantize_affine(W, 8, 16)
+    # 8 bits spread the same 16 grid points over 255 steps: code = 17 k
+    assert list(w8.codes[:16]) == [17 * i for i in range(16)] and w8.codes.size == 32
+
+
+@pytest.mark.parametrize("bits,G", [(4, 32), (4, 64), (4, 128), (8, 32), (8, 64), (8, 128)])
+def test_affine_error_bound(bits, G):
+    W = synth.normal(11, (16, 256), std=0.02)
+    w = oracle.quantize_affine(W, bits, G)
+    Wh = oracle.dequantize(w).astype(np.float64)
+    sc = np.repeat(w.scale.astype(np.float64), G).reshape(W.shape)
+    assert np.all(np.abs(Wh - W) <= 0.5 * sc * (1 + 1e-5) + 1e-7)
+    lo = W.reshape(-1, G).min(1)
+    hi = W.reshape(-1, G).max(1)
+    assert np.array_equal(w.bias, lo)
+    # the group's min and max reconstruct (up to fp32 rounding)
+    assert np.allclose(Wh.reshape(-1, G).min(1), lo, atol=1e-7)
+    assert np.allclose(Wh.reshape(-1, G).max(1), hi, atol=2e-7)
+    assert w.codes.size * 8 // bits == W.size
+
+
+# ------------------------------------------------------ forward / backward
+
+def _small_layer(fmt="nf4", O=96, I=128, R=5, r=4, alpha=8.0, seed=21):
+    W = synth.normal(seed, (O, I), std=0.02)
+    w = oracle.quantize_nf4(W, 64, 3) if fmt == "nf4" else oracle.quantize_affine(W, 4, 32)
+    X = synth.normal(seed + 1, (R, I))
+    A = synth.normal(seed + 2, (r, I), std=0.02)
+    Bm = synth.normal(seed + 3, (O, r), std=0.02)
+    dY = synth.normal(seed + 4, (R, O))
+    return w, X, A, Bm, dY, r, alpha
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "affine"])
+def test_forward_equals_dense_gemm_on_dequantized(fmt):
+    w, X, A, Bm, dY, r, alpha = _small_layer(fmt)
+    Wh = oracle.dequantize(w).astype(np.float64)
+    Y, U = oracle.linear_fwd(w, X, A, Bm, r, alpha)
+    s = float(np.float32(alpha) / np.float32(r))
+    X64, A64, B64 = X.astype(np.float64), A.astype(np.float64), Bm.astype(np.float64)
+    assert np.allclose(U, X64 @ A64.T, rtol=1e-12, atol=1e-13)
+    assert np.allclose(Y, X64 @ Wh.T + s * (X64 @ A64.T) @ B64.T, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "affine"])
+def test_backward_equals_dense_formulas(fmt):
+    w, X, A, Bm, dY, r, alpha = _small_layer(fmt)
+    Wh = oracle.dequantize(w).astype(np.float64)
+    dX, dA, dB = oracle.linear_bwd(w, X, dY, A, Bm, r, alpha)
+    s = float(np.float32(alpha) / np.float32(r))
+    X64, A64, B64, G = (a.astype(np.float64) for a in (X, A, Bm, dY))
+    assert np.allclose(dX, G @ Wh + s * (G @ B64) @ A64, rtol=1e-12, atol=1e-12)
+    assert np.allclose(dA, s * (G @ B64).T @ X64, rtol=1e-12, atol=1e-12)
+    assert np.allclose(dB, s * G.T @ (X64 @ A64.T), rtol=1e-12, atol=1e-12)
+
+
+def test_gradients_by_central_differences():
+    """L = <Y, dY> is linear in X, in A and in B separately, so a central
+    difference with an exactly representable step is the derivative up to
+    fp64 rounding of L."""
+    R, O, I, r, alpha = 3, 128, 128, 2, 4.0
+    w, X, A, Bm, dY, r, alpha = _small_layer("nf4", O=O, I=I, R=R, r=r, alpha=alpha, seed=40)
+    q = lambda a: (np.round(a * 1024) / 1024).astype(np.float32)   # exact fp32 +- h
+    X, A, Bm = q(X), q(A * 16), q(Bm * 16)
+    dY = dY.astype(np.float32)
+    h = np.float32(2.0 ** -4)
+
+    def L(X_, A_, B_):
+        Y, _ = oracle.linear_fwd(w, X_, A_, B_, r, alpha)
+        return float(np.sum(Y * dY.astype(np.float64)))
+
+    dX, dA, dB = oracle.linear_bwd(w, X, dY, A, Bm, r, alpha)
+    rng = np.random.default_rng(0)
+    for name, arr, grad in (("X", X, dX), ("A", A, dA), ("B", Bm, dB)):
+        for _ in range(6):
+            idx = tuple(int(rng.integers(0, n)) for n in arr.shape)
+            p, m = arr.copy(), arr.copy()
+            p[idx] += h
+            m[idx] -= h
+            args_p = {"X": (p, A, Bm), "A": (X, p, Bm), "B": (X, A, p)}[name]
+            args_m = {"X": (m, A, Bm), "A": (X, m, Bm), "B": (X, A, m)}[name]
+            fd = (L(*args_p) - L(*args_m)) / (2 * float(h))
+            assert fd == pytest.approx(grad[idx], rel=1e-7, abs=1e-9), (name, idx)
+
+
+def test_special_cases_zero_adapter_and_identity_input():
+    w, X, A, Bm, dY, r, alpha = _small_layer("nf4", O=64, I=128, R=4)
+    Wh = oracle.dequantize(w).astype(np.float64)
+    Z = np.zeros_like(Bm)
+    Y, _ = oracle.linear_fwd(w, X, A, Z, r, alpha)
+    assert np.allclose(Y, X.astype(np.float64) @ Wh.T, rtol=1e-12, atol=1e-12)
+    _, dA, _ = oracle.linear_bwd(w, X, dY, A, Z, r, alpha)
+    assert np.all(dA == 0)
+    Y0, _ = oracle.linear_fwd(w, X, A, Bm, r, 0.0)
+    assert np.allclose(Y0, X.astype(np.float64) @ Wh.T, rtol=1e-12, atol=1e-12)
+    eye = np.eye(128, dtype=np.float32)
+    Yi, _ = oracle.linear_fwd(w, eye, A, Z, r, alpha)
+    assert np.array_equal(Yi, Wh.T)
+
+
+def test_row_subsets_match_full():
+    w, X, A, Bm, dY, r, alpha = _small_layer("nf4", R=9)
+    rows = np.array([0, 3, 8])
+    Y, U = oracle.linear_fwd(w, X, A, Bm, r, alpha)
+    Ys, Us = oracle.linear_fwd(w, X, A, Bm, r, alpha, rows=rows)
+    assert np.array_equal(Ys, Y[rows]) and np.array_equal(Us, U[rows])
+    dX, dA, dB = oracle.linear_bwd(w, X, dY, A, Bm, r, alpha)
+    dXs, dAs, dBs = oracle.linear_bwd(w, X, dY, A, Bm, r, alpha, rows=rows)
+    assert np.array_equal(dXs, dX[rows]) and np.array_equal(dAs, dA) and np.array_equal(dBs, dB)
+
+
+def test_synth_streams_are_stable():
+    a = synth.normal(1234, 1001)
+    b = synth.normal(1234, 1001)
+    assert np.array_equal(a, b)
+    assert abs(float(a.mean())) < 0.1 and abs(float(a.std()) - 1) < 0.1
+    wide, bits = synth.bf16_round(np.array([1.0, 1.00390625, 1.005859375, -2.5], np.float32))
+    assert list(wide) == [1.0, 1.0, 1.0078125, -2.5]
