@@ -1,0 +1,246 @@
+/*
+ * qlora.h -- C ABI of libqlora: the QLoRA linear layer on one NVIDIA B200
+ * (sm_100a).  A frozen base weight stored as blockwise NF4 with
+ * double-quantized scales (or as affine 4/8-bit groups), plus a trainable
+ * fp32 rank-r LoRA adapter:
+ *
+ *   forward   Y  = X W_hat^T + s (X A^T) B^T             s = alpha / r
+ *   backward  dX = dY W_hat  + s (dY B) A
+ *             dA = s (dY B)^T X          dB = s dY^T (X A^T)
+ *   (no weight gradient: the base is frozen)
+ *
+ * Sources (page title, section):
+ *   "QLoRA Fine-Tuning" (Riftco Transformer how-to): "NF4 representation"
+ *     (format, double quantization, payload sizes) and "Forward and
+ *     backward" (the two sums, one autograd parent, decode inside the sums).
+ *   "QLoRA on Mac -- fine-tuning larger open models on 48 GB", "Design /
+ *     Q-LoRA layer" (base + (alpha/r)(x A^T) B^T with fp32 A/B).
+ *   "LoRA vs QLoRA on Apple Silicon ... in MLX", "Method" (affine
+ *     group-wise 4/8-bit quantization with fp32 scale and bias).
+ *
+ * Conventions for every entry point:
+ *   - All array arguments are DEVICE pointers owned by the caller, unless a
+ *     comment says "host".  Matrices are row-major and dense.
+ *   - The library never allocates device memory.  Scratch space is a caller
+ *     workspace (`ws`, `ws_bytes`); its required size comes from the
+ *     matching *_workspace_bytes() function.  `ws` must be 256-byte aligned.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Only qlora_quantize_nf4, qlora_quantize_affine and
+ *     qlora_workspace_status synchronize `stream` (to read a device flag).
+ *   - Arguments are validated on the host before anything is launched; a
+ *     rejected call returns a status and enqueues nothing.  Nothing aborts
+ *     and no exception crosses the ABI.
+ *   - Weights are read-only in fwd/bwd.  dA and dB are overwritten, not
+ *     accumulated.
+ *   - Calls on distinct streams with distinct workspaces are thread-safe.
+ *   - If no CUDA device is usable, every compute entry point returns
+ *     QLORA_ERR_CUDA; there is no CPU fallback.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* qlora_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,  /* null pointer, bad enum, negative size      */
+  QLORA_ERR_SHAPE = 2,        /* sizes inconsistent with the format         */
+  QLORA_ERR_ALIGNMENT = 3,    /* pointer or workspace misaligned            */
+  QLORA_ERR_NONFINITE = 4,    /* NaN/Inf weight given to a quantizer        */
+  QLORA_ERR_UNSUPPORTED = 5,  /* valid but not implemented (e.g. r > 64)    */
+  QLORA_ERR_CUDA = 6,         /* a CUDA runtime call failed                 */
+  QLORA_ERR_TIMEOUT = 7,      /* a bounded device wait ran out              */
+  QLORA_ERR_WORKSPACE = 8     /* ws_bytes smaller than required             */
+} qlora_status;
+
+typedef enum {
+  QLORA_FMT_NF4_DQ = 0, /* NF4 codes + u8 scale codes + fp32 t_g + fp32 mu */
+  QLORA_FMT_AFFINE = 2  /* 4/8-bit codes + fp32 scale and bias per group   */
+} qlora_format;
+
+typedef enum {
+  QLORA_COMPUTE_FP32 = 0, /* X, dY, Y, dX are fp32; fp32 SIMT arithmetic     */
+  QLORA_COMPUTE_BF16 = 1  /* X, dY, Y, dX are bf16; bf16 tensor-core operands,
+                             fp32 accumulation                               */
+} qlora_compute;
+
+/*
+ * Non-owning view of a quantized weight W_hat [O x I] (logical row-major,
+ * flat index n = o*I + i).  All pointers are device memory.
+ *   NF4_DQ:  block = B (weights per absmax block), group = C (blocks per
+ *            second-level group), bits = 4.
+ *            codes        ceil(N/2) bytes, weight 2j in the low nibble of
+ *                         byte j, 2j+1 in the high nibble
+ *            scale_codes  M = ceil(N/B) bytes q_b
+ *            group_absmax S = ceil(M/C) floats t_g
+ *            mean         1 float mu
+ *   AFFINE:  block = G (weights per group), group ignored, bits = 4 or 8.
+ *            codes        ceil(N*bits/8) bytes (4-bit: low nibble first)
+ *            scale, bias  ceil(N/G) floats each
+ *            w_hat = scale_g * code + bias_g
+ * The fwd/bwd entry points require I % block == 0 (blocks never straddle
+ * rows); the quantizers and qlora_dequantize accept any N.
+ */
+typedef struct {
+  int32_t fmt; /* qlora_format */
+  int64_t O, I;
+  int32_t block, group, bits;
+  const uint8_t* codes;
+  const uint8_t* scale_codes;
+  const float* group_absmax;
+  const float* mean;
+  const float* scale;
+  const float* bias;
+} qlora_weight;
+
+/* Human-readable name of a status (static string, never NULL). */
+const char* qlora_status_string(qlora_status st);
+
+/*
+ * HOST.  Writes the library's 16 fp32 NF4 levels (ascending, c[7] = 0) to
+ * the host array `out`.  Source: "QLoRA: Fine-Tuning Under Memory
+ * Constraints", "Understand what NF4 chooses" (levels follow a normal
+ * distribution) and "QLoRA Fine-Tuning", "NF4 representation" (fixed
+ * 16-value codebook): normal quantiles at probabilities spaced evenly from
+ * delta = ((1-1/30)+(1-1/32))/2 down to 1/2 (8 positive, 7 negative, plus
+ * zero), divided by the largest, rounded to fp32.
+ */
+qlora_status qlora_nf4_codebook(float out[16]);
+
+/*
+ * HOST.  Payload bytes of the double-quantized format: ceil(N/2) + M + 4S
+ * + 4 ("QLoRA Fine-Tuning", "NF4 representation").  0 on bad arguments.
+ */
+size_t qlora_nf4_payload_bytes(int64_t N, int32_t B, int32_t C);
+
+/* HOST.  Workspace bytes qlora_quantize_nf4 needs for N weights. */
+size_t qlora_quantize_nf4_workspace_bytes(int64_t N, int32_t B, int32_t C);
+
+/*
+ * Quantize W [O x I] fp32 to NF4 with double-quantized scales
+ * ("QLoRA Fine-Tuning", "NF4 representation"):
+ *   s_b = max |w| over block b (B consecutive weights of the flat order);
+ *   code = nearest of the 16 levels to fp32(w / s_b), ties to the lower
+ *   level; an all-zero block gets s_b = 0 and the zero level (code 7);
+ *   mu = mean of s_b (fp64 sums: sequential within each group of C blocks,
+ *   then over groups; rounded to fp32);
+ *   t_g = max |fp32(s_b - mu)| over group g;
+ *   q_b = 128 + clamp(round(fp32(fp32(127 (s_b - mu)) / t_g)), -127, 127),
+ *   round half away from zero; q_b = 128 when t_g = 0.
+ * Outputs (device): codes [ceil(N/2)], scale_codes [M], t [S], mu [1].
+ * Bit-exact and deterministic.  Synchronizes `stream` at the end to read
+ * the non-finite flag: returns QLORA_ERR_NONFINITE (outputs undefined) if
+ * W holds a NaN or Inf.  N = 0 is valid (mu = 0).
+ */
+qlora_status qlora_quantize_nf4(const float* W, int64_t O, int64_t I, int32_t B, int32_t C,
+                                uint8_t* codes, uint8_t* scale_codes, float* t, float* mu,
+                                void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/* HOST.  Workspace bytes qlora_quantize_affine needs. */
+size_t qlora_quantize_affine_workspace_bytes(int64_t N, int32_t bits, int32_t G);
+
+/*
+ * Affine group-wise quantization ("LoRA vs QLoRA on Apple Silicon",
+ * "Method"; the pages print no formula -- the plain min/max scheme):
+ *   per group of G weights: bias = min, scale = fp32(fp32(max - min) /
+ *   (2^bits - 1)), code = clamp(round(fp32(fp32(w - bias) / scale)), 0,
+ *   2^bits - 1) (0 when scale = 0).  4-bit codes pack low nibble first.
+ * Outputs: codes [ceil(N*bits/8)], scale [ceil(N/G)], bias [ceil(N/G)].
+ * Synchronizes `stream`; QLORA_ERR_NONFINITE for NaN/Inf or an infinite
+ * range.
+ */
+qlora_status qlora_quantize_affine(const float* W, int64_t O, int64_t I, int32_t bits, int32_t G,
+                                   uint8_t* codes, float* scale, float* bias, void* ws,
+                                   size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * Diagnostic dequantization ("QLoRA Fine-Tuning", "NF4 representation":
+ * dequantize() is an explicit diagnostic/export operation that the training
+ * kernels never call).  W_hat [O x I] fp32:
+ *   NF4_DQ: c[code] * s_hat_b,  s_hat_b = clamp(mu + fp32(fp32(t_g (q_b -
+ *           128)) / 127), 0, FLT_MAX);
+ *   AFFINE: fp32(scale_g * code) + bias_g.
+ * Bit-exact.  Never used by qlora_linear_fwd / qlora_linear_bwd.
+ */
+qlora_status qlora_dequantize(const qlora_weight* w, float* W_hat, qlora_stream_t stream);
+
+/* op codes for qlora_linear_workspace_bytes */
+#define QLORA_OP_FWD 0
+#define QLORA_OP_BWD 1
+
+/* HOST.  Workspace bytes of qlora_linear_fwd (op 0) or qlora_linear_bwd (op 1). */
+size_t qlora_linear_workspace_bytes(const qlora_weight* w, int64_t R, int32_t r, int32_t op,
+                                    int32_t compute);
+
+/*
+ * QLoRA linear forward ("QLoRA Fine-Tuning", "Forward and backward";
+ * "QLoRA on Mac", "Design / Q-LoRA layer"):
+ *   U = X A^T                      [R x r] fp32
+ *   Y = X W_hat^T + s U B^T        [R x O]
+ * X [R x I] and Y [R x O] are fp32 (QLORA_COMPUTE_FP32) or bf16
+ * (QLORA_COMPUTE_BF16); A [r x I] and B [O x r] are fp32; s = alpha / r in
+ * fp32.  U_out (nullable) receives U for reuse by the backward pass.
+ * Every weight is decoded from its nibble and block scale inside the
+ * kernels; no full-size floating-point weight is formed.  R = 0 is valid.
+ * bf16 mode: W_hat and the adapter operands enter the tensor cores as bf16,
+ * accumulation is fp32, Y is rounded to bf16 once.
+ * Requires 1 <= r <= 64 and I % block == 0.
+ */
+qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, const float* A,
+                              const float* B, int32_t r, float alpha, int32_t compute, void* Y,
+                              float* U_out, void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * QLoRA linear backward (vector-Jacobian product; "QLoRA Fine-Tuning",
+ * "Forward and backward": the node's only parent is the input, so there is
+ * no weight gradient; the LoRA factors get the ordinary chain rule):
+ *   V  = dY B                      [R x r]
+ *   dX = dY W_hat + s V A          [R x I]  (nullable: skipped)
+ *   dA = s V^T X                   [r x I]  (nullable: skipped)
+ *   dB = s dY^T U                  [O x r]  (nullable: skipped)
+ * U_in (nullable) is U = X A^T from the forward; when NULL it is
+ * recomputed.  Types as in qlora_linear_fwd; dA and dB are fp32 and
+ * overwritten.
+ */
+qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* dY, int64_t R,
+                              const float* A, const float* B, int32_t r, float alpha,
+                              const float* U_in, int32_t compute, void* dX, float* dA, float* dB,
+                              void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * Reads the device error word that the kernels of the last call using
+ * workspace `ws` may have set (bounded waits that ran out, device-side
+ * argument checks).  Synchronizes `stream`.  Returns QLORA_OK or the first
+ * error recorded (e.g. QLORA_ERR_TIMEOUT).
+ */
+qlora_status qlora_workspace_status(const void* ws, qlora_stream_t stream);
+
+/*
+ * Failure-detection self test: launches one tiny kernel that waits on an
+ * mbarrier nothing ever arrives on, with a wait limit of `limit_us`
+ * microseconds (1..1000000).  The wait gives up, the kernel records
+ * QLORA_ERR_TIMEOUT in `ws` (>= 256 bytes) and returns; the context stays
+ * usable.  Returns the status read back (QLORA_ERR_TIMEOUT when the
+ * mechanism works).  Synchronizes `stream`.
+ */
+qlora_status qlora_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us,
+                                         qlora_stream_t stream);
+
+/*
+ * HOST.  Number of CUDA kernels the library launched in this process so far
+ * (counted on the host at each launch).
+ */
+uint64_t qlora_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H_ */

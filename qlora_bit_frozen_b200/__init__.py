@@ -1,0 +1,226 @@
+"""QLoRA linear layer on NVIDIA B200: Python binding of libqlora.
+
+Thin marshalling over the C ABI declared in include/qlora.h: each function
+here has the name of the C entry point it calls, takes torch tensors, and
+passes their device pointers and the current CUDA stream.  Every step of the
+computation runs in the library's CUDA kernels; torch only allocates device
+memory (outputs and workspaces) and provides the stream.  There is no CPU
+fallback: without the built library or a CUDA device the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+from . import _ffi
+from ._ffi import (COMPUTE_BF16, COMPUTE_FP32, FMT_AFFINE, FMT_NF4_DQ, OP_BWD, OP_FWD,
+                   qlora_weight)
+
+__all__ = [
+    "QLoraError", "QuantizedWeight", "qlora_status_string", "qlora_nf4_codebook",
+    "qlora_nf4_payload_bytes", "qlora_quantize_nf4", "qlora_quantize_affine", "qlora_dequantize",
+    "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
+    "qlora_workspace_status", "qlora_selftest_wait_timeout", "qlora_kernel_launch_count",
+    "COMPUTE_FP32", "COMPUTE_BF16", "FMT_NF4_DQ", "FMT_AFFINE", "workspace",
+]
+
+
+class QLoraError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = int(status)
+        msg = _ffi.load().qlora_status_string(self.status).decode()
+        super().__init__(f"{where}: {msg} (status {self.status})" if where else msg)
+
+
+def _check(status: int, where: str):
+    if status != _ffi.OK:
+        raise QLoraError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A 256-byte aligned device workspace of at least nbytes (torch allocates)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class QuantizedWeight:
+    """Device buffers of a frozen quantized weight (immutable by convention)."""
+    fmt: int
+    O: int
+    I: int
+    block: int
+    group: int
+    bits: int
+    codes: torch.Tensor
+    scale_codes: Optional[torch.Tensor] = None
+    group_absmax: Optional[torch.Tensor] = None
+    mean: Optional[torch.Tensor] = None
+    scale: Optional[torch.Tensor] = None
+    bias: Optional[torch.Tensor] = None
+
+    def c_struct(self) -> qlora_weight:
+        return qlora_weight(self.fmt, self.O, self.I, self.block, self.group, self.bits,
+                            *(t.data_ptr() if t is not None and t.numel() > 0 else None
+                              for t in (self.codes, self.scale_codes, self.group_absmax, self.mean,
+                                        self.scale, self.bias)))
+
+    def payload_bytes(self) -> int:
+        ts = [self.codes, self.scale_codes, self.group_absmax, self.mean, self.scale, self.bias]
+        return sum(t.numel() * t.element_size() for t in ts if t is not None)
+
+
+def qlora_status_string(status: int) -> str:
+    return _ffi.load().qlora_status_string(int(status)).decode()
+
+
+def qlora_nf4_codebook():
+    out = (ctypes.c_float * 16)()
+    _check(_ffi.load().qlora_nf4_codebook(out), "qlora_nf4_codebook")
+    return [float(v) for v in out]
+
+
+def qlora_nf4_payload_bytes(N: int, B: int = 64, C: int = 256) -> int:
+    return int(_ffi.load().qlora_nf4_payload_bytes(N, B, C))
+
+
+def qlora_quantize_nf4(W: torch.Tensor, B: int = 64, C: int = 256, stream=None) -> QuantizedWeight:
+    """NF4 + double-quantized scales of a CUDA fp32 [O x I] matrix (synchronizes the stream)."""
+    lib = _ffi.load()
+    if W.dim() != 2 or W.dtype != torch.float32 or not W.is_cuda:
+        raise ValueError("W must be a CUDA float32 matrix")
+    W = W.contiguous()
+    O, I = W.shape
+    N = O * I
+    M = -(-N // B)
+    S = -(-M // C)
+    dev = W.device
+    codes = torch.empty((N + 1) // 2, dtype=torch.uint8, device=dev)
+    q = torch.empty(M, dtype=torch.uint8, device=dev)
+    t = torch.empty(S, dtype=torch.float32, device=dev)
+    mu = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = workspace(lib.qlora_quantize_nf4_workspace_bytes(N, B, C), dev)
+    st = lib.qlora_quantize_nf4(_ptr(W), O, I, B, C, _ptr(codes), _ptr(q), _ptr(t), _ptr(mu), _ptr(ws),
+                                ws.numel(), _stream(stream))
+    _check(st, "qlora_quantize_nf4")
+    return QuantizedWeight(FMT_NF4_DQ, O, I, B, C, 4, codes, q, t, mu)
+
+
+def qlora_quantize_affine(W: torch.Tensor, bits: int = 4, G: int = 64, stream=None) -> QuantizedWeight:
+    """Affine group-wise 4/8-bit codes with fp32 scale and bias (synchronizes the stream)."""
+    lib = _ffi.load()
+    if W.dim() != 2 or W.dtype != torch.float32 or not W.is_cuda:
+        raise ValueError("W must be a CUDA float32 matrix")
+    W = W.contiguous()
+    O, I = W.shape
+    N = O * I
+    ng = -(-N // G)
+    dev = W.device
+    codes = torch.empty(N if bits == 8 else (N + 1) // 2, dtype=torch.uint8, device=dev)
+    scale = torch.empty(ng, dtype=torch.float32, device=dev)
+    bias = torch.empty(ng, dtype=torch.float32, device=dev)
+    ws = workspace(lib.qlora_quantize_affine_workspace_bytes(N, bits, G), dev)
+    st = lib.qlora_quantize_affine(_ptr(W), O, I, bits, G, _ptr(codes), _ptr(scale), _ptr(bias), _ptr(ws),
+                                   ws.numel(), _stream(stream))
+    _check(st, "qlora_quantize_affine")
+    return QuantizedWeight(FMT_AFFINE, O, I, G, 0, bits, codes, scale=scale, bias=bias)
+
+
+def qlora_dequantize(w: QuantizedWeight, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Diagnostic fp32 reconstruction of the whole weight (never used by fwd/bwd)."""
+    lib = _ffi.load()
+    if out is None:
+        out = torch.empty((w.O, w.I), dtype=torch.float32, device=w.codes.device)
+    cw = w.c_struct()
+    _check(lib.qlora_dequantize(ctypes.byref(cw), _ptr(out), _stream(stream)), "qlora_dequantize")
+    return out
+
+
+def qlora_linear_workspace_bytes(w: QuantizedWeight, R: int, r: int, op: int, compute: int) -> int:
+    cw = w.c_struct()
+    return int(_ffi.load().qlora_linear_workspace_bytes(ctypes.byref(cw), R, r, op, compute))
+
+
+def _compute_of(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return COMPUTE_BF16
+    if t.dtype == torch.float32:
+        return COMPUTE_FP32
+    raise ValueError("activations must be bfloat16 or float32")
+
+
+def qlora_linear_fwd(w: QuantizedWeight, X: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                     Y: Optional[torch.Tensor] = None, U_out: Optional[torch.Tensor] = None,
+                     ws: Optional[torch.Tensor] = None, stream=None,
+                     want_u: bool = True) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Y = X W_hat^T + (alpha/r)(X A^T) B^T; returns (Y, U = X A^T)."""
+    lib = _ffi.load()
+    R = X.shape[0]
+    r = A.shape[0]
+    compute = _compute_of(X)
+    if Y is None:
+        Y = torch.empty((R, w.O), dtype=X.dtype, device=X.device)
+    if U_out is None and want_u:
+        U_out = torch.empty((R, r), dtype=torch.float32, device=X.device)
+    if ws is None:
+        ws = workspace(qlora_linear_workspace_bytes(w, R, r, OP_FWD, compute), X.device)
+    cw = w.c_struct()
+    st = lib.qlora_linear_fwd(ctypes.byref(cw), _ptr(X), R, _ptr(A), _ptr(B), r, float(alpha), compute,
+                              _ptr(Y), _ptr(U_out), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "qlora_linear_fwd")
+    return Y, U_out
+
+
+def qlora_linear_bwd(w: QuantizedWeight, X: Optional[torch.Tensor], dY: torch.Tensor, A: torch.Tensor,
+                     B: torch.Tensor, alpha: float, U: Optional[torch.Tensor] = None,
+                     want_dx: bool = True, want_da: bool = True, want_db: bool = True,
+                     dX: Optional[torch.Tensor] = None, dA: Optional[torch.Tensor] = None,
+                     dB: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """(dX, dA, dB) of the QLoRA linear layer (no weight gradient)."""
+    lib = _ffi.load()
+    R = dY.shape[0]
+    r = A.shape[0]
+    compute = _compute_of(dY)
+    dev = dY.device
+    if want_dx and dX is None:
+        dX = torch.empty((R, w.I), dtype=dY.dtype, device=dev)
+    if want_da and dA is None:
+        dA = torch.empty((r, w.I), dtype=torch.float32, device=dev)
+    if want_db and dB is None:
+        dB = torch.empty((w.O, r), dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(qlora_linear_workspace_bytes(w, R, r, OP_BWD, compute), dev)
+    cw = w.c_struct()
+    st = lib.qlora_linear_bwd(ctypes.byref(cw), _ptr(X), _ptr(dY), R, _ptr(A), _ptr(B), r, float(alpha),
+                              _ptr(U), compute, _ptr(dX if want_dx else None), _ptr(dA if want_da else None),
+                              _ptr(dB if want_db else None), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "qlora_linear_bwd")
+    return (dX if want_dx else None), (dA if want_da else None), (dB if want_db else None)
+
+
+def qlora_workspace_status(ws: torch.Tensor, stream=None) -> int:
+    """Device error word of the last call that used ws (synchronizes)."""
+    return int(_ffi.load().qlora_workspace_status(_ptr(ws), _stream(stream)))
+
+
+def qlora_selftest_wait_timeout(limit_us: int = 1000, stream=None, device="cuda") -> int:
+    ws = workspace(256, device)
+    return int(_ffi.load().qlora_selftest_wait_timeout(_ptr(ws), ws.numel(), int(limit_us), _stream(stream)))
+
+
+def qlora_kernel_launch_count() -> int:
+    return int(_ffi.load().qlora_kernel_launch_count())

@@ -1,0 +1,333 @@
+// api.cu -- the extern "C" entry points of libqlora (declared in qlora.h):
+// host-side argument checks, workspace layout and kernel dispatch.
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_gemm.h"
+
+namespace qlora {
+
+std::atomic<uint64_t> g_launches{0};
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+qlora_status device_ready() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return QLORA_ERR_CUDA;
+  }
+  return QLORA_OK;
+}
+
+// Reads header words 0..2 of a workspace after synchronizing the stream.
+qlora_status read_header(const void* ws, cudaStream_t st, uint32_t out[3]) {
+  uint32_t h[4] = {0, 0, 0, 0};
+  cudaError_t e = cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  out[0] = h[0];
+  out[1] = h[1];
+  out[2] = h[2];
+  return QLORA_OK;
+}
+
+int64_t nf4_blocks(int64_t N, int32_t B) { return (N + B - 1) / B; }
+
+qlora_status check_weight(const qlora_weight* w, bool for_linear) {
+  if (!w) return QLORA_ERR_INVALID_ARG;
+  if (w->O < 0 || w->I < 0 || w->block < 1) return QLORA_ERR_SHAPE;
+  const int64_t N = w->O * w->I;
+  if (w->fmt == QLORA_FMT_NF4_DQ) {
+    if (w->bits != 4 || w->group < 1) return QLORA_ERR_SHAPE;
+    if (N > 0 && (!w->codes || !w->scale_codes || !w->group_absmax || !w->mean))
+      return QLORA_ERR_INVALID_ARG;
+  } else if (w->fmt == QLORA_FMT_AFFINE) {
+    if (w->bits != 4 && w->bits != 8) return QLORA_ERR_SHAPE;
+    if (N > 0 && (!w->codes || !w->scale || !w->bias)) return QLORA_ERR_INVALID_ARG;
+  } else {
+    return QLORA_ERR_INVALID_ARG;
+  }
+  if (for_linear && w->I % w->block != 0) return QLORA_ERR_SHAPE;
+  return QLORA_OK;
+}
+
+WView view_of(const qlora_weight* w) {
+  WView v;
+  v.fmt = w->fmt;
+  v.O = w->O;
+  v.I = w->I;
+  v.block = w->block;
+  v.group = w->group < 1 ? 1 : w->group;
+  v.bits = w->bits;
+  v.codes = w->codes;
+  v.qcodes = w->scale_codes;
+  v.t = w->group_absmax;
+  v.mu = w->mean;
+  v.scale = w->scale;
+  v.bias = w->bias;
+  return v;
+}
+
+// ---------------------------------------------------------------- layouts
+
+struct FwdLayout {
+  size_t u = 0, tc = 0, total = 0;
+};
+struct BwdLayout {
+  size_t u = 0, v = 0, red = 0, tc = 0, total = 0;
+};
+
+FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t compute) {
+  FwdLayout L;
+  size_t off = kWsHeader;
+  L.u = off;
+  off += align_up((size_t)R * r * 4, 256);
+  L.tc = off;
+  if (compute == QLORA_COMPUTE_BF16) off += tc_fwd_ws(view_of(w), R);
+  L.total = off;
+  return L;
+}
+
+BwdLayout bwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t compute) {
+  BwdLayout L;
+  size_t off = kWsHeader;
+  L.u = off;
+  off += align_up((size_t)R * r * 4, 256);
+  L.v = off;
+  off += align_up((size_t)R * r * 4, 256);
+  L.red = off;
+  size_t red = coldot_ws(R, w->I, r);
+  size_t red2 = coldot_ws(R, w->O, r);
+  off += red > red2 ? red : red2;
+  L.tc = off;
+  if (compute == QLORA_COMPUTE_BF16) off += tc_dx_ws(view_of(w), R);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+}  // namespace qlora
+
+using namespace qlora;
+
+extern "C" {
+
+const char* qlora_status_string(qlora_status st) {
+  switch (st) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_SHAPE: return "inconsistent shape";
+    case QLORA_ERR_ALIGNMENT: return "misaligned pointer or workspace";
+    case QLORA_ERR_NONFINITE: return "non-finite weight";
+    case QLORA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case QLORA_ERR_CUDA: return "CUDA runtime error";
+    case QLORA_ERR_TIMEOUT: return "bounded device wait ran out";
+    case QLORA_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+qlora_status qlora_nf4_codebook(float out[16]) {
+  if (!out) return QLORA_ERR_INVALID_ARG;
+  memcpy(out, kNF4Host, sizeof(kNF4Host));
+  return QLORA_OK;
+}
+
+size_t qlora_nf4_payload_bytes(int64_t N, int32_t B, int32_t C) {
+  if (N < 0 || B < 1 || C < 1) return 0;
+  const int64_t M = nf4_blocks(N, B);
+  const int64_t S = (M + C - 1) / C;
+  return (size_t)((N + 1) / 2 + M + 4 * S + 4);
+}
+
+size_t qlora_quantize_nf4_workspace_bytes(int64_t N, int32_t B, int32_t C) {
+  if (N < 0 || B < 1 || C < 1) return 0;
+  return nf4_quantize_ws(N, B, C);
+}
+
+qlora_status qlora_quantize_nf4(const float* W, int64_t O, int64_t I, int32_t B, int32_t C,
+                                uint8_t* codes, uint8_t* scale_codes, float* t, float* mu,
+                                void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (O < 0 || I < 0 || B < 1 || C < 1) return QLORA_ERR_SHAPE;
+  const int64_t N = O * I;
+  if (!mu || !ws) return QLORA_ERR_INVALID_ARG;
+  if (N > 0 && (!W || !codes || !scale_codes || !t)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
+  if (ws_bytes < nf4_quantize_ws(N, B, C)) return QLORA_ERR_WORKSPACE;
+  qlora_status st = device_ready();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  st = cuda_status(launch_nf4_quantize(W, N, B, C, codes, scale_codes, t, mu, ws, s));
+  if (st != QLORA_OK) return st;
+  uint32_t h[3];
+  st = read_header(ws, s, h);
+  if (st != QLORA_OK) return st;
+  if (h[2]) return QLORA_ERR_NONFINITE;
+  return h[0] ? (qlora_status)h[0] : QLORA_OK;
+}
+
+size_t qlora_quantize_affine_workspace_bytes(int64_t N, int32_t bits, int32_t G) {
+  (void)N;
+  (void)bits;
+  (void)G;
+  return kWsHeader;
+}
+
+qlora_status qlora_quantize_affine(const float* W, int64_t O, int64_t I, int32_t bits, int32_t G,
+                                   uint8_t* codes, float* scale, float* bias, void* ws,
+                                   size_t ws_bytes, qlora_stream_t stream) {
+  if (O < 0 || I < 0 || G < 1) return QLORA_ERR_SHAPE;
+  if (bits != 4 && bits != 8) return QLORA_ERR_SHAPE;
+  const int64_t N = O * I;
+  if (!ws) return QLORA_ERR_INVALID_ARG;
+  if (N > 0 && (!W || !codes || !scale || !bias)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
+  if (ws_bytes < kWsHeader) return QLORA_ERR_WORKSPACE;
+  qlora_status st = device_ready();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  st = cuda_status(launch_affine_quantize(W, N, bits, G, codes, scale, bias, ws, s));
+  if (st != QLORA_OK) return st;
+  uint32_t h[3];
+  st = read_header(ws, s, h);
+  if (st != QLORA_OK) return st;
+  if (h[2]) return QLORA_ERR_NONFINITE;
+  return h[0] ? (qlora_status)h[0] : QLORA_OK;
+}
+
+qlora_status qlora_dequantize(const qlora_weight* w, float* W_hat, qlora_stream_t stream) {
+  qlora_status st = check_weight(w, false);
+  if (st != QLORA_OK) return st;
+  if (w->O * w->I > 0 && !W_hat) return QLORA_ERR_INVALID_ARG;
+  st = device_ready();
+  if (st != QLORA_OK) return st;
+  return cuda_status(launch_dequantize(view_of(w), W_hat, (cudaStream_t)stream));
+}
+
+size_t qlora_linear_workspace_bytes(const qlora_weight* w, int64_t R, int32_t r, int32_t op,
+                                    int32_t compute) {
+  if (!w || R < 0 || r < 1 || r > 64) return 0;
+  if (compute != QLORA_COMPUTE_FP32 && compute != QLORA_COMPUTE_BF16) return 0;
+  if (op == QLORA_OP_FWD) return fwd_layout(w, R, r, compute).total;
+  if (op == QLORA_OP_BWD) return bwd_layout(w, R, r, compute).total;
+  return 0;
+}
+
+static qlora_status check_linear_common(const qlora_weight* w, int64_t R, const float* A,
+                                        const float* B, int32_t r, int32_t compute, void* ws) {
+  qlora_status st = check_weight(w, true);
+  if (st != QLORA_OK) return st;
+  if (R < 0) return QLORA_ERR_SHAPE;
+  if (r < 1) return QLORA_ERR_SHAPE;
+  if (r > 64) return QLORA_ERR_UNSUPPORTED;
+  if (compute != QLORA_COMPUTE_FP32 && compute != QLORA_COMPUTE_BF16) return QLORA_ERR_INVALID_ARG;
+  if (!A || !B || !ws) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
+  return QLORA_OK;
+}
+
+qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, const float* A,
+                              const float* B, int32_t r, float alpha, int32_t compute, void* Y,
+                              float* U_out, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status st = check_linear_common(w, R, A, B, r, compute, ws);
+  if (st != QLORA_OK) return st;
+  if (R > 0 && (!X || !Y)) return QLORA_ERR_INVALID_ARG;
+  const FwdLayout L = fwd_layout(w, R, r, compute);
+  if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  st = device_ready();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader, s);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  if (R == 0) return QLORA_OK;
+  const float sc = alpha / (float)r;
+  float* U = U_out ? U_out : (float*)((char*)ws + L.u);
+  const WView v = view_of(w);
+  const bool bf16 = compute == QLORA_COMPUTE_BF16;
+  if (bf16 && tc_fwd_supported(v, X, Y, R)) {
+    e = launch_rowdot(X, true, R, w->I, A, false, r, U, s);
+    if (e == cudaSuccess)
+      e = launch_tc_fwd(v, X, R, U, B, r, sc, Y, (char*)ws + L.tc, (uint32_t*)ws, s);
+  } else {
+    e = launch_simt_fwd(v, X, R, A, B, r, sc, bf16, Y, U, s);
+  }
+  return cuda_status(e);
+}
+
+qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* dY, int64_t R,
+                              const float* A, const float* B, int32_t r, float alpha,
+                              const float* U_in, int32_t compute, void* dX, float* dA, float* dB,
+                              void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  qlora_status st = check_linear_common(w, R, A, B, r, compute, ws);
+  if (st != QLORA_OK) return st;
+  if (R > 0 && !dY) return QLORA_ERR_INVALID_ARG;
+  if (R > 0 && (dA || (dB && !U_in)) && !X) return QLORA_ERR_INVALID_ARG;
+  const BwdLayout L = bwd_layout(w, R, r, compute);
+  if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
+  st = device_ready();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader, s);
+  if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  const bool bf16 = compute == QLORA_COMPUTE_BF16;
+  const float sc = alpha / (float)r;
+  const WView v = view_of(w);
+  float* V = (float*)((char*)ws + L.v);
+  void* red = (char*)ws + L.red;
+  // V = dY B  (B is [O x r]: L(k = o, j) = B[o*r + j])
+  if (dX || dA) e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s);
+  if (e == cudaSuccess && dX) {
+    if (bf16 && tc_dx_supported(v, dY, dX, R))
+      e = launch_tc_dx(v, dY, R, V, A, r, sc, dX, (char*)ws + L.tc, (uint32_t*)ws, s);
+    else
+      e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s);
+  }
+  // dA = s V^T X   [r x I]
+  if (e == cudaSuccess && dA) e = launch_coldot(X, bf16, R, w->I, V, r, sc, false, dA, red, s);
+  // dB = s dY^T U  [O x r]
+  if (e == cudaSuccess && dB) {
+    const float* U = U_in;
+    if (!U) {
+      float* Uw = (float*)((char*)ws + L.u);
+      e = launch_rowdot(X, bf16, R, w->I, A, false, r, Uw, s);
+      U = Uw;
+    }
+    if (e == cudaSuccess) e = launch_coldot(dY, bf16, R, w->O, U, r, sc, true, dB, red, s);
+  }
+  return cuda_status(e);
+}
+
+qlora_status qlora_workspace_status(const void* ws, qlora_stream_t stream) {
+  if (!ws) return QLORA_ERR_INVALID_ARG;
+  qlora_status st = device_ready();
+  if (st != QLORA_OK) return st;
+  uint32_t h[3];
+  st = read_header(ws, (cudaStream_t)stream, h);
+  if (st != QLORA_OK) return st;
+  return h[0] ? (qlora_status)h[0] : QLORA_OK;
+}
+
+qlora_status qlora_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t limit_us,
+                                         qlora_stream_t stream) {
+  if (!ws) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
+  if (ws_bytes < kWsHeader) return QLORA_ERR_WORKSPACE;
+  if (limit_us < 1 || limit_us > 1000000) return QLORA_ERR_INVALID_ARG;
+  qlora_status st = device_ready();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemsetAsync(ws, 0, kWsHeader, s) != cudaSuccess) return QLORA_ERR_CUDA;
+  st = cuda_status(launch_wait_selftest((uint32_t*)ws, (uint64_t)limit_us * 1000ull, s));
+  if (st != QLORA_OK) return st;
+  return qlora_workspace_status(ws, stream);
+}
+
+uint64_t qlora_kernel_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// internal.h -- host-side declarations shared by the libqlora translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "qlora.h"
+
+namespace qlora {
+
+struct WView;
+
+extern std::atomic<uint64_t> g_launches;
+inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bounded-wait limit for device spin loops, nanoseconds.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// quantize.cu
+cudaError_t launch_nf4_quantize(const float* W, int64_t N, int32_t B, int32_t C, uint8_t* codes,
+                                uint8_t* qcodes, float* t, float* mu, void* ws, cudaStream_t st);
+size_t nf4_quantize_ws(int64_t N, int32_t B, int32_t C);
+cudaError_t launch_affine_quantize(const float* W, int64_t N, int32_t bits, int32_t G,
+                                   uint8_t* codes, float* scale, float* bias, void* ws,
+                                   cudaStream_t st);
+cudaError_t launch_dequantize(const WView& w, float* out, cudaStream_t st);
+
+// simt.cu -- generic (SIMT) linear kernels, both compute modes
+cudaError_t launch_simt_fwd(const WView& w, const void* X, int64_t R, const float* A,
+                            const float* B, int32_t r, float s, bool bf16, void* Y, float* U,
+                            cudaStream_t st);
+cudaError_t launch_simt_dx(const WView& w, const void* dY, int64_t R, const float* A,
+                           const float* V, int32_t r, float s, bool bf16, void* dX,
+                           cudaStream_t st);
+// adapter side products
+cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const float* L,
+                          bool l_is_kr, int32_t r, float* out, cudaStream_t st);
+size_t coldot_ws(int64_t R, int64_t N, int32_t r);
+cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
+                          int32_t r, float s, bool out_nr, float* out, void* ws,
+                          cudaStream_t st);
+// bf16 operand staging for the tensor-core path
+cudaError_t launch_pad_rows_bf16(const float* src, int64_t rows, int32_t r, float mul,
+                                 uint16_t* dst, cudaStream_t st);
+cudaError_t launch_pad_cols_bf16(const float* src, int32_t r, int64_t cols, float mul,
+                                 uint16_t* dst, cudaStream_t st);
+cudaError_t launch_splitk_reduce(const float* part, int32_t splits, int64_t R, int64_t N,
+                                 bool bf16_out, void* out, cudaStream_t st, float scale = 1.0f);
+
+// selftest
+cudaError_t launch_wait_selftest(uint32_t* ws_header, uint64_t limit_ns, cudaStream_t st);
+
+}  // namespace qlora

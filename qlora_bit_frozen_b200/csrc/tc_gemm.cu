@@ -1,0 +1,556 @@
+// tc_gemm.cu -- tcgen05 / TMEM kernels of the QLoRA linear layer (sm_100a).
+//
+// Forward  Y  = X W_hat^T + s U B^T     ("QLoRA Fine-Tuning", "Forward and
+// Input    dX = dY W_hat + s V A         backward"; "QLoRA on Mac",
+// gradient                               "Design / Q-LoRA layer")
+//
+// The frozen weight never exists as a floating-point matrix in HBM: packed
+// NF4 nibbles arrive in shared memory by TMA, decoder warps turn each
+// 64-weight block into bf16 (codebook level times the double-quant block
+// scale rebuilt from q_b, t_g and mu) directly in the 128-byte-swizzled
+// layout the tensor core reads, and tcgen05.mma accumulates in TMEM.
+//
+// Orientation: the decoded weight tile is the MMA "A" operand (M = 128
+// weight-side rows: output features in the forward, input features in the
+// input gradient) and the activation tile is the "B" operand (N = a tile of
+// tokens, 16..256).  Small token counts therefore cost no wasted MMA rows,
+// and the same kernel serves the bandwidth-bound and the tensor-bound
+// regimes (split-K supplies parallelism when there are few tiles).
+//   forward : A = W_hat[o, i] tile, K-major (i contiguous)   -> a_major = K
+//   dX      : A = W_hat^T[i, o] tile, MN-major (i contiguous) -> a_major = MN
+// Both layouts consist of 128-byte rows holding 64 consecutive weights of
+// one W row, i.e. exactly one NF4 block, so one decode routine serves both.
+//
+// The adapter term is one extra K step of the same accumulation: its A
+// operand is bf16(s B) (forward) or bf16(s A)^T (dX), zero-padded to 64
+// along the rank, and its B operand is bf16 U or V, all loaded by TMA.
+//
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator and
+// MMA issuer, warps 2..5 decoders, then epilogue (TMEM -> registers ->
+// global).  Every mbarrier wait is bounded (%globaltimer); on expiry the
+// CTA records QLORA_ERR_TIMEOUT in the workspace header, stops issuing
+// work, waits (bounded) for its copies in flight, frees TMEM and exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc_gemm.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr int kBM = 128;             // weight-side rows per CTA (MMA M)
+constexpr int kBK = 64;              // reduction step (one NF4 block)
+constexpr int kDecWarps = 4;         // decoder / epilogue warps
+constexpr int kThreads = 32 * (2 + kDecWarps);
+constexpr int kWTile = kBM * kBK * 2;  // decoded weight tile bytes (16 KB)
+constexpr int kPkTile = kBM * kBK / 2; // packed nibbles per step (4 KB)
+
+struct TcParams {
+  int64_t R;         // tokens
+  int32_t Mw;        // weight-side extent (O forward, I input gradient)
+  int32_t KB;        // reduction steps of 64
+  int32_t I;         // W row length
+  int32_t kb_per_split;
+  int32_t r_slices;  // ceil(r / 16): MMA K=16 slices of the adapter step
+  uint32_t C;        // scale-group size in blocks
+  const uint8_t* qcodes;
+  const float* t;
+  const float* mu;
+  void* out;         // bf16 [R x Mw], or fp32 partials [splits][R][Mw]
+  int32_t partial;
+  uint32_t* err;
+  uint64_t wait_ns;
+};
+
+// UMMA shared-memory descriptor, 128-byte swizzle (sm_100 version field).
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  d |= 2ull << 61;
+  return d;
+}
+
+// kind::f16 instruction descriptor: bf16 x bf16 -> fp32, B K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+template <int BN>
+struct Smem {
+  static constexpr int kAct = BN * kBK * 2;
+  static constexpr int kStage = kWTile + kAct + kPkTile;
+};
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+
+// Decode one 64-weight NF4 block (32 packed bytes at pk) with block scale s
+// into one 128-byte swizzled row at row_addr (row index within its 8-row
+// atom = sw).
+__device__ __forceinline__ void decode_row(const uint8_t* pk, float s, uint32_t row_addr,
+                                           uint32_t sw, const float* lut) {
+  const uint4 p0 = *reinterpret_cast<const uint4*>(pk);
+  const uint4 p1 = *reinterpret_cast<const uint4*>(pk + 16);
+  const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = weights 8j .. 8j+7 = packed word j
+    uint32_t o[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t byte = (w[j] >> (8 * b)) & 0xFFu;
+      const float lo = __fmul_rn(lut[byte & 15u], s);
+      const float hi = __fmul_rn(lut[byte >> 4], s);
+      o[b] = pack_bf16x2(lo, hi);
+    }
+    st_shared_v4(row_addr + ((j ^ sw) << 4), o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <bool DX, int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
+                      const __grid_constant__ CUtensorMap tm_pk,
+                      const __grid_constant__ CUtensorMap tm_aact,
+                      const __grid_constant__ CUtensorMap tm_aw, const TcParams p) {
+  using L = Smem<BN>;
+  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  constexpr uint32_t kIdesc = idesc_bf16(kBM, BN, DX);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* wdec = smem;                               // STAGES x 16 KB
+  uint8_t* act = wdec + STAGES * kWTile;              // STAGES x BN*128
+  uint8_t* pk = act + STAGES * L::kAct;               // STAGES x 4 KB
+  uint64_t* bars = (uint64_t*)(pk + STAGES * kPkTile);
+  uint64_t* full_act = bars;
+  uint64_t* full_pk = bars + STAGES;
+  uint64_t* dec = bars + 2 * STAGES;
+  uint64_t* empty = bars + 3 * STAGES;
+  uint64_t* acc_full = bars + 4 * STAGES;
+  volatile uint32_t* tmem_slot = (volatile uint32_t*)(acc_full + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+  float* lut = (float*)(abort_flag + 3);  // 16 floats
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kBM;
+  const int64_t n0 = (int64_t)blockIdx.y * BN;
+  const int split = blockIdx.z;
+  const int kb_lo = split * p.kb_per_split;
+  const int kb_hi = min(p.KB, kb_lo + p.kb_per_split);
+  const int has_ad = split == 0 ? 1 : 0;  // adapter step rides with split 0
+  const int T = (kb_hi - kb_lo) + has_ad;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full_act[s]), 1);
+      mbar_init(smem_u32(&full_pk[s]), 1);
+      mbar_init(smem_u32(&dec[s]), kDecWarps);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(acc_full), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 16) lut[threadIdx.x] = kNF4[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int it = 0; it < T; ++it) {
+        const int s = it % STAGES;
+        if (*abort_flag) break;
+        if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, p.wait_ns, p.err, 0x101)) {
+          *abort_flag = 1;
+          break;
+        }
+        const uint32_t fa = smem_u32(&full_act[s]), fp = smem_u32(&full_pk[s]);
+        if (has_ad && it == 0) {
+          mbar_arrive_expect_tx(fa, L::kAct + kWTile);
+          tma_load_2d(smem_u32(act + s * L::kAct), &tm_aact, fa, 0, (int32_t)n0);
+          if (!DX) {
+            tma_load_2d(smem_u32(wdec + s * kWTile), &tm_aw, fa, 0, m0);
+          } else {
+            tma_load_2d(smem_u32(wdec + s * kWTile), &tm_aw, fa, m0, 0);
+            tma_load_2d(smem_u32(wdec + s * kWTile + kWTile / 2), &tm_aw, fa, m0 + 64, 0);
+          }
+          mbar_arrive(fp);  // no packed data in the adapter step
+        } else {
+          const int kb = kb_lo + it - has_ad;
+          mbar_arrive_expect_tx(fa, L::kAct);
+          tma_load_2d(smem_u32(act + s * L::kAct), &tm_act, fa, kb * kBK, (int32_t)n0);
+          mbar_arrive_expect_tx(fp, kPkTile);
+          if (!DX)
+            tma_load_2d(smem_u32(pk + s * kPkTile), &tm_pk, fp, kb * (kBK / 2), m0);
+          else
+            tma_load_2d(smem_u32(pk + s * kPkTile), &tm_pk, fp, m0 / 2, kb * kBK);
+        }
+        issued = it + 1;
+      }
+      if (*abort_flag) {  // let copies in flight land before the CTA exits
+        for (int it = issued - STAGES < 0 ? 0 : issued - STAGES; it < issued; ++it) {
+          const int s = it % STAGES;
+          mbar_wait(smem_u32(&full_act[s]), (it / STAGES) & 1, p.wait_ns, nullptr, 0);
+          mbar_wait(smem_u32(&full_pk[s]), (it / STAGES) & 1, p.wait_ns, nullptr, 0);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      for (int it = 0; it < T; ++it) {
+        const int s = it % STAGES;
+        if (*abort_flag) break;
+        const uint32_t par = (it / STAGES) & 1;
+        if (!mbar_wait(smem_u32(&full_act[s]), par, p.wait_ns, p.err, 0x201) ||
+            !mbar_wait(smem_u32(&dec[s]), par, p.wait_ns, p.err, 0x202)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(wdec + s * kWTile);
+        const uint32_t b0 = smem_u32(act + s * L::kAct);
+        const int nsl = (has_ad && it == 0) ? p.r_slices : kBK / 16;
+        for (int kk = 0; kk < nsl; ++kk) {
+          const uint64_t ad = DX ? sdesc(a0 + kk * 2048, 8192, 1024) : sdesc(a0 + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc(b0 + kk * 32, 16, 1024);
+          umma_bf16(tmem, ad, bd, kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(smem_u32(&empty[s]));
+      }
+      umma_commit(smem_u32(acc_full));
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ decoders
+    const int u = threadIdx.x - 64;  // unit 0..127
+    const float mu = __ldg(p.mu);
+    const uint32_t bpr = (uint32_t)(p.I / kBK);  // blocks per W row
+    // unit -> (W row, block column, smem row) for a given step kb
+    auto block_of = [&](int kb) -> uint32_t {
+      if (!DX) return (uint32_t)(m0 + u) * bpr + (uint32_t)kb;
+      return (uint32_t)(kb * kBK + (u & 63)) * bpr + (uint32_t)(m0 / kBK) + (uint32_t)(u >> 6);
+    };
+    const uint32_t row_off = DX ? (uint32_t)((u >> 6) * (kWTile / 2) + (u & 63) * 128) : (uint32_t)u * 128;
+    const uint32_t sw = DX ? (uint32_t)(u & 7) : (uint32_t)(u & 7);
+    const uint32_t pk_off = DX ? (uint32_t)((u & 63) * 64 + (u >> 6) * 32) : (uint32_t)u * 32;
+    uint32_t q_next = 0;
+    float t_next = 0.0f;
+    if (T > has_ad) {
+      const uint32_t b = block_of(kb_lo);
+      q_next = __ldg(p.qcodes + b);
+      t_next = __ldg(p.t + b / p.C);
+    }
+    bool ok = true;
+    for (int it = 0; it < T; ++it) {
+      const int s = it % STAGES;
+      const uint32_t par = (it / STAGES) & 1;
+      const bool adapter = has_ad && it == 0;
+      float sc = 0.0f;
+      if (!adapter) {
+        sc = decode_block_scale(q_next, t_next, mu);
+        const int kb_n = kb_lo + it - has_ad + 1;
+        if (kb_n < kb_hi) {
+          const uint32_t b = block_of(kb_n);
+          q_next = __ldg(p.qcodes + b);
+          t_next = __ldg(p.t + b / p.C);
+        }
+      }
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
+      bool w_ok = mbar_wait(smem_u32(&empty[s]), par ^ 1, p.wait_ns, p.err, 0x301) &&
+                  mbar_wait(smem_u32(&full_pk[s]), par, p.wait_ns, p.err, 0x302);
+      if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
+      if (!adapter)
+        decode_row(pk + s * kPkTile + pk_off, sc, smem_u32(wdec + s * kWTile) + row_off, sw, lut);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&dec[s]));
+    }
+    // ------------------------------------------------------------ epilogue
+    const bool acc_ok = mbar_wait(smem_u32(acc_full), 0, p.wait_ns, p.err, 0x401);
+    tc_fence_after();
+    const bool aborted = __any_sync(0xffffffffu, !ok || !acc_ok || *abort_flag != 0);
+    if (!aborted) {
+      const int quad = warp & 3;  // TMEM lane quarter this warp may read
+      const int mw = m0 + quad * 32 + lane;
+      const size_t Mw = (size_t)p.Mw;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int64_t tok = n0 + c0 + j;
+          if (c0 + j < BN && tok < p.R) {
+            const float f = __uint_as_float(v[j]);
+            if (p.partial)
+              ((float*)p.out)[((size_t)split * (size_t)p.R + (size_t)tok) * Mw + mw] = f;
+            else
+              ((__nv_bfloat16*)p.out)[(size_t)tok * Mw + mw] = __float2bfloat16_rn(f);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+using EncodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiled)f;
+  }
+  return fn;
+}
+
+// 2D row-major tensor [rows x cols] of `esize`-byte elements, box [br x bc].
+bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
+              uint64_t rows, uint32_t bc, uint32_t br, bool swz128) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)esize};
+  cuuint32_t box[2] = {bc, br};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swz128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms_cached() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int BN>
+constexpr int stages_for() {
+  return BN >= 256 ? 4 : (BN >= 128 ? 5 : 4);
+}
+
+template <int BN>
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)stages_for<BN>() * Smem<BN>::kStage + 5 * 8 * stages_for<BN>() + 8 + 16 +
+         64 + 64;
+}
+
+template <bool DX, int BN>
+cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
+                      const CUtensorMap& d, const TcParams& p, cudaStream_t st) {
+  constexpr int S = stages_for<BN>();
+  auto kern = tc_qlinear_kernel<DX, BN, S>;
+  const size_t sm = smem_bytes<BN>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, sm, st>>>(a, b, c, d, p);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <bool DX>
+cudaError_t launch_plan(const TcPlan& pl, dim3 grid, const CUtensorMap& a, const CUtensorMap& b,
+                        const CUtensorMap& c, const CUtensorMap& d, const TcParams& p,
+                        cudaStream_t st) {
+  switch (pl.bn) {
+    case 16: return launch_bn<DX, 16>(grid, a, b, c, d, p, st);
+    case 32: return launch_bn<DX, 32>(grid, a, b, c, d, p, st);
+    case 64: return launch_bn<DX, 64>(grid, a, b, c, d, p, st);
+    case 128: return launch_bn<DX, 128>(grid, a, b, c, d, p, st);
+    default: return launch_bn<DX, 256>(grid, a, b, c, d, p, st);
+  }
+}
+
+bool ptr_aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+bool common_supported(const WView& w, int64_t R) {
+  if (w.fmt != QLORA_FMT_NF4_DQ || w.block != kBK || w.group < 1) return false;
+  if (R <= 0 || R > (int64_t)INT32_MAX - 256) return false;
+  if (w.I % 128 != 0 || w.O % 128 != 0) return false;
+  if (w.O > INT32_MAX || w.I > INT32_MAX) return false;
+  if ((w.O * w.I) / kBK >= (int64_t)UINT32_MAX) return false;
+  if (!ptr_aligned(w.codes, 16)) return false;
+  return encode_fn() != nullptr;
+}
+
+size_t partial_bytes(const TcPlan& pl, int64_t R, int64_t Mw) {
+  return pl.splits > 1 ? align_up((size_t)pl.splits * (size_t)R * (size_t)Mw * 4, 256) : 0;
+}
+
+}  // namespace
+
+TcPlan tc_plan(int64_t Mw, int64_t KB, int64_t R) {
+  TcPlan pl;
+  pl.bn = R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : R <= 128 ? 128 : 256;
+  pl.stages = 0;
+  const int64_t tiles = (Mw / kBM) * ((R + pl.bn - 1) / pl.bn);
+  int64_t splits = 1;
+  const int sms = num_sms_cached();
+  if (tiles > 0 && tiles < sms) {
+    splits = (2 * sms + tiles - 1) / tiles;
+    const int64_t max_splits = KB / 4 > 0 ? KB / 4 : 1;
+    if (splits > max_splits) splits = max_splits;
+  }
+  pl.kb_per_split = (int)((KB + splits - 1) / splits);
+  pl.splits = (int)((KB + pl.kb_per_split - 1) / pl.kb_per_split);
+  return pl;
+}
+
+bool tc_fwd_supported(const WView& w, const void* X, const void* Y, int64_t R) {
+  return common_supported(w, R) && ptr_aligned(X, 16) && ptr_aligned(Y, 2);
+}
+
+bool tc_dx_supported(const WView& w, const void* dY, const void* dX, int64_t R) {
+  return common_supported(w, R) && ptr_aligned(dY, 16) && ptr_aligned(dX, 2);
+}
+
+// Workspace: U_pad / V_pad bf16 [R x 64], the adapter weight operand bf16
+// (fwd: [O x 64]; dX: [64 x I]), split-K partials.
+size_t tc_fwd_ws(const WView& w, int64_t R) {
+  const TcPlan pl = tc_plan(w.O, w.I / kBK, R);
+  return align_up((size_t)R * 128, 256) + align_up((size_t)w.O * 128, 256) +
+         partial_bytes(pl, R, w.O);
+}
+
+size_t tc_dx_ws(const WView& w, int64_t R) {
+  const TcPlan pl = tc_plan(w.I, w.O / kBK, R);
+  return align_up((size_t)R * 128, 256) + align_up((size_t)w.I * 128, 256) +
+         partial_bytes(pl, R, w.I);
+}
+
+cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float* U,
+                          const float* B, int32_t r, float s, void* Y, void* tcws,
+                          uint32_t* hdr, cudaStream_t st) {
+  const int64_t O = w.O, I = w.I;
+  const TcPlan pl = tc_plan(O, I / kBK, R);
+  uint16_t* upad = (uint16_t*)tcws;
+  uint16_t* bpad = (uint16_t*)((char*)tcws + align_up((size_t)R * 128, 256));
+  float* part = (float*)((char*)bpad + align_up((size_t)O * 128, 256));
+  cudaError_t e = launch_pad_rows_bf16(U, R, r, 1.0f, upad, st);
+  if (e == cudaSuccess) e = launch_pad_rows_bf16(B, O, r, s, bpad, st);
+  if (e != cudaSuccess) return e;
+  CUtensorMap m_act, m_pk, m_aact, m_aw;
+  const uint32_t bn = (uint32_t)pl.bn;
+  if (!make_map(&m_act, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, R, 64, bn, true) ||
+      !make_map(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I / 2, O, 32, 128, false) ||
+      !make_map(&m_aact, upad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, true) ||
+      !make_map(&m_aw, bpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, O, 64, 128, true))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.R = R;
+  p.Mw = (int32_t)O;
+  p.KB = (int32_t)(I / kBK);
+  p.I = (int32_t)I;
+  p.kb_per_split = pl.kb_per_split;
+  p.r_slices = (r + 15) / 16;
+  p.C = (uint32_t)w.group;
+  p.qcodes = w.qcodes;
+  p.t = w.t;
+  p.mu = w.mu;
+  p.partial = pl.splits > 1;
+  p.out = pl.splits > 1 ? (void*)part : Y;
+  p.err = hdr;
+  p.wait_ns = kWaitLimitNs;
+  dim3 grid((unsigned)(O / kBM), (unsigned)((R + pl.bn - 1) / pl.bn), (unsigned)pl.splits);
+  e = launch_plan<false>(pl, grid, m_act, m_pk, m_aact, m_aw, p, st);
+  if (e != cudaSuccess || pl.splits == 1) return e;
+  return launch_splitk_reduce(part, pl.splits, R, O, true, Y, st);
+}
+
+cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float* V,
+                         const float* A, int32_t r, float s, void* dX, void* tcws, uint32_t* hdr,
+                         cudaStream_t st) {
+  const int64_t O = w.O, I = w.I;
+  const TcPlan pl = tc_plan(I, O / kBK, R);
+  uint16_t* vpad = (uint16_t*)tcws;
+  uint16_t* apad = (uint16_t*)((char*)tcws + align_up((size_t)R * 128, 256));
+  float* part = (float*)((char*)apad + align_up((size_t)I * 128, 256));
+  cudaError_t e = launch_pad_rows_bf16(V, R, r, 1.0f, vpad, st);
+  if (e == cudaSuccess) e = launch_pad_cols_bf16(A, r, I, s, apad, st);
+  if (e != cudaSuccess) return e;
+  CUtensorMap m_act, m_pk, m_aact, m_aw;
+  const uint32_t bn = (uint32_t)pl.bn;
+  if (!make_map(&m_act, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, O, R, 64, bn, true) ||
+      !make_map(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I / 2, O, 64, 64, false) ||
+      !make_map(&m_aact, vpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, true) ||
+      !make_map(&m_aw, apad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, 64, 64, 64, true))
+    return cudaErrorInvalidValue;
+  TcParams p;
+  p.R = R;
+  p.Mw = (int32_t)I;
+  p.KB = (int32_t)(O / kBK);
+  p.I = (int32_t)I;
+  p.kb_per_split = pl.kb_per_split;
+  p.r_slices = (r + 15) / 16;
+  p.C = (uint32_t)w.group;
+  p.qcodes = w.qcodes;
+  p.t = w.t;
+  p.mu = w.mu;
+  p.partial = pl.splits > 1;
+  p.out = pl.splits > 1 ? (void*)part : dX;
+  p.err = hdr;
+  p.wait_ns = kWaitLimitNs;
+  dim3 grid((unsigned)(I / kBM), (unsigned)((R + pl.bn - 1) / pl.bn), (unsigned)pl.splits);
+  e = launch_plan<true>(pl, grid, m_act, m_pk, m_aact, m_aw, p, st);
+  if (e != cudaSuccess || pl.splits == 1) return e;
+  return launch_splitk_reduce(part, pl.splits, R, I, true, dX, st);
+}
+
+// Failure-detection self test: one thread waits on an mbarrier that nothing
+// arrives on; the bounded wait gives up and records QLORA_ERR_TIMEOUT.
+__global__ void wait_selftest_kernel(uint32_t* hdr, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    mbar_wait(smem_u32(&bar), 0, limit_ns, hdr, 0x901);
+  }
+}
+
+cudaError_t launch_wait_selftest(uint32_t* ws_header, uint64_t limit_ns, cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(ws_header, limit_ns);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

@@ -1,0 +1,110 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every declared
+entry point, and its host logic (argument checks, sizes, codebook) behaves.
+No call here launches a kernel."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from qlora_bit_frozen_b200 import _ffi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _ffi.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(qlora_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_ffi.SIGNATURES), "binding and header disagree"
+
+
+def test_codebook_matches_oracle_bitwise(lib):
+    out = (ctypes.c_float * 16)()
+    assert lib.qlora_nf4_codebook(out) == 0
+    got = np.array(list(out), np.float32)
+    _, ref = oracle.nf4_codebook()
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("N,B,C", [(0, 64, 256), (1, 64, 256), (101, 64, 256), (65536, 64, 256),
+                                   (89128960, 64, 256), (231, 16, 3)])
+def test_payload_bytes_match_oracle(lib, N, B, C):
+    assert lib.qlora_nf4_payload_bytes(N, B, C) == oracle.nf4_payload_bytes(N, B, C)
+
+
+def test_bad_arguments_rejected_before_launch(lib):
+    ws = ctypes.create_string_buffer(1024)
+    wsp = ctypes.c_void_p((ctypes.addressof(ws) + 255) // 256 * 256)
+    # negative shape, zero block, null outputs, misaligned workspace
+    assert lib.qlora_quantize_nf4(None, -1, 4, 64, 256, None, None, None, None, wsp, 512, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_quantize_nf4(None, 4, 4, 0, 256, None, None, None, None, wsp, 512, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_quantize_nf4(None, 4, 64, 64, 256, None, None, None, None, wsp, 512, None) == _ffi.ERR_INVALID_ARG
+    mis = ctypes.c_void_p(wsp.value + 8)
+    dummy = ctypes.c_void_p(wsp.value)
+    assert lib.qlora_quantize_nf4(dummy, 4, 64, 64, 256, dummy, dummy, dummy, dummy, mis, 512, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_quantize_nf4(dummy, 4, 64, 64, 256, dummy, dummy, dummy, dummy, wsp, 16, None) == _ffi.ERR_WORKSPACE
+    assert lib.qlora_quantize_affine(dummy, 4, 64, 3, 64, dummy, dummy, dummy, wsp, 512, None) == _ffi.ERR_SHAPE
+
+    w = _ffi.qlora_weight(_ffi.FMT_NF4_DQ, 64, 128, 64, 256, 4, wsp.value, wsp.value, wsp.value, wsp.value, None, None)
+    P = ctypes.byref(w)
+    # r out of range, bad compute enum, null adapters, I not a multiple of the block
+    assert lib.qlora_linear_fwd(P, dummy, 4, dummy, dummy, 65, 1.0, 1, dummy, None, wsp, 1 << 20, None) == _ffi.ERR_UNSUPPORTED
+    assert lib.qlora_linear_fwd(P, dummy, 4, dummy, dummy, 0, 1.0, 1, dummy, None, wsp, 1 << 20, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_linear_fwd(P, dummy, 4, dummy, dummy, 8, 1.0, 7, dummy, None, wsp, 1 << 20, None) == _ffi.ERR_INVALID_ARG
+    assert lib.qlora_linear_fwd(P, dummy, 4, None, dummy, 8, 1.0, 1, dummy, None, wsp, 1 << 20, None) == _ffi.ERR_INVALID_ARG
+    assert lib.qlora_linear_fwd(P, dummy, 4, dummy, dummy, 8, 1.0, 1, dummy, None, wsp, 16, None) == _ffi.ERR_WORKSPACE
+    w.I = 100
+    assert lib.qlora_linear_fwd(P, dummy, 4, dummy, dummy, 8, 1.0, 1, dummy, None, wsp, 1 << 20, None) == _ffi.ERR_SHAPE
+    w.I = 128
+    w.fmt = 9
+    assert lib.qlora_dequantize(P, dummy, None) == _ffi.ERR_INVALID_ARG
+    w.fmt = _ffi.FMT_AFFINE
+    w.bits = 3
+    assert lib.qlora_dequantize(P, dummy, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_dequantize(None, dummy, None) == _ffi.ERR_INVALID_ARG
+
+
+def test_workspace_sizes_are_consistent(lib):
+    w = _ffi.qlora_weight(_ffi.FMT_NF4_DQ, 2048, 1024, 64, 256, 4, None, None, None, None, None, None)
+    P = ctypes.byref(w)
+    for R in (0, 1, 16, 130, 4096):
+        for op in (0, 1):
+            for comp in (0, 1):
+                n = lib.qlora_linear_workspace_bytes(P, R, 8, op, comp)
+                assert n >= 256 and n % 256 == 0
+    assert lib.qlora_linear_workspace_bytes(P, 16, 65, 0, 1) == 0
+    assert lib.qlora_linear_workspace_bytes(P, 16, 8, 2, 1) == 0
+
+
+def test_status_strings(lib):
+    for s in range(9):
+        assert lib.qlora_status_string(s)
+
+
+def test_no_device_means_error_not_fallback(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    ws = ctypes.create_string_buffer(4096)
+    wsp = ctypes.c_void_p((ctypes.addressof(ws) + 255) // 256 * 256)
+    d = ctypes.c_void_p(wsp.value)
+    st = lib.qlora_quantize_nf4(d, 1, 64, 64, 256, d, d, d, d, wsp, 2048, None)
+    assert st == _ffi.ERR_CUDA
