@@ -1,0 +1,481 @@
+"""Benchmark of the QLoRA linear hot path on B200.
+
+One step = forward + backward (Y, U, dX, dA, dB) of every linear of the
+workload, on one batch of synthetic inputs already resident in HBM.  The
+frozen weights are quantized once before timing (load time, as in training).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  Timing: CUDA events on the launching stream
+around each step, L2 flushed (a 2x-L2 buffer write) between timed steps
+outside the events, barrier + synchronize on both sides of the timed loop,
+max over ranks.  Under torchrun each rank runs a data-parallel replica on
+its own tokens and the adapter gradients dA/dB are summed across ranks with
+NCCL every step (the one exchange data parallelism needs).
+
+--impl reference times the CPU oracle (oracle/, plain C, fp64) on this
+host's cores on a bounded row sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s (large R) & packed-weight HBM GB/s (small R), % roofline"
+DEFAULT_WORKLOAD = "qwen3_0.6b_attn_qv"
+
+
+def algorithmic_flops(wl: synth.Workload, R: int) -> float:
+    """4 R O I + 6 R r (I + O) per linear (fwd + bwd; no recompute, no decode ops)."""
+    return float(sum(4.0 * R * l.O * l.I + 6.0 * R * wl.r * (l.I + l.O) for l in wl.linears))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+class Layer:
+    """Device buffers of one linear: quantized weight, adapters, inputs,
+    outputs and workspaces (all allocated before timing)."""
+
+    def __init__(self, q, torch, wl, li, R, rank_seed):
+        lin = wl.linears[li]
+        dev = "cuda"
+        W = synth.weight(wl, li)
+        A, B = synth.adapters(wl, li)
+        Wd = torch.from_numpy(W).to(dev)
+        self.w = q.qlora_quantize_nf4(Wd, wl.block, wl.group)
+        del Wd
+        self.A = torch.from_numpy(A).to(dev)
+        self.B = torch.from_numpy(B).to(dev)
+        # activations: per rank, distinct tokens (seeded), bf16
+        xs = synth.normal(wl.seed(li, "X") + 7919 * rank_seed, (R, lin.I))
+        ds = synth.normal(wl.seed(li, "dY") + 7919 * rank_seed, (R, lin.O))
+        _, xb = synth.bf16_round(xs)
+        _, db = synth.bf16_round(ds)
+        self.x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.dy_host = torch.from_numpy(db.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.X = self.x_host.to(dev)
+        self.dY = self.dy_host.to(dev)
+        self.Y = torch.empty((R, lin.O), dtype=torch.bfloat16, device=dev)
+        self.U = torch.empty((R, wl.r), dtype=torch.float32, device=dev)
+        self.dX = torch.empty((R, lin.I), dtype=torch.bfloat16, device=dev)
+        self.dA = torch.empty((wl.r, lin.I), dtype=torch.float32, device=dev)
+        self.dB = torch.empty((lin.O, wl.r), dtype=torch.float32, device=dev)
+        self.dA_host = torch.empty_like(self.dA, device="cpu").pin_memory()
+        self.dB_host = torch.empty_like(self.dB, device="cpu").pin_memory()
+        self.ws_f = q.workspace(q.qlora_linear_workspace_bytes(self.w, R, wl.r, 0, q.COMPUTE_BF16))
+        self.ws_b = q.workspace(q.qlora_linear_workspace_bytes(self.w, R, wl.r, 1, q.COMPUTE_BF16))
+        self.alpha = wl.alpha
+
+    def step(self, q, X=None, dY=None):
+        X = self.X if X is None else X
+        dY = self.dY if dY is None else dY
+        q.qlora_linear_fwd(self.w, X, self.A, self.B, self.alpha, Y=self.Y, U_out=self.U, ws=self.ws_f)
+        q.qlora_linear_bwd(self.w, X, dY, self.A, self.B, self.alpha, U=self.U, dX=self.dX, dA=self.dA,
+                           dB=self.dB, ws=self.ws_b)
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import qlora_bit_frozen_b200 as q
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    wl = synth.workload(args.workload)
+    R = wl.R
+    layers = [Layer(q, torch, wl, li, R, rank) for li in range(len(wl.linears))]
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def allreduce_grads():
+        if world > 1:
+            for L in layers:
+                dist.all_reduce(L.dA)
+                dist.all_reduce(L.dB)
+
+    def step():
+        for L in layers:
+            L.step(q)
+        allreduce_grads()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    barrier()
+    for L in layers:
+        assert q.qlora_workspace_status(L.ws_f) == 0 and q.qlora_workspace_status(L.ws_b) == 0
+
+    # ------------------------------------------------ timed region (device)
+    clocks = ClockSampler(local)
+    clocks.start()
+    q.qlora_kernel_timing_enable(64 * max(1, args.steps) * len(layers))
+    launches0 = q.qlora_kernel_launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    barrier()
+    launches = q.qlora_kernel_launch_count() - launches0
+    recs = q.qlora_kernel_timing_collect(64 * max(1, args.steps) * len(layers))
+    q.qlora_kernel_timing_enable(0)
+    clk = clocks.stop()
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    flops_step = algorithmic_flops(wl, R)
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+
+    # ---------------------------------------- end to end through the API
+    h2d = sum(L.x_host.numel() * 2 + L.dy_host.numel() * 2 for L in layers)
+    d2h = sum(L.dA.numel() * 4 + L.dB.numel() * 4 for L in layers)
+    xs = [torch.empty_like(L.X) for L in layers]
+    dys = [torch.empty_like(L.dY) for L in layers]
+
+    def e2e_step():
+        for L, X, dY in zip(layers, xs, dys):
+            X.copy_(L.x_host, non_blocking=True)
+            dY.copy_(L.dy_host, non_blocking=True)
+            L.step(q, X, dY)
+        allreduce_grads()
+        for L in layers:
+            L.dA_host.copy_(L.dA, non_blocking=True)
+            L.dB_host.copy_(L.dB, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        e2e_step()
+    barrier()
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        ee[i][0].record(stream)
+        e2e_step()
+        ee[i][1].record(stream)
+    barrier()
+    ems = sum(a.elapsed_time(b) for a, b in ee)
+    if world > 1:
+        t = torch.tensor([ems], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    e2e_value = flops_step * world / (ems / args.steps * 1e-3) / 1e12
+
+    # ------------------------------------------------------------- roofline
+    peaks = load_peaks()
+    by_kind = {}
+    for kind, kms, kfl in recs:
+        d = by_kind.setdefault(kind, [0.0, 0.0, 0])
+        d[0] += kms
+        d[1] += kfl
+        d[2] += 1
+    dom = max(by_kind.items(), key=lambda kv: kv[1][0]) if by_kind else None
+    roofline = None
+    kernels = {}
+    for kind, (kms, kfl, n) in sorted(by_kind.items()):
+        name = "tc_qlinear_fwd" if kind == 0 else "tc_qlinear_dx"
+        kernels[name] = {"launches": n, "ms_total": round(kms, 4),
+                         "tflops": round(kfl / (kms * 1e-3) / 1e12, 2) if kms > 0 else None,
+                         "share_of_step": round(kms / ms, 4) if ms > 0 else None}
+    if dom is not None:
+        kind, (kms, kfl, n) = dom
+        achieved = kfl / (kms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roofline = {"bound": "tensor", "kernel": "tc_qlinear_fwd" if kind == 0 else "tc_qlinear_dx",
+                    "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / peak, 4), "traffic": None,
+                    "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                    "flops_per_launch": kfl / n, "avg_launch_ms": kms / n}
+
+    small = None
+    if args.small_r and world == 1:
+        small = run_small_r(q, torch, peaks, args)
+
+    quant = None
+    if world == 1:
+        quant = time_quantize(q, torch, wl)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_rows)
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights and adapters)",
+            "config": {"workload": wl.name, "tokens_per_gpu": R,
+                       "linears": [[l.name, l.O, l.I] for l in wl.linears], "r": wl.r, "alpha": wl.alpha,
+                       "nf4_block": wl.block, "dq_group": wl.group, "compute": "bf16, fp32 accumulate",
+                       "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                       "l2": "flushed between timed steps (2x L2 write, outside the events)"},
+            "roofline": roofline, "kernels": kernels,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ems / args.steps, 5)},
+            "clocks": clk, "gpu_launches": int(launches),
+            "small_r": small, "quantize": quant,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_small_r(q, torch, peaks, args):
+    """Bandwidth-bound regime: R in {1, 16} against W [4096 x 4096] and
+    [12288 x 4096] (NF4, B=64, C=256), forward and dX, GB/s on packed weight
+    bytes.  Cold L2: rotating weight copies totalling >= 4x L2, captured in
+    a CUDA graph."""
+    out = {}
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    for name in ("bw_sweep_4096", "bw_sweep_12288"):
+        wl = synth.workload(name)
+        lin = wl.linears[0]
+        W = torch.from_numpy(synth.weight(wl, 0)).cuda()
+        base = q.qlora_quantize_nf4(W, 64, 256)
+        del W
+        payload = base.payload_bytes()
+        ncopy = max(2, math.ceil(4 * l2 / payload))
+        copies = [base] + [q.QuantizedWeight(base.fmt, base.O, base.I, base.block, base.group, base.bits,
+                                             base.codes.clone(), base.scale_codes.clone(),
+                                             base.group_absmax.clone(), base.mean.clone())
+                           for _ in range(ncopy - 1)]
+        A = torch.from_numpy(synth.adapters(wl, 0)[0]).cuda()
+        B = torch.from_numpy(synth.adapters(wl, 0)[1]).cuda()
+        for R in (1, 16):
+            X = torch.randn((R, lin.I), device="cuda").to(torch.bfloat16)
+            dY = torch.randn((R, lin.O), device="cuda").to(torch.bfloat16)
+            Y = torch.empty((R, lin.O), device="cuda", dtype=torch.bfloat16)
+            dX = torch.empty((R, lin.I), device="cuda", dtype=torch.bfloat16)
+            U = torch.empty((R, wl.r), device="cuda")
+            wsf = q.workspace(q.qlora_linear_workspace_bytes(base, R, wl.r, 0, 1))
+            wsb = q.workspace(q.qlora_linear_workspace_bytes(base, R, wl.r, 1, 1))
+            res = {}
+            for op in ("fwd", "dx"):
+                def call(w):
+                    if op == "fwd":
+                        q.qlora_linear_fwd(w, X, A, B, wl.alpha, Y=Y, U_out=U, ws=wsf)
+                    else:
+                        q.qlora_linear_bwd(w, None, dY, A, B, wl.alpha, U=U, want_da=False, want_db=False,
+                                           dX=dX, ws=wsb)
+                for w in copies:
+                    call(w)
+                torch.cuda.synchronize()
+                s = torch.cuda.Stream()
+                s.wait_stream(torch.cuda.current_stream())
+                g = torch.cuda.CUDAGraph()
+                reps = max(64, ncopy)
+                with torch.cuda.graph(g, stream=s):
+                    for k in range(reps):
+                        call(copies[k % ncopy])
+                torch.cuda.synchronize()
+                g.replay()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                g.replay()
+                e1.record()
+                torch.cuda.synchronize()
+                t_call = e0.elapsed_time(e1) / reps
+                gbs = payload / (t_call * 1e-3) / 1e9
+                res[op] = {"us_per_call": round(t_call * 1e3, 3), "packed_GBps": round(gbs, 1),
+                           "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+                del g
+            out[f"{name}_R{R}"] = {"packed_bytes": int(payload), **res}
+        del copies, base
+        torch.cuda.empty_cache()
+    out["peak_GBps"] = peaks["hbm_gbs"]
+    out["peak_source"] = f"{peaks['source']} HBM copy bandwidth"
+    out["timing"] = f"CUDA graph of >= 64 calls rotating weight copies >= 4x L2"
+    return out
+
+
+def time_quantize(q, torch, wl):
+    """Load-time NF4 + double-quant encode of the workload's weights (ms)."""
+    Ws = [torch.from_numpy(synth.weight(wl, li)).cuda() for li in range(len(wl.linears))]
+    for W in Ws:
+        q.qlora_quantize_nf4(W)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for W in Ws:
+        q.qlora_quantize_nf4(W)  # synchronizes (reads the non-finite flag)
+    dt = time.perf_counter() - t0
+    n = sum(W.numel() for W in Ws)
+    return {"ms": round(dt * 1e3, 3), "weights": int(n), "GBps_fp32_in": round(n * 4 / dt / 1e9, 1),
+            "note": "host wall clock incl. the flag read-back synchronization"}
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(wl, rows):
+    """The oracle (plain C, fp64, OpenMP) on the first `rows` tokens of every
+    linear: Y, U, dX, dA, dB.  TFLOP/s on the algorithmic flops of the sample."""
+    import oracle
+    R = min(rows, wl.R)
+    t_total = 0.0
+    for li in range(len(wl.linears)):
+        W = synth.weight(wl, li)
+        A, B = synth.adapters(wl, li)
+        xw, _, dw, _ = synth.activations(wl, li, R)
+        ow = oracle.quantize_nf4(W, wl.block, wl.group)
+        t0 = time.perf_counter()
+        oracle.linear_fwd(ow, xw, A, B, wl.r, wl.alpha)
+        oracle.linear_bwd(ow, xw, dw, A, B, wl.r, wl.alpha)
+        t_total += time.perf_counter() - t0
+    fl = algorithmic_flops(wl, R)
+    return {"value": round(fl / t_total / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": round(t_total, 3),
+            "sample": f"first {R} of {wl.R} tokens of every linear of {wl.name}; Y, U, dX, dA, dB in fp64"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, bounded row sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    wl = synth.workload(args.workload)
+    R = min(args.cpu_rows, wl.R)
+    prep = []
+    for li in range(len(wl.linears)):
+        W = synth.weight(wl, li)
+        A, B = synth.adapters(wl, li)
+        xw, _, dw, _ = synth.activations(wl, li, R)
+        prep.append((oracle.quantize_nf4(W, wl.block, wl.group), xw, dw, A, B))
+
+    def step():
+        for ow, xw, dw, A, B in prep:
+            oracle.linear_fwd(ow, xw, A, B, wl.r, wl.alpha)
+            oracle.linear_bwd(ow, xw, dw, A, B, wl.r, wl.alpha)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    fl = algorithmic_flops(wl, R)
+    value = fl * args.steps / dt / 1e12
+    sample = f"first {R} of {wl.R} tokens of every linear of {wl.name} per step; Y, U, dX, dA, dB in fp64"
+    line = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "tokens_sampled": R, "r": wl.r, "alpha": wl.alpha},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOADS[1:])
+    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-small-r", dest="small_r", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

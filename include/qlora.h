@@ -239,6 +239,24 @@ qlora_status qlora_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t lim
  */
 uint64_t qlora_kernel_launch_count(void);
 
+/*
+ * HOST.  Kernel timing instrumentation.  With max_records > 0 the library
+ * records a CUDA event pair on the launching stream around each launch of
+ * its tensor-core GEMM kernels (up to max_records launches; events are
+ * created here, no device memory is allocated); 0 disables and drops
+ * pending records.
+ */
+qlora_status qlora_kernel_timing_enable(int32_t max_records);
+
+/*
+ * HOST.  Waits for the recorded event pairs, writes up to `max` launch
+ * durations (milliseconds) to ms[] and each launch's kind to kind[]
+ * (0 = forward GEMM, 1 = input-gradient GEMM) and its algorithmic flop count
+ * to flops[] (host arrays; any may be NULL), clears the records and returns
+ * how many were written (negative on a CUDA error).
+ */
+int32_t qlora_kernel_timing_collect(float* ms, int32_t* kind, double* flops, int32_t max);
+
 #ifdef __cplusplus
 }
 #endif

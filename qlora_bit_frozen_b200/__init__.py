@@ -24,6 +24,7 @@ __all__ = [
     "qlora_nf4_payload_bytes", "qlora_quantize_nf4", "qlora_quantize_affine", "qlora_dequantize",
     "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_workspace_status", "qlora_selftest_wait_timeout", "qlora_kernel_launch_count",
+    "qlora_kernel_timing_enable", "qlora_kernel_timing_collect",
     "COMPUTE_FP32", "COMPUTE_BF16", "FMT_NF4_DQ", "FMT_AFFINE", "workspace",
 ]
 
@@ -224,3 +225,18 @@ def qlora_selftest_wait_timeout(limit_us: int = 1000, stream=None, device="cuda"
 
 def qlora_kernel_launch_count() -> int:
     return int(_ffi.load().qlora_kernel_launch_count())
+
+
+def qlora_kernel_timing_enable(max_records: int) -> None:
+    _check(_ffi.load().qlora_kernel_timing_enable(int(max_records)), "qlora_kernel_timing_enable")
+
+
+def qlora_kernel_timing_collect(max_records: int = 4096):
+    """[(kind, ms, flops)] of the tensor-core GEMM launches recorded since enable."""
+    ms = (ctypes.c_float * max_records)()
+    kind = (ctypes.c_int32 * max_records)()
+    fl = (ctypes.c_double * max_records)()
+    n = _ffi.load().qlora_kernel_timing_collect(ms, kind, fl, max_records)
+    if n < 0:
+        raise QLoraError(_ffi.ERR_CUDA, "qlora_kernel_timing_collect")
+    return [(int(kind[i]), float(ms[i]), float(fl[i])) for i in range(n)]

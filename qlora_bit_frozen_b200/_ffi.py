@@ -65,6 +65,8 @@ SIGNATURES = {
     "qlora_workspace_status": (ctypes.c_int, [_P, _P]),
     "qlora_selftest_wait_timeout": (ctypes.c_int, [_P, _sz, _u32, _P]),
     "qlora_kernel_launch_count": (ctypes.c_uint64, []),
+    "qlora_kernel_timing_enable": (ctypes.c_int, [_i32]),
+    "qlora_kernel_timing_collect": (ctypes.c_int32, [_P, _P, _P, _i32]),
 }
 
 _lib = None

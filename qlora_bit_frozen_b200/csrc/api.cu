@@ -2,6 +2,9 @@
 // host-side argument checks, workspace layout and kernel dispatch.
 #include <string.h>
 
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 #include "internal.h"
 #include "tc_gemm.h"
@@ -9,6 +12,48 @@
 namespace qlora {
 
 std::atomic<uint64_t> g_launches{0};
+
+// ------------------------------------------------- kernel timing records
+namespace {
+struct TimingRec {
+  cudaEvent_t a, b;
+  int kind;
+  double flops;
+};
+std::mutex g_tmu;
+std::vector<TimingRec> g_trecs;
+int g_tmax = 0;
+}  // namespace
+
+int timing_begin(cudaStream_t st, int kind, double flops) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  if ((int)g_trecs.size() >= g_tmax) return -1;
+  TimingRec r;
+  if (cudaEventCreate(&r.a) != cudaSuccess) return -1;
+  if (cudaEventCreate(&r.b) != cudaSuccess) {
+    cudaEventDestroy(r.a);
+    return -1;
+  }
+  r.kind = kind;
+  r.flops = flops;
+  cudaEventRecord(r.a, st);
+  g_trecs.push_back(r);
+  return (int)g_trecs.size() - 1;
+}
+
+void timing_end(int slot, cudaStream_t st) {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_tmu);
+  if (slot < (int)g_trecs.size()) cudaEventRecord(g_trecs[slot].b, st);
+}
+
+static void timing_clear_locked() {
+  for (auto& r : g_trecs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  g_trecs.clear();
+}
 
 namespace {
 
@@ -329,5 +374,36 @@ qlora_status qlora_selftest_wait_timeout(void* ws, size_t ws_bytes, uint32_t lim
 }
 
 uint64_t qlora_kernel_launch_count(void) { return g_launches.load(); }
+
+qlora_status qlora_kernel_timing_enable(int32_t max_records) {
+  if (max_records < 0) return QLORA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_tmu);
+  timing_clear_locked();
+  g_tmax = max_records;
+  return QLORA_OK;
+}
+
+int32_t qlora_kernel_timing_collect(float* ms, int32_t* kind, double* flops, int32_t max) {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  int32_t n = 0;
+  for (auto& r : g_trecs) {
+    if (n >= max) break;
+    if (cudaEventSynchronize(r.b) != cudaSuccess) {
+      timing_clear_locked();
+      return -1;
+    }
+    float t = 0.0f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
+      timing_clear_locked();
+      return -1;
+    }
+    if (ms) ms[n] = t;
+    if (kind) kind[n] = r.kind;
+    if (flops) flops[n] = r.flops;
+    ++n;
+  }
+  timing_clear_locked();
+  return n;
+}
 
 }  // extern "C"

@@ -55,4 +55,8 @@ cudaError_t launch_splitk_reduce(const float* part, int32_t splits, int64_t R, i
 // selftest
 cudaError_t launch_wait_selftest(uint32_t* ws_header, uint64_t limit_ns, cudaStream_t st);
 
+// kernel timing instrumentation (api.cu): returns a slot to record into, or -1
+int timing_begin(cudaStream_t st, int kind, double flops);
+void timing_end(int slot, cudaStream_t st);
+
 }  // namespace qlora

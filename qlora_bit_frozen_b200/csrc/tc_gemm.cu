@@ -55,6 +55,7 @@ struct TcParams {
   int32_t I;         // W row length
   int32_t kb_per_split;
   int32_t r_slices;  // ceil(r / 16): MMA K=16 slices of the adapter step
+  int32_t rank;      // r (for the algorithmic flop count only)
   uint32_t C;        // scale-group size in blocks
   const uint8_t* qcodes;
   const float* t;
@@ -383,7 +384,11 @@ cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, con
   const size_t sm = smem_bytes<BN>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
+  const double flops = 2.0 * (double)p.R * (double)p.Mw * (double)p.KB * kBK +
+                       2.0 * (double)p.R * (double)p.Mw * (double)p.rank;
+  const int slot = timing_begin(st, DX ? 1 : 0, flops);
   kern<<<grid, kThreads, sm, st>>>(a, b, c, d, p);
+  timing_end(slot, st);
   count_launch();
   return cudaGetLastError();
 }
@@ -483,6 +488,7 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   p.I = (int32_t)I;
   p.kb_per_split = pl.kb_per_split;
   p.r_slices = (r + 15) / 16;
+  p.rank = r;
   p.C = (uint32_t)w.group;
   p.qcodes = w.qcodes;
   p.t = w.t;
@@ -522,6 +528,7 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   p.I = (int32_t)I;
   p.kb_per_split = pl.kb_per_split;
   p.r_slices = (r + 15) / 16;
+  p.rank = r;
   p.C = (uint32_t)w.group;
   p.qcodes = w.qcodes;
   p.t = w.t;
