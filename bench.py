@@ -166,11 +166,10 @@ def run_gpu(args):
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    from qlora_bit_frozen_b200 import dp
+
     def allreduce_grads():
-        if world > 1:
-            for L in layers:
-                dist.all_reduce(L.dA)
-                dist.all_reduce(L.dB)
+        dp.allreduce_adapter_grads([g for L in layers for g in (L.dA, L.dB)])
 
     def step():
         for L in layers:
@@ -186,31 +185,48 @@ def run_gpu(args):
         flush.zero_()
         step()
     barrier()
-    for L in layers:
-        assert q.qlora_workspace_status(L.ws_f) == 0 and q.qlora_workspace_status(L.ws_b) == 0
 
     # ------------------------------------------------ timed region (device)
+    # One step is captured once in a CUDA graph (no host launch gaps in the
+    # device timing); the library records an event pair around each of its
+    # tensor-core GEMM launches inside the graph.
+    nrec = 16 * len(layers)
+    q.qlora_kernel_timing_enable(nrec)
+    n_before = q.qlora_kernel_launch_count()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
+        step()
+    kernels_per_step = q.qlora_kernel_launch_count() - n_before
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
+    barrier()
     clocks = ClockSampler(local)
     clocks.start()
-    q.qlora_kernel_timing_enable(64 * max(1, args.steps) * len(layers))
-    launches0 = q.qlora_kernel_launch_count()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    recs = []
     barrier()
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
-        step()
+        graph.replay()
         ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        try:
+            recs.extend(q.qlora_kernel_timing_collect(nrec))
+        except q.QLoraError as e:  # keep the step timing; report no roofline
+            print(f"kernel timing unavailable: {e}", file=sys.stderr)
     barrier()
-    launches = q.qlora_kernel_launch_count() - launches0
-    recs = q.qlora_kernel_timing_collect(64 * max(1, args.steps) * len(layers))
-    q.qlora_kernel_timing_enable(0)
     clk = clocks.stop()
-    ms = sum(a.elapsed_time(b) for a, b in ev)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    launches = kernels_per_step * args.steps
+    ms = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), device="cuda")
+    del graph
+    q.qlora_kernel_timing_enable(0)
+    for L in layers:
+        assert q.qlora_workspace_status(L.ws_f) == 0 and q.qlora_workspace_status(L.ws_b) == 0
     ms_per_step = ms / args.steps
     flops_step = algorithmic_flops(wl, R)
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
@@ -241,11 +257,7 @@ def run_gpu(args):
         e2e_step()
         ee[i][1].record(stream)
     barrier()
-    ems = sum(a.elapsed_time(b) for a, b in ee)
-    if world > 1:
-        t = torch.tensor([ems], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
+    ems = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in ee), device="cuda")
     e2e_value = flops_step * world / (ems / args.steps * 1e-3) / 1e12
 
     # ------------------------------------------------------------- roofline
@@ -303,7 +315,8 @@ def run_gpu(args):
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ems / args.steps, 5)},
-            "clocks": clk, "gpu_launches": int(launches),
+            "clocks": clk, "gpu_launches": int(launches), "kernels_per_step": int(kernels_per_step),
+            "timing": "device step captured once in a CUDA graph and replayed; CUDA events around each replay",
             "small_r": small, "quantize": quant,
         }
         print(json.dumps(line), flush=True)
@@ -425,7 +438,7 @@ def run_reference(args):
         return
     import oracle
     wl = synth.workload(args.workload)
-    R = min(args.cpu_rows, wl.R)
+    R = min(args.ref_rows, wl.R)
     prep = []
     for li in range(len(wl.linears)):
         W = synth.weight(wl, li)
@@ -465,7 +478,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOADS[1:])
-    ap.add_argument("--cpu-rows", type=int, default=512)
+    ap.add_argument("--cpu-rows", type=int, default=1 << 30,
+                    help="tokens of the CPU-baseline sample (default: the whole workload)")
+    ap.add_argument("--ref-rows", type=int, default=1024, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-r", dest="small_r", action="store_false")
     args = ap.parse_args()

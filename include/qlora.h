@@ -252,8 +252,10 @@ qlora_status qlora_kernel_timing_enable(int32_t max_records);
  * HOST.  Waits for the recorded event pairs, writes up to `max` launch
  * durations (milliseconds) to ms[] and each launch's kind to kind[]
  * (0 = forward GEMM, 1 = input-gradient GEMM) and its algorithmic flop count
- * to flops[] (host arrays; any may be NULL), clears the records and returns
- * how many were written (negative on a CUDA error).
+ * to flops[] (host arrays; any may be NULL) and returns how many were
+ * written (negative on a CUDA error).  Records are kept (launches captured
+ * in a CUDA graph re-record the same events at every replay, so collect
+ * after each replay); qlora_kernel_timing_enable() drops them.
  */
 int32_t qlora_kernel_timing_collect(float* ms, int32_t* kind, double* flops, int32_t max);
 

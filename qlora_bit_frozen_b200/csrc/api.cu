@@ -25,6 +25,16 @@ std::vector<TimingRec> g_trecs;
 int g_tmax = 0;
 }  // namespace
 
+// Under stream capture an event record must be an external event node to
+// record at every replay of the graph.
+static void record_event(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, st);
+}
+
 int timing_begin(cudaStream_t st, int kind, double flops) {
   std::lock_guard<std::mutex> lk(g_tmu);
   if ((int)g_trecs.size() >= g_tmax) return -1;
@@ -36,7 +46,7 @@ int timing_begin(cudaStream_t st, int kind, double flops) {
   }
   r.kind = kind;
   r.flops = flops;
-  cudaEventRecord(r.a, st);
+  record_event(r.a, st);
   g_trecs.push_back(r);
   return (int)g_trecs.size() - 1;
 }
@@ -44,7 +54,7 @@ int timing_begin(cudaStream_t st, int kind, double flops) {
 void timing_end(int slot, cudaStream_t st) {
   if (slot < 0) return;
   std::lock_guard<std::mutex> lk(g_tmu);
-  if (slot < (int)g_trecs.size()) cudaEventRecord(g_trecs[slot].b, st);
+  if (slot < (int)g_trecs.size()) record_event(g_trecs[slot].b, st);
 }
 
 static void timing_clear_locked() {
@@ -296,9 +306,9 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
   const WView v = view_of(w);
   const bool bf16 = compute == QLORA_COMPUTE_BF16;
   if (bf16 && tc_fwd_supported(v, X, Y, R)) {
-    e = launch_rowdot(X, true, R, w->I, A, false, r, U, s);
-    if (e == cudaSuccess)
-      e = launch_tc_fwd(v, X, R, U, B, r, sc, Y, (char*)ws + L.tc, (uint32_t*)ws, s);
+    void* tcws = (char*)ws + L.tc;
+    e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws));
+    if (e == cudaSuccess) e = launch_tc_fwd(v, X, R, U, B, r, sc, Y, tcws, (uint32_t*)ws, s);
   } else {
     e = launch_simt_fwd(v, X, R, A, B, r, sc, bf16, Y, U, s);
   }
@@ -325,11 +335,14 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   const WView v = view_of(w);
   float* V = (float*)((char*)ws + L.v);
   void* red = (char*)ws + L.red;
-  // V = dY B  (B is [O x r]: L(k = o, j) = B[o*r + j])
-  if (dX || dA) e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s);
+  // V = dY B  (B is [O x r]: L(k = o, j) = B[o*r + j]); its padded bf16 copy
+  // feeds the tensor-core kernel's adapter step
+  const bool tc = dX && bf16 && tc_dx_supported(v, dY, dX, R);
+  void* tcws = (char*)ws + L.tc;
+  if (dX || dA) e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, tc ? tc_act_pad(tcws) : nullptr);
   if (e == cudaSuccess && dX) {
-    if (bf16 && tc_dx_supported(v, dY, dX, R))
-      e = launch_tc_dx(v, dY, R, V, A, r, sc, dX, (char*)ws + L.tc, (uint32_t*)ws, s);
+    if (tc)
+      e = launch_tc_dx(v, dY, R, V, A, r, sc, dX, tcws, (uint32_t*)ws, s);
     else
       e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s);
   }
@@ -388,21 +401,14 @@ int32_t qlora_kernel_timing_collect(float* ms, int32_t* kind, double* flops, int
   int32_t n = 0;
   for (auto& r : g_trecs) {
     if (n >= max) break;
-    if (cudaEventSynchronize(r.b) != cudaSuccess) {
-      timing_clear_locked();
-      return -1;
-    }
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return -1;
     float t = 0.0f;
-    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) {
-      timing_clear_locked();
-      return -1;
-    }
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return -1;
     if (ms) ms[n] = t;
     if (kind) kind[n] = r.kind;
     if (flops) flops[n] = r.flops;
     ++n;
   }
-  timing_clear_locked();
   return n;
 }
 

@@ -38,8 +38,10 @@ cudaError_t launch_simt_dx(const WView& w, const void* dY, int64_t R, const floa
                            const float* V, int32_t r, float s, bool bf16, void* dX,
                            cudaStream_t st);
 // adapter side products
+// adapter.cu
 cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const float* L,
-                          bool l_is_kr, int32_t r, float* out, cudaStream_t st);
+                          bool l_is_kr, int32_t r, float* out, cudaStream_t st,
+                          uint16_t* pad = nullptr);
 size_t coldot_ws(int64_t R, int64_t N, int32_t r);
 cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
                           int32_t r, float s, bool out_nr, float* out, void* ws,

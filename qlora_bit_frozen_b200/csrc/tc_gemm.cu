@@ -43,7 +43,8 @@ namespace {
 
 constexpr int kBM = 128;             // weight-side rows per CTA (MMA M)
 constexpr int kBK = 64;              // reduction step (one NF4 block)
-constexpr int kDecWarps = 4;         // decoder / epilogue warps
+constexpr int kDecGroups = 2;        // decoder groups (alternate K steps)
+constexpr int kDecWarps = 4 * kDecGroups;  // decoder / epilogue warps
 constexpr int kThreads = 32 * (2 + kDecWarps);
 constexpr int kWTile = kBM * kBK * 2;  // decoded weight tile bytes (16 KB)
 constexpr int kPkTile = kBM * kBK / 2; // packed nibbles per step (4 KB)
@@ -98,27 +99,90 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // Decode one 64-weight NF4 block (32 packed bytes at pk) with block scale s
 // into one 128-byte swizzled row at row_addr (row index within its 8-row
 // atom = sw).
+//
+// The 16 possible outputs bf16(fp32(c[k] * s)) are formed once per block
+// and kept in registers as two byte planes (low and high byte of each bf16,
+// 4 entries per register); each group of 4 nibbles then selects its bytes
+// with byte permutes: one permute per plane and per half of the table
+// (nibble bits 0..2), one to pick the half (nibble bit 3) and two to
+// interleave the planes back into bf16 pairs.  No shared-memory lookups.
 __device__ __forceinline__ void decode_row(const uint8_t* pk, float s, uint32_t row_addr,
-                                           uint32_t sw, const float* lut) {
+                                           uint32_t sw) {
+  uint32_t P[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    P[j] = pack_bf16x2(__fmul_rn(kNF4[2 * j], s), __fmul_rn(kNF4[2 * j + 1], s));
+  // byte planes: L[q] / H[q] hold the low / high bytes of entries 4q .. 4q+3
+  const uint32_t L0 = __byte_perm(P[0], P[1], 0x6420), H0 = __byte_perm(P[0], P[1], 0x7531);
+  const uint32_t L1 = __byte_perm(P[2], P[3], 0x6420), H1 = __byte_perm(P[2], P[3], 0x7531);
+  const uint32_t L2 = __byte_perm(P[4], P[5], 0x6420), H2 = __byte_perm(P[4], P[5], 0x7531);
+  const uint32_t L3 = __byte_perm(P[6], P[7], 0x6420), H3 = __byte_perm(P[6], P[7], 0x7531);
   const uint4 p0 = *reinterpret_cast<const uint4*>(pk);
   const uint4 p1 = *reinterpret_cast<const uint4*>(pk + 16);
   const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = weights 8j .. 8j+7 = packed word j
+  for (int j = 0; j < 8; ++j) {  // word j = weights 8j .. 8j+7 (nibble i = weight 8j+i)
     uint32_t o[4];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const uint32_t byte = (w[j] >> (8 * b)) & 0xFFu;
-      const float lo = __fmul_rn(lut[byte & 15u], s);
-      const float hi = __fmul_rn(lut[byte >> 4], s);
-      o[b] = pack_bf16x2(lo, hi);
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t x = h ? (w[j] >> 16) : w[j];  // 4 nibbles in the low 16 bits
+      const uint32_t s7 = x & 0x7777u;
+      const uint32_t alo = __byte_perm(L0, L1, s7), blo = __byte_perm(L2, L3, s7);
+      const uint32_t ahi = __byte_perm(H0, H1, s7), bhi = __byte_perm(H2, H3, s7);
+      const uint32_t sb = ((x >> 1) & 0x4444u) | 0x3210u;  // bit 3 -> second half
+      const uint32_t lo = __byte_perm(alo, blo, sb), hi = __byte_perm(ahi, bhi, sb);
+      o[2 * h] = __byte_perm(lo, hi, 0x5140);
+      o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
     }
     st_shared_v4(row_addr + ((j ^ sw) << 4), o[0], o[1], o[2], o[3]);
   }
 }
 
+// TMEM accumulator columns [c_begin, c_end) of this warp's 32 lanes ->
+// global memory: bf16 outputs, or fp32 split-K partials.
+__device__ __noinline__ void epilogue_store(uint32_t tmem, int quad, int lane, int m0, int64_t n0,
+                                            int c_begin, int c_end, int split, const TcParams& p) {
+  const int mw = m0 + quad * 32 + lane;
+  const size_t Mw = (size_t)p.Mw;
+#pragma unroll 1
+  for (int c0 = c_begin; c0 < c_end; c0 += 32) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
+    tmem_ld_wait();
+    // one token per j: 32 lanes store 32 consecutive weight-side entries
+    const int64_t tok0 = n0 + c0;
+    const int jmax = (int)min((int64_t)min(32, c_end - c0), p.R - tok0);
+    if (p.partial) {
+      float* dst = (float*)p.out + ((size_t)split * (size_t)p.R + (size_t)tok0) * Mw + mw;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < jmax) *dst = __uint_as_float(v[j]);
+        dst += Mw;
+      }
+    } else {
+      __nv_bfloat16* dst = (__nv_bfloat16*)p.out + (size_t)tok0 * Mw + mw;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j < jmax) *dst = __float2bfloat16_rn(__uint_as_float(v[j]));
+        dst += Mw;
+      }
+    }
+  }
+}
+
+template <int BN>
+constexpr int stages_for() {
+  return BN >= 256 ? 4 : (BN >= 64 ? 3 : 4);
+}
+// CTAs per SM the kernel is built for (tiles up to 128 tokens leave room
+// in shared memory, TMEM and registers for two).
+template <int BN>
+constexpr int min_ctas() {
+  return BN >= 256 ? 1 : 2;
+}
+
 template <bool DX, int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, min_ctas<BN>())
     tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_pk,
                       const __grid_constant__ CUtensorMap tm_aact,
@@ -140,7 +204,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = bars + 4 * STAGES;
   volatile uint32_t* tmem_slot = (volatile uint32_t*)(acc_full + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
-  float* lut = (float*)(abort_flag + 3);  // 16 floats
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kBM;
@@ -155,14 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_u32(&full_act[s]), 1);
       mbar_init(smem_u32(&full_pk[s]), 1);
-      mbar_init(smem_u32(&dec[s]), kDecWarps);
+      mbar_init(smem_u32(&dec[s]), 4);  // the 4 warps of one decoder group
       mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (threadIdx.x < 16) lut[threadIdx.x] = kNF4[threadIdx.x];
   if (warp == 1) {
     tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
     tmem_relinquish();
@@ -243,35 +305,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ decoders
-    const int u = threadIdx.x - 64;  // unit 0..127
+    // Two groups of 4 warps; group g decodes the steps it = g, g+2, ...
+    const int group = (warp - 2) >> 2;
+    const int u = threadIdx.x - 64 - 128 * group;  // unit 0..127 within the group
     const float mu = __ldg(p.mu);
     const uint32_t bpr = (uint32_t)(p.I / kBK);  // blocks per W row
-    // unit -> (W row, block column, smem row) for a given step kb
+    // unit -> NF4 block index for step kb
     auto block_of = [&](int kb) -> uint32_t {
       if (!DX) return (uint32_t)(m0 + u) * bpr + (uint32_t)kb;
       return (uint32_t)(kb * kBK + (u & 63)) * bpr + (uint32_t)(m0 / kBK) + (uint32_t)(u >> 6);
     };
     const uint32_t row_off = DX ? (uint32_t)((u >> 6) * (kWTile / 2) + (u & 63) * 128) : (uint32_t)u * 128;
-    const uint32_t sw = DX ? (uint32_t)(u & 7) : (uint32_t)(u & 7);
+    const uint32_t sw = (uint32_t)(u & 7);
     const uint32_t pk_off = DX ? (uint32_t)((u & 63) * 64 + (u >> 6) * 32) : (uint32_t)u * 32;
+    auto kb_of = [&](int it) { return kb_lo + it - has_ad; };
+    int it = group;
     uint32_t q_next = 0;
     float t_next = 0.0f;
-    if (T > has_ad) {
-      const uint32_t b = block_of(kb_lo);
+    if (it < T && !(has_ad && it == 0)) {
+      const uint32_t b = block_of(kb_of(it));
+      q_next = __ldg(p.qcodes + b);
+      t_next = __ldg(p.t + b / p.C);
+    } else if (it + kDecGroups < T) {
+      const uint32_t b = block_of(kb_of(it + kDecGroups));
       q_next = __ldg(p.qcodes + b);
       t_next = __ldg(p.t + b / p.C);
     }
     bool ok = true;
-    for (int it = 0; it < T; ++it) {
+    for (; it < T; it += kDecGroups) {
       const int s = it % STAGES;
       const uint32_t par = (it / STAGES) & 1;
       const bool adapter = has_ad && it == 0;
       float sc = 0.0f;
       if (!adapter) {
         sc = decode_block_scale(q_next, t_next, mu);
-        const int kb_n = kb_lo + it - has_ad + 1;
-        if (kb_n < kb_hi) {
-          const uint32_t b = block_of(kb_n);
+        if (it + kDecGroups < T) {  // prefetch the scale inputs of this group's next step
+          const uint32_t b = block_of(kb_of(it + kDecGroups));
           q_next = __ldg(p.qcodes + b);
           t_next = __ldg(p.t + b / p.C);
         }
@@ -281,37 +350,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                   mbar_wait(smem_u32(&full_pk[s]), par, p.wait_ns, p.err, 0x302);
       if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
       if (!adapter)
-        decode_row(pk + s * kPkTile + pk_off, sc, smem_u32(wdec + s * kWTile) + row_off, sw, lut);
+        decode_row(pk + s * kPkTile + pk_off, sc, smem_u32(wdec + s * kWTile) + row_off, sw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&dec[s]));
     }
     // ------------------------------------------------------------ epilogue
+    // Warp w reads TMEM lanes 32*(w%4) .. +31; the two groups split the
+    // token columns (group 0 alone when the tile is narrower than 64).
     const bool acc_ok = mbar_wait(smem_u32(acc_full), 0, p.wait_ns, p.err, 0x401);
     tc_fence_after();
     const bool aborted = __any_sync(0xffffffffu, !ok || !acc_ok || *abort_flag != 0);
-    if (!aborted) {
-      const int quad = warp & 3;  // TMEM lane quarter this warp may read
-      const int mw = m0 + quad * 32 + lane;
-      const size_t Mw = (size_t)p.Mw;
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int64_t tok = n0 + c0 + j;
-          if (c0 + j < BN && tok < p.R) {
-            const float f = __uint_as_float(v[j]);
-            if (p.partial)
-              ((float*)p.out)[((size_t)split * (size_t)p.R + (size_t)tok) * Mw + mw] = f;
-            else
-              ((__nv_bfloat16*)p.out)[(size_t)tok * Mw + mw] = __float2bfloat16_rn(f);
-          }
-        }
-      }
-    }
+    constexpr int kColsPerGroup = BN >= 64 ? BN / kDecGroups : BN;
+    const int c_begin = BN >= 64 ? group * kColsPerGroup : 0;
+    const int c_end = BN >= 64 ? c_begin + kColsPerGroup : (group == 0 ? BN : 0);
+    if (!aborted) epilogue_store(tmem, warp & 3, lane, m0, n0, c_begin, c_end, split, p);
   }
   tc_fence_before();
   __syncthreads();
@@ -366,11 +419,6 @@ int num_sms_cached() {
 }
 
 template <int BN>
-constexpr int stages_for() {
-  return BN >= 256 ? 4 : (BN >= 128 ? 5 : 4);
-}
-
-template <int BN>
 constexpr size_t smem_bytes() {
   return 1024 + (size_t)stages_for<BN>() * Smem<BN>::kStage + 5 * 8 * stages_for<BN>() + 8 + 16 +
          64 + 64;
@@ -382,8 +430,12 @@ cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, con
   constexpr int S = stages_for<BN>();
   auto kern = tc_qlinear_kernel<DX, BN, S>;
   const size_t sm = smem_bytes<BN>();
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
+  static bool attr_set = false;  // once per instantiation (keeps graph capture free of it)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   const double flops = 2.0 * (double)p.R * (double)p.Mw * (double)p.KB * kBK +
                        2.0 * (double)p.R * (double)p.Mw * (double)p.rank;
   const int slot = timing_begin(st, DX ? 1 : 0, flops);
@@ -426,11 +478,17 @@ size_t partial_bytes(const TcPlan& pl, int64_t R, int64_t Mw) {
 
 TcPlan tc_plan(int64_t Mw, int64_t KB, int64_t R) {
   TcPlan pl;
-  pl.bn = R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : R <= 128 ? 128 : 256;
-  pl.stages = 0;
-  const int64_t tiles = (Mw / kBM) * ((R + pl.bn - 1) / pl.bn);
-  int64_t splits = 1;
   const int sms = num_sms_cached();
+  const int64_t mt = Mw / kBM;
+  // Token tile: the smallest power of two >= R (16..256); at large R, halve
+  // it (down to 64) while the grid is below one wave, rather than split K.
+  int bn = 16;
+  while (bn < 256 && bn < R) bn *= 2;
+  while (bn > 64 && mt * ((R + bn - 1) / bn) < sms) bn /= 2;
+  pl.bn = bn;
+  pl.stages = 0;
+  const int64_t tiles = mt * ((R + bn - 1) / bn);
+  int64_t splits = 1;
   if (tiles > 0 && tiles < sms) {
     splits = (2 * sms + tiles - 1) / tiles;
     const int64_t max_splits = KB / 4 > 0 ? KB / 4 : 1;
@@ -471,8 +529,8 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   uint16_t* upad = (uint16_t*)tcws;
   uint16_t* bpad = (uint16_t*)((char*)tcws + align_up((size_t)R * 128, 256));
   float* part = (float*)((char*)bpad + align_up((size_t)O * 128, 256));
-  cudaError_t e = launch_pad_rows_bf16(U, R, r, 1.0f, upad, st);
-  if (e == cudaSuccess) e = launch_pad_rows_bf16(B, O, r, s, bpad, st);
+  (void)U;  // its bf16 copy upad was written by the rowdot kernel that made U
+  cudaError_t e = launch_pad_rows_bf16(B, O, r, s, bpad, st);
   if (e != cudaSuccess) return e;
   CUtensorMap m_act, m_pk, m_aact, m_aw;
   const uint32_t bn = (uint32_t)pl.bn;
@@ -511,8 +569,8 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   uint16_t* vpad = (uint16_t*)tcws;
   uint16_t* apad = (uint16_t*)((char*)tcws + align_up((size_t)R * 128, 256));
   float* part = (float*)((char*)apad + align_up((size_t)I * 128, 256));
-  cudaError_t e = launch_pad_rows_bf16(V, R, r, 1.0f, vpad, st);
-  if (e == cudaSuccess) e = launch_pad_cols_bf16(A, r, I, s, apad, st);
+  (void)V;  // its bf16 copy vpad was written by the rowdot kernel that made V
+  cudaError_t e = launch_pad_cols_bf16(A, r, I, s, apad, st);
   if (e != cudaSuccess) return e;
   CUtensorMap m_act, m_pk, m_aact, m_aw;
   const uint32_t bn = (uint32_t)pl.bn;

@@ -22,6 +22,11 @@ bool tc_dx_supported(const WView& w, const void* dY, const void* dX, int64_t R);
 size_t tc_fwd_ws(const WView& w, int64_t R);
 size_t tc_dx_ws(const WView& w, int64_t R);
 
+// The first R*128 bytes of the tensor-core workspace hold the bf16 copy of
+// U (forward) or V (input gradient), zero-padded to 64 columns; the caller
+// fills it (launch_rowdot's pad output) before the launch.
+inline uint16_t* tc_act_pad(void* tcws) { return (uint16_t*)tcws; }
+
 // Y = X W_hat^T + s U B^T  (bf16 in/out, fp32 accumulation in TMEM).
 cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float* U,
                           const float* B, int32_t r, float s, void* Y, void* tcws,

@@ -244,3 +244,30 @@ def test_workspace_status_clean_after_tensor_core_calls():
     q.qlora_linear_fwd(gw, d["xd"], A, B, 16.0, ws=ws)
     assert q.qlora_workspace_status(ws) == 0
     assert q.qlora_kernel_launch_count() > n0
+
+
+def test_kernel_timing_inside_cuda_graph():
+    wl = synth.workload("qwen3_0.6b_attn_qv", R=512)
+    d = layer_inputs(wl, 0)
+    gw = q.qlora_quantize_nf4(to_dev_f32(d["W"]))
+    A, B = to_dev_f32(d["A"]), to_dev_f32(d["B"])
+    Y = torch.empty((512, 2048), dtype=torch.bfloat16, device="cuda")
+    U = torch.empty((512, 8), device="cuda")
+    ws = q.workspace(q.qlora_linear_workspace_bytes(gw, 512, 8, 0, 1))
+    q.qlora_linear_fwd(gw, d["xd"], A, B, 16.0, Y=Y, U_out=U, ws=ws)  # first call outside capture
+    torch.cuda.synchronize()
+    q.qlora_kernel_timing_enable(8)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=s, capture_error_mode="thread_local"):
+        q.qlora_linear_fwd(gw, d["xd"], A, B, 16.0, Y=Y, U_out=U, ws=ws)
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        recs = q.qlora_kernel_timing_collect(8)
+        assert len(recs) == 1 and recs[0][0] == 0 and recs[0][1] > 0 and recs[0][2] > 0
+    del g
+    q.qlora_kernel_timing_enable(0)
+    oY, _ = oracle.linear_fwd(oracle.quantize_nf4(d["W"]), d["x"], d["A"], d["B"], 8, 16.0)
+    assert rel_fro(to_host(Y), oY) <= TOL["bf16"]
