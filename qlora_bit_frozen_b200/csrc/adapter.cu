@@ -3,20 +3,23 @@
 // "QLoRA on Mac", "Design / Q-LoRA layer": the adapter branch is
 // (alpha/r)(x A^T) B^T with fp32 A, B.  Forward needs U = X A^T; the
 // backward chain rule needs V = dY B, dA = s V^T X and dB = s dY^T U.
-// All four read one activation matrix once and touch an r-wide factor, so
-// they are bound by HBM bandwidth on X / dY, not by arithmetic:
+// Each reads one activation matrix once and touches an r-wide factor, so
+// they are bound by HBM bandwidth on X / dY; the kernels are written to
+// keep many independent loads in flight (every load of a chunk is issued
+// before any of it is used):
 //
-//  * rowdot: out[m, j] = sum_k P[m, k] L(k, j) (U with L = A^T, V with L = B).
-//    Each warp owns 2 rows; lanes stride K four elements at a time; a
-//    256-wide chunk of L is staged in shared memory once per block and read
-//    as conflict-free float4; the 32 lane partials are combined with a
-//    butterfly.  Also writes the bf16 copy zero-padded to 64 columns that
-//    the tensor-core kernels use as their extra K step.
-//  * coldot: partial[split][j][n] = sum over the split's rows of
-//    aux[m, j] P[m, n] (dA with aux = V, P = X; dB with aux = U, P = dY).
-//    One thread per two columns, the aux rows broadcast from shared memory;
-//    the splits are then summed in split order (deterministic) and scaled
-//    by s, writing dA as [r x I] and dB as [O x r].
+//  * rowdot: out[m, j] = sum_k P[m, k] L(k, j)  (U: L = A^T; V: L = B).
+//    A 32 KB chunk of L is staged in shared memory per block; each warp owns
+//    RW rows, each lane loads 8 consecutive elements of every row per 256
+//    columns; lane partials are combined with a butterfly.  It also writes
+//    the bf16 copy zero-padded to 64 columns that the tensor-core kernels
+//    use as their extra K step, and (extra blocks of the same launch) the
+//    zero-padded bf16(s B) / bf16(s A) operand of that step.
+//  * coldot: out(j, n) = s sum_m aux[m, j] P[m, n]  (dA: aux = V, P = X;
+//    dB: aux = U, P = dY).  A block is 32 column threads x 8 row lanes over a
+//    slice of the rows; the 8 row lanes are summed in shared memory, the
+//    slices then in slice order by a second kernel (deterministic), which
+//    applies s and writes dA as [r x I] or dB as [O x r].
 #include "common.cuh"
 #include "internal.h"
 
@@ -24,111 +27,534 @@ namespace qlora {
 
 namespace {
 
-constexpr int kRowThreads = 256;
-constexpr int kRowsPerWarp = 2;
-constexpr int kRowsPerBlock = kRowsPerWarp * (kRowThreads / 32);
+constexpr int kThreads = 256;
 
-template <typename T>
-struct Vec4;
-template <>
-struct Vec4<float> {
-  __device__ static void load(const float* p, float (&x)[4]) {
-    const float4 v = *reinterpret_cast<const float4*>(p);
-    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-  }
-};
-template <>
-struct Vec4<__nv_bfloat16> {
-  __device__ static void load(const __nv_bfloat16* p, float (&x)[4]) {
-    const uint2 v = *reinterpret_cast<const uint2*>(p);
-    x[0] = __uint_as_float(v.x << 16); x[1] = __uint_as_float(v.x & 0xFFFF0000u);
-    x[2] = __uint_as_float(v.y << 16); x[3] = __uint_as_float(v.y & 0xFFFF0000u);
-  }
-};
-
-// K chunk staged per block: RMAX x KC floats stay within 32 KB.
-template <int RMAX>
-constexpr int kc_for() {
-  return RMAX <= 32 ? 256 : 128;
+// 16-byte global -> shared copy, asynchronous; bytes past src_bytes are
+// filled with zeros (src_bytes = 0 for padding rows/columns).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-template <typename T, int RMAX>
-__global__ void __launch_bounds__(kRowThreads) rowdot_kernel(const T* __restrict__ P, int64_t R,
-                                                             int64_t K, const float* __restrict__ L,
-                                                             int l_is_kr, int r,
-                                                             float* __restrict__ out,
-                                                             uint16_t* __restrict__ out_pad) {
-  constexpr int kKC = kc_for<RMAX>();
-  __shared__ __align__(16) float Ls[RMAX * kKC];  // Ls[j * kKC + k]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row0 = ((int64_t)blockIdx.x * (kRowThreads / 32) + warp) * kRowsPerWarp;
-  const bool vec = (K % 4) == 0;
-  float acc[kRowsPerWarp][RMAX];
+// ----------------------------------------------------------------- loads
+
+template <typename T, int E>
+__device__ __forceinline__ void load_vec(const T* p, float (&x)[E]);
+
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 8>(const __nv_bfloat16* p, float (&x)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int q = 0; q < kRowsPerWarp; ++q)
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&x)[4]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  x[0] = __uint_as_float(v.x << 16);
+  x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(v.y << 16);
+  x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+}
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 2>(const __nv_bfloat16* p, float (&x)[2]) {
+  const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
+  x[0] = __uint_as_float(v << 16);
+  x[1] = __uint_as_float(v & 0xFFFF0000u);
+}
+template <>
+__device__ __forceinline__ void load_vec<__nv_bfloat16, 1>(const __nv_bfloat16* p, float (&x)[1]) {
+  x[0] = __bfloat162float(*p);
+}
+template <>
+__device__ __forceinline__ void load_vec<float, 8>(const float* p, float (&x)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *reinterpret_cast<const float4*>(p + 4);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+template <>
+__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&x)[4]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void load_vec<float, 2>(const float* p, float (&x)[2]) {
+  const float2 a = *reinterpret_cast<const float2*>(p);
+  x[0] = a.x; x[1] = a.y;
+}
+template <>
+__device__ __forceinline__ void load_vec<float, 1>(const float* p, float (&x)[1]) {
+  x[0] = *p;
+}
+
+// E elements starting at p, element i valid when i < nvalid (others 0).
+template <typename T, int E>
+__device__ __forceinline__ void load_elems(const T* p, int nvalid, bool vec_ok, float (&x)[E]) {
+  if (vec_ok && nvalid >= E) {
+    load_vec<T, E>(p, x);
+  } else {
+#pragma unroll
+    for (int i = 0; i < E; ++i) x[i] = i < nvalid ? to_f32<T>(p[i]) : 0.0f;
+  }
+}
+
+// E elements kept in their storage format (32-bit words) until used, so a
+// chunk's loads can all be in flight without converting them first.
+template <typename T, int E>
+struct Raw {
+  static constexpr int kBytes = E * (int)sizeof(T);
+  static constexpr int W = (kBytes + 3) / 4;
+  uint32_t w[W];
+  __device__ __forceinline__ void load(const T* p, int nvalid, bool vec_ok) {
+    if (vec_ok && nvalid >= E) {
+      if constexpr (kBytes == 32) {
+        const uint4 a = *reinterpret_cast<const uint4*>(p);
+        const uint4 b = *reinterpret_cast<const uint4*>(p + 16 / (int)sizeof(T));
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+      } else if constexpr (kBytes == 16) {
+        const uint4 v = *reinterpret_cast<const uint4*>(p);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+      } else if constexpr (kBytes == 8) {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        w[0] = v.x; w[1] = v.y;
+      } else if constexpr (kBytes == 4) {
+        w[0] = *reinterpret_cast<const uint32_t*>(p);
+      } else {
+        w[0] = *reinterpret_cast<const unsigned short*>(p);
+      }
+    } else {
+      float x[E];
+#pragma unroll
+      for (int i = 0; i < E; ++i) x[i] = i < nvalid ? to_f32<T>(p[i]) : 0.0f;
+      set(x);
+    }
+  }
+  __device__ __forceinline__ void set(const float (&x)[E]) {
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int i = 0; i < W; ++i) {
+        const uint32_t lo = __float_as_uint(x[2 * i]) >> 16;
+        const uint32_t hi = 2 * i + 1 < E ? (__float_as_uint(x[2 * i + 1]) & 0xFFFF0000u) : 0u;
+        w[i] = lo | hi;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < W; ++i) w[i] = __float_as_uint(x[i]);
+    }
+  }
+  __device__ __forceinline__ float at(int i) const {
+    if constexpr (sizeof(T) == 2)
+      return __uint_as_float((i & 1) ? (w[i >> 1] & 0xFFFF0000u) : (w[i >> 1] << 16));
+    else
+      return __uint_as_float(w[i]);
+  }
+};
+
+// ---------------------------------------------------------------- pad job
+
+// Zero-padded bf16 copy of an r-wide fp32 factor times mul:
+//   mode 0: dst[rows x 64] from src[rows x r]   (bf16(s B), [O x 64])
+//   mode 1: dst[64 x cols] from src[r x cols]   (bf16(s A), [64 x I])
+struct PadJob {
+  const float* src;
+  uint16_t* dst;
+  int64_t extent;  // rows (mode 0) or cols (mode 1)
+  int r;
+  int mode;
+  float mul;
+  int blocks;  // launch blocks reserved for this job (0 = none)
+};
+
+__device__ void run_pad_job(const PadJob& j, int64_t blk) {
+  const int64_t total = 64 * j.extent;
+  for (int64_t e = blk * kThreads * 8 + threadIdx.x; e < min(total, (blk + 1) * kThreads * 8);
+       e += kThreads) {
+    float v;
+    if (j.mode == 0) {
+      const int64_t m = e >> 6;
+      const int c = (int)(e & 63);
+      v = c < j.r ? __fmul_rn(j.mul, j.src[m * j.r + c]) : 0.0f;
+    } else {
+      const int64_t row = e / j.extent;
+      v = row < j.r ? __fmul_rn(j.mul, j.src[e]) : 0.0f;
+    }
+    j.dst[e] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  }
+}
+
+// ------------------------------------------------------------------ rowdot
+
+// Block = 8 warps = (8 / KS) row groups x KS column groups.  A warp owns RW
+// rows and the 256-wide K steps kg, kg + KS, ...; each lane loads 8
+// consecutive elements of each of its rows per step (all rows' loads in
+// flight together) and reads the matching 8 x r factor values through L1
+// (they are shared by the RW rows).  Lane partials are combined with a
+// butterfly, column groups (KS > 1, for few rows) in shared memory in a fixed
+// order.
+template <typename T, int RMAX, int RW, int KS>
+__global__ void __launch_bounds__(kThreads) rowdot_kernel(const T* __restrict__ P, int64_t R,
+                                                          int64_t K, const float* __restrict__ L,
+                                                          int l_is_kr, int r,
+                                                          float* __restrict__ out,
+                                                          uint16_t* __restrict__ out_pad,
+                                                          int row_blocks, PadJob job) {
+  if ((int)blockIdx.x >= row_blocks) {
+    run_pad_job(job, (int64_t)blockIdx.x - row_blocks);
+    return;
+  }
+  constexpr int EPL = 8;
+  constexpr int STEP = 32 * EPL;  // 256 columns per warp step
+  constexpr int RG = 8 / KS;      // row groups per block
+  __shared__ float red[KS > 1 ? KS : 1][RW][RMAX];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rg = warp % RG, kg = warp / RG;
+  const int64_t row0 = ((int64_t)blockIdx.x * RG + rg) * RW;
+  const bool vec_ok = (K % EPL) == 0 && ((uintptr_t)P % (EPL * sizeof(T))) == 0;
+  const bool l_vec = ((uintptr_t)L % 16) == 0 && (l_is_kr ? (r % 4) == 0 : (K % 4) == 0);
+  float acc[RW][RMAX];
+#pragma unroll
+  for (int q = 0; q < RW; ++q)
 #pragma unroll
     for (int j = 0; j < RMAX; ++j) acc[q][j] = 0.0f;
 
-  for (int64_t k0 = 0; k0 < K; k0 += kKC) {
-    const int kc = (int)min((int64_t)kKC, K - k0);
-    __syncthreads();
-    for (int e = threadIdx.x; e < kc * r; e += kRowThreads) {
-      int j, k;
-      float v;
-      if (l_is_kr) {
-        k = e / r;
-        j = e - k * r;
-        v = L[(k0 + k) * r + j];
-      } else {
-        j = e / kc;
-        k = e - j * kc;
-        v = L[(int64_t)j * K + k0 + k];
-      }
-      Ls[j * kKC + k] = v;
+  for (int64_t k0 = (int64_t)kg * STEP; k0 < K; k0 += (int64_t)KS * STEP) {
+    const int64_t k = k0 + lane * EPL;
+    const int nk = (int)max((int64_t)0, min((int64_t)EPL, K - k));
+    Raw<T, EPL> x[RW];
+#pragma unroll
+    for (int q = 0; q < RW; ++q) {
+      const int64_t m = row0 + q;
+      x[q].load(P + m * K + k, m < R ? nk : 0, vec_ok);
     }
-    __syncthreads();
+    if (nk == 0) continue;
 #pragma unroll
-    for (int t = 0; t < kKC / 128; ++t) {
-      const int kk = t * 128 + lane * 4;
-      if (kk >= kc) break;
-      float x[kRowsPerWarp][4];
+    for (int j = 0; j < RMAX; ++j) {
+      if (j < r) {
+        float l[EPL];
+        if (!l_is_kr) {  // L[j * K + k]
+          const float* lp = L + (int64_t)j * K + k;
+          if (l_vec && nk == EPL) {
+            const float4 a = __ldg(reinterpret_cast<const float4*>(lp));
+            const float4 b = __ldg(reinterpret_cast<const float4*>(lp + 4));
+            l[0] = a.x; l[1] = a.y; l[2] = a.z; l[3] = a.w;
+            l[4] = b.x; l[5] = b.y; l[6] = b.z; l[7] = b.w;
+          } else {
 #pragma unroll
-      for (int q = 0; q < kRowsPerWarp; ++q) {
-        const int64_t m = row0 + q;
-        if (m < R && vec && kk + 4 <= kc) {
-          Vec4<T>::load(P + m * K + k0 + kk, x[q]);
-        } else {
+            for (int e = 0; e < EPL; ++e) l[e] = e < nk ? __ldg(lp + e) : 0.0f;
+          }
+        } else {  // L[k * r + j]
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            x[q][e] = (m < R && kk + e < kc) ? to_f32<T>(P[m * K + k0 + kk + e]) : 0.0f;
+          for (int e = 0; e < EPL; ++e) l[e] = e < nk ? __ldg(L + (k + e) * r + j) : 0.0f;
         }
-      }
-      const int kmax = kc - kk;  // entries of Ls past kc are stale: mask them
 #pragma unroll
-      for (int j = 0; j < RMAX; ++j) {
-        if (j < r) {
-          const float4 l = *reinterpret_cast<const float4*>(&Ls[j * kKC + kk]);
-          const float lv[4] = {l.x, kmax > 1 ? l.y : 0.0f, kmax > 2 ? l.z : 0.0f,
-                               kmax > 3 ? l.w : 0.0f};
+        for (int q = 0; q < RW; ++q)
 #pragma unroll
-          for (int q = 0; q < kRowsPerWarp; ++q)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[q][j] = fmaf(x[q][e], lv[e], acc[q][j]);
-        }
+          for (int e = 0; e < EPL; ++e) acc[q][j] = fmaf(x[q].at(e), l[e], acc[q][j]);
       }
     }
   }
 #pragma unroll
-  for (int q = 0; q < kRowsPerWarp; ++q)
+  for (int q = 0; q < RW; ++q)
+#pragma unroll
+    for (int j = 0; j < RMAX; ++j)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[q][j] += __shfl_xor_sync(0xffffffffu, acc[q][j], o);
+  if constexpr (KS > 1) {
+    if (lane == 0)
+#pragma unroll
+      for (int q = 0; q < RW; ++q)
+#pragma unroll
+        for (int j = 0; j < RMAX; ++j) red[kg][q][j] = acc[q][j];
+    __syncthreads();
+    if (kg != 0) return;
+#pragma unroll
+    for (int q = 0; q < RW; ++q)
+#pragma unroll
+      for (int j = 0; j < RMAX; ++j) {
+        float v = red[0][q][j];
+#pragma unroll
+        for (int g = 1; g < KS; ++g) v += red[g][q][j];
+        acc[q][j] = v;
+      }
+  }
+#pragma unroll
+  for (int q = 0; q < RW; ++q) {
+    const int64_t m = row0 + q;
+    if (m >= R) continue;
+    float a0 = 0.0f, a1 = 0.0f;  // columns lane and lane + 32, picked without dynamic indexing
+#pragma unroll
+    for (int j = 0; j < RMAX; ++j) {
+      if (j == lane) a0 = acc[q][j];
+      if (j == lane + 32) a1 = acc[q][j];
+    }
+    if (lane < r) out[m * r + lane] = a0;
+    if (lane + 32 < r) out[m * r + lane + 32] = a1;
+    if (out_pad) {
+      out_pad[m * 64 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(lane < r ? a0 : 0.0f));
+      out_pad[m * 64 + lane + 32] =
+          __bfloat16_as_ushort(__float2bfloat16_rn(lane + 32 < r ? a1 : 0.0f));
+    }
+  }
+}
+
+// ------------------------------------------------------------------ coldot
+
+template <int RMAX>
+constexpr int col_cpt() {
+  return RMAX <= 8 ? 8 : RMAX <= 16 ? 4 : RMAX <= 32 ? 2 : 1;  // CPT * RMAX = 64
+}
+constexpr int kRowLanes = kThreads / 32;
+constexpr int kUnroll = 8;
+
+// Block (x, y) = column range x (32 threads x CPT columns) over row slice y,
+// 8 row lanes per column thread, 8 rows in flight per lane.  The row lanes
+// are summed in shared memory; the slice sums go to `part`; the last block
+// of column range x to finish (ticket counter) adds the slices in slice
+// order, scales by s and writes the result: dA as [r x N] (out_nr = 0) or
+// dB as [N x r] (out_nr = 1).  With one slice it writes directly.
+template <typename T, int RMAX>
+__global__ void __launch_bounds__(kThreads) coldot_kernel(const T* __restrict__ P, int64_t R,
+                                                          int64_t N, const float* __restrict__ aux,
+                                                          int r, int64_t rows_per_split,
+                                                          int splits, float s, int out_nr,
+                                                          float* __restrict__ part,
+                                                          unsigned* __restrict__ tickets,
+                                                          float* __restrict__ out) {
+  constexpr int CPT = col_cpt<RMAX>();
+  constexpr int NV = CPT * RMAX;  // accumulators per thread (64)
+  __shared__ float red[4][NV][32];  // 32 KB: row-lane reduction staging
+  __shared__ unsigned is_last;
+  const int c = threadIdx.x & 31, tr = threadIdx.x >> 5;
+  const int64_t nb = (int64_t)blockIdx.x * (32 * CPT);
+  const int64_t n0 = nb + (int64_t)c * CPT;
+  const int64_t m_lo = (int64_t)blockIdx.y * rows_per_split;
+  const int64_t m_hi = min(R, m_lo + rows_per_split);
+  const bool vec_ok = (N % CPT) == 0 && ((uintptr_t)P % (CPT * sizeof(T))) == 0;
+  const int nvalid = (int)max((int64_t)0, min((int64_t)CPT, N - n0));
+  const bool aux_vec = (r % 4) == 0 && ((uintptr_t)aux % 16) == 0;
+  float acc[CPT][RMAX];
+#pragma unroll
+  for (int cc = 0; cc < CPT; ++cc)
+#pragma unroll
+    for (int j = 0; j < RMAX; ++j) acc[cc][j] = 0.0f;
+
+  for (int64_t m = m_lo + tr; m < m_hi; m += kRowLanes * kUnroll) {
+    Raw<T, CPT> p[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t mu = m + (int64_t)u * kRowLanes;
+      p[u].load(P + mu * N + n0, mu < m_hi ? nvalid : 0, vec_ok);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t mu = m + (int64_t)u * kRowLanes;
+      if (mu >= m_hi) break;
+      const float* arow = aux + mu * r;
+#pragma unroll
+      for (int j = 0; j < RMAX; j += 4) {
+        if (j < r) {
+          float a[4];
+          if (aux_vec) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(arow + j));
+            a[0] = f.x; a[1] = f.y; a[2] = f.z; a[3] = f.w;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = j + i < r ? __ldg(arow + j + i) : 0.0f;
+          }
+#pragma unroll
+          for (int cc = 0; cc < CPT; ++cc)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (j + i < RMAX) acc[cc][j + i] = fmaf(a[i], p[u].at(cc), acc[cc][j + i]);
+        }
+      }
+    }
+  }
+  // sum the 8 row lanes (warps): 8 -> 4 -> 2 -> 1 through shared memory
+#pragma unroll
+  for (int half = 4; half >= 1; half >>= 1) {
+    __syncthreads();
+    if (tr >= half && tr < 2 * half) {
+#pragma unroll
+      for (int cc = 0; cc < CPT; ++cc)
+#pragma unroll
+        for (int j = 0; j < RMAX; ++j) red[tr - half][cc * RMAX + j][c] = acc[cc][j];
+    }
+    __syncthreads();
+    if (tr < half) {
+#pragma unroll
+      for (int cc = 0; cc < CPT; ++cc)
+#pragma unroll
+        for (int j = 0; j < RMAX; ++j) acc[cc][j] += red[tr][cc * RMAX + j][c];
+    }
+  }
+  if (splits == 1) {
+    if (tr == 0)
+#pragma unroll
+      for (int j = 0; j < RMAX; ++j)
+#pragma unroll
+        for (int cc = 0; cc < CPT; ++cc)
+          if (j < r && cc < nvalid) {
+            const int64_t n = n0 + cc;
+            out[out_nr ? n * r + j : (int64_t)j * N + n] = s * acc[cc][j];
+          }
+    return;
+  }
+  if (tr == 0) {
+    float* dst = part + (int64_t)blockIdx.y * r * N;
+#pragma unroll
+    for (int j = 0; j < RMAX; ++j)
+#pragma unroll
+      for (int cc = 0; cc < CPT; ++cc)
+        if (j < r && cc < nvalid) dst[(int64_t)j * N + n0 + cc] = acc[cc][j];
+    __threadfence();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(&tickets[blockIdx.x], 1u) == (unsigned)splits - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  // this block's columns [nb, nb + 32 * CPT) x r: sum the slices in order
+  const int ncols = (int)min((int64_t)(32 * CPT), N - nb);
+  const int64_t rN = (int64_t)r * N;
+  for (int e = threadIdx.x; e < ncols * r; e += kThreads) {
+    const int j = e / ncols, cc = e - j * ncols;
+    const int64_t idx = (int64_t)j * N + nb + cc;
+    float v = 0.0f;
+    int k = 0;
+    for (; k + 8 <= splits; k += 8) {
+      float t[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) t[u] = __ldcg(part + (int64_t)(k + u) * rN + idx);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v += t[u];
+    }
+    for (; k < splits; ++k) v += __ldcg(part + (int64_t)k * rN + idx);
+    const int64_t n = nb + cc;
+    out[out_nr ? n * r + j : idx] = s * v;
+  }
+  if (threadIdx.x == 0) tickets[blockIdx.x] = 0;  // ready for the next call
+}
+
+// ------------------------------------------- pipelined kernels (16-byte rows)
+//
+// Used when every row of P starts on a 16-byte boundary.  A block streams
+// tiles of P (and of the r-wide factor) through a 4-stage cp.async ring in
+// shared memory, so each block keeps ~3 tiles of loads in flight whatever
+// its register use; threads compute from shared memory.
+
+constexpr int kStages = 4;
+
+// rowdot: block = 16 rows (2 per warp); tile = KT columns of P and of
+// L [r x K] (KT * RMAX = 2048 floats = 8 KB).  Lane l owns columns
+// l*EPL .. l*EPL+EPL-1 of the tile.
+template <typename T, int RMAX>
+struct RowPipe {
+  static constexpr int RB = 16;
+  static constexpr int KT = 2048 / RMAX;
+  static constexpr int EPL = KT / 32;
+  static constexpr int XB = RB * KT * (int)sizeof(T);
+  static constexpr int LB = RMAX * KT * 4;
+  static constexpr int STAGE = XB + LB;
+  static constexpr int SMEM = kStages * STAGE;
+};
+
+template <typename T, int RMAX>
+__global__ void __launch_bounds__(kThreads) rowdot_pipe_kernel(
+    const T* __restrict__ P, int64_t R, int64_t K, const float* __restrict__ L, int r,
+    float* __restrict__ out, uint16_t* __restrict__ out_pad, int row_blocks, PadJob job) {
+  if ((int)blockIdx.x >= row_blocks) {
+    run_pad_job(job, (int64_t)blockIdx.x - row_blocks);
+    return;
+  }
+  using C = RowPipe<T, RMAX>;
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t rb0 = (int64_t)blockIdx.x * C::RB;
+  const int ntiles = (int)((K + C::KT - 1) / C::KT);
+  constexpr int XCH = C::XB / 16, LCH = C::LB / 16;  // 16-byte chunks per tile
+  constexpr int ROWCH = C::KT * (int)sizeof(T) / 16;  // chunks per P row
+  constexpr int LROWCH = C::KT * 4 / 16;               // chunks per L row
+
+  auto issue = [&](int t) {
+    const int stg = t % kStages;
+    const uint32_t xs = (uint32_t)__cvta_generic_to_shared(sm + stg * C::STAGE);
+    const uint32_t ls = xs + C::XB;
+    const int64_t k0 = (int64_t)t * C::KT;
+    for (int c = threadIdx.x; c < XCH; c += kThreads) {
+      const int row = c / ROWCH, cc = c - row * ROWCH;
+      const int64_t m = rb0 + row;
+      const int64_t k = k0 + (int64_t)cc * (16 / (int)sizeof(T));
+      const int64_t rem = (K - k) * (int64_t)sizeof(T);
+      const uint32_t nb = (m < R && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
+      cp_async16(xs + c * 16, nb ? (const void*)(P + m * K + k) : (const void*)P, nb);
+    }
+    for (int c = threadIdx.x; c < LCH; c += kThreads) {
+      const int j = c / LROWCH, cc = c - j * LROWCH;
+      const int64_t k = k0 + (int64_t)cc * 4;
+      const int64_t rem = (K - k) * 4;
+      const uint32_t nb = (j < r && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
+      cp_async16(ls + c * 16, nb ? (const void*)(L + (int64_t)j * K + k) : (const void*)L, nb);
+    }
+  };
+
+  float acc[2][RMAX];
+#pragma unroll
+  for (int q = 0; q < 2; ++q)
+#pragma unroll
+    for (int j = 0; j < RMAX; ++j) acc[q][j] = 0.0f;
+#pragma unroll
+  for (int t = 0; t < kStages - 1; ++t) {
+    if (t < ntiles) issue(t);
+    cp_async_commit();
+  }
+  for (int t = 0; t < ntiles; ++t) {
+    cp_async_wait<kStages - 2>();
+    __syncthreads();
+    if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
+    cp_async_commit();
+    const uint8_t* xs = sm + (t % kStages) * C::STAGE;
+    const float* ls = (const float*)(xs + C::XB);
+    float x[2][C::EPL];
+#pragma unroll
+    for (int q = 0; q < 2; ++q)
+      load_vec<T, C::EPL>((const T*)xs + (warp * 2 + q) * C::KT + lane * C::EPL, x[q]);
+#pragma unroll
+    for (int j = 0; j < RMAX; ++j) {
+      if (j < r) {
+        float l[C::EPL];
+        load_vec<float, C::EPL>(ls + j * C::KT + lane * C::EPL, l);
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int e = 0; e < C::EPL; ++e) acc[q][j] = fmaf(x[q][e], l[e], acc[q][j]);
+      }
+    }
+  }
+  cp_async_wait<0>();
+#pragma unroll
+  for (int q = 0; q < 2; ++q)
 #pragma unroll
     for (int j = 0; j < RMAX; ++j)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc[q][j] += __shfl_xor_sync(0xffffffffu, acc[q][j], o);
 #pragma unroll
-  for (int q = 0; q < kRowsPerWarp; ++q) {
-    const int64_t m = row0 + q;
+  for (int q = 0; q < 2; ++q) {
+    const int64_t m = rb0 + warp * 2 + q;
     if (m >= R) continue;
-    // lane l writes columns l and l + 32 (selected without dynamic indexing)
     float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
     for (int j = 0; j < RMAX; ++j) {
@@ -145,87 +571,138 @@ __global__ void __launch_bounds__(kRowThreads) rowdot_kernel(const T* __restrict
   }
 }
 
-constexpr int kColThreads = 256;
-constexpr int kColsPerThread = 2;
-constexpr int kColsPerBlock = kColThreads * kColsPerThread;
-constexpr int kMC = 64;  // aux rows staged per chunk
+// coldot: block = 512 columns (2 per thread) over a row slice; tile = 32
+// rows of P (32 KB bf16) and the matching 32 rows of aux [R x r].
+template <typename T, int RMAX>
+struct ColPipe {
+  static constexpr int NC = 512;
+  static constexpr int RT = 32;
+  static constexpr int PB = RT * NC * (int)sizeof(T);
+  static constexpr int AB = RT * RMAX * 4;
+  static constexpr int STAGE = PB + AB;
+  static constexpr int SMEM = kStages * STAGE;
+};
 
 template <typename T, int RMAX>
-__global__ void __launch_bounds__(kColThreads) coldot_kernel(const T* __restrict__ P, int64_t R,
-                                                             int64_t N, const float* __restrict__ aux,
-                                                             int r, int64_t rows_per_split,
-                                                             float* __restrict__ part) {
-  __shared__ __align__(16) float As[kMC * RMAX];  // As[mm * RMAX + j]
-  const int64_t n = ((int64_t)blockIdx.x * kColThreads + threadIdx.x) * kColsPerThread;
+__global__ void __launch_bounds__(kThreads) coldot_pipe_kernel(
+    const T* __restrict__ P, int64_t R, int64_t N, const float* __restrict__ aux, int r,
+    int64_t rows_per_split, float* __restrict__ part) {
+  using C = ColPipe<T, RMAX>;
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int64_t nb = (int64_t)blockIdx.x * C::NC;
   const int64_t m_lo = (int64_t)blockIdx.y * rows_per_split;
   const int64_t m_hi = min(R, m_lo + rows_per_split);
-  const bool pair = (n + 1 < N) && ((N & 1) == 0);
-  float acc[kColsPerThread][RMAX];
-#pragma unroll
-  for (int c = 0; c < kColsPerThread; ++c)
-#pragma unroll
-    for (int j = 0; j < RMAX; ++j) acc[c][j] = 0.0f;
-  for (int64_t m0 = m_lo; m0 < m_hi; m0 += kMC) {
-    const int mc = (int)min((int64_t)kMC, m_hi - m0);
-    __syncthreads();
-    for (int e = threadIdx.x; e < mc * RMAX; e += kColThreads) {
-      const int mm = e / RMAX, j = e - mm * RMAX;
-      As[e] = j < r ? aux[(m0 + mm) * r + j] : 0.0f;
+  const int ntiles = (int)((m_hi - m_lo + C::RT - 1) / C::RT);
+  constexpr int PCH = C::PB / 16;
+  constexpr int ROWCH = C::NC * (int)sizeof(T) / 16;
+  const int ach_row = (r * 4 + 15) / 16;  // 16-byte chunks per aux row (r*4 bytes, padded)
+
+  auto issue = [&](int t) {
+    const int stg = t % kStages;
+    const uint32_t ps = (uint32_t)__cvta_generic_to_shared(sm + stg * C::STAGE);
+    const uint32_t as = ps + C::PB;
+    const int64_t r0 = m_lo + (int64_t)t * C::RT;
+    for (int c = threadIdx.x; c < PCH; c += kThreads) {
+      const int row = c / ROWCH, cc = c - row * ROWCH;
+      const int64_t m = r0 + row;
+      const int64_t n = nb + (int64_t)cc * (16 / (int)sizeof(T));
+      const int64_t rem = (N - n) * (int64_t)sizeof(T);
+      const uint32_t bytes = (m < m_hi && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
+      cp_async16(ps + c * 16, bytes ? (const void*)(P + m * N + n) : (const void*)P, bytes);
     }
-    __syncthreads();
-    if (n < N) {
-      for (int mm = 0; mm < mc; ++mm) {
-        float p0, p1 = 0.0f;
-        const T* row = P + (m0 + mm) * N + n;
-        if (pair) {
-          if constexpr (sizeof(T) == 2) {
-            const uint32_t v = *reinterpret_cast<const uint32_t*>(row);
-            p0 = __uint_as_float(v << 16);
-            p1 = __uint_as_float(v & 0xFFFF0000u);
-          } else {
-            const float2 v = *reinterpret_cast<const float2*>(row);
-            p0 = v.x;
-            p1 = v.y;
-          }
-        } else {
-          p0 = to_f32<T>(row[0]);
-          if (n + 1 < N) p1 = to_f32<T>(row[1]);
-        }
+    // aux rows r0 .. r0+RT of [R x r] are contiguous: r0*r .. (r0+RT)*r floats
+    const int64_t a0 = r0 * r;
+    const int64_t a_end = min(m_hi, r0 + C::RT) * r;
+    const int nch = (C::RT * r * 4 + 15) / 16;
+    for (int c = threadIdx.x; c < nch; c += kThreads) {
+      const int64_t e = a0 + (int64_t)c * 4;
+      const int64_t rem = (a_end - e) * 4;
+      const uint32_t bytes = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
+      cp_async16(as + c * 16, bytes ? (const void*)(aux + e) : (const void*)aux, bytes);
+    }
+    (void)ach_row;
+  };
+
+  float acc[2][RMAX];
 #pragma unroll
-        for (int j = 0; j < RMAX; j += 4) {
-          const float4 a = *reinterpret_cast<const float4*>(&As[mm * RMAX + j]);
-          acc[0][j] = fmaf(a.x, p0, acc[0][j]);
-          acc[0][j + 1] = fmaf(a.y, p0, acc[0][j + 1]);
-          acc[0][j + 2] = fmaf(a.z, p0, acc[0][j + 2]);
-          acc[0][j + 3] = fmaf(a.w, p0, acc[0][j + 3]);
-          acc[1][j] = fmaf(a.x, p1, acc[1][j]);
-          acc[1][j + 1] = fmaf(a.y, p1, acc[1][j + 1]);
-          acc[1][j + 2] = fmaf(a.z, p1, acc[1][j + 2]);
-          acc[1][j + 3] = fmaf(a.w, p1, acc[1][j + 3]);
+  for (int q = 0; q < 2; ++q)
+#pragma unroll
+    for (int j = 0; j < RMAX; ++j) acc[q][j] = 0.0f;
+#pragma unroll
+  for (int t = 0; t < kStages - 1; ++t) {
+    if (t < ntiles) issue(t);
+    cp_async_commit();
+  }
+  const int col = threadIdx.x * 2;  // local column pair
+  for (int t = 0; t < ntiles; ++t) {
+    cp_async_wait<kStages - 2>();
+    __syncthreads();
+    if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
+    cp_async_commit();
+    const uint8_t* ps = sm + (t % kStages) * C::STAGE;
+    const float* as = (const float*)(ps + C::PB);  // row-major [RT x r]
+    const int rows = (int)min((int64_t)C::RT, m_hi - (m_lo + (int64_t)t * C::RT));
+    for (int row = 0; row < rows; ++row) {
+      float pv[2];
+      load_vec<T, 2>((const T*)ps + row * C::NC + col, pv);
+      const float* ar = as + row * r;
+#pragma unroll
+      for (int j = 0; j < RMAX; j += 4) {
+        if (j < r) {
+          float a[4];
+          if ((r & 3) == 0) {
+            load_vec<float, 4>(ar + j, a);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = j + i < r ? ar[j + i] : 0.0f;
+          }
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[0][j + i] = fmaf(a[i], pv[0], acc[0][j + i]);
+            acc[1][j + i] = fmaf(a[i], pv[1], acc[1][j + i]);
+          }
         }
       }
     }
   }
+  cp_async_wait<0>();
   float* dst = part + (int64_t)blockIdx.y * r * N;
 #pragma unroll
   for (int j = 0; j < RMAX; ++j) {
     if (j < r) {
+      const int64_t n = nb + col;
       if (n < N) dst[(int64_t)j * N + n] = acc[0][j];
       if (n + 1 < N) dst[(int64_t)j * N + n + 1] = acc[1][j];
     }
   }
 }
 
-// out = s * sum over splits (in order) of part[split][j][n];
+// out = s * sum over slices of part[slice][j][n], one warp per output
+// element (lanes take slices l, l+32, ...; fixed butterfly order).
 // out_nr == 0: out[j * N + n] (dA);  1: out[n * r + j] (dB).
-__global__ void coldot_reduce_kernel(const float* __restrict__ part, int splits, int64_t N, int r,
-                                     float s, int out_nr, float* __restrict__ out) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // e = j * N + n
-  if (e >= (int64_t)r * N) return;
-  float acc = 0.0f;
-  for (int k = 0; k < splits; ++k) acc += part[(int64_t)k * r * N + e];
-  const int64_t j = e / N, n = e - j * N;
-  out[out_nr ? n * r + j : e] = s * acc;
+__global__ void slice_reduce_kernel(const float* __restrict__ part, int splits, int64_t N, int r,
+                                    float s, int out_nr, float* __restrict__ out) {
+  const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // e = j * N + n
+  const int lane = threadIdx.x & 31;
+  const int64_t rN = (int64_t)r * N;
+  if (e >= rN) return;
+  float v = 0.0f;
+  for (int k = lane; k < splits; k += 32) v += part[(int64_t)k * rN + e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) {
+    const int64_t j = e / N, n = e - j * N;
+    out[out_nr ? n * r + j : e] = s * v;
+  }
+}
+
+// dst[j * K + k] = src[k * r + j]: B [K x r] -> B^T [r x K].
+__global__ void transpose_kr_kernel(const float* __restrict__ src, int64_t K, int r,
+                                    float* __restrict__ dst) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // e = j * K + k
+  if (e >= (int64_t)r * K) return;
+  const int64_t j = e / K, k = e - j * K;
+  dst[e] = src[k * r + j];
 }
 
 inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
@@ -241,93 +718,233 @@ int sm_count() {
   return n;
 }
 
-template <typename T, int RMAX>
-void rowdot_launch(const void* P, int64_t R, int64_t K, const float* L, bool l_is_kr, int r,
-                   float* out, uint16_t* pad, cudaStream_t st) {
-  rowdot_kernel<T, RMAX><<<cdiv(R, kRowsPerBlock), kRowThreads, 0, st>>>(
-      (const T*)P, R, K, L, l_is_kr ? 1 : 0, r, out, pad);
+template <typename T, int RMAX, int RW, int KS>
+void rowdot_go(unsigned grid, const void* P, int64_t R, int64_t K, const float* L, bool l_is_kr,
+               int r, float* out, uint16_t* pad, int row_blocks, PadJob job, cudaStream_t st) {
+  rowdot_kernel<T, RMAX, RW, KS><<<grid, kThreads, 0, st>>>((const T*)P, R, K, L, l_is_kr, r, out,
+                                                            pad, row_blocks, job);
 }
 
 template <typename T, int RMAX>
-void coldot_launch(const void* P, int64_t R, int64_t N, const float* aux, int r, int64_t rps,
-                   int splits, float* part, cudaStream_t st) {
-  dim3 grid(cdiv(N, kColsPerBlock), (unsigned)splits);
-  coldot_kernel<T, RMAX><<<grid, kColThreads, 0, st>>>((const T*)P, R, N, aux, r, rps, part);
+cudaError_t rowdot_dispatch(const void* P, int64_t R, int64_t K, const float* L, bool l_is_kr,
+                            int r, float* out, uint16_t* pad, PadJob job, cudaStream_t st) {
+  // Many rows: one column group, RW rows per warp (RW * RMAX <= 64) while
+  // that leaves >= one block per SM.  Few rows: the 8 warps split K.
+  constexpr int RWMAX = 64 / RMAX < 4 ? 64 / RMAX : 4;
+  const int sms = sm_count();
+  int row_blocks = 0;
+  unsigned grid = 0;
+  if (R <= 64) {
+    row_blocks = (int)R;  // one row per block, 8 warps over K
+    grid = (unsigned)(row_blocks + job.blocks);
+    if (grid) rowdot_go<T, RMAX, 1, 8>(grid, P, R, K, L, l_is_kr, r, out, pad, row_blocks, job, st);
+  } else {
+    int rw = RWMAX;
+    while (rw > 1 && (R + 8 * rw - 1) / (8 * rw) < sms) rw /= 2;
+    row_blocks = (int)cdiv(R, 8 * rw);
+    grid = (unsigned)(row_blocks + job.blocks);
+    if (rw >= 4)
+      rowdot_go<T, RMAX, RWMAX, 1>(grid, P, R, K, L, l_is_kr, r, out, pad, row_blocks, job, st);
+    else if (rw == 2)
+      rowdot_go<T, RMAX, (RWMAX >= 2 ? 2 : 1), 1>(grid, P, R, K, L, l_is_kr, r, out, pad,
+                                                  row_blocks, job, st);
+    else
+      rowdot_go<T, RMAX, 1, 1>(grid, P, R, K, L, l_is_kr, r, out, pad, row_blocks, job, st);
+  }
+  if (grid == 0) return cudaSuccess;
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t rowdot_r(const void* P, int64_t R, int64_t K, const float* L, bool l_is_kr, int r,
+                     float* out, uint16_t* pad, PadJob job, cudaStream_t st) {
+  if (r <= 8) return rowdot_dispatch<T, 8>(P, R, K, L, l_is_kr, r, out, pad, job, st);
+  if (r <= 16) return rowdot_dispatch<T, 16>(P, R, K, L, l_is_kr, r, out, pad, job, st);
+  if (r <= 32) return rowdot_dispatch<T, 32>(P, R, K, L, l_is_kr, r, out, pad, job, st);
+  return rowdot_dispatch<T, 64>(P, R, K, L, l_is_kr, r, out, pad, job, st);
+}
+
+template <typename Kern>
+cudaError_t set_smem_once(Kern k, int bytes, bool& done) {
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
+template <int RMAX>
+cudaError_t rowdot_pipe_go(const __nv_bfloat16* P, int64_t R, int64_t K, const float* L, int r,
+                           float* out, uint16_t* pad, PadJob job, cudaStream_t st) {
+  using C = RowPipe<__nv_bfloat16, RMAX>;
+  static bool attr = false;
+  auto kern = rowdot_pipe_kernel<__nv_bfloat16, RMAX>;
+  cudaError_t e = set_smem_once(kern, C::SMEM, attr);
+  if (e != cudaSuccess) return e;
+  const int row_blocks = (int)cdiv(R, C::RB);
+  const unsigned grid = (unsigned)(row_blocks + job.blocks);
+  if (grid == 0) return cudaSuccess;
+  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, K, L, r, out, pad, row_blocks, job);
+  count_launch();
+  return cudaGetLastError();
 }
 
 struct ColPlan {
   int splits;
   int64_t rows_per_split;
+  unsigned colblocks;
 };
 
-ColPlan col_plan(int64_t R, int64_t N) {
+ColPlan col_plan(int64_t R, int64_t N, int r) {
+  const int cpt = r <= 8 ? 8 : r <= 16 ? 4 : r <= 32 ? 2 : 1;
   ColPlan c;
-  const int64_t colblocks = (N + kColsPerBlock - 1) / kColsPerBlock;
-  int64_t splits = (2 * (int64_t)sm_count() + colblocks - 1) / colblocks;
+  c.colblocks = cdiv(N, 32 * cpt);
+  int64_t splits = ((int64_t)sm_count() + c.colblocks - 1) / c.colblocks;  // ~one wave
+  const int64_t max_splits = (R + 127) / 128;
+  if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
-  int64_t rps = (R + splits - 1) / splits;
-  rps = (rps + kMC - 1) / kMC * kMC;
-  if (rps < kMC) rps = kMC;
-  c.rows_per_split = rps;
-  c.splits = (int)(R > 0 ? (R + rps - 1) / rps : 1);
+  c.rows_per_split = R > 0 ? (R + splits - 1) / splits : 1;
+  c.splits = (int)(R > 0 ? (R + c.rows_per_split - 1) / c.rows_per_split : 1);
   return c;
+}
+
+template <typename T, int RMAX>
+void coldot_launch(const void* P, int64_t R, int64_t N, const float* aux, int r, const ColPlan& c,
+                   float s, bool out_nr, float* part, unsigned* tickets, float* out,
+                   cudaStream_t st) {
+  dim3 grid(c.colblocks, (unsigned)c.splits);
+  coldot_kernel<T, RMAX><<<grid, kThreads, 0, st>>>((const T*)P, R, N, aux, r, c.rows_per_split,
+                                                    c.splits, s, out_nr ? 1 : 0, part, tickets,
+                                                    out);
+}
+
+template <typename T>
+void coldot_r(const void* P, int64_t R, int64_t N, const float* aux, int r, const ColPlan& c,
+              float s, bool out_nr, float* part, unsigned* tickets, float* out, cudaStream_t st) {
+  if (r <= 8) coldot_launch<T, 8>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
+  else if (r <= 16) coldot_launch<T, 16>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
+  else if (r <= 32) coldot_launch<T, 32>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
+  else coldot_launch<T, 64>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
 }
 
 }  // namespace
 
-// out[m, j] = sum_k P[m, k] * L(k, j);  L(k, j) = L[k*r + j] if l_is_kr else L[j*K + k].
-// pad (nullable): bf16 copy [R x 64], columns r..63 zero.
 cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const float* L,
-                          bool l_is_kr, int32_t r, float* out, cudaStream_t st, uint16_t* pad) {
-  if (R == 0) return cudaSuccess;
-  if (bf16) {
-    if (r <= 8) rowdot_launch<__nv_bfloat16, 8>(P, R, K, L, l_is_kr, r, out, pad, st);
-    else if (r <= 16) rowdot_launch<__nv_bfloat16, 16>(P, R, K, L, l_is_kr, r, out, pad, st);
-    else if (r <= 32) rowdot_launch<__nv_bfloat16, 32>(P, R, K, L, l_is_kr, r, out, pad, st);
-    else rowdot_launch<__nv_bfloat16, 64>(P, R, K, L, l_is_kr, r, out, pad, st);
-  } else {
-    if (r <= 8) rowdot_launch<float, 8>(P, R, K, L, l_is_kr, r, out, pad, st);
-    else if (r <= 16) rowdot_launch<float, 16>(P, R, K, L, l_is_kr, r, out, pad, st);
-    else if (r <= 32) rowdot_launch<float, 32>(P, R, K, L, l_is_kr, r, out, pad, st);
-    else rowdot_launch<float, 64>(P, R, K, L, l_is_kr, r, out, pad, st);
+                          bool l_is_kr, int32_t r, float* out, cudaStream_t st, uint16_t* pad,
+                          const float* side_src, int64_t side_extent, int side_mode,
+                          float side_mul, uint16_t* side_dst, float* lt_ws) {
+  PadJob job{side_src, side_dst, side_extent, r, side_mode, side_mul, 0};
+  if (side_dst && side_extent > 0) job.blocks = (int)cdiv(64 * side_extent, kThreads * 8);
+  // pipelined path: bf16 rows on 16-byte boundaries, factor rows as [r x K]
+  const bool rows16 = bf16 && (K % 8) == 0 && ((uintptr_t)P % 16) == 0;
+  if (rows16 && R > 64 && (!l_is_kr || lt_ws)) {
+    const float* Lr = L;
+    if (l_is_kr) {  // B [K x r] -> B^T [r x K] in the caller's scratch
+      transpose_kr_kernel<<<cdiv((int64_t)r * K, 256), 256, 0, st>>>(L, K, r, lt_ws);
+      count_launch();
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      Lr = lt_ws;
+    }
+    if (((uintptr_t)Lr % 16) == 0) {
+      const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
+      if (r <= 8) return rowdot_pipe_go<8>(Pb, R, K, Lr, r, out, pad, job, st);
+      if (r <= 16) return rowdot_pipe_go<16>(Pb, R, K, Lr, r, out, pad, job, st);
+      if (r <= 32) return rowdot_pipe_go<32>(Pb, R, K, Lr, r, out, pad, job, st);
+      return rowdot_pipe_go<64>(Pb, R, K, Lr, r, out, pad, job, st);
+    }
   }
+  if (bf16) return rowdot_r<__nv_bfloat16>(P, R, K, L, l_is_kr, r, out, pad, job, st);
+  return rowdot_r<float>(P, R, K, L, l_is_kr, r, out, pad, job, st);
+}
+
+namespace {
+
+struct PipePlan {
+  int splits;
+  int64_t rows_per_split;
+  unsigned colblocks;
+};
+
+PipePlan pipe_plan(int64_t R, int64_t N) {
+  PipePlan c;
+  c.colblocks = cdiv(N, ColPipe<__nv_bfloat16, 8>::NC);
+  int64_t splits = (2 * (int64_t)sm_count() + c.colblocks - 1) / c.colblocks;
+  const int64_t max_splits = (R + 63) / 64;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  int64_t rps = (R + splits - 1) / splits;
+  rps = (rps + 31) / 32 * 32;  // aux tiles start on 16-byte boundaries
+  if (rps < 32) rps = 32;
+  c.rows_per_split = rps;
+  c.splits = R > 0 ? (int)((R + rps - 1) / rps) : 1;
+  return c;
+}
+
+bool coldot_pipe_ok(const void* P, bool bf16, int64_t R, int64_t N, const float* aux) {
+  return bf16 && R > 0 && (N % 8) == 0 && ((uintptr_t)P % 16) == 0 && ((uintptr_t)aux % 16) == 0;
+}
+
+template <int RMAX>
+cudaError_t coldot_pipe_go(const __nv_bfloat16* P, int64_t R, int64_t N, const float* aux, int r,
+                           const PipePlan& c, float* part, cudaStream_t st) {
+  using C = ColPipe<__nv_bfloat16, RMAX>;
+  static bool attr = false;
+  auto kern = coldot_pipe_kernel<__nv_bfloat16, RMAX>;
+  cudaError_t e = set_smem_once(kern, C::SMEM, attr);
+  if (e != cudaSuccess) return e;
+  dim3 grid(c.colblocks, (unsigned)c.splits);
+  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, N, aux, r, c.rows_per_split, part);
   count_launch();
   return cudaGetLastError();
 }
 
+}  // namespace
+
+// Workspace: the larger of the pipelined path (slice sums) and the
+// streaming path (tickets + slice sums).
 size_t coldot_ws(int64_t R, int64_t N, int32_t r) {
-  const ColPlan c = col_plan(R, N);
-  return align_up((size_t)c.splits * (size_t)r * (size_t)N * 4, 256);
+  const ColPlan c = col_plan(R, N, r);
+  size_t a = c.splits <= 1 ? 0
+                           : align_up((size_t)c.colblocks * 4, 256) +
+                                 align_up((size_t)c.splits * (size_t)r * (size_t)N * 4, 256);
+  const PipePlan pp = pipe_plan(R, N);
+  size_t b = align_up((size_t)pp.splits * (size_t)r * (size_t)N * 4, 256);
+  return a > b ? a : b;
 }
 
-// out = s * aux^T P:  out(j, n) = s * sum_m aux[m, j] * P[m, n];
-// out_nr == false: out is [r x N] (dA);  true: out is [N x r] (dB).
 cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
                           int32_t r, float s, bool out_nr, float* out, void* ws,
                           cudaStream_t st) {
   if (N == 0) return cudaSuccess;
-  const ColPlan c = col_plan(R, N);
-  float* part = (float*)ws;
-  if (R == 0) {
-    cudaError_t e = cudaMemsetAsync(out, 0, (size_t)r * (size_t)N * 4, st);
-    return e;
+  if (R == 0) return cudaMemsetAsync(out, 0, (size_t)r * (size_t)N * 4, st);
+  if (coldot_pipe_ok(P, bf16, R, N, aux)) {
+    const PipePlan c = pipe_plan(R, N);
+    float* part = (float*)ws;
+    const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
+    cudaError_t e;
+    if (r <= 8) e = coldot_pipe_go<8>(Pb, R, N, aux, r, c, part, st);
+    else if (r <= 16) e = coldot_pipe_go<16>(Pb, R, N, aux, r, c, part, st);
+    else if (r <= 32) e = coldot_pipe_go<32>(Pb, R, N, aux, r, c, part, st);
+    else e = coldot_pipe_go<64>(Pb, R, N, aux, r, c, part, st);
+    if (e != cudaSuccess) return e;
+    const int64_t outs = (int64_t)r * N;
+    slice_reduce_kernel<<<cdiv(outs * 32, 256), 256, 0, st>>>(part, c.splits, N, r, s,
+                                                              out_nr ? 1 : 0, out);
+    count_launch();
+    return cudaGetLastError();
   }
-  if (bf16) {
-    if (r <= 8) coldot_launch<__nv_bfloat16, 8>(P, R, N, aux, r, c.rows_per_split, c.splits, part, st);
-    else if (r <= 16) coldot_launch<__nv_bfloat16, 16>(P, R, N, aux, r, c.rows_per_split, c.splits, part, st);
-    else if (r <= 32) coldot_launch<__nv_bfloat16, 32>(P, R, N, aux, r, c.rows_per_split, c.splits, part, st);
-    else coldot_launch<__nv_bfloat16, 64>(P, R, N, aux, r, c.rows_per_split, c.splits, part, st);
-  } else {
-    if (r <= 8) coldot_launch<float, 8>(P, R, N, aux, r, c.rows_per_split, c.splits, part, st);
-    else if (r <= 16) coldot_launch<float, 16>(P, R, N, aux, r, c.rows_per_split, c.splits, part, st);
-    else if (r <= 32) coldot_launch<float, 32>(P, R, N, aux, r, c.rows_per_split, c.splits, part, st);
-    else coldot_launch<float, 64>(P, R, N, aux, r, c.rows_per_split, c.splits, part, st);
+  const ColPlan c = col_plan(R, N, r);
+  unsigned* tickets = (unsigned*)ws;
+  float* part = (float*)((char*)ws + align_up((size_t)c.colblocks * 4, 256));
+  if (c.splits > 1) {
+    cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)c.colblocks * 4, st);
+    if (e != cudaSuccess) return e;
   }
-  count_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  coldot_reduce_kernel<<<cdiv((int64_t)r * N, 256), 256, 0, st>>>(part, c.splits, N, r, s,
-                                                                    out_nr ? 1 : 0, out);
+  if (bf16)
+    coldot_r<__nv_bfloat16>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
+  else
+    coldot_r<float>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
   count_launch();
   return cudaGetLastError();
 }

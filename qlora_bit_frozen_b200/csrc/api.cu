@@ -135,7 +135,7 @@ struct FwdLayout {
   size_t u = 0, tc = 0, total = 0;
 };
 struct BwdLayout {
-  size_t u = 0, v = 0, red = 0, tc = 0, total = 0;
+  size_t u = 0, v = 0, bt = 0, red = 0, tc = 0, total = 0;
 };
 
 FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t compute) {
@@ -156,6 +156,8 @@ BwdLayout bwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
   off += align_up((size_t)R * r * 4, 256);
   L.v = off;
   off += align_up((size_t)R * r * 4, 256);
+  L.bt = off;  // B^T [r x O] for the pipelined V = dY B
+  off += align_up((size_t)r * w->O * 4, 256);
   L.red = off;
   size_t red = coldot_ws(R, w->I, r);
   size_t red2 = coldot_ws(R, w->O, r);
@@ -307,7 +309,8 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
   const bool bf16 = compute == QLORA_COMPUTE_BF16;
   if (bf16 && tc_fwd_supported(v, X, Y, R)) {
     void* tcws = (char*)ws + L.tc;
-    e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws));
+    e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws), B, w->O, 0, sc,
+                      tc_w_pad(tcws, R));
     if (e == cudaSuccess) e = launch_tc_fwd(v, X, R, U, B, r, sc, Y, tcws, (uint32_t*)ws, s);
   } else {
     e = launch_simt_fwd(v, X, R, A, B, r, sc, bf16, Y, U, s);
@@ -339,7 +342,14 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   // feeds the tensor-core kernel's adapter step
   const bool tc = dX && bf16 && tc_dx_supported(v, dY, dX, R);
   void* tcws = (char*)ws + L.tc;
-  if (dX || dA) e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, tc ? tc_act_pad(tcws) : nullptr);
+  if (dX || dA) {
+    if (tc)
+      e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, tc_act_pad(tcws), A, w->I, 1, sc,
+                        tc_w_pad(tcws, R), (float*)((char*)ws + L.bt));
+    else
+      e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, nullptr, nullptr, 0, 0, 1.0f,
+                        nullptr, (float*)((char*)ws + L.bt));
+  }
   if (e == cudaSuccess && dX) {
     if (tc)
       e = launch_tc_dx(v, dY, R, V, A, r, sc, dX, tcws, (uint32_t*)ws, s);

@@ -39,9 +39,17 @@ cudaError_t launch_simt_dx(const WView& w, const void* dY, int64_t R, const floa
                            cudaStream_t st);
 // adapter side products
 // adapter.cu
+//   out[m, j] = sum_k P[m, k] L(k, j); pad (nullable): its bf16 copy [R x 64].
+//   Optional side job in the same launch (side_dst != nullptr): the
+//   zero-padded bf16(side_mul * src) operand, mode 0: [extent x 64] from
+//   src [extent x r]; mode 1: [64 x extent] from src [r x extent].
+//   lt_ws (nullable, r*K floats): scratch for L^T when l_is_kr, which lets
+//   the pipelined kernel read the factor row-wise.
 cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const float* L,
                           bool l_is_kr, int32_t r, float* out, cudaStream_t st,
-                          uint16_t* pad = nullptr);
+                          uint16_t* pad = nullptr, const float* side_src = nullptr,
+                          int64_t side_extent = 0, int side_mode = 0, float side_mul = 1.0f,
+                          uint16_t* side_dst = nullptr, float* lt_ws = nullptr);
 size_t coldot_ws(int64_t R, int64_t N, int32_t r);
 cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
                           int32_t r, float s, bool out_nr, float* out, void* ws,

@@ -96,7 +96,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-// Decode one 64-weight NF4 block (32 packed bytes at pk) with block scale s
+// Decode one 64-weight NF4 block (packed bytes 0..15 at pk_lo, 16..31 at
+// pk_hi) with block scale s
 // into one 128-byte swizzled row at row_addr (row index within its 8-row
 // atom = sw).
 //
@@ -106,8 +107,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // with byte permutes: one permute per plane and per half of the table
 // (nibble bits 0..2), one to pick the half (nibble bit 3) and two to
 // interleave the planes back into bf16 pairs.  No shared-memory lookups.
-__device__ __forceinline__ void decode_row(const uint8_t* pk, float s, uint32_t row_addr,
-                                           uint32_t sw) {
+__device__ __forceinline__ void decode_row(const uint8_t* pk_lo, const uint8_t* pk_hi, float s,
+                                           uint32_t row_addr, uint32_t sw) {
   uint32_t P[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j)
@@ -117,8 +118,8 @@ __device__ __forceinline__ void decode_row(const uint8_t* pk, float s, uint32_t 
   const uint32_t L1 = __byte_perm(P[2], P[3], 0x6420), H1 = __byte_perm(P[2], P[3], 0x7531);
   const uint32_t L2 = __byte_perm(P[4], P[5], 0x6420), H2 = __byte_perm(P[4], P[5], 0x7531);
   const uint32_t L3 = __byte_perm(P[6], P[7], 0x6420), H3 = __byte_perm(P[6], P[7], 0x7531);
-  const uint4 p0 = *reinterpret_cast<const uint4*>(pk);
-  const uint4 p1 = *reinterpret_cast<const uint4*>(pk + 16);
+  const uint4 p0 = *reinterpret_cast<const uint4*>(pk_lo);
+  const uint4 p1 = *reinterpret_cast<const uint4*>(pk_hi);
   const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
   for (int j = 0; j < 8; ++j) {  // word j = weights 8j .. 8j+7 (nibble i = weight 8j+i)
@@ -138,34 +139,48 @@ __device__ __forceinline__ void decode_row(const uint8_t* pk, float s, uint32_t 
   }
 }
 
-// TMEM accumulator columns [c_begin, c_end) of this warp's 32 lanes ->
-// global memory: bf16 outputs, or fp32 split-K partials.
-__device__ __noinline__ void epilogue_store(uint32_t tmem, int quad, int lane, int m0, int64_t n0,
-                                            int c_begin, int c_end, int split, const TcParams& p) {
-  const int mw = m0 + quad * 32 + lane;
-  const size_t Mw = (size_t)p.Mw;
+// TMA bulk tensor store of a shared-memory box (3D map: weight-side
+// column, token, split); coordinates past the tensor edge are not written.
+__device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int32_t x, int32_t y,
+                                             int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(tmap),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// TMEM accumulator columns [c_begin, c_end) (tokens) of this warp's 32
+// lanes (weight-side rows 32*quad + lane) -> the group's staging area `ep`
+// laid out as two boxes [ncols tokens][64 weight-side columns] (rows 0..63
+// and 64..127 of the tile), bf16 outputs or fp32 split-K partials.
+template <bool PARTIAL>
+__device__ __forceinline__ void epilogue_stage(uint32_t tmem, int quad, int lane, int c_begin,
+                                               int c_end, int ncols, uint8_t* ep) {
+  constexpr int ES = PARTIAL ? 4 : 2;
+  const int half = quad >> 1, col64 = (quad & 1) * 32 + lane;
+  uint8_t* base = ep + ((size_t)half * ncols * 64 + col64) * ES;
 #pragma unroll 1
   for (int c0 = c_begin; c0 < c_end; c0 += 32) {
     uint32_t v[32];
     tmem_ld_32x32b_x32(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)c0, v);
     tmem_ld_wait();
-    // one token per j: 32 lanes store 32 consecutive weight-side entries
-    const int64_t tok0 = n0 + c0;
-    const int jmax = (int)min((int64_t)min(32, c_end - c0), p.R - tok0);
-    if (p.partial) {
-      float* dst = (float*)p.out + ((size_t)split * (size_t)p.R + (size_t)tok0) * Mw + mw;
+    uint8_t* dst = base + (size_t)(c0 - c_begin) * 64 * ES;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (j < jmax) *dst = __uint_as_float(v[j]);
-        dst += Mw;
+    for (int j = 0; j < 32; ++j) {
+      if (c0 + j < c_end) {
+        if (PARTIAL)
+          *reinterpret_cast<uint32_t*>(dst) = v[j];
+        else
+          *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(__uint_as_float(v[j]));
       }
-    } else {
-      __nv_bfloat16* dst = (__nv_bfloat16*)p.out + (size_t)tok0 * Mw + mw;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if (j < jmax) *dst = __float2bfloat16_rn(__uint_as_float(v[j]));
-        dst += Mw;
-      }
+      dst += 64 * ES;
     }
   }
 }
@@ -186,7 +201,8 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
     tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_pk,
                       const __grid_constant__ CUtensorMap tm_aact,
-                      const __grid_constant__ CUtensorMap tm_aw, const TcParams p) {
+                      const __grid_constant__ CUtensorMap tm_aw,
+                      const __grid_constant__ CUtensorMap tm_out, const TcParams p) {
   using L = Smem<BN>;
   constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, BN, DX);
@@ -317,7 +333,20 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
     };
     const uint32_t row_off = DX ? (uint32_t)((u >> 6) * (kWTile / 2) + (u & 63) * 128) : (uint32_t)u * 128;
     const uint32_t sw = (uint32_t)(u & 7);
-    const uint32_t pk_off = DX ? (uint32_t)((u & 63) * 64 + (u >> 6) * 32) : (uint32_t)u * 32;
+    // Packed tile as TMA wrote it: forward 128 rows x 32 B with the 32-byte
+    // swizzle (16-byte half c of row y at c ^ bit 2 of y), dX 64 rows x 64 B
+    // with the 64-byte swizzle (chunk c of row y at c ^ bits 1..2 of y).
+    // Eight consecutive lanes then hit eight different bank groups.
+    uint32_t pk_lo, pk_hi;
+    if (!DX) {
+      const uint32_t x = (uint32_t)(u >> 2) & 1u;
+      pk_lo = (uint32_t)u * 32 + ((0u ^ x) << 4);
+      pk_hi = (uint32_t)u * 32 + ((1u ^ x) << 4);
+    } else {
+      const uint32_t o = (uint32_t)(u & 63), h = (uint32_t)(u >> 6), x = (o >> 1) & 3u;
+      pk_lo = o * 64 + (((2 * h) ^ x) << 4);
+      pk_hi = o * 64 + (((2 * h + 1) ^ x) << 4);
+    }
     auto kb_of = [&](int it) { return kb_lo + it - has_ad; };
     int it = group;
     uint32_t q_next = 0;
@@ -350,21 +379,47 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
                   mbar_wait(smem_u32(&full_pk[s]), par, p.wait_ns, p.err, 0x302);
       if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
       if (!adapter)
-        decode_row(pk + s * kPkTile + pk_off, sc, smem_u32(wdec + s * kWTile) + row_off, sw);
+        decode_row(pk + s * kPkTile + pk_lo, pk + s * kPkTile + pk_hi, sc,
+                   smem_u32(wdec + s * kWTile) + row_off, sw);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&dec[s]));
     }
-    // ------------------------------------------------------------ epilogue
-    // Warp w reads TMEM lanes 32*(w%4) .. +31; the two groups split the
-    // token columns (group 0 alone when the tile is narrower than 64).
+    // the accumulator is complete once acc_full fires
     const bool acc_ok = mbar_wait(smem_u32(acc_full), 0, p.wait_ns, p.err, 0x401);
-    tc_fence_after();
-    const bool aborted = __any_sync(0xffffffffu, !ok || !acc_ok || *abort_flag != 0);
+    if (!ok || !acc_ok) *abort_flag = 1;
+  }
+  // All roles are past the main loop: the stage buffers are free and the
+  // abort flag is final (and the same for every thread after this barrier).
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp >= 2 && *abort_flag == 0) {
+    // ---------------------------------------------------------- epilogue
+    // Warp w reads TMEM lanes 32*(w%4) .. +31; the two decoder groups split
+    // the token columns (group 0 alone when the tile is narrower than 64).
+    // Each group stages its columns in the freed stage buffers and one
+    // thread writes them with two TMA stores (weight-side rows 0..63, 64..127).
+    const int group = (warp - 2) >> 2;
     constexpr int kColsPerGroup = BN >= 64 ? BN / kDecGroups : BN;
     const int c_begin = BN >= 64 ? group * kColsPerGroup : 0;
     const int c_end = BN >= 64 ? c_begin + kColsPerGroup : (group == 0 ? BN : 0);
-    if (!aborted) epilogue_store(tmem, warp & 3, lane, m0, n0, c_begin, c_end, split, p);
+    if (c_end > c_begin) {
+      const int es = p.partial ? 4 : 2;
+      uint8_t* ep = smem + (size_t)group * 2 * kColsPerGroup * 64 * es;
+      if (p.partial)
+        epilogue_stage<true>(tmem, warp & 3, lane, c_begin, c_end, kColsPerGroup, ep);
+      else
+        epilogue_stage<false>(tmem, warp & 3, lane, c_begin, c_end, kColsPerGroup, ep);
+      fence_proxy_async_smem();
+      named_bar_sync(1 + group, 128);
+      if (((warp - 2) & 3) == 0 && lane == 0) {
+        const int32_t y = (int32_t)(n0 + c_begin);
+        tma_store_3d(&tm_out, smem_u32(ep), m0, y, split);
+        tma_store_3d(&tm_out, smem_u32(ep + (size_t)kColsPerGroup * 64 * es), m0 + 64, y, split);
+        bulk_commit_and_wait_read();
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -393,7 +448,7 @@ EncodeTiled encode_fn() {
 
 // 2D row-major tensor [rows x cols] of `esize`-byte elements, box [br x bc].
 bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
-              uint64_t rows, uint32_t bc, uint32_t br, bool swz128) {
+              uint64_t rows, uint32_t bc, uint32_t br, CUtensorMapSwizzle swz) {
   EncodeTiled enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -402,8 +457,26 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
   cuuint32_t es[2] = {1, 1};
   CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   swz128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   swz,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3D output map [splits][rows][cols] of `esize`-byte elements, box
+// [1][br][64] (one 64-column half of a tile), no swizzle.
+bool make_out_map(CUtensorMap* m, const void* base, bool fp32, uint64_t cols, uint64_t rows,
+                  uint64_t splits, uint32_t br) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t es = fp32 ? 4 : 2;
+  cuuint64_t dims[3] = {cols, rows, splits};
+  cuuint64_t strides[2] = {cols * es, cols * rows * es};
+  cuuint32_t box[3] = {64, br, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -424,10 +497,20 @@ constexpr size_t smem_bytes() {
          64 + 64;
 }
 
+// Columns of the token tile each decoder group stores, and the staging
+// bytes that takes (worst case fp32); it must fit in the stage buffers.
+template <int BN>
+constexpr int cols_per_group() {
+  return BN >= 64 ? BN / kDecGroups : BN;
+}
+
 template <bool DX, int BN>
 cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
-                      const CUtensorMap& d, const TcParams& p, cudaStream_t st) {
+                      const CUtensorMap& d, const CUtensorMap& o, const TcParams& p,
+                      cudaStream_t st) {
   constexpr int S = stages_for<BN>();
+  static_assert((BN >= 64 ? 2 : 1) * 2 * cols_per_group<BN>() * 64 * 4 <= S * (kWTile + Smem<BN>::kAct),
+                "epilogue staging must fit in the stage buffers");
   auto kern = tc_qlinear_kernel<DX, BN, S>;
   const size_t sm = smem_bytes<BN>();
   static bool attr_set = false;  // once per instantiation (keeps graph capture free of it)
@@ -439,7 +522,7 @@ cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, con
   const double flops = 2.0 * (double)p.R * (double)p.Mw * (double)p.KB * kBK +
                        2.0 * (double)p.R * (double)p.Mw * (double)p.rank;
   const int slot = timing_begin(st, DX ? 1 : 0, flops);
-  kern<<<grid, kThreads, sm, st>>>(a, b, c, d, p);
+  kern<<<grid, kThreads, sm, st>>>(a, b, c, d, o, p);
   timing_end(slot, st);
   count_launch();
   return cudaGetLastError();
@@ -447,16 +530,18 @@ cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, con
 
 template <bool DX>
 cudaError_t launch_plan(const TcPlan& pl, dim3 grid, const CUtensorMap& a, const CUtensorMap& b,
-                        const CUtensorMap& c, const CUtensorMap& d, const TcParams& p,
-                        cudaStream_t st) {
+                        const CUtensorMap& c, const CUtensorMap& d, const CUtensorMap& o,
+                        const TcParams& p, cudaStream_t st) {
   switch (pl.bn) {
-    case 16: return launch_bn<DX, 16>(grid, a, b, c, d, p, st);
-    case 32: return launch_bn<DX, 32>(grid, a, b, c, d, p, st);
-    case 64: return launch_bn<DX, 64>(grid, a, b, c, d, p, st);
-    case 128: return launch_bn<DX, 128>(grid, a, b, c, d, p, st);
-    default: return launch_bn<DX, 256>(grid, a, b, c, d, p, st);
+    case 16: return launch_bn<DX, 16>(grid, a, b, c, d, o, p, st);
+    case 32: return launch_bn<DX, 32>(grid, a, b, c, d, o, p, st);
+    case 64: return launch_bn<DX, 64>(grid, a, b, c, d, o, p, st);
+    case 128: return launch_bn<DX, 128>(grid, a, b, c, d, o, p, st);
+    default: return launch_bn<DX, 256>(grid, a, b, c, d, o, p, st);
   }
 }
+
+int group_cols(int bn) { return bn >= 64 ? bn / kDecGroups : bn; }
 
 bool ptr_aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
@@ -500,11 +585,11 @@ TcPlan tc_plan(int64_t Mw, int64_t KB, int64_t R) {
 }
 
 bool tc_fwd_supported(const WView& w, const void* X, const void* Y, int64_t R) {
-  return common_supported(w, R) && ptr_aligned(X, 16) && ptr_aligned(Y, 2);
+  return common_supported(w, R) && ptr_aligned(X, 16) && ptr_aligned(Y, 16);
 }
 
 bool tc_dx_supported(const WView& w, const void* dY, const void* dX, int64_t R) {
-  return common_supported(w, R) && ptr_aligned(dY, 16) && ptr_aligned(dX, 2);
+  return common_supported(w, R) && ptr_aligned(dY, 16) && ptr_aligned(dX, 16);
 }
 
 // Workspace: U_pad / V_pad bf16 [R x 64], the adapter weight operand bf16
@@ -529,15 +614,17 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   uint16_t* upad = (uint16_t*)tcws;
   uint16_t* bpad = (uint16_t*)((char*)tcws + align_up((size_t)R * 128, 256));
   float* part = (float*)((char*)bpad + align_up((size_t)O * 128, 256));
-  (void)U;  // its bf16 copy upad was written by the rowdot kernel that made U
-  cudaError_t e = launch_pad_rows_bf16(B, O, r, s, bpad, st);
-  if (e != cudaSuccess) return e;
+  // upad (bf16 U) and bpad (bf16(s B)) were written by the rowdot launch that made U
+  (void)U;
+  (void)B;
+  (void)s;
+  cudaError_t e = cudaSuccess;
   CUtensorMap m_act, m_pk, m_aact, m_aw;
   const uint32_t bn = (uint32_t)pl.bn;
-  if (!make_map(&m_act, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, R, 64, bn, true) ||
-      !make_map(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I / 2, O, 32, 128, false) ||
-      !make_map(&m_aact, upad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, true) ||
-      !make_map(&m_aw, bpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, O, 64, 128, true))
+  if (!make_map(&m_act, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I / 2, O, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !make_map(&m_aact, upad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&m_aw, bpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, O, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   TcParams p;
   p.R = R;
@@ -555,8 +642,12 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   p.out = pl.splits > 1 ? (void*)part : Y;
   p.err = hdr;
   p.wait_ns = kWaitLimitNs;
+  CUtensorMap m_out;
+  if (!make_out_map(&m_out, p.out, pl.splits > 1, (uint64_t)O, (uint64_t)R, (uint64_t)pl.splits,
+                    (uint32_t)group_cols(pl.bn)))
+    return cudaErrorInvalidValue;
   dim3 grid((unsigned)(O / kBM), (unsigned)((R + pl.bn - 1) / pl.bn), (unsigned)pl.splits);
-  e = launch_plan<false>(pl, grid, m_act, m_pk, m_aact, m_aw, p, st);
+  e = launch_plan<false>(pl, grid, m_act, m_pk, m_aact, m_aw, m_out, p, st);
   if (e != cudaSuccess || pl.splits == 1) return e;
   return launch_splitk_reduce(part, pl.splits, R, O, true, Y, st);
 }
@@ -569,15 +660,17 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   uint16_t* vpad = (uint16_t*)tcws;
   uint16_t* apad = (uint16_t*)((char*)tcws + align_up((size_t)R * 128, 256));
   float* part = (float*)((char*)apad + align_up((size_t)I * 128, 256));
-  (void)V;  // its bf16 copy vpad was written by the rowdot kernel that made V
-  cudaError_t e = launch_pad_cols_bf16(A, r, I, s, apad, st);
-  if (e != cudaSuccess) return e;
+  // vpad (bf16 V) and apad (bf16(s A)) were written by the rowdot launch that made V
+  (void)V;
+  (void)A;
+  (void)s;
+  cudaError_t e = cudaSuccess;
   CUtensorMap m_act, m_pk, m_aact, m_aw;
   const uint32_t bn = (uint32_t)pl.bn;
-  if (!make_map(&m_act, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, O, R, 64, bn, true) ||
-      !make_map(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I / 2, O, 64, 64, false) ||
-      !make_map(&m_aact, vpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, true) ||
-      !make_map(&m_aw, apad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, 64, 64, 64, true))
+  if (!make_map(&m_act, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, O, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I / 2, O, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map(&m_aact, vpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&m_aw, apad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, 64, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   TcParams p;
   p.R = R;
@@ -595,8 +688,12 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   p.out = pl.splits > 1 ? (void*)part : dX;
   p.err = hdr;
   p.wait_ns = kWaitLimitNs;
+  CUtensorMap m_out;
+  if (!make_out_map(&m_out, p.out, pl.splits > 1, (uint64_t)I, (uint64_t)R, (uint64_t)pl.splits,
+                    (uint32_t)group_cols(pl.bn)))
+    return cudaErrorInvalidValue;
   dim3 grid((unsigned)(I / kBM), (unsigned)((R + pl.bn - 1) / pl.bn), (unsigned)pl.splits);
-  e = launch_plan<true>(pl, grid, m_act, m_pk, m_aact, m_aw, p, st);
+  e = launch_plan<true>(pl, grid, m_act, m_pk, m_aact, m_aw, m_out, p, st);
   if (e != cudaSuccess || pl.splits == 1) return e;
   return launch_splitk_reduce(part, pl.splits, R, I, true, dX, st);
 }

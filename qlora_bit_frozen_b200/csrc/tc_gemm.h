@@ -26,6 +26,12 @@ size_t tc_dx_ws(const WView& w, int64_t R);
 // U (forward) or V (input gradient), zero-padded to 64 columns; the caller
 // fills it (launch_rowdot's pad output) before the launch.
 inline uint16_t* tc_act_pad(void* tcws) { return (uint16_t*)tcws; }
+// Next region: the adapter-step weight operand, bf16(s B) [O x 64] in the
+// forward or bf16(s A) [64 x I] in the input gradient, also filled by the
+// caller (launch_rowdot's side job).
+inline uint16_t* tc_w_pad(void* tcws, int64_t R) {
+  return (uint16_t*)((char*)tcws + (((size_t)R * 128 + 255) / 256) * 256);
+}
 
 // Y = X W_hat^T + s U B^T  (bf16 in/out, fp32 accumulation in TMEM).
 cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float* U,
