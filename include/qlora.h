@@ -143,6 +143,29 @@ qlora_status qlora_quantize_nf4(const float* W, int64_t O, int64_t I, int32_t B,
                                 uint8_t* codes, uint8_t* scale_codes, float* t, float* mu,
                                 void* ws, size_t ws_bytes, qlora_stream_t stream);
 
+/*
+ * qlora_quantize_nf4 for callers that cannot allocate device memory (the
+ * pages have no counterpart; this is an interface convenience).  A plugin
+ * inside a framework whose caching allocator owns the device memory, or a
+ * plain C caller with no allocator, may be unable to provide the workspace
+ * qlora_quantize_nf4 needs; this entry point takes none and calls no
+ * allocation routine.  Its scratch is one file-scope device array of
+ * 8 MiB that every GPU loading the library holds until the process exits;
+ * that covers qlora_quantize_nf4_workspace_bytes(N, B, C) <= 8 MiB (at B = 64,
+ * C = 256 about 133 million weights).  Larger inputs return
+ * QLORA_ERR_WORKSPACE (use qlora_quantize_nf4 with a workspace instead).
+ * Same arguments (minus the workspace), outputs, bit-exact results and
+ * synchronization as qlora_quantize_nf4.
+ * The first call on a device looks up the array's device address there
+ * (with that device current); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents: calls that overlap on the GPU (another stream, another host
+ * thread on the same device) race and must be serialized by the caller.
+ */
+qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t O, int64_t I, int32_t B, int32_t C,
+                                        uint8_t* codes, uint8_t* scale_codes, float* t, float* mu,
+                                        qlora_stream_t stream);
+
 /* HOST.  Workspace bytes qlora_quantize_affine needs. */
 size_t qlora_quantize_affine_workspace_bytes(int64_t N, int32_t bits, int32_t G);
 

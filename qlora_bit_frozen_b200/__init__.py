@@ -21,7 +21,8 @@ from ._ffi import (COMPUTE_BF16, COMPUTE_FP32, FMT_AFFINE, FMT_NF4_DQ, OP_BWD, O
 
 __all__ = [
     "QLoraError", "QuantizedWeight", "qlora_status_string", "qlora_nf4_codebook",
-    "qlora_nf4_payload_bytes", "qlora_quantize_nf4", "qlora_quantize_affine", "qlora_dequantize",
+    "qlora_nf4_payload_bytes", "qlora_quantize_nf4", "qlora_quantize_nf4_noalloc", "qlora_quantize_affine",
+    "qlora_dequantize",
     "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_workspace_status", "qlora_selftest_wait_timeout", "qlora_kernel_launch_count",
     "qlora_kernel_timing_enable", "qlora_kernel_timing_collect",
@@ -118,6 +119,29 @@ def qlora_quantize_nf4(W: torch.Tensor, B: int = 64, C: int = 256, stream=None) 
     st = lib.qlora_quantize_nf4(_ptr(W), O, I, B, C, _ptr(codes), _ptr(q), _ptr(t), _ptr(mu), _ptr(ws),
                                 ws.numel(), _stream(stream))
     _check(st, "qlora_quantize_nf4")
+    return QuantizedWeight(FMT_NF4_DQ, O, I, B, C, 4, codes, q, t, mu)
+
+
+def qlora_quantize_nf4_noalloc(W: torch.Tensor, B: int = 64, C: int = 256, stream=None) -> QuantizedWeight:
+    """As qlora_quantize_nf4, for callers that cannot supply a workspace: the
+    library's fixed device scratch is used (see include/qlora.h).  The output
+    buffers are still the caller's; calls sharing the scratch must not overlap."""
+    lib = _ffi.load()
+    if W.dim() != 2 or W.dtype != torch.float32 or not W.is_cuda:
+        raise ValueError("W must be a CUDA float32 matrix")
+    W = W.contiguous()
+    O, I = W.shape
+    N = O * I
+    M = -(-N // B)
+    S = -(-M // C)
+    dev = W.device
+    codes = torch.empty((N + 1) // 2, dtype=torch.uint8, device=dev)
+    q = torch.empty(M, dtype=torch.uint8, device=dev)
+    t = torch.empty(S, dtype=torch.float32, device=dev)
+    mu = torch.empty(1, dtype=torch.float32, device=dev)
+    st = lib.qlora_quantize_nf4_noalloc(_ptr(W), O, I, B, C, _ptr(codes), _ptr(q), _ptr(t), _ptr(mu),
+                                        _stream(stream))
+    _check(st, "qlora_quantize_nf4_noalloc")
     return QuantizedWeight(FMT_NF4_DQ, O, I, B, C, 4, codes, q, t, mu)
 
 

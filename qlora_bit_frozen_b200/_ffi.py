@@ -55,6 +55,7 @@ SIGNATURES = {
     "qlora_nf4_payload_bytes": (_sz, [_i64, _i32, _i32]),
     "qlora_quantize_nf4_workspace_bytes": (_sz, [_i64, _i32, _i32]),
     "qlora_quantize_nf4": (ctypes.c_int, [_P, _i64, _i64, _i32, _i32, _P, _P, _P, _P, _P, _sz, _P]),
+    "qlora_quantize_nf4_noalloc": (ctypes.c_int, [_P, _i64, _i64, _i32, _i32, _P, _P, _P, _P, _P]),
     "qlora_quantize_affine_workspace_bytes": (_sz, [_i64, _i32, _i32]),
     "qlora_quantize_affine": (ctypes.c_int, [_P, _i64, _i64, _i32, _i32, _P, _P, _P, _P, _sz, _P]),
     "qlora_dequantize": (ctypes.c_int, [_W, _P, _P]),

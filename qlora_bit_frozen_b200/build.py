@@ -15,7 +15,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libqlora.so")
 
-SOURCES = ["api.cu", "quantize.cu", "simt.cu", "adapter.cu", "tc_gemm.cu"]
+SOURCES = ["api.cu", "quantize.cu", "simt.cu", "adapter.cu", "tc_gemm.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "internal.h", "tc_gemm.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
