@@ -458,18 +458,32 @@ __global__ void __launch_bounds__(kThreads) coldot_kernel(const T* __restrict__ 
 
 constexpr int kStages = 4;
 
-// rowdot: block = 16 rows (2 per warp); tile = KT columns of P and of
-// L [r x K] (KT * RMAX = 2048 floats = 8 KB).  Lane l owns columns
-// l*EPL .. l*EPL+EPL-1 of the tile.
+// Lane l of a warp owns the tile columns {128 h + 4 l + e : h < H, e < 4}
+// (H = KT / 128) when KT >= 128, else {l * E + e : e < E} (E = KT / 32):
+// consecutive lanes then read consecutive 16-byte (or 8-byte) words of a
+// shared-memory row, free of bank conflicts.
+template <int KT>
+struct LaneCols {
+  static constexpr int E = KT >= 128 ? 4 : KT / 32;  // elements per group
+  static constexpr int H = KT >= 128 ? KT / 128 : 1;  // groups per lane
+  static constexpr int N = E * H;                      // elements per lane
+  __device__ static int col(int lane, int h) { return KT >= 128 ? 128 * h + 4 * lane : lane * E; }
+};
+
+// rowdot: block = 8 warps x RW rows (RW * RMAX <= 64 accumulators per
+// thread); tile = KT columns of P and of L [r x K] (KT * RMAX = 2048 floats).
 template <typename T, int RMAX>
 struct RowPipe {
-  static constexpr int RB = 16;
+  static constexpr int RW = 64 / RMAX >= 4 ? 4 : 64 / RMAX;
+  static constexpr int RB = 8 * RW;
   static constexpr int KT = 2048 / RMAX;
-  static constexpr int EPL = KT / 32;
   static constexpr int XB = RB * KT * (int)sizeof(T);
   static constexpr int LB = RMAX * KT * 4;
   static constexpr int STAGE = XB + LB;
   static constexpr int SMEM = kStages * STAGE;
+  static constexpr int XTOT = XB / 16, LTOT = LB / 16;  // 16-byte copies per tile
+  static constexpr int XCH = (XTOT + kThreads - 1) / kThreads;  // per thread (some idle)
+  static constexpr int LCH = (LTOT + kThreads - 1) / kThreads;
 };
 
 template <typename T, int RMAX>
@@ -481,39 +495,56 @@ __global__ void __launch_bounds__(kThreads) rowdot_pipe_kernel(
     return;
   }
   using C = RowPipe<T, RMAX>;
+  using LC = LaneCols<C::KT>;
+  constexpr int EPC = 16 / (int)sizeof(T);          // elements per 16-byte copy
+  constexpr int ROWCH = C::KT / EPC;                // copies per P row of a tile
+  constexpr int LROWCH = C::KT / 4;                 // copies per L row of a tile
   extern __shared__ __align__(16) uint8_t sm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t rb0 = (int64_t)blockIdx.x * C::RB;
   const int ntiles = (int)((K + C::KT - 1) / C::KT);
-  constexpr int XCH = C::XB / 16, LCH = C::LB / 16;  // 16-byte chunks per tile
-  constexpr int ROWCH = C::KT * (int)sizeof(T) / 16;  // chunks per P row
-  constexpr int LROWCH = C::KT * 4 / 16;               // chunks per L row
-
+  // fixed copy slots of this thread: P rows/cols and L rows/cols
+  int xrow[C::XCH], xcol[C::XCH], lrow[C::LCH], lcol[C::LCH];
+#pragma unroll
+  for (int i = 0; i < C::XCH; ++i) {
+    const int c = threadIdx.x + kThreads * i;
+    xrow[i] = c / ROWCH;
+    xcol[i] = (c - xrow[i] * ROWCH) * EPC;
+  }
+#pragma unroll
+  for (int i = 0; i < C::LCH; ++i) {
+    const int c = threadIdx.x + kThreads * i;
+    lrow[i] = c / LROWCH;
+    lcol[i] = (c - lrow[i] * LROWCH) * 4;
+  }
   auto issue = [&](int t) {
-    const int stg = t % kStages;
-    const uint32_t xs = (uint32_t)__cvta_generic_to_shared(sm + stg * C::STAGE);
+    const uint32_t xs = (uint32_t)__cvta_generic_to_shared(sm + (t % kStages) * C::STAGE);
     const uint32_t ls = xs + C::XB;
     const int64_t k0 = (int64_t)t * C::KT;
-    for (int c = threadIdx.x; c < XCH; c += kThreads) {
-      const int row = c / ROWCH, cc = c - row * ROWCH;
-      const int64_t m = rb0 + row;
-      const int64_t k = k0 + (int64_t)cc * (16 / (int)sizeof(T));
+#pragma unroll
+    for (int i = 0; i < C::XCH; ++i) {
+      if (threadIdx.x + kThreads * i >= C::XTOT) break;
+      const int64_t m = rb0 + xrow[i], k = k0 + xcol[i];
       const int64_t rem = (K - k) * (int64_t)sizeof(T);
       const uint32_t nb = (m < R && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
-      cp_async16(xs + c * 16, nb ? (const void*)(P + m * K + k) : (const void*)P, nb);
+      cp_async16(xs + (uint32_t)(xrow[i] * ROWCH * 16 + xcol[i] * (int)sizeof(T)),
+                 nb ? (const void*)(P + m * K + k) : (const void*)P, nb);
     }
-    for (int c = threadIdx.x; c < LCH; c += kThreads) {
-      const int j = c / LROWCH, cc = c - j * LROWCH;
-      const int64_t k = k0 + (int64_t)cc * 4;
+#pragma unroll
+    for (int i = 0; i < C::LCH; ++i) {
+      if (threadIdx.x + kThreads * i >= C::LTOT) break;
+      const int64_t k = k0 + lcol[i];
       const int64_t rem = (K - k) * 4;
-      const uint32_t nb = (j < r && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
-      cp_async16(ls + c * 16, nb ? (const void*)(L + (int64_t)j * K + k) : (const void*)L, nb);
+      const uint32_t nb = (lrow[i] < r && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
+      cp_async16(ls + (uint32_t)(lrow[i] * C::KT * 4 + lcol[i] * 4),
+                 nb ? (const void*)(L + (int64_t)lrow[i] * K + k) : (const void*)L, nb);
     }
   };
 
-  float acc[2][RMAX];
+  constexpr int RW = C::RW;
+  float acc[RW][RMAX];
 #pragma unroll
-  for (int q = 0; q < 2; ++q)
+  for (int q = 0; q < RW; ++q)
 #pragma unroll
     for (int j = 0; j < RMAX; ++j) acc[q][j] = 0.0f;
 #pragma unroll
@@ -528,32 +559,44 @@ __global__ void __launch_bounds__(kThreads) rowdot_pipe_kernel(
     cp_async_commit();
     const uint8_t* xs = sm + (t % kStages) * C::STAGE;
     const float* ls = (const float*)(xs + C::XB);
-    float x[2][C::EPL];
+    float x[RW][LC::N];
 #pragma unroll
-    for (int q = 0; q < 2; ++q)
-      load_vec<T, C::EPL>((const T*)xs + (warp * 2 + q) * C::KT + lane * C::EPL, x[q]);
+    for (int q = 0; q < RW; ++q)
+#pragma unroll
+      for (int h = 0; h < LC::H; ++h) {
+        float v[LC::E];
+        load_vec<T, LC::E>((const T*)xs + (warp * RW + q) * C::KT + LC::col(lane, h), v);
+#pragma unroll
+        for (int e = 0; e < LC::E; ++e) x[q][h * LC::E + e] = v[e];
+      }
 #pragma unroll
     for (int j = 0; j < RMAX; ++j) {
       if (j < r) {
-        float l[C::EPL];
-        load_vec<float, C::EPL>(ls + j * C::KT + lane * C::EPL, l);
+        float l[LC::N];
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
+        for (int h = 0; h < LC::H; ++h) {
+          float v[LC::E];
+          load_vec<float, LC::E>(ls + j * C::KT + LC::col(lane, h), v);
 #pragma unroll
-          for (int e = 0; e < C::EPL; ++e) acc[q][j] = fmaf(x[q][e], l[e], acc[q][j]);
+          for (int e = 0; e < LC::E; ++e) l[h * LC::E + e] = v[e];
+        }
+#pragma unroll
+        for (int q = 0; q < RW; ++q)
+#pragma unroll
+          for (int e = 0; e < LC::N; ++e) acc[q][j] = fmaf(x[q][e], l[e], acc[q][j]);
       }
     }
   }
   cp_async_wait<0>();
 #pragma unroll
-  for (int q = 0; q < 2; ++q)
+  for (int q = 0; q < RW; ++q)
 #pragma unroll
     for (int j = 0; j < RMAX; ++j)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) acc[q][j] += __shfl_xor_sync(0xffffffffu, acc[q][j], o);
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    const int64_t m = rb0 + warp * 2 + q;
+  for (int q = 0; q < RW; ++q) {
+    const int64_t m = rb0 + warp * RW + q;
     if (m >= R) continue;
     float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
@@ -571,56 +614,61 @@ __global__ void __launch_bounds__(kThreads) rowdot_pipe_kernel(
   }
 }
 
-// coldot: block = 512 columns (2 per thread) over a row slice; tile = 32
-// rows of P (32 KB bf16) and the matching 32 rows of aux [R x r].
+// coldot: block = 128 threads x 2 columns = 256 columns over a row slice;
+// tile = 32 rows of P (16 KB bf16) and the matching 32 rows of aux [R x r].
+constexpr int kColThreadsP = 128;
+constexpr int kColStages = 3;
 template <typename T, int RMAX>
 struct ColPipe {
-  static constexpr int NC = 512;
+  static constexpr int NC = 256;
   static constexpr int RT = 32;
   static constexpr int PB = RT * NC * (int)sizeof(T);
   static constexpr int AB = RT * RMAX * 4;
   static constexpr int STAGE = PB + AB;
-  static constexpr int SMEM = kStages * STAGE;
+  static constexpr int SMEM = kColStages * STAGE;
+  static constexpr int PCH = PB / 16 / kColThreadsP;  // 16-byte copies per thread per tile
 };
 
 template <typename T, int RMAX>
-__global__ void __launch_bounds__(kThreads) coldot_pipe_kernel(
+__global__ void __launch_bounds__(kColThreadsP) coldot_pipe_kernel(
     const T* __restrict__ P, int64_t R, int64_t N, const float* __restrict__ aux, int r,
     int64_t rows_per_split, float* __restrict__ part) {
   using C = ColPipe<T, RMAX>;
+  constexpr int EPC = 16 / (int)sizeof(T);
+  constexpr int ROWCH = C::NC / EPC;
   extern __shared__ __align__(16) uint8_t sm[];
   const int64_t nb = (int64_t)blockIdx.x * C::NC;
   const int64_t m_lo = (int64_t)blockIdx.y * rows_per_split;
   const int64_t m_hi = min(R, m_lo + rows_per_split);
   const int ntiles = (int)((m_hi - m_lo + C::RT - 1) / C::RT);
-  constexpr int PCH = C::PB / 16;
-  constexpr int ROWCH = C::NC * (int)sizeof(T) / 16;
-  const int ach_row = (r * 4 + 15) / 16;  // 16-byte chunks per aux row (r*4 bytes, padded)
-
+  int prow[C::PCH], pcol[C::PCH];
+#pragma unroll
+  for (int i = 0; i < C::PCH; ++i) {
+    const int c = threadIdx.x + kColThreadsP * i;
+    prow[i] = c / ROWCH;
+    pcol[i] = (c - prow[i] * ROWCH) * EPC;
+  }
+  const int ach = (C::RT * r * 4 + 15) / 16;  // aux copies per tile (<= 2 * RMAX)
   auto issue = [&](int t) {
-    const int stg = t % kStages;
-    const uint32_t ps = (uint32_t)__cvta_generic_to_shared(sm + stg * C::STAGE);
+    const uint32_t ps = (uint32_t)__cvta_generic_to_shared(sm + (t % kColStages) * C::STAGE);
     const uint32_t as = ps + C::PB;
     const int64_t r0 = m_lo + (int64_t)t * C::RT;
-    for (int c = threadIdx.x; c < PCH; c += kThreads) {
-      const int row = c / ROWCH, cc = c - row * ROWCH;
-      const int64_t m = r0 + row;
-      const int64_t n = nb + (int64_t)cc * (16 / (int)sizeof(T));
+#pragma unroll
+    for (int i = 0; i < C::PCH; ++i) {
+      const int64_t m = r0 + prow[i], n = nb + pcol[i];
       const int64_t rem = (N - n) * (int64_t)sizeof(T);
       const uint32_t bytes = (m < m_hi && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
-      cp_async16(ps + c * 16, bytes ? (const void*)(P + m * N + n) : (const void*)P, bytes);
+      cp_async16(ps + (uint32_t)(prow[i] * ROWCH * 16 + pcol[i] * (int)sizeof(T)),
+                 bytes ? (const void*)(P + m * N + n) : (const void*)P, bytes);
     }
-    // aux rows r0 .. r0+RT of [R x r] are contiguous: r0*r .. (r0+RT)*r floats
-    const int64_t a0 = r0 * r;
+    // aux rows r0 .. r0+RT of [R x r] are contiguous
     const int64_t a_end = min(m_hi, r0 + C::RT) * r;
-    const int nch = (C::RT * r * 4 + 15) / 16;
-    for (int c = threadIdx.x; c < nch; c += kThreads) {
-      const int64_t e = a0 + (int64_t)c * 4;
+    for (int c = threadIdx.x; c < ach; c += kColThreadsP) {
+      const int64_t e = r0 * r + (int64_t)c * 4;
       const int64_t rem = (a_end - e) * 4;
       const uint32_t bytes = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
       cp_async16(as + c * 16, bytes ? (const void*)(aux + e) : (const void*)aux, bytes);
     }
-    (void)ach_row;
   };
 
   float acc[2][RMAX];
@@ -629,17 +677,17 @@ __global__ void __launch_bounds__(kThreads) coldot_pipe_kernel(
 #pragma unroll
     for (int j = 0; j < RMAX; ++j) acc[q][j] = 0.0f;
 #pragma unroll
-  for (int t = 0; t < kStages - 1; ++t) {
+  for (int t = 0; t < kColStages - 1; ++t) {
     if (t < ntiles) issue(t);
     cp_async_commit();
   }
   const int col = threadIdx.x * 2;  // local column pair
   for (int t = 0; t < ntiles; ++t) {
-    cp_async_wait<kStages - 2>();
+    cp_async_wait<kColStages - 2>();
     __syncthreads();
-    if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
+    if (t + kColStages - 1 < ntiles) issue(t + kColStages - 1);
     cp_async_commit();
-    const uint8_t* ps = sm + (t % kStages) * C::STAGE;
+    const uint8_t* ps = sm + (t % kColStages) * C::STAGE;
     const float* as = (const float*)(ps + C::PB);  // row-major [RT x r]
     const int rows = (int)min((int64_t)C::RT, m_hi - (m_lo + (int64_t)t * C::RT));
     for (int row = 0; row < rows; ++row) {
@@ -677,22 +725,38 @@ __global__ void __launch_bounds__(kThreads) coldot_pipe_kernel(
   }
 }
 
-// out = s * sum over slices of part[slice][j][n], one warp per output
-// element (lanes take slices l, l+32, ...; fixed butterfly order).
-// out_nr == 0: out[j * N + n] (dA);  1: out[n * r + j] (dB).
-__global__ void slice_reduce_kernel(const float* __restrict__ part, int splits, int64_t N, int r,
-                                    float s, int out_nr, float* __restrict__ out) {
-  const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // e = j * N + n
-  const int lane = threadIdx.x & 31;
+// out = s * sum over slices of part[slice][j][n].  Block = 8 warps over 32
+// consecutive outputs e (= j * N + n): warp w sums slices w, w+8, ... for
+// lane-th output (coalesced across lanes), then the 8 warp sums are added in
+// warp order.  out_nr == 0: out[j * N + n] (dA);  1: out[n * r + j] (dB).
+__global__ void __launch_bounds__(256) slice_reduce_kernel(const float* __restrict__ part, int splits,
+                                                           int64_t N, int r, float s, int out_nr,
+                                                           float* __restrict__ out) {
+  __shared__ float red[8][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t rN = (int64_t)r * N;
-  if (e >= rN) return;
+  const int64_t e = (int64_t)blockIdx.x * 32 + lane;
   float v = 0.0f;
-  for (int k = lane; k < splits; k += 32) v += part[(int64_t)k * rN + e];
+  if (e < rN) {
+    int k = warp;
+    for (; k + 8 * 3 < splits; k += 8 * 4) {
+      const float a = part[(int64_t)k * rN + e], b = part[(int64_t)(k + 8) * rN + e];
+      const float c = part[(int64_t)(k + 16) * rN + e], d = part[(int64_t)(k + 24) * rN + e];
+      v += a;
+      v += b;
+      v += c;
+      v += d;
+    }
+    for (; k < splits; k += 8) v += part[(int64_t)k * rN + e];
+  }
+  red[warp][lane] = v;
+  __syncthreads();
+  if (warp == 0 && e < rN) {
+    float t = red[0][lane];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if (lane == 0) {
+    for (int w = 1; w < 8; ++w) t += red[w][lane];
     const int64_t j = e / N, n = e - j * N;
-    out[out_nr ? n * r + j : e] = s * v;
+    out[out_nr ? n * r + j : e] = s * t;
   }
 }
 
@@ -835,27 +899,29 @@ cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const 
                           float side_mul, uint16_t* side_dst, float* lt_ws) {
   PadJob job{side_src, side_dst, side_extent, r, side_mode, side_mul, 0};
   if (side_dst && side_extent > 0) job.blocks = (int)cdiv(64 * side_extent, kThreads * 8);
-  // pipelined path: bf16 rows on 16-byte boundaries, factor rows as [r x K]
-  const bool rows16 = bf16 && (K % 8) == 0 && ((uintptr_t)P % 16) == 0;
-  if (rows16 && R > 64 && (!l_is_kr || lt_ws)) {
-    const float* Lr = L;
-    if (l_is_kr) {  // B [K x r] -> B^T [r x K] in the caller's scratch
-      transpose_kr_kernel<<<cdiv((int64_t)r * K, 256), 256, 0, st>>>(L, K, r, lt_ws);
-      count_launch();
-      cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-      Lr = lt_ws;
-    }
-    if (((uintptr_t)Lr % 16) == 0) {
-      const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
-      if (r <= 8) return rowdot_pipe_go<8>(Pb, R, K, Lr, r, out, pad, job, st);
-      if (r <= 16) return rowdot_pipe_go<16>(Pb, R, K, Lr, r, out, pad, job, st);
-      if (r <= 32) return rowdot_pipe_go<32>(Pb, R, K, Lr, r, out, pad, job, st);
-      return rowdot_pipe_go<64>(Pb, R, K, Lr, r, out, pad, job, st);
-    }
+  // With scratch for it, a factor given as [K x r] is transposed first so
+  // every path below reads factor rows ([r x K]) contiguously.
+  const float* Lr = L;
+  bool lkr = l_is_kr;
+  if (l_is_kr && lt_ws && R > 0) {
+    transpose_kr_kernel<<<cdiv((int64_t)r * K, 256), 256, 0, st>>>(L, K, r, lt_ws);
+    count_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    Lr = lt_ws;
+    lkr = false;
   }
-  if (bf16) return rowdot_r<__nv_bfloat16>(P, R, K, L, l_is_kr, r, out, pad, job, st);
-  return rowdot_r<float>(P, R, K, L, l_is_kr, r, out, pad, job, st);
+  // pipelined path: more than 64 bf16 rows on 16-byte boundaries
+  const bool rows16 = bf16 && (K % 8) == 0 && ((uintptr_t)P % 16) == 0;
+  if (rows16 && R > 64 && !lkr && ((uintptr_t)Lr % 16) == 0 && (K % 4) == 0) {
+    const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
+    if (r <= 8) return rowdot_pipe_go<8>(Pb, R, K, Lr, r, out, pad, job, st);
+    if (r <= 16) return rowdot_pipe_go<16>(Pb, R, K, Lr, r, out, pad, job, st);
+    if (r <= 32) return rowdot_pipe_go<32>(Pb, R, K, Lr, r, out, pad, job, st);
+    return rowdot_pipe_go<64>(Pb, R, K, Lr, r, out, pad, job, st);
+  }
+  if (bf16) return rowdot_r<__nv_bfloat16>(P, R, K, Lr, lkr, r, out, pad, job, st);
+  return rowdot_r<float>(P, R, K, Lr, lkr, r, out, pad, job, st);
 }
 
 namespace {
@@ -894,7 +960,7 @@ cudaError_t coldot_pipe_go(const __nv_bfloat16* P, int64_t R, int64_t N, const f
   cudaError_t e = set_smem_once(kern, C::SMEM, attr);
   if (e != cudaSuccess) return e;
   dim3 grid(c.colblocks, (unsigned)c.splits);
-  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, N, aux, r, c.rows_per_split, part);
+  kern<<<grid, kColThreadsP, C::SMEM, st>>>(P, R, N, aux, r, c.rows_per_split, part);
   count_launch();
   return cudaGetLastError();
 }
@@ -929,8 +995,8 @@ cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const 
     else e = coldot_pipe_go<64>(Pb, R, N, aux, r, c, part, st);
     if (e != cudaSuccess) return e;
     const int64_t outs = (int64_t)r * N;
-    slice_reduce_kernel<<<cdiv(outs * 32, 256), 256, 0, st>>>(part, c.splits, N, r, s,
-                                                              out_nr ? 1 : 0, out);
+    slice_reduce_kernel<<<cdiv(outs, 32), 256, 0, st>>>(part, c.splits, N, r, s, out_nr ? 1 : 0,
+                                                        out);
     count_launch();
     return cudaGetLastError();
   }
