@@ -188,18 +188,24 @@ def run_gpu(args):
 
     # ------------------------------------------------ timed region (device)
     # One step is captured once in a CUDA graph (no host launch gaps in the
-    # device timing); the library records an event pair around each of its
-    # tensor-core GEMM launches inside the graph.
-    nrec = 16 * len(layers)
-    q.qlora_kernel_timing_enable(nrec)
+    # device timing) and replayed K times between CUDA events.  A second
+    # graph of the same step, with the library's event pair around each
+    # tensor-core GEMM launch, is then replayed K times for the per-kernel
+    # durations; those events also hold each launch back until the one
+    # before it has finished (no programmatic overlap), so the step time
+    # comes from the first pass only.
+    def capture():
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+            step()
+        torch.cuda.synchronize()
+        return g
+
     n_before = q.qlora_kernel_launch_count()
-    graph = torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream()
-    cap.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.graph(graph, stream=cap, capture_error_mode="thread_local"):
-        step()
+    graph = capture()
     kernels_per_step = q.qlora_kernel_launch_count() - n_before
-    torch.cuda.synchronize()
     for _ in range(args.warmup):
         flush.zero_()
         graph.replay()
@@ -207,23 +213,33 @@ def run_gpu(args):
     clocks = ClockSampler(local)
     clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    recs = []
     barrier()
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
         graph.replay()
         ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        try:
-            recs.extend(q.qlora_kernel_timing_collect(nrec))
-        except q.QLoraError as e:  # keep the step timing; report no roofline
-            print(f"kernel timing unavailable: {e}", file=sys.stderr)
     barrier()
     clk = clocks.stop()
     launches = kernels_per_step * args.steps
     ms = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), device="cuda")
     del graph
+
+    nrec = 16 * len(layers)
+    q.qlora_kernel_timing_enable(nrec)
+    tgraph = capture()
+    tgraph.replay()  # warm-up; each replay re-records the same event pairs
+    torch.cuda.synchronize()
+    recs = []
+    for i in range(args.steps):
+        flush.zero_()
+        tgraph.replay()
+        torch.cuda.synchronize()
+        try:
+            recs.extend(q.qlora_kernel_timing_collect(nrec))
+        except q.QLoraError as e:  # keep the step timing; report no roofline
+            print(f"kernel timing unavailable: {e}", file=sys.stderr)
+    del tgraph
     q.qlora_kernel_timing_enable(0)
     for L in layers:
         assert q.qlora_workspace_status(L.ws_f) == 0 and q.qlora_workspace_status(L.ws_b) == 0
@@ -316,7 +332,7 @@ def run_gpu(args):
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ems / args.steps, 5)},
             "clocks": clk, "gpu_launches": int(launches), "kernels_per_step": int(kernels_per_step),
-            "timing": "device step captured once in a CUDA graph and replayed; CUDA events around each replay",
+            "timing": "device step captured once in a CUDA graph and replayed; CUDA events around each replay; per-kernel durations from a second pass with events around each tensor-core launch",
             "small_r": small, "quantize": quant,
         }
         print(json.dumps(line), flush=True)

@@ -211,6 +211,8 @@ __global__ void __launch_bounds__(kThreads) rowdot_kernel(const T* __restrict__ 
                                                           float* __restrict__ out,
                                                           uint16_t* __restrict__ out_pad,
                                                           int row_blocks, PadJob job) {
+  // the tensor-core kernel queued next may start its weight stream now
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if ((int)blockIdx.x >= row_blocks) {
     run_pad_job(job, (int64_t)blockIdx.x - row_blocks);
     return;
@@ -490,6 +492,8 @@ template <typename T, int RMAX>
 __global__ void __launch_bounds__(kThreads) rowdot_pipe_kernel(
     const T* __restrict__ P, int64_t R, int64_t K, const float* __restrict__ L, int r,
     float* __restrict__ out, uint16_t* __restrict__ out_pad, int row_blocks, PadJob job) {
+  // the tensor-core kernel queued next may start its weight stream now
+  if (threadIdx.x == 0) griddep_launch_dependents();
   if ((int)blockIdx.x >= row_blocks) {
     run_pad_job(job, (int64_t)blockIdx.x - row_blocks);
     return;
@@ -725,6 +729,368 @@ __global__ void __launch_bounds__(kColThreadsP) coldot_pipe_kernel(
   }
 }
 
+// ------------------------------------------------------ tensor-core path
+//
+// The same products on the tensor cores (mma.sync m16n8k16, bf16 operands,
+// fp32 accumulation).  The activation operand is exact in bf16.  The fp32
+// factor x is split into bf16 hi = bf16(x) and lo = bf16(x - hi) (x - hi is
+// exact in fp32) and both halves are multiplied: the factor keeps 16
+// significant bits (relative error <= 2^-16), against 24 in the FMA form.
+// That removes the r FMAs per activation element from the issue slots; the
+// kernels are then bound by HBM on the activation, not by instructions.
+
+constexpr int kMmaStages = 4;
+constexpr int kMaxTickets = 1024;  // zeroed counters the caller provides
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+// c += A (16 x 16, row) * B (16 x 8, col)
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// (x, y) -> bf16 pairs hi = (bf16(x), bf16(y)) and lo = bf16 of the remainders
+__device__ __forceinline__ void split_bf16(float x, float y, uint32_t& hi, uint32_t& lo) {
+  hi = pack_bf16x2(x, y);
+  lo = pack_bf16x2(x - __uint_as_float(hi << 16), y - __uint_as_float(hi & 0xFFFF0000u));
+}
+// B fragment pair of one n-tile from an fp32 factor tile, hi/lo halves
+// accumulated into c.  f(k, n) gives the factor entry (0 outside).
+template <typename F>
+__device__ __forceinline__ void mma_split(float (&c)[4], const uint32_t (&a)[4], int k0, int n,
+                                          F f) {
+  uint32_t h0, l0, h1, l1;
+  split_bf16(f(k0, n), f(k0 + 1, n), h0, l0);
+  split_bf16(f(k0 + 8, n), f(k0 + 9, n), h1, l1);
+  mma16816(c, a, h0, h1);
+  mma16816(c, a, l0, l1);
+}
+
+// rowdot on the tensor cores: out[m, j] = sum_k P[m, k] L(k, j).
+// Block = 8 warps = 4 row groups (16 rows each, 64 rows per block) x 2 K
+// groups (alternate 16-column chunks); a stage holds KT = 128 columns of
+// the 64 rows (rows padded by 16 bytes: conflict-free ldmatrix) and the
+// matching factor tile, as given: [r x KT] rows when L is [r x K] (A),
+// [KT x r] when L is [K x r] (B).  Grid = row blocks x K splits; with
+// several splits each writes a partial and the last block of a row block
+// to finish (ticket) adds them in split order.  The final values go out as
+// fp32 [R x r] and, optionally, bf16 zero-padded to 64 columns.
+template <int NT, bool LKR>
+struct RowMma {
+  static constexpr int RB = 64, KT = 128;
+  static constexpr int NP = 8 * NT;                    // padded rank
+  static constexpr int PSTR = KT * 2 + 16;             // bytes per P row in smem
+  static constexpr int PB = RB * PSTR;
+  static constexpr int LSTRF = KT + 8;                 // floats per L row ([r x K] case)
+  static constexpr int LB = LKR ? KT * NP * 4 : NP * LSTRF * 4;
+  static constexpr int STAGE = PB + LB;
+  static constexpr int TSTR = NP + 1;                  // result tile row stride (floats)
+  static constexpr int RED = 4 * 32 * NT * 4 * 4;      // K-group combine buffer
+  static constexpr int TILE = RB * TSTR * 4;
+  static constexpr int SMEM = kMmaStages * STAGE + (RED > TILE ? RED : TILE);
+};
+
+template <int NT, bool LKR>
+__global__ void __launch_bounds__(kThreads) rowdot_mma_kernel(
+    const __nv_bfloat16* __restrict__ P, int64_t R, int64_t K, const float* __restrict__ L,
+    int r, int row_blocks, int ksplit, int tiles_per_split, float* __restrict__ out,
+    uint16_t* __restrict__ out_pad, float* __restrict__ part, unsigned* __restrict__ tickets,
+    PadJob job) {
+  // the tensor-core kernel queued next may start its weight stream now
+  if (threadIdx.x == 0) griddep_launch_dependents();
+  if ((int)blockIdx.x >= row_blocks * ksplit) {
+    run_pad_job(job, (int64_t)blockIdx.x - row_blocks * ksplit);
+    return;
+  }
+  using C = RowMma<NT, LKR>;
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ int s_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rb = (int)blockIdx.x % row_blocks, ks = (int)blockIdx.x / row_blocks;
+  const int64_t m0 = (int64_t)rb * C::RB;
+  const int ntiles = (int)((K + C::KT - 1) / C::KT);
+  const int t_lo = ks * tiles_per_split, t_hi = min(ntiles, t_lo + tiles_per_split);
+
+  auto issue = [&](int t) {
+    const uint32_t ps = (uint32_t)__cvta_generic_to_shared(sm + ((t - t_lo) % kMmaStages) * C::STAGE);
+    const uint32_t ls = ps + C::PB;
+    const int64_t k0 = (int64_t)t * C::KT;
+    // P: 64 rows x 16 chunks of 16 bytes
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = threadIdx.x + kThreads * i, row = c >> 4, ch = c & 15;
+      const int64_t m = m0 + row, k = k0 + ch * 8;
+      const int64_t rem = (K - k) * 2;
+      const uint32_t nb = (m < R && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
+      cp_async16(ps + (uint32_t)(row * C::PSTR + ch * 16), nb ? (const void*)(P + m * K + k) : (const void*)P, nb);
+    }
+    if (LKR) {  // contiguous [KT x r] floats
+      const int64_t base = k0 * r, total = K * (int64_t)r;
+      const int nch = (C::KT * r) / 4;
+      for (int c = threadIdx.x; c < nch; c += kThreads) {
+        const int64_t e = base + (int64_t)c * 4;
+        const int64_t rem = (total - e) * 4;
+        const uint32_t nb = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
+        cp_async16(ls + (uint32_t)c * 16, nb ? (const void*)(L + e) : (const void*)L, nb);
+      }
+    } else {  // NP rows of KT floats, rows >= r zero
+      for (int c = threadIdx.x; c < C::NP * (C::KT / 4); c += kThreads) {
+        const int j = c / (C::KT / 4), ch = c % (C::KT / 4);
+        const int64_t k = k0 + ch * 4;
+        const int64_t rem = (K - k) * 4;
+        const uint32_t nb = (j < r && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
+        cp_async16(ls + (uint32_t)(j * C::LSTRF + ch * 4) * 4,
+                   nb ? (const void*)(L + (int64_t)j * K + k) : (const void*)L, nb);
+      }
+    }
+  };
+
+  const int rg = warp & 3, kg = warp >> 2;
+  const int g = lane >> 2, tq = lane & 3;
+  float c[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) c[n][0] = c[n][1] = c[n][2] = c[n][3] = 0.0f;
+
+#pragma unroll
+  for (int i = 0; i < kMmaStages - 1; ++i) {
+    if (t_lo + i < t_hi) issue(t_lo + i);
+    cp_async_commit();
+  }
+  for (int t = t_lo; t < t_hi; ++t) {
+    cp_async_wait<kMmaStages - 2>();
+    __syncthreads();
+    if (t + kMmaStages - 1 < t_hi) issue(t + kMmaStages - 1);
+    cp_async_commit();
+    const uint8_t* stage = sm + ((t - t_lo) % kMmaStages) * C::STAGE;
+    const uint32_t ps = (uint32_t)__cvta_generic_to_shared(stage);
+    const float* ls = (const float*)(stage + C::PB);
+#pragma unroll
+    for (int q = 0; q < C::KT / 32; ++q) {
+      const int kc = 2 * q + kg;  // 16-column chunk
+      uint32_t a[4];
+      ldsm_x4(ps + (uint32_t)((16 * rg + (lane & 15)) * C::PSTR + (kc * 16 + (lane >> 4) * 8) * 2), a);
+      const int kb = kc * 16 + 2 * tq;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        if (LKR)
+          mma_split(c[n], a, kb, 8 * n + g,
+                    [&](int k, int j) { return j < r ? ls[k * r + j] : 0.0f; });
+        else
+          mma_split(c[n], a, kb, 8 * n + g, [&](int k, int j) { return ls[j * C::LSTRF + k]; });
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  // combine the two K groups, then stage the 64 x NP result tile
+  float* red = (float*)(sm + kMmaStages * C::STAGE);
+  if (kg == 1) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) red[((rg * 32 + lane) * NT + n) * 4 + e] = c[n][e];
+  }
+  __syncthreads();
+  if (kg == 0) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) c[n][e] += red[((rg * 32 + lane) * NT + n) * 4 + e];
+  }
+  __syncthreads();
+  float* tile = red;  // [64][TSTR]
+  if (kg == 0) {
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int col = 8 * n + 2 * tq, row = 16 * rg + g;
+      tile[row * C::TSTR + col] = c[n][0];
+      tile[row * C::TSTR + col + 1] = c[n][1];
+      tile[(row + 8) * C::TSTR + col] = c[n][2];
+      tile[(row + 8) * C::TSTR + col + 1] = c[n][3];
+    }
+  }
+  __syncthreads();
+  if (ksplit > 1) {
+    for (int e = threadIdx.x; e < C::RB * C::NP; e += kThreads) {
+      const int row = e / C::NP, col = e % C::NP;
+      const int64_t m = m0 + row;
+      if (m < R) part[((int64_t)ks * R + m) * C::NP + col] = tile[row * C::TSTR + col];
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&tickets[rb], 1u) == (unsigned)(ksplit - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int e = threadIdx.x; e < C::RB * C::NP; e += kThreads) {
+      const int row = e / C::NP, col = e % C::NP;
+      const int64_t m = m0 + row;
+      float v = 0.0f;
+      if (m < R)
+        for (int q = 0; q < ksplit; ++q) v += __ldcg(part + ((int64_t)q * R + m) * C::NP + col);
+      tile[row * C::TSTR + col] = v;
+    }
+    if (threadIdx.x == 0) tickets[rb] = 0;  // ready for the next launch
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < C::RB * 64; e += kThreads) {
+    const int row = e >> 6, col = e & 63;
+    const int64_t m = m0 + row;
+    if (m >= R) continue;
+    const float v = col < r ? tile[row * C::TSTR + col] : 0.0f;
+    if (col < r) out[m * r + col] = v;
+    if (out_pad) out_pad[m * 64 + col] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  }
+}
+
+// coldot on the tensor cores: out(j, n) = s sum_m aux[m, j] P[m, n].
+// D[n, j] = sum_m P^T[n, m] aux[m, j]: the P tile [64 rows x 128 columns]
+// is read transposed by ldmatrix.trans.  Block = 8 warps x 16 columns;
+// grid = column blocks x row splits, the last block of a column block to
+// finish (ticket) adds the split partials in split order, scales by s and
+// writes dA as [r x N] (out_nr = 0) or dB as [N x r] (out_nr = 1).
+template <int NT>
+struct ColMma {
+  static constexpr int NC = 128, RT = 64;
+  static constexpr int NP = 8 * NT;
+  static constexpr int PSTR = NC * 2 + 16;
+  static constexpr int PB = RT * PSTR;
+  static constexpr int AB = RT * NP * 4;               // aux tile [RT x r] (stride r)
+  static constexpr int STAGE = PB + AB;
+  static constexpr int TSTR = NP + 1;
+  static constexpr int TILE = NC * TSTR * 4;
+  static constexpr int SMEM = kMmaStages * STAGE + TILE;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads) coldot_mma_kernel(
+    const __nv_bfloat16* __restrict__ P, int64_t R, int64_t N, const float* __restrict__ aux,
+    int r, int col_blocks, int splits, int tiles_per_split, float s, int out_nr,
+    float* __restrict__ out, float* __restrict__ part, unsigned* __restrict__ tickets) {
+  using C = ColMma<NT>;
+  extern __shared__ __align__(16) uint8_t sm[];
+  __shared__ int s_last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cb = (int)blockIdx.x, sp = (int)blockIdx.y;
+  const int64_t n0 = (int64_t)cb * C::NC;
+  const int ntiles = (int)((R + C::RT - 1) / C::RT);
+  const int t_lo = sp * tiles_per_split, t_hi = min(ntiles, t_lo + tiles_per_split);
+
+  auto issue = [&](int t) {
+    const uint32_t ps = (uint32_t)__cvta_generic_to_shared(sm + ((t - t_lo) % kMmaStages) * C::STAGE);
+    const uint32_t as = ps + C::PB;
+    const int64_t mt = (int64_t)t * C::RT;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {  // 64 rows x 16 chunks
+      const int c = threadIdx.x + kThreads * i, row = c >> 4, ch = c & 15;
+      const int64_t m = mt + row, n = n0 + ch * 8;
+      const int64_t rem = (N - n) * 2;
+      const uint32_t nb = (m < R && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
+      cp_async16(ps + (uint32_t)(row * C::PSTR + ch * 16), nb ? (const void*)(P + m * N + n) : (const void*)P, nb);
+    }
+    const int64_t base = mt * r, total = R * (int64_t)r;  // contiguous [RT x r]
+    const int nch = (C::RT * r) / 4;
+    for (int c = threadIdx.x; c < nch; c += kThreads) {
+      const int64_t e = base + (int64_t)c * 4;
+      const int64_t rem = (total - e) * 4;
+      const uint32_t nb = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
+      cp_async16(as + (uint32_t)c * 16, nb ? (const void*)(aux + e) : (const void*)aux, nb);
+    }
+  };
+
+  const int g = lane >> 2, tq = lane & 3;
+  float c[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) c[n][0] = c[n][1] = c[n][2] = c[n][3] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kMmaStages - 1; ++i) {
+    if (t_lo + i < t_hi) issue(t_lo + i);
+    cp_async_commit();
+  }
+  // ldmatrix.trans source rows: matrix q = lane / 8 covers columns
+  // 8 (q & 1) .. +7 and rows 8 (q >> 1) .. +7 of the 16 x 16 block
+  const int lrow = (lane & 7) + 8 * (lane >> 4), lcol = 16 * warp + 8 * ((lane >> 3) & 1);
+  for (int t = t_lo; t < t_hi; ++t) {
+    cp_async_wait<kMmaStages - 2>();
+    __syncthreads();
+    if (t + kMmaStages - 1 < t_hi) issue(t + kMmaStages - 1);
+    cp_async_commit();
+    const uint8_t* stage = sm + ((t - t_lo) % kMmaStages) * C::STAGE;
+    const uint32_t ps = (uint32_t)__cvta_generic_to_shared(stage);
+    const float* as = (const float*)(stage + C::PB);
+#pragma unroll
+    for (int kc = 0; kc < C::RT / 16; ++kc) {
+      uint32_t a[4];
+      ldsm_x4_t(ps + (uint32_t)((kc * 16 + lrow) * C::PSTR + lcol * 2), a);
+      const int kb = kc * 16 + 2 * tq;
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+        mma_split(c[n], a, kb, 8 * n + g,
+                  [&](int k, int j) { return j < r ? as[k * r + j] : 0.0f; });
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+  float* tile = (float*)(sm + kMmaStages * C::STAGE);  // [NC][TSTR]: D[n][j]
+#pragma unroll
+  for (int n = 0; n < NT; ++n) {
+    const int col = 8 * n + 2 * tq, row = 16 * warp + g;
+    tile[row * C::TSTR + col] = c[n][0];
+    tile[row * C::TSTR + col + 1] = c[n][1];
+    tile[(row + 8) * C::TSTR + col] = c[n][2];
+    tile[(row + 8) * C::TSTR + col + 1] = c[n][3];
+  }
+  __syncthreads();
+  if (splits > 1) {
+    for (int e = threadIdx.x; e < C::NC * C::NP; e += kThreads) {
+      const int row = e / C::NP, col = e % C::NP;
+      const int64_t n = n0 + row;
+      if (n < N) part[((int64_t)sp * N + n) * C::NP + col] = tile[row * C::TSTR + col];
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&tickets[cb], 1u) == (unsigned)(splits - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int e = threadIdx.x; e < C::NC * C::NP; e += kThreads) {
+      const int row = e / C::NP, col = e % C::NP;
+      const int64_t n = n0 + row;
+      float v = 0.0f;
+      if (n < N)
+        for (int q = 0; q < splits; ++q) v += __ldcg(part + ((int64_t)q * N + n) * C::NP + col);
+      tile[row * C::TSTR + col] = v;
+    }
+    if (threadIdx.x == 0) tickets[cb] = 0;  // ready for the next launch
+    __syncthreads();
+  }
+  if (out_nr) {  // dB [N x r]: consecutive threads along j then n
+    for (int e = threadIdx.x; e < C::NC * r; e += kThreads) {
+      const int row = e / r, j = e % r;
+      const int64_t n = n0 + row;
+      if (n < N) out[n * r + j] = s * tile[row * C::TSTR + j];
+    }
+  } else {  // dA [r x N]: consecutive threads along n
+    for (int e = threadIdx.x; e < C::NC * r; e += kThreads) {
+      const int j = e / C::NC, row = e % C::NC;
+      const int64_t n = n0 + row;
+      if (n < N) out[(int64_t)j * N + n] = s * tile[row * C::TSTR + j];
+    }
+  }
+}
+
 // out = s * sum over slices of part[slice][j][n].  Block = 8 warps over 32
 // consecutive outputs e (= j * N + n): warp w sums slices w, w+8, ... for
 // lane-th output (coalesced across lanes), then the 8 warp sums are added in
@@ -891,14 +1257,103 @@ void coldot_r(const void* P, int64_t R, int64_t N, const float* aux, int r, cons
   else coldot_launch<T, 64>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
 }
 
+struct MmaPlan {
+  int blocks;          // row blocks (rowdot) or column blocks (coldot)
+  int splits;          // K splits (rowdot) or row splits (coldot)
+  int tiles_per_split;
+};
+
+// ~two waves of 256-thread blocks; a split only where the blocks alone
+// leave SMs idle, and only with ticket counters to spare.
+MmaPlan mma_plan(int64_t blocks, int64_t ntiles, bool can_split) {
+  MmaPlan pl;
+  pl.blocks = (int)blocks;
+  int64_t splits = 1;
+  if (can_split && blocks > 0 && blocks <= kMaxTickets && blocks < sm_count()) {
+    splits = (2 * (int64_t)sm_count()) / blocks;
+    if (splits > ntiles) splits = ntiles;
+    if (splits < 1) splits = 1;
+  }
+  pl.tiles_per_split = (int)((ntiles + splits - 1) / splits);
+  if (pl.tiles_per_split < 1) pl.tiles_per_split = 1;
+  pl.splits = (int)((ntiles + pl.tiles_per_split - 1) / pl.tiles_per_split);
+  if (pl.splits < 1) pl.splits = 1;
+  return pl;
+}
+
+int rank_tiles(int r) { return r <= 8 ? 1 : r <= 16 ? 2 : r <= 32 ? 4 : 8; }
+
+MmaPlan rowdot_mma_plan(int64_t R, int64_t K, bool can_split) {
+  return mma_plan(cdiv(R, 64), cdiv(K, 128), can_split);
+}
+MmaPlan coldot_mma_plan(int64_t R, int64_t N, bool can_split) {
+  return mma_plan(cdiv(N, 128), cdiv(R, 64), can_split);
+}
+
+bool rowdot_mma_ok(const void* P, bool bf16, int64_t K, const float* L) {
+  return bf16 && (K % 8) == 0 && ((uintptr_t)P % 16) == 0 && ((uintptr_t)L % 16) == 0;
+}
+
+template <int NT, bool LKR>
+cudaError_t rowdot_mma_go(const __nv_bfloat16* P, int64_t R, int64_t K, const float* L, int r,
+                          const MmaPlan& pl, float* out, uint16_t* pad, float* part,
+                          unsigned* tickets, PadJob job, cudaStream_t st) {
+  using C = RowMma<NT, LKR>;
+  static bool attr = false;
+  auto kern = rowdot_mma_kernel<NT, LKR>;
+  cudaError_t e = set_smem_once(kern, C::SMEM, attr);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)(pl.blocks * pl.splits + job.blocks);
+  if (grid == 0) return cudaSuccess;
+  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, K, L, r, pl.blocks, pl.splits, pl.tiles_per_split,
+                                        out, pad, part, tickets, job);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <bool LKR>
+cudaError_t rowdot_mma_r(const __nv_bfloat16* P, int64_t R, int64_t K, const float* L, int r,
+                         const MmaPlan& pl, float* out, uint16_t* pad, float* part,
+                         unsigned* tickets, PadJob job, cudaStream_t st) {
+  switch (rank_tiles(r)) {
+    case 1: return rowdot_mma_go<1, LKR>(P, R, K, L, r, pl, out, pad, part, tickets, job, st);
+    case 2: return rowdot_mma_go<2, LKR>(P, R, K, L, r, pl, out, pad, part, tickets, job, st);
+    case 4: return rowdot_mma_go<4, LKR>(P, R, K, L, r, pl, out, pad, part, tickets, job, st);
+    default: return rowdot_mma_go<8, LKR>(P, R, K, L, r, pl, out, pad, part, tickets, job, st);
+  }
+}
+
+template <int NT>
+cudaError_t coldot_mma_go(const __nv_bfloat16* P, int64_t R, int64_t N, const float* aux, int r,
+                          const MmaPlan& pl, float s, bool out_nr, float* out, float* part,
+                          unsigned* tickets, cudaStream_t st) {
+  using C = ColMma<NT>;
+  static bool attr = false;
+  auto kern = coldot_mma_kernel<NT>;
+  cudaError_t e = set_smem_once(kern, C::SMEM, attr);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)pl.blocks, (unsigned)pl.splits);
+  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, N, aux, r, pl.blocks, pl.splits, pl.tiles_per_split,
+                                        s, out_nr ? 1 : 0, out, part, tickets);
+  count_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const float* L,
                           bool l_is_kr, int32_t r, float* out, cudaStream_t st, uint16_t* pad,
                           const float* side_src, int64_t side_extent, int side_mode,
-                          float side_mul, uint16_t* side_dst, float* lt_ws) {
+                          float side_mul, uint16_t* side_dst, float* lt_ws, float* part_ws,
+                          unsigned* tickets) {
   PadJob job{side_src, side_dst, side_extent, r, side_mode, side_mul, 0};
   if (side_dst && side_extent > 0) job.blocks = (int)cdiv(64 * side_extent, kThreads * 8);
+  if (R > 0 && rowdot_mma_ok(P, bf16, K, L)) {  // tensor cores, either factor layout
+    const MmaPlan pl = rowdot_mma_plan(R, K, part_ws != nullptr && tickets != nullptr);
+    const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
+    if (l_is_kr) return rowdot_mma_r<true>(Pb, R, K, L, r, pl, out, pad, part_ws, tickets, job, st);
+    return rowdot_mma_r<false>(Pb, R, K, L, r, pl, out, pad, part_ws, tickets, job, st);
+  }
   // With scratch for it, a factor given as [K x r] is transposed first so
   // every path below reads factor rows ([r x K]) contiguously.
   const float* Lr = L;
@@ -967,6 +1422,11 @@ cudaError_t coldot_pipe_go(const __nv_bfloat16* P, int64_t R, int64_t N, const f
 
 }  // namespace
 
+size_t rowdot_ws(int64_t R, int64_t K, int32_t r) {
+  const MmaPlan pl = rowdot_mma_plan(R, K, true);
+  return pl.splits > 1 ? align_up((size_t)pl.splits * (size_t)R * 8 * rank_tiles(r) * 4, 256) : 0;
+}
+
 // Workspace: the larger of the pipelined path (slice sums) and the
 // streaming path (tickets + slice sums).
 size_t coldot_ws(int64_t R, int64_t N, int32_t r) {
@@ -976,14 +1436,29 @@ size_t coldot_ws(int64_t R, int64_t N, int32_t r) {
                                  align_up((size_t)c.splits * (size_t)r * (size_t)N * 4, 256);
   const PipePlan pp = pipe_plan(R, N);
   size_t b = align_up((size_t)pp.splits * (size_t)r * (size_t)N * 4, 256);
+  const MmaPlan mp = coldot_mma_plan(R, N, true);
+  const size_t cm =
+      mp.splits > 1 ? align_up((size_t)mp.splits * (size_t)N * 8 * rank_tiles(r) * 4, 256) : 0;
+  if (cm > b) b = cm;
   return a > b ? a : b;
 }
 
 cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
                           int32_t r, float s, bool out_nr, float* out, void* ws,
-                          cudaStream_t st) {
+                          cudaStream_t st, unsigned* tickets) {
   if (N == 0) return cudaSuccess;
   if (R == 0) return cudaMemsetAsync(out, 0, (size_t)r * (size_t)N * 4, st);
+  if (coldot_pipe_ok(P, bf16, R, N, aux)) {  // tensor cores
+    const MmaPlan pl = coldot_mma_plan(R, N, tickets != nullptr);
+    const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
+    float* part = (float*)ws;
+    switch (rank_tiles(r)) {
+      case 1: return coldot_mma_go<1>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
+      case 2: return coldot_mma_go<2>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
+      case 4: return coldot_mma_go<4>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
+      default: return coldot_mma_go<8>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
+    }
+  }
   if (coldot_pipe_ok(P, bf16, R, N, aux)) {
     const PipePlan c = pipe_plan(R, N);
     float* part = (float*)ws;
@@ -1001,16 +1476,16 @@ cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const 
     return cudaGetLastError();
   }
   const ColPlan c = col_plan(R, N, r);
-  unsigned* tickets = (unsigned*)ws;
+  unsigned* slice_tickets = (unsigned*)ws;
   float* part = (float*)((char*)ws + align_up((size_t)c.colblocks * 4, 256));
   if (c.splits > 1) {
-    cudaError_t e = cudaMemsetAsync(tickets, 0, (size_t)c.colblocks * 4, st);
+    cudaError_t e = cudaMemsetAsync(slice_tickets, 0, (size_t)c.colblocks * 4, st);
     if (e != cudaSuccess) return e;
   }
   if (bf16)
-    coldot_r<__nv_bfloat16>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
+    coldot_r<__nv_bfloat16>(P, R, N, aux, r, c, s, out_nr, part, slice_tickets, out, st);
   else
-    coldot_r<float>(P, R, N, aux, r, c, s, out_nr, part, tickets, out, st);
+    coldot_r<float>(P, R, N, aux, r, c, s, out_nr, part, slice_tickets, out, st);
   count_launch();
   return cudaGetLastError();
 }

@@ -51,6 +51,11 @@ int timing_begin(cudaStream_t st, int kind, double flops) {
   return (int)g_trecs.size() - 1;
 }
 
+bool timing_enabled() {
+  std::lock_guard<std::mutex> lk(g_tmu);
+  return g_tmax > 0;
+}
+
 void timing_end(int slot, cudaStream_t st) {
   if (slot < 0) return;
   std::lock_guard<std::mutex> lk(g_tmu);
@@ -131,8 +136,12 @@ WView view_of(const qlora_weight* w) {
 
 // ---------------------------------------------------------------- layouts
 
+// Every layout starts with the status header and the ticket counters, both
+// zeroed by one memset at the start of the call.
+constexpr size_t kWsZeroed = kWsHeader + kWsTickets;
+
 struct FwdLayout {
-  size_t u = 0, tc = 0, total = 0;
+  size_t u = 0, red = 0, tc = 0, total = 0;
 };
 struct BwdLayout {
   size_t u = 0, v = 0, bt = 0, red = 0, tc = 0, total = 0;
@@ -140,9 +149,11 @@ struct BwdLayout {
 
 FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t compute) {
   FwdLayout L;
-  size_t off = kWsHeader;
+  size_t off = kWsZeroed;
   L.u = off;
   off += align_up((size_t)R * r * 4, 256);
+  L.red = off;  // split partials of U = X A^T
+  off += rowdot_ws(R, w->I, r);
   L.tc = off;
   if (compute == QLORA_COMPUTE_BF16) off += tc_fwd_ws(view_of(w), R);
   L.total = off;
@@ -151,7 +162,7 @@ FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
 
 BwdLayout bwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t compute) {
   BwdLayout L;
-  size_t off = kWsHeader;
+  size_t off = kWsZeroed;
   L.u = off;
   off += align_up((size_t)R * r * 4, 256);
   L.v = off;
@@ -159,9 +170,12 @@ BwdLayout bwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
   L.bt = off;  // B^T [r x O] for the pipelined V = dY B
   off += align_up((size_t)r * w->O * 4, 256);
   L.red = off;
+  // partials of the four side products, used one after another
   size_t red = coldot_ws(R, w->I, r);
-  size_t red2 = coldot_ws(R, w->O, r);
-  off += red > red2 ? red : red2;
+  const size_t more[3] = {coldot_ws(R, w->O, r), rowdot_ws(R, w->O, r), rowdot_ws(R, w->I, r)};
+  for (size_t m : more)
+    if (m > red) red = m;
+  off += red;
   L.tc = off;
   if (compute == QLORA_COMPUTE_BF16) off += tc_dx_ws(view_of(w), R);
   L.total = off;
@@ -300,9 +314,11 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
   st = device_ready();
   if (st != QLORA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader, s);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kWsZeroed, s);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
   if (R == 0) return QLORA_OK;
+  unsigned* tickets = (unsigned*)((char*)ws + kWsHeader);
+  float* red = (float*)((char*)ws + L.red);
   const float sc = alpha / (float)r;
   float* U = U_out ? U_out : (float*)((char*)ws + L.u);
   const WView v = view_of(w);
@@ -310,7 +326,7 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
   if (bf16 && tc_fwd_supported(v, X, Y, R)) {
     void* tcws = (char*)ws + L.tc;
     e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws), B, w->O, 0, sc,
-                      tc_w_pad(tcws, R));
+                      tc_w_pad(tcws, R), nullptr, red, tickets);
     if (e == cudaSuccess) e = launch_tc_fwd(v, X, R, U, B, r, sc, Y, tcws, (uint32_t*)ws, s);
   } else {
     e = launch_simt_fwd(v, X, R, A, B, r, sc, bf16, Y, U, s);
@@ -331,8 +347,9 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   st = device_ready();
   if (st != QLORA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader, s);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kWsZeroed, s);
   if (e != cudaSuccess) return QLORA_ERR_CUDA;
+  unsigned* tickets = (unsigned*)((char*)ws + kWsHeader);
   const bool bf16 = compute == QLORA_COMPUTE_BF16;
   const float sc = alpha / (float)r;
   const WView v = view_of(w);
@@ -343,12 +360,14 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   const bool tc = dX && bf16 && tc_dx_supported(v, dY, dX, R);
   void* tcws = (char*)ws + L.tc;
   if (dX || dA) {
+    float* bt = (float*)((char*)ws + L.bt);
+    float* part = (float*)red;
     if (tc)
       e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, tc_act_pad(tcws), A, w->I, 1, sc,
-                        tc_w_pad(tcws, R), (float*)((char*)ws + L.bt));
+                        tc_w_pad(tcws, R), bt, part, tickets);
     else
       e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, nullptr, nullptr, 0, 0, 1.0f,
-                        nullptr, (float*)((char*)ws + L.bt));
+                        nullptr, bt, part, tickets);
   }
   if (e == cudaSuccess && dX) {
     if (tc)
@@ -357,16 +376,19 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
       e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s);
   }
   // dA = s V^T X   [r x I]
-  if (e == cudaSuccess && dA) e = launch_coldot(X, bf16, R, w->I, V, r, sc, false, dA, red, s);
+  if (e == cudaSuccess && dA)
+    e = launch_coldot(X, bf16, R, w->I, V, r, sc, false, dA, red, s, tickets);
   // dB = s dY^T U  [O x r]
   if (e == cudaSuccess && dB) {
     const float* U = U_in;
     if (!U) {
       float* Uw = (float*)((char*)ws + L.u);
-      e = launch_rowdot(X, bf16, R, w->I, A, false, r, Uw, s);
+      e = launch_rowdot(X, bf16, R, w->I, A, false, r, Uw, s, nullptr, nullptr, 0, 0, 1.0f,
+                        nullptr, nullptr, (float*)red, tickets);
       U = Uw;
     }
-    if (e == cudaSuccess) e = launch_coldot(dY, bf16, R, w->O, U, r, sc, true, dB, red, s);
+    if (e == cudaSuccess)
+      e = launch_coldot(dY, bf16, R, w->O, U, r, sc, true, dB, red, s, tickets);
   }
   return cuda_status(e);
 }

@@ -18,6 +18,11 @@ inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_o
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Zeroed ticket counters after the workspace status header (1024 x u32):
+// zeroed with the header at the start of every linear call; kernels that
+// take one leave it zero again.
+constexpr size_t kWsTickets = 4096;
+
 // Bounded-wait limit for device spin loops, nanoseconds.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -49,18 +54,27 @@ cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const 
                           bool l_is_kr, int32_t r, float* out, cudaStream_t st,
                           uint16_t* pad = nullptr, const float* side_src = nullptr,
                           int64_t side_extent = 0, int side_mode = 0, float side_mul = 1.0f,
-                          uint16_t* side_dst = nullptr, float* lt_ws = nullptr);
+                          uint16_t* side_dst = nullptr, float* lt_ws = nullptr,
+                          float* part_ws = nullptr, unsigned* tickets = nullptr);
+// part_ws (rowdot_ws bytes) and tickets (kWsTickets bytes, zero on entry
+// and left zero) let the bf16 tensor-core path split K across blocks.
+size_t rowdot_ws(int64_t R, int64_t K, int32_t r);
 size_t coldot_ws(int64_t R, int64_t N, int32_t r);
+// tickets: as for launch_rowdot (nullptr: no row splits on the tensor-core path)
 cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
                           int32_t r, float s, bool out_nr, float* out, void* ws,
-                          cudaStream_t st);
+                          cudaStream_t st, unsigned* tickets = nullptr);
 // bf16 operand staging for the tensor-core path
 cudaError_t launch_pad_rows_bf16(const float* src, int64_t rows, int32_t r, float mul,
                                  uint16_t* dst, cudaStream_t st);
 cudaError_t launch_pad_cols_bf16(const float* src, int32_t r, int64_t cols, float mul,
                                  uint16_t* dst, cudaStream_t st);
+// out = scale * sum of the split partials.  pdl: launched with a
+// programmatic dependency on the kernel before it (which must have
+// triggered its dependents); the kernel waits for that grid first.
 cudaError_t launch_splitk_reduce(const float* part, int32_t splits, int64_t R, int64_t N,
-                                 bool bf16_out, void* out, cudaStream_t st, float scale = 1.0f);
+                                 bool bf16_out, void* out, cudaStream_t st, float scale = 1.0f,
+                                 bool pdl = false);
 
 // selftest
 cudaError_t launch_wait_selftest(uint32_t* ws_header, uint64_t limit_ns, cudaStream_t st);
@@ -68,5 +82,7 @@ cudaError_t launch_wait_selftest(uint32_t* ws_header, uint64_t limit_ns, cudaStr
 // kernel timing instrumentation (api.cu): returns a slot to record into, or -1
 int timing_begin(cudaStream_t st, int kind, double flops);
 void timing_end(int slot, cudaStream_t st);
+// true while kernel timing is switched on (launches then keep plain stream order)
+bool timing_enabled();
 
 }  // namespace qlora

@@ -117,11 +117,29 @@ __global__ void pad_cols_bf16_kernel(const float* __restrict__ src, int32_t r, i
 template <typename TO>
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int32_t splits, int64_t MN,
                                      float scale, TO* __restrict__ out) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= MN) return;
-  float acc = 0.0f;
-  for (int sidx = 0; sidx < splits; ++sidx) acc += part[(int64_t)sidx * MN + e];
-  out[e] = from_f32<TO>(scale * acc);
+  griddep_wait();  // the partials come from the launch just before
+  const int64_t e4 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (e4 >= MN) return;
+  if ((MN & 3) == 0) {
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int sidx = 0; sidx < splits; ++sidx) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(part + (int64_t)sidx * MN + e4));
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    out[e4] = from_f32<TO>(scale * acc.x);
+    out[e4 + 1] = from_f32<TO>(scale * acc.y);
+    out[e4 + 2] = from_f32<TO>(scale * acc.z);
+    out[e4 + 3] = from_f32<TO>(scale * acc.w);
+    return;
+  }
+  for (int64_t e = e4; e < e4 + 4 && e < MN; ++e) {
+    float acc = 0.0f;
+    for (int sidx = 0; sidx < splits; ++sidx) acc += part[(int64_t)sidx * MN + e];
+    out[e] = from_f32<TO>(scale * acc);
+  }
 }
 
 inline unsigned cdiv(int64_t a, int64_t b) { return (unsigned)((a + b - 1) / b); }
@@ -177,16 +195,26 @@ cudaError_t launch_pad_cols_bf16(const float* src, int32_t r, int64_t cols, floa
 }
 
 cudaError_t launch_splitk_reduce(const float* part, int32_t splits, int64_t R, int64_t N,
-                                 bool bf16_out, void* out, cudaStream_t st, float scale) {
+                                 bool bf16_out, void* out, cudaStream_t st, float scale, bool pdl) {
   const int64_t MN = R * N;
   if (MN == 0) return cudaSuccess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cdiv(MN, 1024));
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  cudaError_t e;
   if (bf16_out)
-    splitk_reduce_kernel<__nv_bfloat16><<<cdiv(MN, 256), 256, 0, st>>>(part, splits, MN, scale,
-                                                                        (__nv_bfloat16*)out);
+    e = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<__nv_bfloat16>, part, splits, MN, scale,
+                           (__nv_bfloat16*)out);
   else
-    splitk_reduce_kernel<float><<<cdiv(MN, 256), 256, 0, st>>>(part, splits, MN, scale, (float*)out);
+    e = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel<float>, part, splits, MN, scale, (float*)out);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace qlora

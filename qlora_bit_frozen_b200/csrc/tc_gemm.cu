@@ -67,6 +67,41 @@ struct TcParams {
   uint64_t wait_ns;
 };
 
+constexpr int pow2_at_least(int x) {
+  int p = 32;
+  while (p < x) p *= 2;
+  return p;
+}
+
+// Shared-memory and TMEM plan of one instantiation.
+//   in ring  : NIN stages of {token tile [BN x 64] bf16, packed tile 4 KB},
+//              filled by TMA, released by the MMA that consumed them
+//   dec ring : NDEC decoded weight tiles, bf16 [128 x 64]; in TMEM (forward:
+//              the MMA reads A from TMEM) or in shared memory (input
+//              gradient: A is read MN-major through a descriptor)
+//   adw      : the adapter step's A operand (16 KB, loaded once)
+// Tiles of up to 128 tokens stay under half the SM's shared memory and TMEM
+// so that two CTAs share an SM.
+template <bool DX, int BN>
+struct Cfg {
+  static constexpr int kAct = BN * kBK * 2;
+  static constexpr int NIN = DX ? (BN >= 256 ? 4 : BN >= 128 ? 3 : BN >= 64 ? 5 : BN >= 32 ? 6 : 8)
+                                : (BN >= 256 ? 5 : BN >= 128 ? 4 : BN >= 64 ? 6 : BN >= 32 ? 8 : 12);
+  static constexpr int NDEC = DX ? (BN >= 256 ? 3 : 2) : (BN >= 128 ? 4 : 6);
+  static constexpr int kAccCols = BN < 32 ? 32 : BN;
+  static constexpr int kTmemCols = pow2_at_least(DX ? kAccCols : kAccCols + NDEC * 32);
+  static constexpr int kWdec = DX ? NDEC * kWTile : 0;
+  static constexpr int kRing = NIN * (kAct + kPkTile) + kWdec;  // also the epilogue staging
+  static constexpr int kBars = 8 * (2 * NIN + 2 * NDEC + 1) + 16;
+  static constexpr int kSmem = 1024 + kRing + kWTile + kBars;
+  static constexpr int kMinCtas = BN >= 256 ? 1 : 2;
+  static_assert(kMinCtas == 1 || (kSmem <= 113 * 1024 && 2 * kTmemCols <= 512),
+                "two CTAs per SM must fit");
+  static_assert(kMinCtas == 2 || (kSmem <= 227 * 1024 && kTmemCols <= 512), "one CTA must fit");
+  // more than 76 KB keeps a third CTA (and a third TMEM allocation) off the SM
+  static_assert(kSmem > 76 * 1024, "at most two CTAs per SM");
+};
+
 // UMMA shared-memory descriptor, 128-byte swizzle (sm_100 version field).
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
@@ -83,12 +118,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn) {
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
-template <int BN>
-struct Smem {
-  static constexpr int kAct = BN * kBK * 2;
-  static constexpr int kStage = kWTile + kAct + kPkTile;
-};
-
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
                                              uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
@@ -96,10 +125,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-// Decode one 64-weight NF4 block (packed bytes 0..15 at pk_lo, 16..31 at
-// pk_hi) with block scale s
-// into one 128-byte swizzled row at row_addr (row index within its 8-row
-// atom = sw).
+// Decoding one 64-weight NF4 block with block scale s.
 //
 // The 16 possible outputs bf16(fp32(c[k] * s)) are formed once per block
 // and kept in registers as two byte planes (low and high byte of each bf16,
@@ -107,35 +133,72 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // with byte permutes: one permute per plane and per half of the table
 // (nibble bits 0..2), one to pick the half (nibble bit 3) and two to
 // interleave the planes back into bf16 pairs.  No shared-memory lookups.
-__device__ __forceinline__ void decode_row(const uint8_t* pk_lo, const uint8_t* pk_hi, float s,
-                                           uint32_t row_addr, uint32_t sw) {
+struct Nf4Planes {
+  uint32_t L0, L1, L2, L3, H0, H1, H2, H3;
+};
+
+__device__ __forceinline__ Nf4Planes nf4_planes(float s) {
   uint32_t P[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j)
     P[j] = pack_bf16x2(__fmul_rn(kNF4[2 * j], s), __fmul_rn(kNF4[2 * j + 1], s));
-  // byte planes: L[q] / H[q] hold the low / high bytes of entries 4q .. 4q+3
-  const uint32_t L0 = __byte_perm(P[0], P[1], 0x6420), H0 = __byte_perm(P[0], P[1], 0x7531);
-  const uint32_t L1 = __byte_perm(P[2], P[3], 0x6420), H1 = __byte_perm(P[2], P[3], 0x7531);
-  const uint32_t L2 = __byte_perm(P[4], P[5], 0x6420), H2 = __byte_perm(P[4], P[5], 0x7531);
-  const uint32_t L3 = __byte_perm(P[6], P[7], 0x6420), H3 = __byte_perm(P[6], P[7], 0x7531);
+  Nf4Planes t;
+  t.L0 = __byte_perm(P[0], P[1], 0x6420); t.H0 = __byte_perm(P[0], P[1], 0x7531);
+  t.L1 = __byte_perm(P[2], P[3], 0x6420); t.H1 = __byte_perm(P[2], P[3], 0x7531);
+  t.L2 = __byte_perm(P[4], P[5], 0x6420); t.H2 = __byte_perm(P[4], P[5], 0x7531);
+  t.L3 = __byte_perm(P[6], P[7], 0x6420); t.H3 = __byte_perm(P[6], P[7], 0x7531);
+  return t;
+}
+
+// 8 nibbles (weights 8j .. 8j+7, low nibble first) -> 4 bf16 pairs
+// o[q] = (weight 2q, weight 2q+1) of the 8, low half first.
+__device__ __forceinline__ void nf4_word(const Nf4Planes& t, uint32_t w, uint32_t (&o)[4]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint32_t x = h ? (w >> 16) : w;  // 4 nibbles in the low 16 bits
+    const uint32_t s7 = x & 0x7777u;
+    const uint32_t alo = __byte_perm(t.L0, t.L1, s7), blo = __byte_perm(t.L2, t.L3, s7);
+    const uint32_t ahi = __byte_perm(t.H0, t.H1, s7), bhi = __byte_perm(t.H2, t.H3, s7);
+    const uint32_t sb = ((x >> 1) & 0x4444u) | 0x3210u;  // bit 3 -> second half
+    const uint32_t lo = __byte_perm(alo, blo, sb), hi = __byte_perm(ahi, bhi, sb);
+    o[2 * h] = __byte_perm(lo, hi, 0x5140);
+    o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
+  }
+}
+
+// Block (packed bytes 0..15 at pk_lo, 16..31 at pk_hi) -> one 128-byte
+// swizzled shared-memory row at row_addr (row index within its 8-row atom
+// = sw).
+__device__ __forceinline__ void decode_row_smem(const uint8_t* pk_lo, const uint8_t* pk_hi, float s,
+                                                uint32_t row_addr, uint32_t sw) {
+  const Nf4Planes t = nf4_planes(s);
   const uint4 p0 = *reinterpret_cast<const uint4*>(pk_lo);
   const uint4 p1 = *reinterpret_cast<const uint4*>(pk_hi);
   const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {  // word j = weights 8j .. 8j+7 (nibble i = weight 8j+i)
+  for (int j = 0; j < 8; ++j) {
     uint32_t o[4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t x = h ? (w[j] >> 16) : w[j];  // 4 nibbles in the low 16 bits
-      const uint32_t s7 = x & 0x7777u;
-      const uint32_t alo = __byte_perm(L0, L1, s7), blo = __byte_perm(L2, L3, s7);
-      const uint32_t ahi = __byte_perm(H0, H1, s7), bhi = __byte_perm(H2, H3, s7);
-      const uint32_t sb = ((x >> 1) & 0x4444u) | 0x3210u;  // bit 3 -> second half
-      const uint32_t lo = __byte_perm(alo, blo, sb), hi = __byte_perm(ahi, bhi, sb);
-      o[2 * h] = __byte_perm(lo, hi, 0x5140);
-      o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
-    }
+    nf4_word(t, w[j], o);
     st_shared_v4(row_addr + ((j ^ sw) << 4), o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Block -> 32 registers, v[c] = (weight 2c, weight 2c+1): one TMEM row of
+// the A operand (32 columns of two bf16 each).
+__device__ __forceinline__ void decode_row_regs(const uint8_t* pk_lo, const uint8_t* pk_hi, float s,
+                                                uint32_t (&v)[32]) {
+  const Nf4Planes t = nf4_planes(s);
+  const uint4 p0 = *reinterpret_cast<const uint4*>(pk_lo);
+  const uint4 p1 = *reinterpret_cast<const uint4*>(pk_hi);
+  const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t o[4];
+    nf4_word(t, w[j], o);
+    v[4 * j] = o[0];
+    v[4 * j + 1] = o[1];
+    v[4 * j + 2] = o[2];
+    v[4 * j + 3] = o[3];
   }
 }
 
@@ -185,39 +248,37 @@ __device__ __forceinline__ void epilogue_stage(uint32_t tmem, int quad, int lane
   }
 }
 
+// Columns of the token tile each decoder group stores in the epilogue.
 template <int BN>
-constexpr int stages_for() {
-  return BN >= 256 ? 4 : (BN >= 64 ? 3 : 4);
-}
-// CTAs per SM the kernel is built for (tiles up to 128 tokens leave room
-// in shared memory, TMEM and registers for two).
-template <int BN>
-constexpr int min_ctas() {
-  return BN >= 256 ? 1 : 2;
+constexpr int cols_per_group() {
+  return BN >= 64 ? BN / kDecGroups : BN;
 }
 
-template <bool DX, int BN, int STAGES>
-__global__ void __launch_bounds__(kThreads, min_ctas<BN>())
+template <bool DX, int BN>
+__global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_pk,
                       const __grid_constant__ CUtensorMap tm_aact,
                       const __grid_constant__ CUtensorMap tm_aw,
                       const __grid_constant__ CUtensorMap tm_out, const TcParams p) {
-  using L = Smem<BN>;
-  constexpr uint32_t kTmemCols = BN < 32 ? 32 : BN;
+  using C = Cfg<DX, BN>;
+  constexpr int NIN = C::NIN, NDEC = C::NDEC;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, BN, DX);
+  static_assert((BN >= 64 ? 2 : 1) * 2 * cols_per_group<BN>() * 64 * 4 <= C::kRing,
+                "epilogue staging must fit in the ring buffers");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* wdec = smem;                               // STAGES x 16 KB
-  uint8_t* act = wdec + STAGES * kWTile;              // STAGES x BN*128
-  uint8_t* pk = act + STAGES * L::kAct;               // STAGES x 4 KB
-  uint64_t* bars = (uint64_t*)(pk + STAGES * kPkTile);
-  uint64_t* full_act = bars;
-  uint64_t* full_pk = bars + STAGES;
-  uint64_t* dec = bars + 2 * STAGES;
-  uint64_t* empty = bars + 3 * STAGES;
-  uint64_t* acc_full = bars + 4 * STAGES;
+  uint8_t* act = smem;                        // NIN x BN*128
+  uint8_t* pk = act + NIN * C::kAct;          // NIN x 4 KB
+  uint8_t* wdec = pk + NIN * kPkTile;         // input gradient: NDEC x 16 KB
+  uint8_t* adw = wdec + C::kWdec;             // 16 KB
+  uint64_t* bars = (uint64_t*)(adw + kWTile);
+  uint64_t* full_in = bars;                   // TMA landed (token + packed tile)
+  uint64_t* in_empty = bars + NIN;            // MMA done with the in-ring stage
+  uint64_t* dec_full = bars + 2 * NIN;        // decoded tile written (4 warps)
+  uint64_t* dec_empty = bars + 2 * NIN + NDEC;  // MMA done with the decoded tile
+  uint64_t* acc_full = bars + 2 * NIN + 2 * NDEC;
   volatile uint32_t* tmem_slot = (volatile uint32_t*)(acc_full + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -227,22 +288,27 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
   const int split = blockIdx.z;
   const int kb_lo = split * p.kb_per_split;
   const int kb_hi = min(p.KB, kb_lo + p.kb_per_split);
-  const int has_ad = split == 0 ? 1 : 0;  // adapter step rides with split 0
-  const int T = (kb_hi - kb_lo) + has_ad;
+  const int nk = kb_hi - kb_lo;               // weight K steps of this CTA
+  const int T = nk + (split == 0 ? 1 : 0);    // + the adapter step, last, in split 0
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(&full_act[s]), 1);
-      mbar_init(smem_u32(&full_pk[s]), 1);
-      mbar_init(smem_u32(&dec[s]), 4);  // the 4 warps of one decoder group
-      mbar_init(smem_u32(&empty[s]), 1);
+    // A kernel queued behind this one with a programmatic dependency (the
+    // split-K reduction) may start now; it waits for this grid itself.
+    griddep_launch_dependents();
+    for (int s = 0; s < NIN; ++s) {
+      mbar_init(smem_u32(&full_in[s]), 1);
+      mbar_init(smem_u32(&in_empty[s]), 1);
+    }
+    for (int d = 0; d < NDEC; ++d) {
+      mbar_init(smem_u32(&dec_full[d]), 4);  // the 4 warps of one decoder group
+      mbar_init(smem_u32(&dec_empty[d]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32((const void*)tmem_slot), kTmemCols);
+    tmem_alloc(smem_u32((const void*)tmem_slot), C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -255,41 +321,40 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
     if (lane == 0) {
       int issued = 0;
       for (int it = 0; it < T; ++it) {
-        const int s = it % STAGES;
+        const int s = it % NIN;
         if (*abort_flag) break;
-        if (!mbar_wait(smem_u32(&empty[s]), ((it / STAGES) & 1) ^ 1, p.wait_ns, p.err, 0x101)) {
+        if (!mbar_wait(smem_u32(&in_empty[s]), ((it / NIN) & 1) ^ 1, p.wait_ns, p.err, 0x101)) {
           *abort_flag = 1;
           break;
         }
-        const uint32_t fa = smem_u32(&full_act[s]), fp = smem_u32(&full_pk[s]);
-        if (has_ad && it == 0) {
-          mbar_arrive_expect_tx(fa, L::kAct + kWTile);
-          tma_load_2d(smem_u32(act + s * L::kAct), &tm_aact, fa, 0, (int32_t)n0);
-          if (!DX) {
-            tma_load_2d(smem_u32(wdec + s * kWTile), &tm_aw, fa, 0, m0);
-          } else {
-            tma_load_2d(smem_u32(wdec + s * kWTile), &tm_aw, fa, m0, 0);
-            tma_load_2d(smem_u32(wdec + s * kWTile + kWTile / 2), &tm_aw, fa, m0 + 64, 0);
-          }
-          mbar_arrive(fp);  // no packed data in the adapter step
-        } else {
-          const int kb = kb_lo + it - has_ad;
-          mbar_arrive_expect_tx(fa, L::kAct);
-          tma_load_2d(smem_u32(act + s * L::kAct), &tm_act, fa, kb * kBK, (int32_t)n0);
-          mbar_arrive_expect_tx(fp, kPkTile);
+        const uint32_t fb = smem_u32(&full_in[s]);
+        const uint32_t a_dst = smem_u32(act + s * C::kAct);
+        if (it < nk) {
+          const int kb = kb_lo + it;
+          mbar_arrive_expect_tx(fb, C::kAct + kPkTile);
+          tma_load_2d(a_dst, &tm_act, fb, kb * kBK, (int32_t)n0);
           if (!DX)
-            tma_load_2d(smem_u32(pk + s * kPkTile), &tm_pk, fp, kb * (kBK / 2), m0);
+            tma_load_2d(smem_u32(pk + s * kPkTile), &tm_pk, fb, kb * (kBK / 2), m0);
           else
-            tma_load_2d(smem_u32(pk + s * kPkTile), &tm_pk, fp, m0 / 2, kb * kBK);
+            tma_load_2d(smem_u32(pk + s * kPkTile), &tm_pk, fb, m0 / 2, kb * kBK);
+        } else {
+          // Adapter step: U / V and the scaled factor come from the launch
+          // just before this one, which may still be running.
+          griddep_wait();
+          mbar_arrive_expect_tx(fb, C::kAct + kWTile);
+          tma_load_2d(a_dst, &tm_aact, fb, 0, (int32_t)n0);
+          if (!DX) {
+            tma_load_2d(smem_u32(adw), &tm_aw, fb, 0, m0);
+          } else {
+            tma_load_2d(smem_u32(adw), &tm_aw, fb, m0, 0);
+            tma_load_2d(smem_u32(adw + kWTile / 2), &tm_aw, fb, m0 + 64, 0);
+          }
         }
         issued = it + 1;
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
-        for (int it = issued - STAGES < 0 ? 0 : issued - STAGES; it < issued; ++it) {
-          const int s = it % STAGES;
-          mbar_wait(smem_u32(&full_act[s]), (it / STAGES) & 1, p.wait_ns, nullptr, 0);
-          mbar_wait(smem_u32(&full_pk[s]), (it / STAGES) & 1, p.wait_ns, nullptr, 0);
-        }
+        for (int it = issued - NIN < 0 ? 0 : issued - NIN; it < issued; ++it)
+          mbar_wait(smem_u32(&full_in[it % NIN]), (it / NIN) & 1, p.wait_ns, nullptr, 0);
       }
     }
     __syncwarp();
@@ -297,24 +362,41 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       for (int it = 0; it < T; ++it) {
-        const int s = it % STAGES;
+        const int s = it % NIN;
         if (*abort_flag) break;
-        const uint32_t par = (it / STAGES) & 1;
-        if (!mbar_wait(smem_u32(&full_act[s]), par, p.wait_ns, p.err, 0x201) ||
-            !mbar_wait(smem_u32(&dec[s]), par, p.wait_ns, p.err, 0x202)) {
+        if (!mbar_wait(smem_u32(&full_in[s]), (it / NIN) & 1, p.wait_ns, p.err, 0x201)) {
           *abort_flag = 1;
           break;
         }
-        tc_fence_after();
-        const uint32_t a0 = smem_u32(wdec + s * kWTile);
-        const uint32_t b0 = smem_u32(act + s * L::kAct);
-        const int nsl = (has_ad && it == 0) ? p.r_slices : kBK / 16;
-        for (int kk = 0; kk < nsl; ++kk) {
-          const uint64_t ad = DX ? sdesc(a0 + kk * 2048, 8192, 1024) : sdesc(a0 + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc(b0 + kk * 32, 16, 1024);
-          umma_bf16(tmem, ad, bd, kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+        const uint32_t b0 = smem_u32(act + s * C::kAct);
+        if (it < nk) {
+          const int d = it % NDEC;
+          if (!mbar_wait(smem_u32(&dec_full[d]), (it / NDEC) & 1, p.wait_ns, p.err, 0x202)) {
+            *abort_flag = 1;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t bd = sdesc(b0 + kk * 32, 16, 1024);
+            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+            if (!DX)
+              umma_bf16_ta(tmem, tmem + (uint32_t)(C::kAccCols + d * 32 + kk * 8), bd, kIdesc, acc);
+            else
+              umma_bf16(tmem, sdesc(smem_u32(wdec + d * kWTile) + kk * 2048, 8192, 1024), bd,
+                        kIdesc, acc);
+          }
+          umma_commit(smem_u32(&in_empty[s]));
+          umma_commit(smem_u32(&dec_empty[d]));
+        } else {
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(adw);
+          for (int kk = 0; kk < p.r_slices; ++kk) {
+            const uint64_t ad = DX ? sdesc(a0 + kk * 2048, 8192, 1024) : sdesc(a0 + kk * 32, 16, 1024);
+            umma_bf16(tmem, ad, sdesc(b0 + kk * 32, 16, 1024), kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(&in_empty[s]));
         }
-        umma_commit(smem_u32(&empty[s]));
       }
       umma_commit(smem_u32(acc_full));
     }
@@ -322,21 +404,26 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
   } else {
     // ------------------------------------------------------------ decoders
     // Two groups of 4 warps; group g decodes the steps it = g, g+2, ...
+    // Forward: the thread decodes weight row 32*(warp%4) + lane, its own
+    // TMEM lane, and stores the block's 32 bf16 pairs with one tcgen05.st.
+    // Input gradient: unit u writes one swizzled 128-byte row of the
+    // MN-major shared-memory tile (64 weights of W row kb*64 + u%64).
     const int group = (warp - 2) >> 2;
-    const int u = threadIdx.x - 64 - 128 * group;  // unit 0..127 within the group
+    const int quad = warp & 3;
+    const int u = DX ? (int)threadIdx.x - 64 - 128 * group : 32 * quad + lane;
     const float mu = __ldg(p.mu);
     const uint32_t bpr = (uint32_t)(p.I / kBK);  // blocks per W row
-    // unit -> NF4 block index for step kb
     auto block_of = [&](int kb) -> uint32_t {
       if (!DX) return (uint32_t)(m0 + u) * bpr + (uint32_t)kb;
       return (uint32_t)(kb * kBK + (u & 63)) * bpr + (uint32_t)(m0 / kBK) + (uint32_t)(u >> 6);
     };
-    const uint32_t row_off = DX ? (uint32_t)((u >> 6) * (kWTile / 2) + (u & 63) * 128) : (uint32_t)u * 128;
+    const uint32_t row_off = (uint32_t)((u >> 6) * (kWTile / 2) + (u & 63) * 128);
     const uint32_t sw = (uint32_t)(u & 7);
     // Packed tile as TMA wrote it: forward 128 rows x 32 B with the 32-byte
-    // swizzle (16-byte half c of row y at c ^ bit 2 of y), dX 64 rows x 64 B
-    // with the 64-byte swizzle (chunk c of row y at c ^ bits 1..2 of y).
-    // Eight consecutive lanes then hit eight different bank groups.
+    // swizzle (16-byte half c of row y at c ^ bit 2 of y), input gradient
+    // 64 rows x 64 B with the 64-byte swizzle (chunk c of row y at
+    // c ^ bits 1..2 of y).  Eight consecutive lanes then hit eight
+    // different bank groups.
     uint32_t pk_lo, pk_hi;
     if (!DX) {
       const uint32_t x = (uint32_t)(u >> 2) & 1u;
@@ -347,49 +434,48 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
       pk_lo = o * 64 + (((2 * h) ^ x) << 4);
       pk_hi = o * 64 + (((2 * h + 1) ^ x) << 4);
     }
-    auto kb_of = [&](int it) { return kb_lo + it - has_ad; };
+    const uint32_t tm_row = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)C::kAccCols;
     int it = group;
     uint32_t q_next = 0;
     float t_next = 0.0f;
-    if (it < T && !(has_ad && it == 0)) {
-      const uint32_t b = block_of(kb_of(it));
-      q_next = __ldg(p.qcodes + b);
-      t_next = __ldg(p.t + b / p.C);
-    } else if (it + kDecGroups < T) {
-      const uint32_t b = block_of(kb_of(it + kDecGroups));
+    if (it < nk) {
+      const uint32_t b = block_of(kb_lo + it);
       q_next = __ldg(p.qcodes + b);
       t_next = __ldg(p.t + b / p.C);
     }
     bool ok = true;
-    for (; it < T; it += kDecGroups) {
-      const int s = it % STAGES;
-      const uint32_t par = (it / STAGES) & 1;
-      const bool adapter = has_ad && it == 0;
-      float sc = 0.0f;
-      if (!adapter) {
-        sc = decode_block_scale(q_next, t_next, mu);
-        if (it + kDecGroups < T) {  // prefetch the scale inputs of this group's next step
-          const uint32_t b = block_of(kb_of(it + kDecGroups));
-          q_next = __ldg(p.qcodes + b);
-          t_next = __ldg(p.t + b / p.C);
-        }
+    for (; it < nk; it += kDecGroups) {
+      const int s = it % NIN, d = it % NDEC;
+      const float sc = decode_block_scale(q_next, t_next, mu);
+      if (it + kDecGroups < nk) {  // prefetch the scale inputs of this group's next step
+        const uint32_t b = block_of(kb_lo + it + kDecGroups);
+        q_next = __ldg(p.qcodes + b);
+        t_next = __ldg(p.t + b / p.C);
       }
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-      bool w_ok = mbar_wait(smem_u32(&empty[s]), par ^ 1, p.wait_ns, p.err, 0x301) &&
-                  mbar_wait(smem_u32(&full_pk[s]), par, p.wait_ns, p.err, 0x302);
+      bool w_ok = mbar_wait(smem_u32(&dec_empty[d]), ((it / NDEC) & 1) ^ 1, p.wait_ns, p.err, 0x301) &&
+                  mbar_wait(smem_u32(&full_in[s]), (it / NIN) & 1, p.wait_ns, p.err, 0x302);
       if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
-      if (!adapter)
-        decode_row(pk + s * kPkTile + pk_lo, pk + s * kPkTile + pk_hi, sc,
-                   smem_u32(wdec + s * kWTile) + row_off, sw);
-      fence_proxy_async_smem();
+      const uint8_t* src = pk + s * kPkTile;
+      if (!DX) {
+        tc_fence_after();
+        uint32_t v[32];
+        decode_row_regs(src + pk_lo, src + pk_hi, sc, v);
+        tmem_st_32x32b_x32(tm_row + (uint32_t)(d * 32), v);
+        tmem_st_wait();
+        tc_fence_before();
+      } else {
+        decode_row_smem(src + pk_lo, src + pk_hi, sc, smem_u32(wdec + d * kWTile) + row_off, sw);
+        fence_proxy_async_smem();
+      }
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&dec[s]));
+      if (lane == 0) mbar_arrive(smem_u32(&dec_full[d]));
     }
     // the accumulator is complete once acc_full fires
     const bool acc_ok = mbar_wait(smem_u32(acc_full), 0, p.wait_ns, p.err, 0x401);
     if (!ok || !acc_ok) *abort_flag = 1;
   }
-  // All roles are past the main loop: the stage buffers are free and the
+  // All roles are past the main loop: the ring buffers are free and the
   // abort flag is final (and the same for every thread after this barrier).
   tc_fence_before();
   __syncthreads();
@@ -398,10 +484,10 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
     // ---------------------------------------------------------- epilogue
     // Warp w reads TMEM lanes 32*(w%4) .. +31; the two decoder groups split
     // the token columns (group 0 alone when the tile is narrower than 64).
-    // Each group stages its columns in the freed stage buffers and one
+    // Each group stages its columns in the freed ring buffers and one
     // thread writes them with two TMA stores (weight-side rows 0..63, 64..127).
     const int group = (warp - 2) >> 2;
-    constexpr int kColsPerGroup = BN >= 64 ? BN / kDecGroups : BN;
+    constexpr int kColsPerGroup = cols_per_group<BN>();
     const int c_begin = BN >= 64 ? group * kColsPerGroup : 0;
     const int c_end = BN >= 64 ? c_begin + kColsPerGroup : (group == 0 ? BN : 0);
     if (c_end > c_begin) {
@@ -425,8 +511,11 @@ __global__ void __launch_bounds__(kThreads, min_ctas<BN>())
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
+  // The grid counts as finished only after the launch it depends on has:
+  // whatever runs next in the stream sees that launch's writes too.
+  if (threadIdx.x == 0) griddep_wait();
 }
 
 // ------------------------------------------------------------------ host
@@ -491,41 +580,39 @@ int num_sms_cached() {
   return n;
 }
 
-template <int BN>
-constexpr size_t smem_bytes() {
-  return 1024 + (size_t)stages_for<BN>() * Smem<BN>::kStage + 5 * 8 * stages_for<BN>() + 8 + 16 +
-         64 + 64;
-}
-
-// Columns of the token tile each decoder group stores, and the staging
-// bytes that takes (worst case fp32); it must fit in the stage buffers.
-template <int BN>
-constexpr int cols_per_group() {
-  return BN >= 64 ? BN / kDecGroups : BN;
-}
-
+// The launch waits for the kernel before it in the stream only where the
+// adapter step needs that kernel's output (programmatic dependent launch):
+// the weight stream starts while U / V are still being computed.
 template <bool DX, int BN>
 cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                       const CUtensorMap& d, const CUtensorMap& o, const TcParams& p,
                       cudaStream_t st) {
-  constexpr int S = stages_for<BN>();
-  static_assert((BN >= 64 ? 2 : 1) * 2 * cols_per_group<BN>() * 64 * 4 <= S * (kWTile + Smem<BN>::kAct),
-                "epilogue staging must fit in the stage buffers");
-  auto kern = tc_qlinear_kernel<DX, BN, S>;
-  const size_t sm = smem_bytes<BN>();
+  using Cf = Cfg<DX, BN>;
+  auto kern = tc_qlinear_kernel<DX, BN>;
   static bool attr_set = false;  // once per instantiation (keeps graph capture free of it)
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   const double flops = 2.0 * (double)p.R * (double)p.Mw * (double)p.KB * kBK +
                        2.0 * (double)p.R * (double)p.Mw * (double)p.rank;
   const int slot = timing_begin(st, DX ? 1 : 0, flops);
-  kern<<<grid, kThreads, sm, st>>>(a, b, c, d, o, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)Cf::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // a timing event between the two launches would separate them anyway
+  cfg.attrs = attr;
+  cfg.numAttrs = slot < 0 ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, b, c, d, o, p);
   timing_end(slot, st);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <bool DX>
@@ -566,18 +653,23 @@ TcPlan tc_plan(int64_t Mw, int64_t KB, int64_t R) {
   const int sms = num_sms_cached();
   const int64_t mt = Mw / kBM;
   // Token tile: the smallest power of two >= R (16..256); at large R, halve
-  // it (down to 64) while the grid is below one wave, rather than split K.
+  // it (down to 64) while the grid fills less than 3/4 of a wave, rather
+  // than split K (a 256-token tile reads half the weight bytes per flop of
+  // a 128-token one and wins down to ~0.85 of a wave).
   int bn = 16;
   while (bn < 256 && bn < R) bn *= 2;
-  while (bn > 64 && mt * ((R + bn - 1) / bn) < sms) bn /= 2;
+  while (bn > 64 && 4 * mt * ((R + bn - 1) / bn) < 3 * (int64_t)sms) bn /= 2;
   pl.bn = bn;
   pl.stages = 0;
   const int64_t tiles = mt * ((R + bn - 1) / bn);
+  // Below one wave of tiles, split K so that the grid is one full wave
+  // (two CTAs per SM up to 128-token tiles), at least 4 K steps per split.
   int64_t splits = 1;
   if (tiles > 0 && tiles < sms) {
-    splits = (2 * sms + tiles - 1) / tiles;
+    splits = ((bn >= 256 ? 1 : 2) * (int64_t)sms) / tiles;
     const int64_t max_splits = KB / 4 > 0 ? KB / 4 : 1;
     if (splits > max_splits) splits = max_splits;
+    if (splits < 1) splits = 1;
   }
   pl.kb_per_split = (int)((KB + splits - 1) / splits);
   pl.splits = (int)((KB + pl.kb_per_split - 1) / pl.kb_per_split);
@@ -649,7 +741,7 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   dim3 grid((unsigned)(O / kBM), (unsigned)((R + pl.bn - 1) / pl.bn), (unsigned)pl.splits);
   e = launch_plan<false>(pl, grid, m_act, m_pk, m_aact, m_aw, m_out, p, st);
   if (e != cudaSuccess || pl.splits == 1) return e;
-  return launch_splitk_reduce(part, pl.splits, R, O, true, Y, st);
+  return launch_splitk_reduce(part, pl.splits, R, O, true, Y, st, 1.0f, !timing_enabled());
 }
 
 cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float* V,
@@ -695,7 +787,7 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   dim3 grid((unsigned)(I / kBM), (unsigned)((R + pl.bn - 1) / pl.bn), (unsigned)pl.splits);
   e = launch_plan<true>(pl, grid, m_act, m_pk, m_aact, m_aw, m_out, p, st);
   if (e != cudaSuccess || pl.splits == 1) return e;
-  return launch_splitk_reduce(part, pl.splits, R, I, true, dX, st);
+  return launch_splitk_reduce(part, pl.splits, R, I, true, dX, st, 1.0f, !timing_enabled());
 }
 
 // Failure-detection self test: one thread waits on an mbarrier that nothing
