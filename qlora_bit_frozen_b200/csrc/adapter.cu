@@ -778,6 +778,48 @@ __device__ __forceinline__ void mma_split(float (&c)[4], const uint32_t (&a)[4],
   mma16816(c, a, l0, l1);
 }
 
+// dst[row * tstr + col] = sum over q < nsplit (in q order) of
+// part[q * slice + (row0 + row) * NP + col] for rows < nrows, the whole
+// block cooperating: four consecutive columns per thread and eight slices
+// in flight, so the last block's reduction is not a chain of dependent
+// L2 loads.  part was written by other blocks of this grid: read via L2.
+template <int NP>
+__device__ __forceinline__ void sum_slices(const float* __restrict__ part, int64_t slice,
+                                           int64_t row0, int nrows, int rows, int nsplit,
+                                           float* dst, int tstr) {
+  for (int e4 = threadIdx.x; e4 < rows * (NP / 4); e4 += kThreads) {
+    const int row = e4 / (NP / 4), col = (e4 % (NP / 4)) * 4;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (row < nrows) {
+      const float* p = part + (row0 + row) * NP + col;
+      int q = 0;
+      for (; q + 8 <= nsplit; q += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldcg(reinterpret_cast<const float4*>(p + (q + u) * slice));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          acc.x += v[u].x;
+          acc.y += v[u].y;
+          acc.z += v[u].z;
+          acc.w += v[u].w;
+        }
+      }
+      for (; q < nsplit; ++q) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(p + q * slice));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+    }
+    dst[row * tstr + col] = acc.x;
+    dst[row * tstr + col + 1] = acc.y;
+    dst[row * tstr + col + 2] = acc.z;
+    dst[row * tstr + col + 3] = acc.w;
+  }
+}
+
 // rowdot on the tensor cores: out[m, j] = sum_k P[m, k] L(k, j).
 // Block = 8 warps = 4 row groups (16 rows each, 64 rows per block) x 2 K
 // groups (alternate 16-column chunks); a stage holds KT = 128 columns of
@@ -934,14 +976,8 @@ __global__ void __launch_bounds__(kThreads) rowdot_mma_kernel(
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int e = threadIdx.x; e < C::RB * C::NP; e += kThreads) {
-      const int row = e / C::NP, col = e % C::NP;
-      const int64_t m = m0 + row;
-      float v = 0.0f;
-      if (m < R)
-        for (int q = 0; q < ksplit; ++q) v += __ldcg(part + ((int64_t)q * R + m) * C::NP + col);
-      tile[row * C::TSTR + col] = v;
-    }
+    sum_slices<C::NP>(part, R * C::NP, m0, (int)min((int64_t)C::RB, R - m0), C::RB, ksplit, tile,
+                      C::TSTR);
     if (threadIdx.x == 0) tickets[rb] = 0;  // ready for the next launch
     __syncthreads();
   }
@@ -1065,14 +1101,8 @@ __global__ void __launch_bounds__(kThreads) coldot_mma_kernel(
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int e = threadIdx.x; e < C::NC * C::NP; e += kThreads) {
-      const int row = e / C::NP, col = e % C::NP;
-      const int64_t n = n0 + row;
-      float v = 0.0f;
-      if (n < N)
-        for (int q = 0; q < splits; ++q) v += __ldcg(part + ((int64_t)q * N + n) * C::NP + col);
-      tile[row * C::TSTR + col] = v;
-    }
+    sum_slices<C::NP>(part, N * C::NP, n0, (int)min((int64_t)C::NC, N - n0), C::NC, splits, tile,
+                      C::TSTR);
     if (threadIdx.x == 0) tickets[cb] = 0;  // ready for the next launch
     __syncthreads();
   }

@@ -67,6 +67,9 @@ struct TcParams {
   uint64_t wait_ns;
 };
 
+// K steps per TMA load of the token and packed tiles (see Cfg::G).
+constexpr int tma_group(int bn) { return bn <= 16 ? 4 : bn <= 32 ? 2 : 1; }
+
 constexpr int pow2_at_least(int x) {
   int p = 32;
   while (p < x) p *= 2;
@@ -82,18 +85,26 @@ constexpr int pow2_at_least(int x) {
 //   adw      : the adapter step's A operand (16 KB, loaded once)
 // Tiles of up to 128 tokens stay under half the SM's shared memory and TMEM
 // so that two CTAs share an SM.
+//   G        : K steps per TMA load (small token tiles: one load of the
+//              token and packed tiles covers G ring slots, so the single
+//              producer thread issues a few large copies, not many small ones)
+//   adx      : with G > 1, the adapter step's token tile (U / V), outside
+//              the ring
 template <bool DX, int BN>
 struct Cfg {
   static constexpr int kAct = BN * kBK * 2;
+  static constexpr int G = tma_group(BN);
   static constexpr int NIN = DX ? (BN >= 256 ? 4 : BN >= 128 ? 3 : BN >= 64 ? 5 : BN >= 32 ? 6 : 8)
                                 : (BN >= 256 ? 5 : BN >= 128 ? 4 : BN >= 64 ? 6 : BN >= 32 ? 8 : 12);
+  static_assert(NIN % G == 0, "a TMA group fills whole ring slots");
   static constexpr int NDEC = DX ? (BN >= 256 ? 3 : 2) : (BN >= 128 ? 4 : 6);
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr int kTmemCols = pow2_at_least(DX ? kAccCols : kAccCols + NDEC * 32);
   static constexpr int kWdec = DX ? NDEC * kWTile : 0;
   static constexpr int kRing = NIN * (kAct + kPkTile) + kWdec;  // also the epilogue staging
-  static constexpr int kBars = 8 * (2 * NIN + 2 * NDEC + 1) + 16;
-  static constexpr int kSmem = 1024 + kRing + kWTile + kBars;
+  static constexpr int kAdx = G > 1 ? (kAct + 1023) / 1024 * 1024 : 0;
+  static constexpr int kBars = 8 * (2 * NIN + 2 * NDEC + 2) + 16;
+  static constexpr int kSmem = 1024 + kRing + kWTile + kAdx + kBars;
   static constexpr int kMinCtas = BN >= 256 ? 1 : 2;
   static_assert(kMinCtas == 1 || (kSmem <= 113 * 1024 && 2 * kTmemCols <= 512),
                 "two CTAs per SM must fit");
@@ -152,14 +163,17 @@ __device__ __forceinline__ Nf4Planes nf4_planes(float s) {
 
 // 8 nibbles (weights 8j .. 8j+7, low nibble first) -> 4 bf16 pairs
 // o[q] = (weight 2q, weight 2q+1) of the 8, low half first.
+// A byte permute reads only the low 16 bits of its selector, so the
+// selectors of both 4-nibble halves come from one pass over the word.
 __device__ __forceinline__ void nf4_word(const Nf4Planes& t, uint32_t w, uint32_t (&o)[4]) {
+  const uint32_t s7w = w & 0x77777777u;                            // table index, nibble bits 0..2
+  const uint32_t sbw = ((w >> 1) & 0x44444444u) | 0x32103210u;     // bit 3 -> second half
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint32_t x = h ? (w >> 16) : w;  // 4 nibbles in the low 16 bits
-    const uint32_t s7 = x & 0x7777u;
+    const uint32_t s7 = h ? (s7w >> 16) : s7w;
+    const uint32_t sb = h ? (sbw >> 16) : sbw;
     const uint32_t alo = __byte_perm(t.L0, t.L1, s7), blo = __byte_perm(t.L2, t.L3, s7);
     const uint32_t ahi = __byte_perm(t.H0, t.H1, s7), bhi = __byte_perm(t.H2, t.H3, s7);
-    const uint32_t sb = ((x >> 1) & 0x4444u) | 0x3210u;  // bit 3 -> second half
     const uint32_t lo = __byte_perm(alo, blo, sb), hi = __byte_perm(ahi, bhi, sb);
     o[2 * h] = __byte_perm(lo, hi, 0x5140);
     o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
@@ -273,13 +287,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
   uint8_t* pk = act + NIN * C::kAct;          // NIN x 4 KB
   uint8_t* wdec = pk + NIN * kPkTile;         // input gradient: NDEC x 16 KB
   uint8_t* adw = wdec + C::kWdec;             // 16 KB
-  uint64_t* bars = (uint64_t*)(adw + kWTile);
-  uint64_t* full_in = bars;                   // TMA landed (token + packed tile)
+  uint8_t* adx = adw + kWTile;                // G > 1: adapter token tile
+  uint64_t* bars = (uint64_t*)(adx + C::kAdx);
+  uint64_t* full_in = bars;                   // TMA landed (on the group's first slot)
   uint64_t* in_empty = bars + NIN;            // MMA done with the in-ring stage
   uint64_t* dec_full = bars + 2 * NIN;        // decoded tile written (4 warps)
   uint64_t* dec_empty = bars + 2 * NIN + NDEC;  // MMA done with the decoded tile
   uint64_t* acc_full = bars + 2 * NIN + 2 * NDEC;
-  volatile uint32_t* tmem_slot = (volatile uint32_t*)(acc_full + 1);
+  uint64_t* ad_full = acc_full + 1;           // G > 1: adapter operands landed
+  volatile uint32_t* tmem_slot = (volatile uint32_t*)(ad_full + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -304,8 +320,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       mbar_init(smem_u32(&dec_empty[d]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
+    mbar_init(smem_u32(ad_full), 1);
     *abort_flag = 0;
     fence_mbar_init();
+    prefetch_tensormap(&tm_act);
+    prefetch_tensormap(&tm_pk);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32((const void*)tmem_slot), C::kTmemCols);
@@ -319,27 +338,43 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued = 0;
-      for (int it = 0; it < T; ++it) {
-        const int s = it % NIN;
+      constexpr int G = C::G;
+      int issued = 0;  // K steps whose copies were issued
+      bool ad_issued = false;
+      for (int it0 = 0; it0 < nk; it0 += G) {
+        const int s0 = it0 % NIN, sl = s0 + G - 1, itl = it0 + G - 1;  // group = slots s0 .. sl
         if (*abort_flag) break;
-        if (!mbar_wait(smem_u32(&in_empty[s]), ((it / NIN) & 1) ^ 1, p.wait_ns, p.err, 0x101)) {
+        if (!mbar_wait(smem_u32(&in_empty[sl]), ((itl / NIN) & 1) ^ 1, p.wait_ns, p.err, 0x101)) {
           *abort_flag = 1;
           break;
         }
-        const uint32_t fb = smem_u32(&full_in[s]);
-        const uint32_t a_dst = smem_u32(act + s * C::kAct);
-        if (it < nk) {
-          const int kb = kb_lo + it;
-          mbar_arrive_expect_tx(fb, C::kAct + kPkTile);
-          tma_load_2d(a_dst, &tm_act, fb, kb * kBK, (int32_t)n0);
-          if (!DX)
-            tma_load_2d(smem_u32(pk + s * kPkTile), &tm_pk, fb, kb * (kBK / 2), m0);
-          else
-            tma_load_2d(smem_u32(pk + s * kPkTile), &tm_pk, fb, m0 / 2, kb * kBK);
+        const uint32_t fb = smem_u32(&full_in[s0]);
+        const int kb = kb_lo + it0;
+        mbar_arrive_expect_tx(fb, G * (C::kAct + kPkTile));
+        tma_load_3d(smem_u32(act + s0 * C::kAct), &tm_act, fb, 0, (int32_t)n0, kb);
+        if (!DX)
+          tma_load_3d(smem_u32(pk + s0 * kPkTile), &tm_pk, fb, 0, m0, kb);
+        else
+          tma_load_3d(smem_u32(pk + s0 * kPkTile), &tm_pk, fb, m0 / 2, 0, kb);
+        issued = it0 + G;
+      }
+      if (split == 0 && !*abort_flag) {
+        // Adapter step: U / V and the scaled factor come from the launch
+        // just before this one, which may still be running.
+        uint32_t fb, a_dst;
+        bool ok = true;
+        if (G > 1) {
+          fb = smem_u32(ad_full);
+          a_dst = smem_u32(adx);
         } else {
-          // Adapter step: U / V and the scaled factor come from the launch
-          // just before this one, which may still be running.
+          const int s = nk % NIN;
+          ok = mbar_wait(smem_u32(&in_empty[s]), ((nk / NIN) & 1) ^ 1, p.wait_ns, p.err, 0x102);
+          fb = smem_u32(&full_in[s]);
+          a_dst = smem_u32(act + s * C::kAct);
+        }
+        if (!ok) {
+          *abort_flag = 1;
+        } else {
           griddep_wait();
           mbar_arrive_expect_tx(fb, C::kAct + kWTile);
           tma_load_2d(a_dst, &tm_aact, fb, 0, (int32_t)n0);
@@ -349,12 +384,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
             tma_load_2d(smem_u32(adw), &tm_aw, fb, m0, 0);
             tma_load_2d(smem_u32(adw + kWTile / 2), &tm_aw, fb, m0 + 64, 0);
           }
+          if (G > 1) ad_issued = true;
+          else issued = nk + 1;
         }
-        issued = it + 1;
       }
       if (*abort_flag) {  // let copies in flight land before the CTA exits
-        for (int it = issued - NIN < 0 ? 0 : issued - NIN; it < issued; ++it)
+        const int first = issued - NIN < 0 ? 0 : issued - NIN;
+        for (int it = first - first % G; it < issued; it += G)
           mbar_wait(smem_u32(&full_in[it % NIN]), (it / NIN) & 1, p.wait_ns, nullptr, 0);
+        if (ad_issued) mbar_wait(smem_u32(ad_full), 0, p.wait_ns, nullptr, 0);
       }
     }
     __syncwarp();
@@ -364,11 +402,13 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       for (int it = 0; it < T; ++it) {
         const int s = it % NIN;
         if (*abort_flag) break;
-        if (!mbar_wait(smem_u32(&full_in[s]), (it / NIN) & 1, p.wait_ns, p.err, 0x201)) {
+        const bool ad_sep = C::G > 1 && it == nk;  // adapter step outside the ring
+        const uint32_t fb = ad_sep ? smem_u32(ad_full) : smem_u32(&full_in[s - s % C::G]);
+        if (!mbar_wait(fb, ad_sep ? 0u : (uint32_t)((it / NIN) & 1), p.wait_ns, p.err, 0x201)) {
           *abort_flag = 1;
           break;
         }
-        const uint32_t b0 = smem_u32(act + s * C::kAct);
+        const uint32_t b0 = ad_sep ? smem_u32(adx) : smem_u32(act + s * C::kAct);
         if (it < nk) {
           const int d = it % NDEC;
           if (!mbar_wait(smem_u32(&dec_full[d]), (it / NDEC) & 1, p.wait_ns, p.err, 0x202)) {
@@ -395,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
             const uint64_t ad = DX ? sdesc(a0 + kk * 2048, 8192, 1024) : sdesc(a0 + kk * 32, 16, 1024);
             umma_bf16(tmem, ad, sdesc(b0 + kk * 32, 16, 1024), kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
           }
-          umma_commit(smem_u32(&in_empty[s]));
+          if (!ad_sep) umma_commit(smem_u32(&in_empty[s]));
         }
       }
       umma_commit(smem_u32(acc_full));
@@ -435,26 +475,43 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       pk_hi = o * 64 + (((2 * h + 1) ^ x) << 4);
     }
     const uint32_t tm_row = tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)C::kAccCols;
-    int it = group;
-    uint32_t q_next = 0;
-    float t_next = 0.0f;
-    if (it < nk) {
-      const uint32_t b = block_of(kb_lo + it);
-      q_next = __ldg(p.qcodes + b);
-      t_next = __ldg(p.t + b / p.C);
+    // Scale inputs (q_b, t_g) of this group's next kPf steps are in flight
+    // while it decodes: a rotating window of loads kPf steps ahead hides
+    // the global-memory latency behind kPf tile decodes.
+    constexpr int kPf = 4;
+    uint32_t qw[kPf];
+    float tw[kPf];
+#pragma unroll
+    for (int j = 0; j < kPf; ++j) {
+      const int itj = group + j * kDecGroups;
+      qw[j] = 128u;
+      tw[j] = 0.0f;
+      if (itj < nk) {
+        const uint32_t b = block_of(kb_lo + itj);
+        qw[j] = __ldg(p.qcodes + b);
+        tw[j] = __ldg(p.t + b / p.C);
+      }
     }
     bool ok = true;
-    for (; it < nk; it += kDecGroups) {
+    for (int it = group; it < nk; it += kDecGroups) {
       const int s = it % NIN, d = it % NDEC;
-      const float sc = decode_block_scale(q_next, t_next, mu);
-      if (it + kDecGroups < nk) {  // prefetch the scale inputs of this group's next step
-        const uint32_t b = block_of(kb_lo + it + kDecGroups);
-        q_next = __ldg(p.qcodes + b);
-        t_next = __ldg(p.t + b / p.C);
+      const float sc = decode_block_scale(qw[0], tw[0], mu);
+#pragma unroll
+      for (int j = 0; j + 1 < kPf; ++j) {
+        qw[j] = qw[j + 1];
+        tw[j] = tw[j + 1];
+      }
+      {
+        const int itn = it + kPf * kDecGroups;
+        if (itn < nk) {
+          const uint32_t b = block_of(kb_lo + itn);
+          qw[kPf - 1] = __ldg(p.qcodes + b);
+          tw[kPf - 1] = __ldg(p.t + b / p.C);
+        }
       }
       if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
       bool w_ok = mbar_wait(smem_u32(&dec_empty[d]), ((it / NDEC) & 1) ^ 1, p.wait_ns, p.err, 0x301) &&
-                  mbar_wait(smem_u32(&full_in[s]), (it / NIN) & 1, p.wait_ns, p.err, 0x302);
+                  mbar_wait(smem_u32(&full_in[s - s % C::G]), (it / NIN) & 1, p.wait_ns, p.err, 0x302);
       if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
       const uint8_t* src = pk + s * kPkTile;
       if (!DX) {
@@ -548,6 +605,24 @@ bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esiz
                    CU_TENSOR_MAP_INTERLEAVE_NONE,
                    swz,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3D view {d0, d1, d2} of `esize`-byte elements with byte strides s1 (dim
+// 1) and s2 (dim 2), box {b0, b1, b2}: the token and packed tiles of b2
+// consecutive K steps in one copy, landing as b2 consecutive tiles.
+bool make_map3(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+               CUtensorMapSwizzle swz) {
+  EncodeTiled enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -713,8 +788,12 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   cudaError_t e = cudaSuccess;
   CUtensorMap m_act, m_pk, m_aact, m_aw;
   const uint32_t bn = (uint32_t)pl.bn;
-  if (!make_map(&m_act, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I / 2, O, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B) ||
+  // X as {64 columns, R rows, I/64 K steps}; codes as {32 bytes, O rows, I/64 K steps}
+  const uint32_t g = (uint32_t)tma_group(pl.bn);
+  if (!make_map3(&m_act, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, (uint64_t)R, (uint64_t)(I / 64),
+                 (uint64_t)I * 2, 128, 64, bn, g, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 32, (uint64_t)O, (uint64_t)(I / 64),
+                 (uint64_t)(I / 2), 32, 32, 128, g, CU_TENSOR_MAP_SWIZZLE_32B) ||
       !make_map(&m_aact, upad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&m_aw, bpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, O, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
@@ -759,8 +838,13 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   cudaError_t e = cudaSuccess;
   CUtensorMap m_act, m_pk, m_aact, m_aw;
   const uint32_t bn = (uint32_t)pl.bn;
-  if (!make_map(&m_act, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, O, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, I / 2, O, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B) ||
+  // dY as {64 columns, R rows, O/64 K steps}; codes as {I/2 bytes, 64 rows, O/64 K steps}
+  const uint32_t g = (uint32_t)tma_group(pl.bn);
+  if (!make_map3(&m_act, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, (uint64_t)R, (uint64_t)(O / 64),
+                 (uint64_t)O * 2, 128, 64, bn, g, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(I / 2), 64,
+                 (uint64_t)(O / 64), (uint64_t)(I / 2), (uint64_t)64 * (I / 2), 64, 64, g,
+                 CU_TENSOR_MAP_SWIZZLE_64B) ||
       !make_map(&m_aact, vpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&m_aw, apad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, 64, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
