@@ -19,6 +19,7 @@ host's cores on a bounded row sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -144,6 +145,26 @@ class Layer:
         q.qlora_linear_fwd(self.w, X, self.A, self.B, self.alpha, Y=self.Y, U_out=self.U, ws=self.ws_f)
         q.qlora_linear_bwd(self.w, X, dY, self.A, self.B, self.alpha, U=self.U, dX=self.dX, dA=self.dA,
                            dB=self.dB, ws=self.ws_b)
+
+
+def measured_traffic(workload, kernel):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu
+    capture under profiles/, or None when there is none or the kernel's
+    source has changed since it was taken (the capture records a hash of the
+    source files)."""
+    path = os.path.join(ROOT, "profiles", f"tc_qlinear_traffic_{workload}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for rel in rec.get("source_files", []):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if h.hexdigest() != rec.get("source_sha256"):
+        return None
+    k = rec.get("kernels", {}).get(kernel)
+    return int(k["dram_bytes_per_launch"]) if k else None
 
 
 def run_gpu(args):
@@ -296,9 +317,10 @@ def run_gpu(args):
         kind, (kms, kfl, n) = dom
         achieved = kfl / (kms * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
-        roofline = {"bound": "tensor", "kernel": "tc_qlinear_fwd" if kind == 0 else "tc_qlinear_dx",
+        kname = "tc_qlinear_fwd" if kind == 0 else "tc_qlinear_dx"
+        roofline = {"bound": "tensor", "kernel": kname,
                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                    "frac": round(achieved / peak, 4), "traffic": None,
+                    "frac": round(achieved / peak, 4), "traffic": measured_traffic(wl.name, kname),
                     "peak_source": f"{peaks['source']} bf16 dense (burst)",
                     "flops_per_launch": kfl / n, "avg_launch_ms": kms / n}
 
