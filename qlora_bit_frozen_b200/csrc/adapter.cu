@@ -1,25 +1,21 @@
-// adapter.cu -- the LoRA side products of the QLoRA linear layer, in fp32.
+// adapter.cu -- the LoRA side products of the QLoRA linear layer.
 //
 // "QLoRA on Mac", "Design / Q-LoRA layer": the adapter branch is
 // (alpha/r)(x A^T) B^T with fp32 A, B.  Forward needs U = X A^T; the
 // backward chain rule needs V = dY B, dA = s V^T X and dB = s dY^T U.
 // Each reads one activation matrix once and touches an r-wide factor, so
-// they are bound by HBM bandwidth on X / dY; the kernels are written to
-// keep many independent loads in flight (every load of a chunk is issued
-// before any of it is used):
+// they are bound by HBM bandwidth on X / dY.
 //
-//  * rowdot: out[m, j] = sum_k P[m, k] L(k, j)  (U: L = A^T; V: L = B).
-//    A 32 KB chunk of L is staged in shared memory per block; each warp owns
-//    RW rows, each lane loads 8 consecutive elements of every row per 256
-//    columns; lane partials are combined with a butterfly.  It also writes
-//    the bf16 copy zero-padded to 64 columns that the tensor-core kernels
-//    use as their extra K step, and (extra blocks of the same launch) the
-//    zero-padded bf16(s B) / bf16(s A) operand of that step.
-//  * coldot: out(j, n) = s sum_m aux[m, j] P[m, n]  (dA: aux = V, P = X;
-//    dB: aux = U, P = dY).  A block is 32 column threads x 8 row lanes over a
-//    slice of the rows; the 8 row lanes are summed in shared memory, the
-//    slices then in slice order by a second kernel (deterministic), which
-//    applies s and writes dA as [r x I] or dB as [O x r].
+//  * bf16 activations (the tensor-core configurations): rowdot_mma_kernel
+//    and coldot_mma_kernel run the products on mma.sync with the fp32
+//    factor split into two bf16 halves (16 significant bits kept); few-row
+//    cases split the reduction across blocks and the last block to finish
+//    adds the partials in a fixed order.  rowdot also writes the bf16 copy
+//    of U / V zero-padded to 64 columns and (extra blocks of the same
+//    launch) the zero-padded bf16(s B) / bf16(s A) operand of the
+//    tensor-core kernel's adapter step.
+//  * fp32 activations (fp32 compute mode) and unaligned inputs: the FMA
+//    forms rowdot_kernel / coldot_kernel, fp32 throughout.
 #include "common.cuh"
 #include "internal.h"
 
@@ -46,72 +42,6 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // ----------------------------------------------------------------- loads
 
-template <typename T, int E>
-__device__ __forceinline__ void load_vec(const T* p, float (&x)[E]);
-
-template <>
-__device__ __forceinline__ void load_vec<__nv_bfloat16, 8>(const __nv_bfloat16* p, float (&x)[8]) {
-  const uint4 v = *reinterpret_cast<const uint4*>(p);
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-template <>
-__device__ __forceinline__ void load_vec<__nv_bfloat16, 4>(const __nv_bfloat16* p, float (&x)[4]) {
-  const uint2 v = *reinterpret_cast<const uint2*>(p);
-  x[0] = __uint_as_float(v.x << 16);
-  x[1] = __uint_as_float(v.x & 0xFFFF0000u);
-  x[2] = __uint_as_float(v.y << 16);
-  x[3] = __uint_as_float(v.y & 0xFFFF0000u);
-}
-template <>
-__device__ __forceinline__ void load_vec<__nv_bfloat16, 2>(const __nv_bfloat16* p, float (&x)[2]) {
-  const uint32_t v = *reinterpret_cast<const uint32_t*>(p);
-  x[0] = __uint_as_float(v << 16);
-  x[1] = __uint_as_float(v & 0xFFFF0000u);
-}
-template <>
-__device__ __forceinline__ void load_vec<__nv_bfloat16, 1>(const __nv_bfloat16* p, float (&x)[1]) {
-  x[0] = __bfloat162float(*p);
-}
-template <>
-__device__ __forceinline__ void load_vec<float, 8>(const float* p, float (&x)[8]) {
-  const float4 a = *reinterpret_cast<const float4*>(p);
-  const float4 b = *reinterpret_cast<const float4*>(p + 4);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-}
-template <>
-__device__ __forceinline__ void load_vec<float, 4>(const float* p, float (&x)[4]) {
-  const float4 a = *reinterpret_cast<const float4*>(p);
-  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-}
-template <>
-__device__ __forceinline__ void load_vec<float, 2>(const float* p, float (&x)[2]) {
-  const float2 a = *reinterpret_cast<const float2*>(p);
-  x[0] = a.x; x[1] = a.y;
-}
-template <>
-__device__ __forceinline__ void load_vec<float, 1>(const float* p, float (&x)[1]) {
-  x[0] = *p;
-}
-
-// E elements starting at p, element i valid when i < nvalid (others 0).
-template <typename T, int E>
-__device__ __forceinline__ void load_elems(const T* p, int nvalid, bool vec_ok, float (&x)[E]) {
-  if (vec_ok && nvalid >= E) {
-    load_vec<T, E>(p, x);
-  } else {
-#pragma unroll
-    for (int i = 0; i < E; ++i) x[i] = i < nvalid ? to_f32<T>(p[i]) : 0.0f;
-  }
-}
-
-// E elements kept in their storage format (32-bit words) until used, so a
-// chunk's loads can all be in flight without converting them first.
 template <typename T, int E>
 struct Raw {
   static constexpr int kBytes = E * (int)sizeof(T);
@@ -458,276 +388,6 @@ __global__ void __launch_bounds__(kThreads) coldot_kernel(const T* __restrict__ 
 // shared memory, so each block keeps ~3 tiles of loads in flight whatever
 // its register use; threads compute from shared memory.
 
-constexpr int kStages = 4;
-
-// Lane l of a warp owns the tile columns {128 h + 4 l + e : h < H, e < 4}
-// (H = KT / 128) when KT >= 128, else {l * E + e : e < E} (E = KT / 32):
-// consecutive lanes then read consecutive 16-byte (or 8-byte) words of a
-// shared-memory row, free of bank conflicts.
-template <int KT>
-struct LaneCols {
-  static constexpr int E = KT >= 128 ? 4 : KT / 32;  // elements per group
-  static constexpr int H = KT >= 128 ? KT / 128 : 1;  // groups per lane
-  static constexpr int N = E * H;                      // elements per lane
-  __device__ static int col(int lane, int h) { return KT >= 128 ? 128 * h + 4 * lane : lane * E; }
-};
-
-// rowdot: block = 8 warps x RW rows (RW * RMAX <= 64 accumulators per
-// thread); tile = KT columns of P and of L [r x K] (KT * RMAX = 2048 floats).
-template <typename T, int RMAX>
-struct RowPipe {
-  static constexpr int RW = 64 / RMAX >= 4 ? 4 : 64 / RMAX;
-  static constexpr int RB = 8 * RW;
-  static constexpr int KT = 2048 / RMAX;
-  static constexpr int XB = RB * KT * (int)sizeof(T);
-  static constexpr int LB = RMAX * KT * 4;
-  static constexpr int STAGE = XB + LB;
-  static constexpr int SMEM = kStages * STAGE;
-  static constexpr int XTOT = XB / 16, LTOT = LB / 16;  // 16-byte copies per tile
-  static constexpr int XCH = (XTOT + kThreads - 1) / kThreads;  // per thread (some idle)
-  static constexpr int LCH = (LTOT + kThreads - 1) / kThreads;
-};
-
-template <typename T, int RMAX>
-__global__ void __launch_bounds__(kThreads) rowdot_pipe_kernel(
-    const T* __restrict__ P, int64_t R, int64_t K, const float* __restrict__ L, int r,
-    float* __restrict__ out, uint16_t* __restrict__ out_pad, int row_blocks, PadJob job) {
-  // the tensor-core kernel queued next may start its weight stream now
-  if (threadIdx.x == 0) griddep_launch_dependents();
-  if ((int)blockIdx.x >= row_blocks) {
-    run_pad_job(job, (int64_t)blockIdx.x - row_blocks);
-    return;
-  }
-  using C = RowPipe<T, RMAX>;
-  using LC = LaneCols<C::KT>;
-  constexpr int EPC = 16 / (int)sizeof(T);          // elements per 16-byte copy
-  constexpr int ROWCH = C::KT / EPC;                // copies per P row of a tile
-  constexpr int LROWCH = C::KT / 4;                 // copies per L row of a tile
-  extern __shared__ __align__(16) uint8_t sm[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t rb0 = (int64_t)blockIdx.x * C::RB;
-  const int ntiles = (int)((K + C::KT - 1) / C::KT);
-  // fixed copy slots of this thread: P rows/cols and L rows/cols
-  int xrow[C::XCH], xcol[C::XCH], lrow[C::LCH], lcol[C::LCH];
-#pragma unroll
-  for (int i = 0; i < C::XCH; ++i) {
-    const int c = threadIdx.x + kThreads * i;
-    xrow[i] = c / ROWCH;
-    xcol[i] = (c - xrow[i] * ROWCH) * EPC;
-  }
-#pragma unroll
-  for (int i = 0; i < C::LCH; ++i) {
-    const int c = threadIdx.x + kThreads * i;
-    lrow[i] = c / LROWCH;
-    lcol[i] = (c - lrow[i] * LROWCH) * 4;
-  }
-  auto issue = [&](int t) {
-    const uint32_t xs = (uint32_t)__cvta_generic_to_shared(sm + (t % kStages) * C::STAGE);
-    const uint32_t ls = xs + C::XB;
-    const int64_t k0 = (int64_t)t * C::KT;
-#pragma unroll
-    for (int i = 0; i < C::XCH; ++i) {
-      if (threadIdx.x + kThreads * i >= C::XTOT) break;
-      const int64_t m = rb0 + xrow[i], k = k0 + xcol[i];
-      const int64_t rem = (K - k) * (int64_t)sizeof(T);
-      const uint32_t nb = (m < R && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
-      cp_async16(xs + (uint32_t)(xrow[i] * ROWCH * 16 + xcol[i] * (int)sizeof(T)),
-                 nb ? (const void*)(P + m * K + k) : (const void*)P, nb);
-    }
-#pragma unroll
-    for (int i = 0; i < C::LCH; ++i) {
-      if (threadIdx.x + kThreads * i >= C::LTOT) break;
-      const int64_t k = k0 + lcol[i];
-      const int64_t rem = (K - k) * 4;
-      const uint32_t nb = (lrow[i] < r && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
-      cp_async16(ls + (uint32_t)(lrow[i] * C::KT * 4 + lcol[i] * 4),
-                 nb ? (const void*)(L + (int64_t)lrow[i] * K + k) : (const void*)L, nb);
-    }
-  };
-
-  constexpr int RW = C::RW;
-  float acc[RW][RMAX];
-#pragma unroll
-  for (int q = 0; q < RW; ++q)
-#pragma unroll
-    for (int j = 0; j < RMAX; ++j) acc[q][j] = 0.0f;
-#pragma unroll
-  for (int t = 0; t < kStages - 1; ++t) {
-    if (t < ntiles) issue(t);
-    cp_async_commit();
-  }
-  for (int t = 0; t < ntiles; ++t) {
-    cp_async_wait<kStages - 2>();
-    __syncthreads();
-    if (t + kStages - 1 < ntiles) issue(t + kStages - 1);
-    cp_async_commit();
-    const uint8_t* xs = sm + (t % kStages) * C::STAGE;
-    const float* ls = (const float*)(xs + C::XB);
-    float x[RW][LC::N];
-#pragma unroll
-    for (int q = 0; q < RW; ++q)
-#pragma unroll
-      for (int h = 0; h < LC::H; ++h) {
-        float v[LC::E];
-        load_vec<T, LC::E>((const T*)xs + (warp * RW + q) * C::KT + LC::col(lane, h), v);
-#pragma unroll
-        for (int e = 0; e < LC::E; ++e) x[q][h * LC::E + e] = v[e];
-      }
-#pragma unroll
-    for (int j = 0; j < RMAX; ++j) {
-      if (j < r) {
-        float l[LC::N];
-#pragma unroll
-        for (int h = 0; h < LC::H; ++h) {
-          float v[LC::E];
-          load_vec<float, LC::E>(ls + j * C::KT + LC::col(lane, h), v);
-#pragma unroll
-          for (int e = 0; e < LC::E; ++e) l[h * LC::E + e] = v[e];
-        }
-#pragma unroll
-        for (int q = 0; q < RW; ++q)
-#pragma unroll
-          for (int e = 0; e < LC::N; ++e) acc[q][j] = fmaf(x[q][e], l[e], acc[q][j]);
-      }
-    }
-  }
-  cp_async_wait<0>();
-#pragma unroll
-  for (int q = 0; q < RW; ++q)
-#pragma unroll
-    for (int j = 0; j < RMAX; ++j)
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) acc[q][j] += __shfl_xor_sync(0xffffffffu, acc[q][j], o);
-#pragma unroll
-  for (int q = 0; q < RW; ++q) {
-    const int64_t m = rb0 + warp * RW + q;
-    if (m >= R) continue;
-    float a0 = 0.0f, a1 = 0.0f;
-#pragma unroll
-    for (int j = 0; j < RMAX; ++j) {
-      if (j == lane) a0 = acc[q][j];
-      if (j == lane + 32) a1 = acc[q][j];
-    }
-    if (lane < r) out[m * r + lane] = a0;
-    if (lane + 32 < r) out[m * r + lane + 32] = a1;
-    if (out_pad) {
-      out_pad[m * 64 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(lane < r ? a0 : 0.0f));
-      out_pad[m * 64 + lane + 32] =
-          __bfloat16_as_ushort(__float2bfloat16_rn(lane + 32 < r ? a1 : 0.0f));
-    }
-  }
-}
-
-// coldot: block = 128 threads x 2 columns = 256 columns over a row slice;
-// tile = 32 rows of P (16 KB bf16) and the matching 32 rows of aux [R x r].
-constexpr int kColThreadsP = 128;
-constexpr int kColStages = 3;
-template <typename T, int RMAX>
-struct ColPipe {
-  static constexpr int NC = 256;
-  static constexpr int RT = 32;
-  static constexpr int PB = RT * NC * (int)sizeof(T);
-  static constexpr int AB = RT * RMAX * 4;
-  static constexpr int STAGE = PB + AB;
-  static constexpr int SMEM = kColStages * STAGE;
-  static constexpr int PCH = PB / 16 / kColThreadsP;  // 16-byte copies per thread per tile
-};
-
-template <typename T, int RMAX>
-__global__ void __launch_bounds__(kColThreadsP) coldot_pipe_kernel(
-    const T* __restrict__ P, int64_t R, int64_t N, const float* __restrict__ aux, int r,
-    int64_t rows_per_split, float* __restrict__ part) {
-  using C = ColPipe<T, RMAX>;
-  constexpr int EPC = 16 / (int)sizeof(T);
-  constexpr int ROWCH = C::NC / EPC;
-  extern __shared__ __align__(16) uint8_t sm[];
-  const int64_t nb = (int64_t)blockIdx.x * C::NC;
-  const int64_t m_lo = (int64_t)blockIdx.y * rows_per_split;
-  const int64_t m_hi = min(R, m_lo + rows_per_split);
-  const int ntiles = (int)((m_hi - m_lo + C::RT - 1) / C::RT);
-  int prow[C::PCH], pcol[C::PCH];
-#pragma unroll
-  for (int i = 0; i < C::PCH; ++i) {
-    const int c = threadIdx.x + kColThreadsP * i;
-    prow[i] = c / ROWCH;
-    pcol[i] = (c - prow[i] * ROWCH) * EPC;
-  }
-  const int ach = (C::RT * r * 4 + 15) / 16;  // aux copies per tile (<= 2 * RMAX)
-  auto issue = [&](int t) {
-    const uint32_t ps = (uint32_t)__cvta_generic_to_shared(sm + (t % kColStages) * C::STAGE);
-    const uint32_t as = ps + C::PB;
-    const int64_t r0 = m_lo + (int64_t)t * C::RT;
-#pragma unroll
-    for (int i = 0; i < C::PCH; ++i) {
-      const int64_t m = r0 + prow[i], n = nb + pcol[i];
-      const int64_t rem = (N - n) * (int64_t)sizeof(T);
-      const uint32_t bytes = (m < m_hi && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
-      cp_async16(ps + (uint32_t)(prow[i] * ROWCH * 16 + pcol[i] * (int)sizeof(T)),
-                 bytes ? (const void*)(P + m * N + n) : (const void*)P, bytes);
-    }
-    // aux rows r0 .. r0+RT of [R x r] are contiguous
-    const int64_t a_end = min(m_hi, r0 + C::RT) * r;
-    for (int c = threadIdx.x; c < ach; c += kColThreadsP) {
-      const int64_t e = r0 * r + (int64_t)c * 4;
-      const int64_t rem = (a_end - e) * 4;
-      const uint32_t bytes = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
-      cp_async16(as + c * 16, bytes ? (const void*)(aux + e) : (const void*)aux, bytes);
-    }
-  };
-
-  float acc[2][RMAX];
-#pragma unroll
-  for (int q = 0; q < 2; ++q)
-#pragma unroll
-    for (int j = 0; j < RMAX; ++j) acc[q][j] = 0.0f;
-#pragma unroll
-  for (int t = 0; t < kColStages - 1; ++t) {
-    if (t < ntiles) issue(t);
-    cp_async_commit();
-  }
-  const int col = threadIdx.x * 2;  // local column pair
-  for (int t = 0; t < ntiles; ++t) {
-    cp_async_wait<kColStages - 2>();
-    __syncthreads();
-    if (t + kColStages - 1 < ntiles) issue(t + kColStages - 1);
-    cp_async_commit();
-    const uint8_t* ps = sm + (t % kColStages) * C::STAGE;
-    const float* as = (const float*)(ps + C::PB);  // row-major [RT x r]
-    const int rows = (int)min((int64_t)C::RT, m_hi - (m_lo + (int64_t)t * C::RT));
-    for (int row = 0; row < rows; ++row) {
-      float pv[2];
-      load_vec<T, 2>((const T*)ps + row * C::NC + col, pv);
-      const float* ar = as + row * r;
-#pragma unroll
-      for (int j = 0; j < RMAX; j += 4) {
-        if (j < r) {
-          float a[4];
-          if ((r & 3) == 0) {
-            load_vec<float, 4>(ar + j, a);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = j + i < r ? ar[j + i] : 0.0f;
-          }
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            acc[0][j + i] = fmaf(a[i], pv[0], acc[0][j + i]);
-            acc[1][j + i] = fmaf(a[i], pv[1], acc[1][j + i]);
-          }
-        }
-      }
-    }
-  }
-  cp_async_wait<0>();
-  float* dst = part + (int64_t)blockIdx.y * r * N;
-#pragma unroll
-  for (int j = 0; j < RMAX; ++j) {
-    if (j < r) {
-      const int64_t n = nb + col;
-      if (n < N) dst[(int64_t)j * N + n] = acc[0][j];
-      if (n + 1 < N) dst[(int64_t)j * N + n + 1] = acc[1][j];
-    }
-  }
-}
 
 // ------------------------------------------------------ tensor-core path
 //
@@ -1121,41 +781,6 @@ __global__ void __launch_bounds__(kThreads) coldot_mma_kernel(
   }
 }
 
-// out = s * sum over slices of part[slice][j][n].  Block = 8 warps over 32
-// consecutive outputs e (= j * N + n): warp w sums slices w, w+8, ... for
-// lane-th output (coalesced across lanes), then the 8 warp sums are added in
-// warp order.  out_nr == 0: out[j * N + n] (dA);  1: out[n * r + j] (dB).
-__global__ void __launch_bounds__(256) slice_reduce_kernel(const float* __restrict__ part, int splits,
-                                                           int64_t N, int r, float s, int out_nr,
-                                                           float* __restrict__ out) {
-  __shared__ float red[8][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t rN = (int64_t)r * N;
-  const int64_t e = (int64_t)blockIdx.x * 32 + lane;
-  float v = 0.0f;
-  if (e < rN) {
-    int k = warp;
-    for (; k + 8 * 3 < splits; k += 8 * 4) {
-      const float a = part[(int64_t)k * rN + e], b = part[(int64_t)(k + 8) * rN + e];
-      const float c = part[(int64_t)(k + 16) * rN + e], d = part[(int64_t)(k + 24) * rN + e];
-      v += a;
-      v += b;
-      v += c;
-      v += d;
-    }
-    for (; k < splits; k += 8) v += part[(int64_t)k * rN + e];
-  }
-  red[warp][lane] = v;
-  __syncthreads();
-  if (warp == 0 && e < rN) {
-    float t = red[0][lane];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) t += red[w][lane];
-    const int64_t j = e / N, n = e - j * N;
-    out[out_nr ? n * r + j : e] = s * t;
-  }
-}
-
 // dst[j * K + k] = src[k * r + j]: B [K x r] -> B^T [r x K].
 __global__ void transpose_kr_kernel(const float* __restrict__ src, int64_t K, int r,
                                     float* __restrict__ dst) {
@@ -1231,22 +856,6 @@ cudaError_t set_smem_once(Kern k, int bytes, bool& done) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess) done = true;
   return e;
-}
-
-template <int RMAX>
-cudaError_t rowdot_pipe_go(const __nv_bfloat16* P, int64_t R, int64_t K, const float* L, int r,
-                           float* out, uint16_t* pad, PadJob job, cudaStream_t st) {
-  using C = RowPipe<__nv_bfloat16, RMAX>;
-  static bool attr = false;
-  auto kern = rowdot_pipe_kernel<__nv_bfloat16, RMAX>;
-  cudaError_t e = set_smem_once(kern, C::SMEM, attr);
-  if (e != cudaSuccess) return e;
-  const int row_blocks = (int)cdiv(R, C::RB);
-  const unsigned grid = (unsigned)(row_blocks + job.blocks);
-  if (grid == 0) return cudaSuccess;
-  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, K, L, r, out, pad, row_blocks, job);
-  count_launch();
-  return cudaGetLastError();
 }
 
 struct ColPlan {
@@ -1396,58 +1005,14 @@ cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const 
     Lr = lt_ws;
     lkr = false;
   }
-  // pipelined path: more than 64 bf16 rows on 16-byte boundaries
-  const bool rows16 = bf16 && (K % 8) == 0 && ((uintptr_t)P % 16) == 0;
-  if (rows16 && R > 64 && !lkr && ((uintptr_t)Lr % 16) == 0 && (K % 4) == 0) {
-    const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
-    if (r <= 8) return rowdot_pipe_go<8>(Pb, R, K, Lr, r, out, pad, job, st);
-    if (r <= 16) return rowdot_pipe_go<16>(Pb, R, K, Lr, r, out, pad, job, st);
-    if (r <= 32) return rowdot_pipe_go<32>(Pb, R, K, Lr, r, out, pad, job, st);
-    return rowdot_pipe_go<64>(Pb, R, K, Lr, r, out, pad, job, st);
-  }
   if (bf16) return rowdot_r<__nv_bfloat16>(P, R, K, Lr, lkr, r, out, pad, job, st);
   return rowdot_r<float>(P, R, K, Lr, lkr, r, out, pad, job, st);
 }
 
 namespace {
 
-struct PipePlan {
-  int splits;
-  int64_t rows_per_split;
-  unsigned colblocks;
-};
-
-PipePlan pipe_plan(int64_t R, int64_t N) {
-  PipePlan c;
-  c.colblocks = cdiv(N, ColPipe<__nv_bfloat16, 8>::NC);
-  int64_t splits = (2 * (int64_t)sm_count() + c.colblocks - 1) / c.colblocks;
-  const int64_t max_splits = (R + 63) / 64;
-  if (splits > max_splits) splits = max_splits;
-  if (splits < 1) splits = 1;
-  int64_t rps = (R + splits - 1) / splits;
-  rps = (rps + 31) / 32 * 32;  // aux tiles start on 16-byte boundaries
-  if (rps < 32) rps = 32;
-  c.rows_per_split = rps;
-  c.splits = R > 0 ? (int)((R + rps - 1) / rps) : 1;
-  return c;
-}
-
-bool coldot_pipe_ok(const void* P, bool bf16, int64_t R, int64_t N, const float* aux) {
+bool coldot_mma_ok(const void* P, bool bf16, int64_t R, int64_t N, const float* aux) {
   return bf16 && R > 0 && (N % 8) == 0 && ((uintptr_t)P % 16) == 0 && ((uintptr_t)aux % 16) == 0;
-}
-
-template <int RMAX>
-cudaError_t coldot_pipe_go(const __nv_bfloat16* P, int64_t R, int64_t N, const float* aux, int r,
-                           const PipePlan& c, float* part, cudaStream_t st) {
-  using C = ColPipe<__nv_bfloat16, RMAX>;
-  static bool attr = false;
-  auto kern = coldot_pipe_kernel<__nv_bfloat16, RMAX>;
-  cudaError_t e = set_smem_once(kern, C::SMEM, attr);
-  if (e != cudaSuccess) return e;
-  dim3 grid(c.colblocks, (unsigned)c.splits);
-  kern<<<grid, kColThreadsP, C::SMEM, st>>>(P, R, N, aux, r, c.rows_per_split, part);
-  count_launch();
-  return cudaGetLastError();
 }
 
 }  // namespace
@@ -1457,19 +1022,16 @@ size_t rowdot_ws(int64_t R, int64_t K, int32_t r) {
   return pl.splits > 1 ? align_up((size_t)pl.splits * (size_t)R * 8 * rank_tiles(r) * 4, 256) : 0;
 }
 
-// Workspace: the larger of the pipelined path (slice sums) and the
-// streaming path (tickets + slice sums).
+// Workspace: the larger of the tensor-core path (split partials) and the
+// FMA path (tickets + slice sums).
 size_t coldot_ws(int64_t R, int64_t N, int32_t r) {
   const ColPlan c = col_plan(R, N, r);
   size_t a = c.splits <= 1 ? 0
                            : align_up((size_t)c.colblocks * 4, 256) +
                                  align_up((size_t)c.splits * (size_t)r * (size_t)N * 4, 256);
-  const PipePlan pp = pipe_plan(R, N);
-  size_t b = align_up((size_t)pp.splits * (size_t)r * (size_t)N * 4, 256);
   const MmaPlan mp = coldot_mma_plan(R, N, true);
-  const size_t cm =
+  const size_t b =
       mp.splits > 1 ? align_up((size_t)mp.splits * (size_t)N * 8 * rank_tiles(r) * 4, 256) : 0;
-  if (cm > b) b = cm;
   return a > b ? a : b;
 }
 
@@ -1478,7 +1040,7 @@ cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const 
                           cudaStream_t st, unsigned* tickets) {
   if (N == 0) return cudaSuccess;
   if (R == 0) return cudaMemsetAsync(out, 0, (size_t)r * (size_t)N * 4, st);
-  if (coldot_pipe_ok(P, bf16, R, N, aux)) {  // tensor cores
+  if (coldot_mma_ok(P, bf16, R, N, aux)) {  // tensor cores
     const MmaPlan pl = coldot_mma_plan(R, N, tickets != nullptr);
     const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
     float* part = (float*)ws;
@@ -1488,22 +1050,6 @@ cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const 
       case 4: return coldot_mma_go<4>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
       default: return coldot_mma_go<8>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
     }
-  }
-  if (coldot_pipe_ok(P, bf16, R, N, aux)) {
-    const PipePlan c = pipe_plan(R, N);
-    float* part = (float*)ws;
-    const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
-    cudaError_t e;
-    if (r <= 8) e = coldot_pipe_go<8>(Pb, R, N, aux, r, c, part, st);
-    else if (r <= 16) e = coldot_pipe_go<16>(Pb, R, N, aux, r, c, part, st);
-    else if (r <= 32) e = coldot_pipe_go<32>(Pb, R, N, aux, r, c, part, st);
-    else e = coldot_pipe_go<64>(Pb, R, N, aux, r, c, part, st);
-    if (e != cudaSuccess) return e;
-    const int64_t outs = (int64_t)r * N;
-    slice_reduce_kernel<<<cdiv(outs, 32), 256, 0, st>>>(part, c.splits, N, r, s, out_nr ? 1 : 0,
-                                                        out);
-    count_launch();
-    return cudaGetLastError();
   }
   const ColPlan c = col_plan(R, N, r);
   unsigned* slice_tickets = (unsigned*)ws;

@@ -40,10 +40,6 @@ __device__ __forceinline__ double nf4_mid(int k) {
 // ---------------------------------------------------------------------------
 constexpr size_t kWsHeader = 256;
 
-struct DevErr {
-  uint32_t* word;  // nullptr disables reporting
-};
-
 __device__ __forceinline__ void report_error(uint32_t* ws_header, uint32_t status, uint32_t where) {
   if (ws_header == nullptr) return;
   if (atomicCAS(ws_header, 0u, status) == 0u) ws_header[1] = where;

@@ -64,11 +64,6 @@ size_t coldot_ws(int64_t R, int64_t N, int32_t r);
 cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
                           int32_t r, float s, bool out_nr, float* out, void* ws,
                           cudaStream_t st, unsigned* tickets = nullptr);
-// bf16 operand staging for the tensor-core path
-cudaError_t launch_pad_rows_bf16(const float* src, int64_t rows, int32_t r, float mul,
-                                 uint16_t* dst, cudaStream_t st);
-cudaError_t launch_pad_cols_bf16(const float* src, int32_t r, int64_t cols, float mul,
-                                 uint16_t* dst, cudaStream_t st);
 // out = scale * sum of the split partials.  pdl: launched with a
 // programmatic dependency on the kernel before it (which must have
 // triggered its dependents); the kernel waits for that grid first.

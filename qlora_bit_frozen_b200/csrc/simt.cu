@@ -92,28 +92,6 @@ __global__ void __launch_bounds__(NT) qlinear_simt_kernel(WView w, int64_t M, co
   }
 }
 
-// dst[m, j] = bf16(mul * src[m, j]) for j < r, 0 for r <= j < 64.
-__global__ void pad_rows_bf16_kernel(const float* __restrict__ src, int64_t rows, int32_t r,
-                                     float mul, uint16_t* __restrict__ dst) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= rows * 64) return;
-  const int64_t m = e >> 6;
-  const int j = (int)(e & 63);
-  const float v = j < r ? __fmul_rn(mul, src[m * r + j]) : 0.0f;
-  dst[e] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-
-// dst[j, n] = bf16(mul * src[j, n]) for j < r, 0 for r <= j < 64.
-__global__ void pad_cols_bf16_kernel(const float* __restrict__ src, int32_t r, int64_t cols,
-                                     float mul, uint16_t* __restrict__ dst) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= 64 * cols) return;
-  const int64_t j = e / cols;
-  const float v = j < r ? __fmul_rn(mul, src[e]) : 0.0f;
-  dst[e] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
-
-// out[m, n] = sum over splits (in order) of part[s][m][n].
 template <typename TO>
 __global__ void splitk_reduce_kernel(const float* __restrict__ part, int32_t splits, int64_t MN,
                                      float scale, TO* __restrict__ out) {
@@ -174,22 +152,6 @@ cudaError_t launch_simt_dx(const WView& w, const void* dY, int64_t R, const floa
   else
     qlinear_simt_kernel<float, true><<<grid, NT, 0, st>>>(w, R, (const float*)dY, V, A, r, s,
                                                           (float*)dX);
-  count_launch();
-  return cudaGetLastError();
-}
-
-cudaError_t launch_pad_rows_bf16(const float* src, int64_t rows, int32_t r, float mul,
-                                 uint16_t* dst, cudaStream_t st) {
-  if (rows == 0) return cudaSuccess;
-  pad_rows_bf16_kernel<<<cdiv(rows * 64, 256), 256, 0, st>>>(src, rows, r, mul, dst);
-  count_launch();
-  return cudaGetLastError();
-}
-
-cudaError_t launch_pad_cols_bf16(const float* src, int32_t r, int64_t cols, float mul,
-                                 uint16_t* dst, cudaStream_t st) {
-  if (cols == 0) return cudaSuccess;
-  pad_cols_bf16_kernel<<<cdiv(64 * cols, 256), 256, 0, st>>>(src, r, cols, mul, dst);
   count_launch();
   return cudaGetLastError();
 }

@@ -7,8 +7,9 @@
 // The frozen weight never exists as a floating-point matrix in HBM: packed
 // NF4 nibbles arrive in shared memory by TMA, decoder warps turn each
 // 64-weight block into bf16 (codebook level times the double-quant block
-// scale rebuilt from q_b, t_g and mu) directly in the 128-byte-swizzled
-// layout the tensor core reads, and tcgen05.mma accumulates in TMEM.
+// scale rebuilt from q_b, t_g and mu) in registers and write it where the
+// tensor core reads it (TMEM rows, or 128-byte-swizzled shared-memory rows),
+// and tcgen05.mma accumulates in TMEM.
 //
 // Orientation: the decoded weight tile is the MMA "A" operand (M = 128
 // weight-side rows: output features in the forward, input features in the
@@ -16,20 +17,23 @@
 // tokens, 16..256).  Small token counts therefore cost no wasted MMA rows,
 // and the same kernel serves the bandwidth-bound and the tensor-bound
 // regimes (split-K supplies parallelism when there are few tiles).
-//   forward : A = W_hat[o, i] tile, K-major (i contiguous)   -> a_major = K
-//   dX      : A = W_hat^T[i, o] tile, MN-major (i contiguous) -> a_major = MN
-// Both layouts consist of 128-byte rows holding 64 consecutive weights of
-// one W row, i.e. exactly one NF4 block, so one decode routine serves both.
+//   forward : A = W_hat[o, i] tile, K-major, decoded into TMEM
+//   dX      : A = W_hat^T[i, o] tile, MN-major, decoded into shared memory
+// A 64-weight NF4 block is one row of either tile, so one register decode
+// serves both.
 //
-// The adapter term is one extra K step of the same accumulation: its A
+// The adapter term is the last K step of the same accumulation: its A
 // operand is bf16(s B) (forward) or bf16(s A)^T (dX), zero-padded to 64
-// along the rank, and its B operand is bf16 U or V, all loaded by TMA.
+// along the rank, and its B operand is bf16 U or V, all loaded by TMA once
+// the launch that computed them has finished (programmatic dependent
+// launch: the K loop before it overlaps that launch).
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM allocator and
-// MMA issuer, warps 2..5 decoders, then epilogue (TMEM -> registers ->
-// global).  Every mbarrier wait is bounded (%globaltimer); on expiry the
-// CTA records QLORA_ERR_TIMEOUT in the workspace header, stops issuing
-// work, waits (bounded) for its copies in flight, frees TMEM and exits.
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and
+// MMA issuer, warps 2..9 decoders in two groups of four (alternate K
+// steps), then epilogue (TMEM -> registers -> shared memory -> TMA store).
+// Every mbarrier wait is bounded (%globaltimer); on expiry the CTA records
+// QLORA_ERR_TIMEOUT in the workspace header, stops issuing work, waits
+// (bounded) for its copies in flight, frees TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
