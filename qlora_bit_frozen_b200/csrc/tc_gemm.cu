@@ -62,6 +62,7 @@ struct TcParams {
   int32_t r_slices;  // ceil(r / 16): MMA K=16 slices of the adapter step
   int32_t rank;      // r (for the algorithmic flop count only)
   uint32_t C;        // scale-group size in blocks
+  int32_t c_shift;   // log2(C) when C is a power of two, else -1
   const uint8_t* qcodes;
   const float* t;
   const float* mu;
@@ -308,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
   const int split = blockIdx.z;
   const int kb_lo = split * p.kb_per_split;
   const int kb_hi = min(p.KB, kb_lo + p.kb_per_split);
-  const int nk = kb_hi - kb_lo;               // weight K steps of this CTA
-  const int T = nk + (split == 0 ? 1 : 0);    // + the adapter step, last, in split 0
+  const int nk = kb_hi - kb_lo;               // weight K steps of this CTA (+ the adapter
+                                              // step, last, in split 0)
 
   if (threadIdx.x == 0) {
     // A kernel queued behind this one with a programmatic dependency (the
@@ -345,10 +346,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       constexpr int G = C::G;
       int issued = 0;  // K steps whose copies were issued
       bool ad_issued = false;
+      int s0 = 0;          // first slot of the group (running)
+      uint32_t ph = 0;     // ring cycle parity of the group
       for (int it0 = 0; it0 < nk; it0 += G) {
-        const int s0 = it0 % NIN, sl = s0 + G - 1, itl = it0 + G - 1;  // group = slots s0 .. sl
-        if (*abort_flag) break;
-        if (!mbar_wait(smem_u32(&in_empty[sl]), ((itl / NIN) & 1) ^ 1, p.wait_ns, p.err, 0x101)) {
+        const int sl = s0 + G - 1;  // group = slots s0 .. sl
+        if ((it0 & (8 * G - 1)) == 0 && *abort_flag) break;
+        if (!mbar_wait(smem_u32(&in_empty[sl]), ph ^ 1u, p.wait_ns, p.err, 0x101)) {
           *abort_flag = 1;
           break;
         }
@@ -361,6 +364,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
         else
           tma_load_3d(smem_u32(pk + s0 * kPkTile), &tm_pk, fb, m0 / 2, 0, kb);
         issued = it0 + G;
+        s0 += G;
+        if (s0 == NIN) { s0 = 0; ph ^= 1u; }
       }
       if (split == 0 && !*abort_flag) {
         // Adapter step: U / V and the scaled factor come from the launch
@@ -371,8 +376,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
           fb = smem_u32(ad_full);
           a_dst = smem_u32(adx);
         } else {
-          const int s = nk % NIN;
-          ok = mbar_wait(smem_u32(&in_empty[s]), ((nk / NIN) & 1) ^ 1, p.wait_ns, p.err, 0x102);
+          const int s = nk % NIN;  // G == 1 here: s0 == s, ph its cycle
+          ok = mbar_wait(smem_u32(&in_empty[s]), ph ^ 1u, p.wait_ns, p.err, 0x102);
           fb = smem_u32(&full_in[s]);
           a_dst = smem_u32(act + s * C::kAct);
         }
@@ -402,44 +407,57 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
+    // The loop is one thread's dependent chain, so it keeps it short:
+    // running ring positions instead of divisions, descriptors built once,
+    // both barriers tested together (the bounded blocking wait only when a
+    // test fails), the abort flag read every eighth step.
     if (lane == 0) {
-      for (int it = 0; it < T; ++it) {
-        const int s = it % NIN;
-        if (*abort_flag) break;
-        const bool ad_sep = C::G > 1 && it == nk;  // adapter step outside the ring
-        const uint32_t fb = ad_sep ? smem_u32(ad_full) : smem_u32(&full_in[s - s % C::G]);
-        if (!mbar_wait(fb, ad_sep ? 0u : (uint32_t)((it / NIN) & 1), p.wait_ns, p.err, 0x201)) {
+      constexpr int G = C::G;
+      const uint32_t act0 = smem_u32(act);
+      const uint64_t bdesc0 = sdesc(act0, 16, 1024);
+      const uint64_t adesc0 = sdesc(smem_u32(wdec), 8192, 1024);
+      int s = 0, d = 0;
+      uint32_t ph_in = 0, ph_dec = 0;
+      bool ok = true;
+      for (int it = 0; it < nk; ++it) {
+        if ((it & 7) == 0 && *abort_flag) { ok = false; break; }
+        const uint32_t fb = smem_u32(&full_in[s - s % G]), db = smem_u32(&dec_full[d]);
+        const bool ready = mbar_test(fb, ph_in) & mbar_test(db, ph_dec);
+        if (!ready && (!mbar_wait(fb, ph_in, p.wait_ns, p.err, 0x201) ||
+                       !mbar_wait(db, ph_dec, p.wait_ns, p.err, 0x202))) {
           *abort_flag = 1;
+          ok = false;
           break;
         }
-        const uint32_t b0 = ad_sep ? smem_u32(adx) : smem_u32(act + s * C::kAct);
-        if (it < nk) {
-          const int d = it % NDEC;
-          if (!mbar_wait(smem_u32(&dec_full[d]), (it / NDEC) & 1, p.wait_ns, p.err, 0x202)) {
-            *abort_flag = 1;
-            break;
-          }
-          tc_fence_after();
+        tc_fence_after();
+        const uint64_t bd = bdesc0 + (uint64_t)((uint32_t)(s * C::kAct) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t bd = sdesc(b0 + kk * 32, 16, 1024);
-            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-            if (!DX)
-              umma_bf16_ta(tmem, tmem + (uint32_t)(C::kAccCols + d * 32 + kk * 8), bd, kIdesc, acc);
-            else
-              umma_bf16(tmem, sdesc(smem_u32(wdec + d * kWTile) + kk * 2048, 8192, 1024), bd,
-                        kIdesc, acc);
-          }
-          umma_commit(smem_u32(&in_empty[s]));
-          umma_commit(smem_u32(&dec_empty[d]));
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          if (!DX)
+            umma_bf16_ta(tmem, tmem + (uint32_t)(C::kAccCols + d * 32 + kk * 8), bd + 2 * kk,
+                         kIdesc, acc);
+          else
+            umma_bf16(tmem, adesc0 + (uint64_t)((uint32_t)(d * kWTile + kk * 2048) >> 4),
+                      bd + 2 * kk, kIdesc, acc);
+        }
+        umma_commit(smem_u32(&in_empty[s]));
+        umma_commit(smem_u32(&dec_empty[d]));
+        if (++s == NIN) { s = 0; ph_in ^= 1u; }
+        if (++d == NDEC) { d = 0; ph_dec ^= 1u; }
+      }
+      if (ok && split == 0) {  // adapter step (s is now nk % NIN)
+        const uint32_t fb = G > 1 ? smem_u32(ad_full) : smem_u32(&full_in[s]);
+        const uint32_t b0 = G > 1 ? smem_u32(adx) : act0 + (uint32_t)(s * C::kAct);
+        if (*abort_flag || !mbar_wait(fb, G > 1 ? 0u : ph_in, p.wait_ns, p.err, 0x203)) {
+          *abort_flag = 1;
         } else {
           tc_fence_after();
           const uint32_t a0 = smem_u32(adw);
           for (int kk = 0; kk < p.r_slices; ++kk) {
             const uint64_t ad = DX ? sdesc(a0 + kk * 2048, 8192, 1024) : sdesc(a0 + kk * 32, 16, 1024);
-            umma_bf16(tmem, ad, sdesc(b0 + kk * 32, 16, 1024), kIdesc, (it > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16(tmem, ad, sdesc(b0 + kk * 32, 16, 1024), kIdesc, (nk > 0 || kk > 0) ? 1u : 0u);
           }
-          if (!ad_sep) umma_commit(smem_u32(&in_empty[s]));
         }
       }
       umma_commit(smem_u32(acc_full));
@@ -460,6 +478,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     auto block_of = [&](int kb) -> uint32_t {
       if (!DX) return (uint32_t)(m0 + u) * bpr + (uint32_t)kb;
       return (uint32_t)(kb * kBK + (u & 63)) * bpr + (uint32_t)(m0 / kBK) + (uint32_t)(u >> 6);
+    };
+    // scale group of block b (a shift when the group size is a power of two)
+    auto group_of = [&](uint32_t b) -> uint32_t {
+      return p.c_shift >= 0 ? (b >> p.c_shift) : b / p.C;
     };
     const uint32_t row_off = (uint32_t)((u >> 6) * (kWTile / 2) + (u & 63) * 128);
     const uint32_t sw = (uint32_t)(u & 7);
@@ -493,12 +515,14 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       if (itj < nk) {
         const uint32_t b = block_of(kb_lo + itj);
         qw[j] = __ldg(p.qcodes + b);
-        tw[j] = __ldg(p.t + b / p.C);
+        tw[j] = __ldg(p.t + group_of(b));
       }
     }
     bool ok = true;
+    // running ring positions of this group's steps (it = group, group + 2, ...)
+    int s = group % NIN, d = group % NDEC;
+    uint32_t ph_in = 0, ph_dec = 0;
     for (int it = group; it < nk; it += kDecGroups) {
-      const int s = it % NIN, d = it % NDEC;
       const float sc = decode_block_scale(qw[0], tw[0], mu);
 #pragma unroll
       for (int j = 0; j + 1 < kPf; ++j) {
@@ -510,12 +534,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
         if (itn < nk) {
           const uint32_t b = block_of(kb_lo + itn);
           qw[kPf - 1] = __ldg(p.qcodes + b);
-          tw[kPf - 1] = __ldg(p.t + b / p.C);
+          tw[kPf - 1] = __ldg(p.t + group_of(b));
         }
       }
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-      bool w_ok = mbar_wait(smem_u32(&dec_empty[d]), ((it / NDEC) & 1) ^ 1, p.wait_ns, p.err, 0x301) &&
-                  mbar_wait(smem_u32(&full_in[s - s % C::G]), (it / NIN) & 1, p.wait_ns, p.err, 0x302);
+      if (((it >> 1) & 3) == 0 && __any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
+      const uint32_t eb = smem_u32(&dec_empty[d]), fb = smem_u32(&full_in[s - s % C::G]);
+      bool w_ok = mbar_test(eb, ph_dec ^ 1u) & mbar_test(fb, ph_in);
+      if (!w_ok)
+        w_ok = mbar_wait(eb, ph_dec ^ 1u, p.wait_ns, p.err, 0x301) &&
+               mbar_wait(fb, ph_in, p.wait_ns, p.err, 0x302);
       if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
       const uint8_t* src = pk + s * kPkTile;
       if (!DX) {
@@ -531,6 +558,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&dec_full[d]));
+      s += kDecGroups;
+      if (s >= NIN) { s -= NIN; ph_in ^= 1u; }
+      d += kDecGroups;
+      if (d >= NDEC) { d -= NDEC; ph_dec ^= 1u; }
     }
     // the accumulator is complete once acc_full fires
     const bool acc_ok = mbar_wait(smem_u32(acc_full), 0, p.wait_ns, p.err, 0x401);
@@ -810,6 +841,7 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   p.r_slices = (r + 15) / 16;
   p.rank = r;
   p.C = (uint32_t)w.group;
+  p.c_shift = ((w.group & (w.group - 1)) == 0) ? __builtin_ctz((unsigned)w.group) : -1;
   p.qcodes = w.qcodes;
   p.t = w.t;
   p.mu = w.mu;
@@ -861,6 +893,7 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   p.r_slices = (r + 15) / 16;
   p.rank = r;
   p.C = (uint32_t)w.group;
+  p.c_shift = ((w.group & (w.group - 1)) == 0) ? __builtin_ctz((unsigned)w.group) : -1;
   p.qcodes = w.qcodes;
   p.t = w.t;
   p.mu = w.mu;
