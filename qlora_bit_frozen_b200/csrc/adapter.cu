@@ -489,9 +489,15 @@ __device__ __forceinline__ void sum_slices(const float* __restrict__ part, int64
 // several splits each writes a partial and the last block of a row block
 // to finish (ticket) adds them in split order.  The final values go out as
 // fp32 [R x r] and, optionally, bf16 zero-padded to 64 columns.
+// Ranks above 16 use 64-column stages (a smaller factor tile): three blocks
+// per SM instead of one.
+constexpr int rowmma_kt(int nt) { return nt >= 4 ? 64 : 128; }
+constexpr int colmma_rt(int nt) { return nt >= 4 ? 32 : 64; }
+
 template <int NT, bool LKR>
 struct RowMma {
-  static constexpr int RB = 64, KT = 128;
+  static constexpr int RB = 64, KT = rowmma_kt(NT);
+  static constexpr int PCH = KT / 8;                   // 16-byte chunks per P row
   static constexpr int NP = 8 * NT;                    // padded rank
   static constexpr int PSTR = KT * 2 + 16;             // bytes per P row in smem
   static constexpr int PB = RB * PSTR;
@@ -529,10 +535,10 @@ __global__ void __launch_bounds__(kThreads) rowdot_mma_kernel(
     const uint32_t ps = (uint32_t)__cvta_generic_to_shared(sm + ((t - t_lo) % kMmaStages) * C::STAGE);
     const uint32_t ls = ps + C::PB;
     const int64_t k0 = (int64_t)t * C::KT;
-    // P: 64 rows x 16 chunks of 16 bytes
+    // P: 64 rows x PCH chunks of 16 bytes
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = threadIdx.x + kThreads * i, row = c >> 4, ch = c & 15;
+    for (int i = 0; i < C::RB * C::PCH / kThreads; ++i) {
+      const int c = threadIdx.x + kThreads * i, row = c / C::PCH, ch = c % C::PCH;
       const int64_t m = m0 + row, k = k0 + ch * 8;
       const int64_t rem = (K - k) * 2;
       const uint32_t nb = (m < R && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
@@ -659,7 +665,7 @@ __global__ void __launch_bounds__(kThreads) rowdot_mma_kernel(
 // writes dA as [r x N] (out_nr = 0) or dB as [N x r] (out_nr = 1).
 template <int NT>
 struct ColMma {
-  static constexpr int NC = 128, RT = 64;
+  static constexpr int NC = 128, RT = colmma_rt(NT);
   static constexpr int NP = 8 * NT;
   static constexpr int PSTR = NC * 2 + 16;
   static constexpr int PB = RT * PSTR;
@@ -689,7 +695,7 @@ __global__ void __launch_bounds__(kThreads) coldot_mma_kernel(
     const uint32_t as = ps + C::PB;
     const int64_t mt = (int64_t)t * C::RT;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {  // 64 rows x 16 chunks
+    for (int i = 0; i < C::RT * 16 / kThreads; ++i) {  // RT rows x 16 chunks
       const int c = threadIdx.x + kThreads * i, row = c >> 4, ch = c & 15;
       const int64_t m = mt + row, n = n0 + ch * 8;
       const int64_t rem = (N - n) * 2;
@@ -922,11 +928,11 @@ MmaPlan mma_plan(int64_t blocks, int64_t ntiles, bool can_split) {
 
 int rank_tiles(int r) { return r <= 8 ? 1 : r <= 16 ? 2 : r <= 32 ? 4 : 8; }
 
-MmaPlan rowdot_mma_plan(int64_t R, int64_t K, bool can_split) {
-  return mma_plan(cdiv(R, 64), cdiv(K, 128), can_split);
+MmaPlan rowdot_mma_plan(int64_t R, int64_t K, int r, bool can_split) {
+  return mma_plan(cdiv(R, 64), cdiv(K, rowmma_kt(rank_tiles(r))), can_split);
 }
-MmaPlan coldot_mma_plan(int64_t R, int64_t N, bool can_split) {
-  return mma_plan(cdiv(N, 128), cdiv(R, 64), can_split);
+MmaPlan coldot_mma_plan(int64_t R, int64_t N, int r, bool can_split) {
+  return mma_plan(cdiv(N, 128), cdiv(R, colmma_rt(rank_tiles(r))), can_split);
 }
 
 bool rowdot_mma_ok(const void* P, bool bf16, int64_t K, const float* L) {
@@ -988,7 +994,7 @@ cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const 
   PadJob job{side_src, side_dst, side_extent, r, side_mode, side_mul, 0};
   if (side_dst && side_extent > 0) job.blocks = (int)cdiv(64 * side_extent, kThreads * 8);
   if (R > 0 && rowdot_mma_ok(P, bf16, K, L)) {  // tensor cores, either factor layout
-    const MmaPlan pl = rowdot_mma_plan(R, K, part_ws != nullptr && tickets != nullptr);
+    const MmaPlan pl = rowdot_mma_plan(R, K, r, part_ws != nullptr && tickets != nullptr);
     const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
     if (l_is_kr) return rowdot_mma_r<true>(Pb, R, K, L, r, pl, out, pad, part_ws, tickets, job, st);
     return rowdot_mma_r<false>(Pb, R, K, L, r, pl, out, pad, part_ws, tickets, job, st);
@@ -1018,7 +1024,7 @@ bool coldot_mma_ok(const void* P, bool bf16, int64_t R, int64_t N, const float* 
 }  // namespace
 
 size_t rowdot_ws(int64_t R, int64_t K, int32_t r) {
-  const MmaPlan pl = rowdot_mma_plan(R, K, true);
+  const MmaPlan pl = rowdot_mma_plan(R, K, r, true);
   return pl.splits > 1 ? align_up((size_t)pl.splits * (size_t)R * 8 * rank_tiles(r) * 4, 256) : 0;
 }
 
@@ -1029,7 +1035,7 @@ size_t coldot_ws(int64_t R, int64_t N, int32_t r) {
   size_t a = c.splits <= 1 ? 0
                            : align_up((size_t)c.colblocks * 4, 256) +
                                  align_up((size_t)c.splits * (size_t)r * (size_t)N * 4, 256);
-  const MmaPlan mp = coldot_mma_plan(R, N, true);
+  const MmaPlan mp = coldot_mma_plan(R, N, r, true);
   const size_t b =
       mp.splits > 1 ? align_up((size_t)mp.splits * (size_t)N * 8 * rank_tiles(r) * 4, 256) : 0;
   return a > b ? a : b;
@@ -1041,7 +1047,7 @@ cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const 
   if (N == 0) return cudaSuccess;
   if (R == 0) return cudaMemsetAsync(out, 0, (size_t)r * (size_t)N * 4, st);
   if (coldot_mma_ok(P, bf16, R, N, aux)) {  // tensor cores
-    const MmaPlan pl = coldot_mma_plan(R, N, tickets != nullptr);
+    const MmaPlan pl = coldot_mma_plan(R, N, r, tickets != nullptr);
     const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
     float* part = (float*)ws;
     switch (rank_tiles(r)) {

@@ -103,12 +103,13 @@ struct Cfg {
                                 : (BN >= 256 ? 5 : BN >= 128 ? 4 : BN >= 64 ? 6 : BN >= 32 ? 8 : 12);
   static_assert(NIN % G == 0, "a TMA group fills whole ring slots");
   static constexpr int NDEC = DX ? (BN >= 256 ? 3 : 2) : (BN >= 128 ? 4 : 6);
+  static_assert(NDEC <= NIN, "decoded slots are released through the in-ring barriers");
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr int kTmemCols = pow2_at_least(DX ? kAccCols : kAccCols + NDEC * 32);
   static constexpr int kWdec = DX ? NDEC * kWTile : 0;
   static constexpr int kRing = NIN * (kAct + kPkTile) + kWdec;  // also the epilogue staging
   static constexpr int kAdx = G > 1 ? (kAct + 1023) / 1024 * 1024 : 0;
-  static constexpr int kBars = 8 * (2 * NIN + 2 * NDEC + 2) + 16;
+  static constexpr int kBars = 8 * (2 * NIN + NDEC + 2) + 16;
   static constexpr int kSmem = 1024 + kRing + kWTile + kAdx + kBars;
   static constexpr int kMinCtas = BN >= 256 ? 1 : 2;
   static_assert(kMinCtas == 1 || (kSmem <= 113 * 1024 && 2 * kTmemCols <= 512),
@@ -295,10 +296,9 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
   uint8_t* adx = adw + kWTile;                // G > 1: adapter token tile
   uint64_t* bars = (uint64_t*)(adx + C::kAdx);
   uint64_t* full_in = bars;                   // TMA landed (on the group's first slot)
-  uint64_t* in_empty = bars + NIN;            // MMA done with the in-ring stage
+  uint64_t* in_empty = bars + NIN;            // MMA done with the step of this stage
   uint64_t* dec_full = bars + 2 * NIN;        // decoded tile written (4 warps)
-  uint64_t* dec_empty = bars + 2 * NIN + NDEC;  // MMA done with the decoded tile
-  uint64_t* acc_full = bars + 2 * NIN + 2 * NDEC;
+  uint64_t* acc_full = bars + 2 * NIN + NDEC;
   uint64_t* ad_full = acc_full + 1;           // G > 1: adapter operands landed
   volatile uint32_t* tmem_slot = (volatile uint32_t*)(ad_full + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
@@ -322,7 +322,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     }
     for (int d = 0; d < NDEC; ++d) {
       mbar_init(smem_u32(&dec_full[d]), 4);  // the 4 warps of one decoder group
-      mbar_init(smem_u32(&dec_empty[d]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
     mbar_init(smem_u32(ad_full), 1);
@@ -421,10 +420,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       bool ok = true;
       for (int it = 0; it < nk; ++it) {
         if ((it & 7) == 0 && *abort_flag) { ok = false; break; }
-        const uint32_t fb = smem_u32(&full_in[s - s % G]), db = smem_u32(&dec_full[d]);
-        const bool ready = mbar_test(fb, ph_in) & mbar_test(db, ph_dec);
-        if (!ready && (!mbar_wait(fb, ph_in, p.wait_ns, p.err, 0x201) ||
-                       !mbar_wait(db, ph_dec, p.wait_ns, p.err, 0x202))) {
+        // The decoders waited for this step's TMA group (token and packed
+        // tiles land on the same barrier) before they arrived on dec_full,
+        // so dec_full alone orders the MMA after both copies.
+        const uint32_t db = smem_u32(&dec_full[d]);
+        if (!mbar_wait(db, ph_dec, p.wait_ns, p.err, 0x202)) {
           *abort_flag = 1;
           ok = false;
           break;
@@ -441,8 +441,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
             umma_bf16(tmem, adesc0 + (uint64_t)((uint32_t)(d * kWTile + kk * 2048) >> 4),
                       bd + 2 * kk, kIdesc, acc);
         }
-        umma_commit(smem_u32(&in_empty[s]));
-        umma_commit(smem_u32(&dec_empty[d]));
+        umma_commit(smem_u32(&in_empty[s]));  // frees the in-ring stage and, NDEC steps on, the decoded slot
         if (++s == NIN) { s = 0; ph_in ^= 1u; }
         if (++d == NDEC) { d = 0; ph_dec ^= 1u; }
       }
@@ -521,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     bool ok = true;
     // running ring positions of this group's steps (it = group, group + 2, ...)
     int s = group % NIN, d = group % NDEC;
-    uint32_t ph_in = 0, ph_dec = 0;
+    uint32_t ph_in = 0;
     for (int it = group; it < nk; it += kDecGroups) {
       const float sc = decode_block_scale(qw[0], tw[0], mu);
 #pragma unroll
@@ -538,10 +537,19 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
         }
       }
       if (((it >> 1) & 3) == 0 && __any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
-      const uint32_t eb = smem_u32(&dec_empty[d]), fb = smem_u32(&full_in[s - s % C::G]);
-      bool w_ok = mbar_test(eb, ph_dec ^ 1u) & mbar_test(fb, ph_in);
+      // Decoded slot d was last used by step it - NDEC; the MMA releases a
+      // step by committing to its in-ring stage barrier (NDEC <= NIN, so
+      // that barrier cannot have moved on by a further phase yet).
+      const uint32_t fb = smem_u32(&full_in[s - s % C::G]);
+      uint32_t eb = 0, ep = 0;
+      if (it >= NDEC) {
+        const int j = it - NDEC;
+        eb = smem_u32(&in_empty[j % NIN]);
+        ep = (uint32_t)((j / NIN) & 1);
+      }
+      bool w_ok = mbar_test(fb, ph_in) & (eb == 0 || mbar_test(eb, ep));
       if (!w_ok)
-        w_ok = mbar_wait(eb, ph_dec ^ 1u, p.wait_ns, p.err, 0x301) &&
+        w_ok = (eb == 0 || mbar_wait(eb, ep, p.wait_ns, p.err, 0x301)) &&
                mbar_wait(fb, ph_in, p.wait_ns, p.err, 0x302);
       if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
       const uint8_t* src = pk + s * kPkTile;
@@ -561,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       s += kDecGroups;
       if (s >= NIN) { s -= NIN; ph_in ^= 1u; }
       d += kDecGroups;
-      if (d >= NDEC) { d -= NDEC; ph_dec ^= 1u; }
+      if (d >= NDEC) d -= NDEC;
     }
     // the accumulator is complete once acc_full fires
     const bool acc_ok = mbar_wait(smem_u32(acc_full), 0, p.wait_ns, p.err, 0x401);
