@@ -996,6 +996,17 @@ cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const 
   if (R > 0 && rowdot_mma_ok(P, bf16, K, L)) {  // tensor cores, either factor layout
     const MmaPlan pl = rowdot_mma_plan(R, K, r, part_ws != nullptr && tickets != nullptr);
     const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
+    // A [K x r] factor is read in place, except over large activations
+    // with scratch for it: there one transposing launch (r*K floats) is
+    // repaid by the faster row-major factor path (measured 25-40% on
+    // 8192 x 4096 and 16384 x 17408 activations).
+    if (l_is_kr && lt_ws && R * K >= (int64_t)32 << 20 && ((uintptr_t)lt_ws % 16) == 0) {
+      transpose_kr_kernel<<<cdiv((int64_t)r * K, 256), 256, 0, st>>>(L, K, r, lt_ws);
+      count_launch();
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+      return rowdot_mma_r<false>(Pb, R, K, lt_ws, r, pl, out, pad, part_ws, tickets, job, st);
+    }
     if (l_is_kr) return rowdot_mma_r<true>(Pb, R, K, L, r, pl, out, pad, part_ws, tickets, job, st);
     return rowdot_mma_r<false>(Pb, R, K, L, r, pl, out, pad, part_ws, tickets, job, st);
   }

@@ -158,10 +158,36 @@ def test_bf16_qwen_attention_full():
         _check(_run_layer(wl, li), TOL["bf16"])
 
 
-@pytest.mark.parametrize("R", [1, 16, 100, 128, 130, 256, 1000])
+@pytest.mark.parametrize("R", [1, 16, 17, 31, 32, 48, 64, 100, 128, 130, 256, 1000])
 def test_bf16_ragged_token_counts(R):
+    # 16/32-token tiles (TMA loads of 4 and 2 K steps, adapter tile outside
+    # the ring), 64..256-token tiles, split-K and not, ragged last tile
     wl = synth.workload("qwen3_0.6b_attn_qv", R=R)
     _check(_run_layer(wl, 1), TOL["bf16"])
+
+
+@pytest.mark.parametrize("R", [24, 200])
+def test_bf16_ragged_token_counts_wide_output(R):
+    wl = synth.workload("qwen3_0.6b_attn_qv", R=R)
+    _check(_run_layer(wl, 0), TOL["bf16"])
+
+
+@pytest.mark.parametrize("R", [16, 4096])
+def test_bf16_linear_is_deterministic(R):
+    """Split-K partials and the side-product split partials are reduced in a
+    fixed order: two runs on the same inputs agree bit for bit."""
+    wl = synth.workload("qwen3_0.6b_attn_qv", R=R)
+    d = layer_inputs(wl, 0)
+    gw = q.qlora_quantize_nf4(to_dev_f32(d["W"]))
+    A, B = to_dev_f32(d["A"]), to_dev_f32(d["B"])
+    outs = []
+    for _ in range(2):
+        Y, U = q.qlora_linear_fwd(gw, d["xd"], A, B, wl.alpha)
+        dX, dA, dB = q.qlora_linear_bwd(gw, d["xd"], d["dyd"], A, B, wl.alpha, U=U)
+        torch.cuda.synchronize()
+        outs.append([bf16_bits_of(Y), U.cpu().numpy(), bf16_bits_of(dX), dA.cpu().numpy(), dB.cpu().numpy()])
+    for a, b in zip(outs[0], outs[1]):
+        assert np.array_equal(a, b)
 
 
 def test_bf16_identity_input_recovers_decoded_weight_bitwise():
