@@ -480,6 +480,35 @@ __device__ __forceinline__ void sum_slices(const float* __restrict__ part, int64
   }
 }
 
+// c += A * (B_hi + B_lo) for one n-tile from a split tile in shared memory:
+// hi row n at t + n * ls, lo row n at t + lo_off + n * ls (bf16, k contiguous).
+__device__ __forceinline__ void mma_pairs(float (&c)[4], const uint32_t (&a)[4], const uint16_t* t,
+                                          int ls, int lo_off, int n, int kb) {
+  const uint16_t* h = t + n * ls + kb;
+  const uint16_t* l = h + lo_off;
+  mma16816(c, a, *reinterpret_cast<const uint32_t*>(h), *reinterpret_cast<const uint32_t*>(h + 8));
+  mma16816(c, a, *reinterpret_cast<const uint32_t*>(l), *reinterpret_cast<const uint32_t*>(l + 8));
+}
+
+// Split an r-wide fp32 factor into bf16 hi / lo rows, n-major:
+// dst[j * ld + k] = hi, dst[(NP + j) * ld + k] = lo of F(k, j), where
+// F(k, j) = src[k * r + j] (nr = 1, [n x r]) or src[j * n + k] (nr = 0,
+// [r x n]); zero for j >= r or k >= n, up to the row length ld.
+__global__ void split_factor_kernel(const float* __restrict__ src, int64_t n, int r, int nr, int NP,
+                                    int64_t ld, uint16_t* __restrict__ dst) {
+  const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 2;  // (j, k) pair start
+  if (e >= (int64_t)NP * ld) return;
+  const int64_t j = e / ld, k = e - j * ld;
+  auto f = [&](int64_t kk) -> float {
+    if (j >= r || kk >= n) return 0.0f;
+    return nr ? src[kk * r + j] : src[j * n + kk];
+  };
+  uint32_t h, l;
+  split_bf16(f(k), f(k + 1), h, l);
+  *reinterpret_cast<uint32_t*>(dst + j * ld + k) = h;
+  *reinterpret_cast<uint32_t*>(dst + ((int64_t)NP + j) * ld + k) = l;
+}
+
 // rowdot on the tensor cores: out[m, j] = sum_k P[m, k] L(k, j).
 // Block = 8 warps = 4 row groups (16 rows each, 64 rows per block) x 2 K
 // groups (alternate 16-column chunks); a stage holds KT = 128 columns of
@@ -494,15 +523,21 @@ __device__ __forceinline__ void sum_slices(const float* __restrict__ part, int64
 constexpr int rowmma_kt(int nt) { return nt >= 4 ? 64 : 128; }
 constexpr int colmma_rt(int nt) { return nt >= 4 ? 32 : 64; }
 
-template <int NT, bool LKR>
+// Factor modes: FM 0 fp32 [r x K] rows (A), FM 1 fp32 [K x r] (B), FM 2 the
+// factor already split into bf16 hi / lo rows [2][NP][lstride] (n-major,
+// zero past r and K) by split_factor_kernel: B fragments are then plain
+// bf16 pairs, no per-warp split arithmetic.
+template <int NT, int FM>
 struct RowMma {
+  static constexpr bool LKR = FM == 1;
   static constexpr int RB = 64, KT = rowmma_kt(NT);
   static constexpr int PCH = KT / 8;                   // 16-byte chunks per P row
   static constexpr int NP = 8 * NT;                    // padded rank
   static constexpr int PSTR = KT * 2 + 16;             // bytes per P row in smem
   static constexpr int PB = RB * PSTR;
   static constexpr int LSTRF = KT + 8;                 // floats per L row ([r x K] case)
-  static constexpr int LB = LKR ? KT * NP * 4 : NP * LSTRF * 4;
+  static constexpr int LSTRH = KT + 8;                 // bf16 per split row (FM 2)
+  static constexpr int LB = FM == 2 ? 2 * NP * LSTRH * 2 : LKR ? KT * NP * 4 : NP * LSTRF * 4;
   static constexpr int STAGE = PB + LB;
   static constexpr int TSTR = NP + 1;                  // result tile row stride (floats)
   static constexpr int RED = 4 * 32 * NT * 4 * 4;      // K-group combine buffer
@@ -510,19 +545,20 @@ struct RowMma {
   static constexpr int SMEM = kMmaStages * STAGE + (RED > TILE ? RED : TILE);
 };
 
-template <int NT, bool LKR>
+template <int NT, int FM>
 __global__ void __launch_bounds__(kThreads) rowdot_mma_kernel(
     const __nv_bfloat16* __restrict__ P, int64_t R, int64_t K, const float* __restrict__ L,
-    int r, int row_blocks, int ksplit, int tiles_per_split, float* __restrict__ out,
-    uint16_t* __restrict__ out_pad, float* __restrict__ part, unsigned* __restrict__ tickets,
-    PadJob job) {
+    int64_t lstride, int r, int row_blocks, int ksplit, int tiles_per_split,
+    float* __restrict__ out, uint16_t* __restrict__ out_pad, float* __restrict__ part,
+    unsigned* __restrict__ tickets, PadJob job) {
+  constexpr bool LKR = FM == 1;
   // the tensor-core kernel queued next may start its weight stream now
   if (threadIdx.x == 0) griddep_launch_dependents();
   if ((int)blockIdx.x >= row_blocks * ksplit) {
     run_pad_job(job, (int64_t)blockIdx.x - row_blocks * ksplit);
     return;
   }
-  using C = RowMma<NT, LKR>;
+  using C = RowMma<NT, FM>;
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -544,7 +580,17 @@ __global__ void __launch_bounds__(kThreads) rowdot_mma_kernel(
       const uint32_t nb = (m < R && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
       cp_async16(ps + (uint32_t)(row * C::PSTR + ch * 16), nb ? (const void*)(P + m * K + k) : (const void*)P, nb);
     }
-    if (LKR) {  // contiguous [KT x r] floats
+    if (FM == 2) {  // split rows: 2 x NP rows of KT bf16
+      const uint16_t* Ls = reinterpret_cast<const uint16_t*>(L);
+      for (int c = threadIdx.x; c < 2 * C::NP * (C::KT / 8); c += kThreads) {
+        const int row = c / (C::KT / 8), ch = c % (C::KT / 8);
+        const int64_t k = k0 + ch * 8;
+        const int64_t rem = (lstride - k) * 2;
+        const uint32_t nb = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
+        cp_async16(ls + (uint32_t)(row * C::LSTRH + ch * 8) * 2,
+                   nb ? (const void*)(Ls + row * lstride + k) : (const void*)Ls, nb);
+      }
+    } else if (LKR) {  // contiguous [KT x r] floats
       const int64_t base = k0 * r, total = K * (int64_t)r;
       const int nch = (C::KT * r) / 4;
       for (int c = threadIdx.x; c < nch; c += kThreads) {
@@ -592,7 +638,10 @@ __global__ void __launch_bounds__(kThreads) rowdot_mma_kernel(
       const int kb = kc * 16 + 2 * tq;
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        if (LKR)
+        if (FM == 2)
+          mma_pairs(c[n], a, reinterpret_cast<const uint16_t*>(ls), C::LSTRH, C::NP * C::LSTRH,
+                    8 * n + g, kb);
+        else if (LKR)
           mma_split(c[n], a, kb, 8 * n + g,
                     [&](int k, int j) { return j < r ? ls[k * r + j] : 0.0f; });
         else
@@ -663,25 +712,28 @@ __global__ void __launch_bounds__(kThreads) rowdot_mma_kernel(
 // grid = column blocks x row splits, the last block of a column block to
 // finish (ticket) adds the split partials in split order, scales by s and
 // writes dA as [r x N] (out_nr = 0) or dB as [N x r] (out_nr = 1).
-template <int NT>
+// Aux modes: FM 0 fp32 [R x r]; FM 2 split into bf16 hi / lo rows (as for
+// the rowdot factor).
+template <int NT, int FM>
 struct ColMma {
   static constexpr int NC = 128, RT = colmma_rt(NT);
   static constexpr int NP = 8 * NT;
   static constexpr int PSTR = NC * 2 + 16;
   static constexpr int PB = RT * PSTR;
-  static constexpr int AB = RT * NP * 4;               // aux tile [RT x r] (stride r)
+  static constexpr int ASTRH = RT + 8;                 // bf16 per split row (FM 2)
+  static constexpr int AB = FM == 2 ? 2 * NP * ASTRH * 2 : RT * NP * 4;  // aux tile
   static constexpr int STAGE = PB + AB;
   static constexpr int TSTR = NP + 1;
   static constexpr int TILE = NC * TSTR * 4;
   static constexpr int SMEM = kMmaStages * STAGE + TILE;
 };
 
-template <int NT>
+template <int NT, int FM>
 __global__ void __launch_bounds__(kThreads) coldot_mma_kernel(
     const __nv_bfloat16* __restrict__ P, int64_t R, int64_t N, const float* __restrict__ aux,
-    int r, int col_blocks, int splits, int tiles_per_split, float s, int out_nr,
+    int64_t astride, int r, int col_blocks, int splits, int tiles_per_split, float s, int out_nr,
     float* __restrict__ out, float* __restrict__ part, unsigned* __restrict__ tickets) {
-  using C = ColMma<NT>;
+  using C = ColMma<NT, FM>;
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -702,13 +754,25 @@ __global__ void __launch_bounds__(kThreads) coldot_mma_kernel(
       const uint32_t nb = (m < R && rem > 0) ? (uint32_t)min((int64_t)16, rem) : 0u;
       cp_async16(ps + (uint32_t)(row * C::PSTR + ch * 16), nb ? (const void*)(P + m * N + n) : (const void*)P, nb);
     }
-    const int64_t base = mt * r, total = R * (int64_t)r;  // contiguous [RT x r]
-    const int nch = (C::RT * r) / 4;
-    for (int c = threadIdx.x; c < nch; c += kThreads) {
-      const int64_t e = base + (int64_t)c * 4;
-      const int64_t rem = (total - e) * 4;
-      const uint32_t nb = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
-      cp_async16(as + (uint32_t)c * 16, nb ? (const void*)(aux + e) : (const void*)aux, nb);
+    if (FM == 2) {  // split rows: 2 x NP rows of RT bf16
+      const uint16_t* As = reinterpret_cast<const uint16_t*>(aux);
+      for (int c = threadIdx.x; c < 2 * C::NP * (C::RT / 8); c += kThreads) {
+        const int row = c / (C::RT / 8), ch = c % (C::RT / 8);
+        const int64_t m = mt + ch * 8;
+        const int64_t rem = (astride - m) * 2;
+        const uint32_t nb = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
+        cp_async16(as + (uint32_t)(row * C::ASTRH + ch * 8) * 2,
+                   nb ? (const void*)(As + row * astride + m) : (const void*)As, nb);
+      }
+    } else {
+      const int64_t base = mt * r, total = R * (int64_t)r;  // contiguous [RT x r]
+      const int nch = (C::RT * r) / 4;
+      for (int c = threadIdx.x; c < nch; c += kThreads) {
+        const int64_t e = base + (int64_t)c * 4;
+        const int64_t rem = (total - e) * 4;
+        const uint32_t nb = rem > 0 ? (uint32_t)min((int64_t)16, rem) : 0u;
+        cp_async16(as + (uint32_t)c * 16, nb ? (const void*)(aux + e) : (const void*)aux, nb);
+      }
     }
   };
 
@@ -738,9 +802,14 @@ __global__ void __launch_bounds__(kThreads) coldot_mma_kernel(
       ldsm_x4_t(ps + (uint32_t)((kc * 16 + lrow) * C::PSTR + lcol * 2), a);
       const int kb = kc * 16 + 2 * tq;
 #pragma unroll
-      for (int n = 0; n < NT; ++n)
-        mma_split(c[n], a, kb, 8 * n + g,
-                  [&](int k, int j) { return j < r ? as[k * r + j] : 0.0f; });
+      for (int n = 0; n < NT; ++n) {
+        if (FM == 2)
+          mma_pairs(c[n], a, reinterpret_cast<const uint16_t*>(as), C::ASTRH, C::NP * C::ASTRH,
+                    8 * n + g, kb);
+        else
+          mma_split(c[n], a, kb, 8 * n + g,
+                    [&](int k, int j) { return j < r ? as[k * r + j] : 0.0f; });
+      }
     }
   }
   cp_async_wait<0>();
@@ -939,47 +1008,59 @@ bool rowdot_mma_ok(const void* P, bool bf16, int64_t K, const float* L) {
   return bf16 && (K % 8) == 0 && ((uintptr_t)P % 16) == 0 && ((uintptr_t)L % 16) == 0;
 }
 
-template <int NT, bool LKR>
-cudaError_t rowdot_mma_go(const __nv_bfloat16* P, int64_t R, int64_t K, const float* L, int r,
-                          const MmaPlan& pl, float* out, uint16_t* pad, float* part,
-                          unsigned* tickets, PadJob job, cudaStream_t st) {
-  using C = RowMma<NT, LKR>;
+template <int NT, int FM>
+cudaError_t rowdot_mma_go(const __nv_bfloat16* P, int64_t R, int64_t K, const float* L,
+                          int64_t lstride, int r, const MmaPlan& pl, float* out, uint16_t* pad,
+                          float* part, unsigned* tickets, PadJob job, cudaStream_t st) {
+  using C = RowMma<NT, FM>;
   static bool attr = false;
-  auto kern = rowdot_mma_kernel<NT, LKR>;
+  auto kern = rowdot_mma_kernel<NT, FM>;
   cudaError_t e = set_smem_once(kern, C::SMEM, attr);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(pl.blocks * pl.splits + job.blocks);
   if (grid == 0) return cudaSuccess;
-  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, K, L, r, pl.blocks, pl.splits, pl.tiles_per_split,
-                                        out, pad, part, tickets, job);
+  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, K, L, lstride, r, pl.blocks, pl.splits,
+                                        pl.tiles_per_split, out, pad, part, tickets, job);
   count_launch();
   return cudaGetLastError();
 }
 
-template <bool LKR>
-cudaError_t rowdot_mma_r(const __nv_bfloat16* P, int64_t R, int64_t K, const float* L, int r,
-                         const MmaPlan& pl, float* out, uint16_t* pad, float* part,
-                         unsigned* tickets, PadJob job, cudaStream_t st) {
+template <int FM>
+cudaError_t rowdot_mma_r(const __nv_bfloat16* P, int64_t R, int64_t K, const float* L,
+                         int64_t lstride, int r, const MmaPlan& pl, float* out, uint16_t* pad,
+                         float* part, unsigned* tickets, PadJob job, cudaStream_t st) {
   switch (rank_tiles(r)) {
-    case 1: return rowdot_mma_go<1, LKR>(P, R, K, L, r, pl, out, pad, part, tickets, job, st);
-    case 2: return rowdot_mma_go<2, LKR>(P, R, K, L, r, pl, out, pad, part, tickets, job, st);
-    case 4: return rowdot_mma_go<4, LKR>(P, R, K, L, r, pl, out, pad, part, tickets, job, st);
-    default: return rowdot_mma_go<8, LKR>(P, R, K, L, r, pl, out, pad, part, tickets, job, st);
+    case 1: return rowdot_mma_go<1, FM>(P, R, K, L, lstride, r, pl, out, pad, part, tickets, job, st);
+    case 2: return rowdot_mma_go<2, FM>(P, R, K, L, lstride, r, pl, out, pad, part, tickets, job, st);
+    case 4: return rowdot_mma_go<4, FM>(P, R, K, L, lstride, r, pl, out, pad, part, tickets, job, st);
+    default: return rowdot_mma_go<8, FM>(P, R, K, L, lstride, r, pl, out, pad, part, tickets, job, st);
   }
 }
 
-template <int NT>
-cudaError_t coldot_mma_go(const __nv_bfloat16* P, int64_t R, int64_t N, const float* aux, int r,
-                          const MmaPlan& pl, float s, bool out_nr, float* out, float* part,
-                          unsigned* tickets, cudaStream_t st) {
-  using C = ColMma<NT>;
+// Split the r-wide factor of one product into bf16 hi / lo rows in `dst`
+// (row length ld = extent rounded up to 8).
+cudaError_t split_factor(const float* src, int64_t extent, int r, bool nr, uint16_t* dst,
+                         int64_t* ld, cudaStream_t st) {
+  const int NP = 8 * rank_tiles(r);
+  *ld = (extent + 7) / 8 * 8;
+  const int64_t pairs = (int64_t)NP * *ld / 2;
+  split_factor_kernel<<<cdiv(pairs, 256), 256, 0, st>>>(src, extent, r, nr ? 1 : 0, NP, *ld, dst);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int NT, int FM>
+cudaError_t coldot_mma_go(const __nv_bfloat16* P, int64_t R, int64_t N, const float* aux,
+                          int64_t astride, int r, const MmaPlan& pl, float s, bool out_nr,
+                          float* out, float* part, unsigned* tickets, cudaStream_t st) {
+  using C = ColMma<NT, FM>;
   static bool attr = false;
-  auto kern = coldot_mma_kernel<NT>;
+  auto kern = coldot_mma_kernel<NT, FM>;
   cudaError_t e = set_smem_once(kern, C::SMEM, attr);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)pl.blocks, (unsigned)pl.splits);
-  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, N, aux, r, pl.blocks, pl.splits, pl.tiles_per_split,
-                                        s, out_nr ? 1 : 0, out, part, tickets);
+  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, N, aux, astride, r, pl.blocks, pl.splits,
+                                        pl.tiles_per_split, s, out_nr ? 1 : 0, out, part, tickets);
   count_launch();
   return cudaGetLastError();
 }
@@ -990,7 +1071,7 @@ cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const 
                           bool l_is_kr, int32_t r, float* out, cudaStream_t st, uint16_t* pad,
                           const float* side_src, int64_t side_extent, int side_mode,
                           float side_mul, uint16_t* side_dst, float* lt_ws, float* part_ws,
-                          unsigned* tickets) {
+                          unsigned* tickets, uint16_t* split_ws) {
   PadJob job{side_src, side_dst, side_extent, r, side_mode, side_mul, 0};
   if (side_dst && side_extent > 0) job.blocks = (int)cdiv(64 * side_extent, kThreads * 8);
   if (R > 0 && rowdot_mma_ok(P, bf16, K, L)) {  // tensor cores, either factor layout
@@ -1000,15 +1081,24 @@ cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const 
     // with scratch for it: there one transposing launch (r*K floats) is
     // repaid by the faster row-major factor path (measured 25-40% on
     // 8192 x 4096 and 16384 x 17408 activations).
+    // Above rank 8, one small launch splits the factor into bf16 hi / lo
+    // rows once, instead of every warp of every block splitting it again.
+    if (split_ws && rank_tiles(r) >= 2 && ((uintptr_t)split_ws % 16) == 0) {
+      int64_t ld = 0;
+      cudaError_t e = split_factor(L, K, r, l_is_kr, split_ws, &ld, st);
+      if (e != cudaSuccess) return e;
+      return rowdot_mma_r<2>(Pb, R, K, (const float*)split_ws, ld, r, pl, out, pad, part_ws,
+                             tickets, job, st);
+    }
     if (l_is_kr && lt_ws && R * K >= (int64_t)32 << 20 && ((uintptr_t)lt_ws % 16) == 0) {
       transpose_kr_kernel<<<cdiv((int64_t)r * K, 256), 256, 0, st>>>(L, K, r, lt_ws);
       count_launch();
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
-      return rowdot_mma_r<false>(Pb, R, K, lt_ws, r, pl, out, pad, part_ws, tickets, job, st);
+      return rowdot_mma_r<0>(Pb, R, K, lt_ws, 0, r, pl, out, pad, part_ws, tickets, job, st);
     }
-    if (l_is_kr) return rowdot_mma_r<true>(Pb, R, K, L, r, pl, out, pad, part_ws, tickets, job, st);
-    return rowdot_mma_r<false>(Pb, R, K, L, r, pl, out, pad, part_ws, tickets, job, st);
+    if (l_is_kr) return rowdot_mma_r<1>(Pb, R, K, L, 0, r, pl, out, pad, part_ws, tickets, job, st);
+    return rowdot_mma_r<0>(Pb, R, K, L, 0, r, pl, out, pad, part_ws, tickets, job, st);
   }
   // With scratch for it, a factor given as [K x r] is transposed first so
   // every path below reads factor rows ([r x K]) contiguously.
@@ -1034,6 +1124,11 @@ bool coldot_mma_ok(const void* P, bool bf16, int64_t R, int64_t N, const float* 
 
 }  // namespace
 
+size_t adapter_split_ws(int64_t extent, int32_t r) {
+  if (rank_tiles(r) < 2) return 0;
+  return align_up((size_t)2 * 8 * rank_tiles(r) * (size_t)((extent + 7) / 8 * 8) * 2, 256);
+}
+
 size_t rowdot_ws(int64_t R, int64_t K, int32_t r) {
   const MmaPlan pl = rowdot_mma_plan(R, K, r, true);
   return pl.splits > 1 ? align_up((size_t)pl.splits * (size_t)R * 8 * rank_tiles(r) * 4, 256) : 0;
@@ -1054,18 +1149,29 @@ size_t coldot_ws(int64_t R, int64_t N, int32_t r) {
 
 cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
                           int32_t r, float s, bool out_nr, float* out, void* ws,
-                          cudaStream_t st, unsigned* tickets) {
+                          cudaStream_t st, unsigned* tickets, uint16_t* split_ws) {
   if (N == 0) return cudaSuccess;
   if (R == 0) return cudaMemsetAsync(out, 0, (size_t)r * (size_t)N * 4, st);
   if (coldot_mma_ok(P, bf16, R, N, aux)) {  // tensor cores
     const MmaPlan pl = coldot_mma_plan(R, N, r, tickets != nullptr);
     const __nv_bfloat16* Pb = (const __nv_bfloat16*)P;
     float* part = (float*)ws;
+    if (split_ws && rank_tiles(r) >= 2 && ((uintptr_t)split_ws % 16) == 0) {
+      int64_t ld = 0;
+      cudaError_t e = split_factor(aux, R, r, true, split_ws, &ld, st);
+      if (e != cudaSuccess) return e;
+      const float* sp = (const float*)split_ws;
+      switch (rank_tiles(r)) {
+        case 2: return coldot_mma_go<2, 2>(Pb, R, N, sp, ld, r, pl, s, out_nr, out, part, tickets, st);
+        case 4: return coldot_mma_go<4, 2>(Pb, R, N, sp, ld, r, pl, s, out_nr, out, part, tickets, st);
+        default: return coldot_mma_go<8, 2>(Pb, R, N, sp, ld, r, pl, s, out_nr, out, part, tickets, st);
+      }
+    }
     switch (rank_tiles(r)) {
-      case 1: return coldot_mma_go<1>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
-      case 2: return coldot_mma_go<2>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
-      case 4: return coldot_mma_go<4>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
-      default: return coldot_mma_go<8>(Pb, R, N, aux, r, pl, s, out_nr, out, part, tickets, st);
+      case 1: return coldot_mma_go<1, 0>(Pb, R, N, aux, 0, r, pl, s, out_nr, out, part, tickets, st);
+      case 2: return coldot_mma_go<2, 0>(Pb, R, N, aux, 0, r, pl, s, out_nr, out, part, tickets, st);
+      case 4: return coldot_mma_go<4, 0>(Pb, R, N, aux, 0, r, pl, s, out_nr, out, part, tickets, st);
+      default: return coldot_mma_go<8, 0>(Pb, R, N, aux, 0, r, pl, s, out_nr, out, part, tickets, st);
     }
   }
   const ColPlan c = col_plan(R, N, r);

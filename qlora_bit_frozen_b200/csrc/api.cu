@@ -141,10 +141,10 @@ WView view_of(const qlora_weight* w) {
 constexpr size_t kWsZeroed = kWsHeader + kWsTickets;
 
 struct FwdLayout {
-  size_t u = 0, red = 0, tc = 0, total = 0;
+  size_t u = 0, red = 0, split = 0, tc = 0, total = 0;
 };
 struct BwdLayout {
-  size_t u = 0, v = 0, bt = 0, red = 0, tc = 0, total = 0;
+  size_t u = 0, v = 0, bt = 0, red = 0, split = 0, tc = 0, total = 0;
 };
 
 FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t compute) {
@@ -154,6 +154,8 @@ FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
   off += align_up((size_t)R * r * 4, 256);
   L.red = off;  // split partials of U = X A^T
   off += rowdot_ws(R, w->I, r);
+  L.split = off;  // bf16 hi / lo copy of A (above rank 8)
+  off += adapter_split_ws(w->I, r);
   L.tc = off;
   if (compute == QLORA_COMPUTE_BF16) off += tc_fwd_ws(view_of(w), R);
   L.total = off;
@@ -176,6 +178,12 @@ BwdLayout bwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
   for (size_t m : more)
     if (m > red) red = m;
   off += red;
+  L.split = off;  // bf16 hi / lo copy of B, V, A or U (one at a time)
+  size_t sp = adapter_split_ws(w->O, r);
+  const size_t sps[2] = {adapter_split_ws(w->I, r), adapter_split_ws(R, r)};
+  for (size_t m : sps)
+    if (m > sp) sp = m;
+  off += sp;
   L.tc = off;
   if (compute == QLORA_COMPUTE_BF16) off += tc_dx_ws(view_of(w), R);
   L.total = off;
@@ -326,7 +334,7 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
   if (bf16 && tc_fwd_supported(v, X, Y, R)) {
     void* tcws = (char*)ws + L.tc;
     e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws), B, w->O, 0, sc,
-                      tc_w_pad(tcws, R), nullptr, red, tickets);
+                      tc_w_pad(tcws, R), nullptr, red, tickets, (uint16_t*)((char*)ws + L.split));
     if (e == cudaSuccess) e = launch_tc_fwd(v, X, R, U, B, r, sc, Y, tcws, (uint32_t*)ws, s);
   } else {
     e = launch_simt_fwd(v, X, R, A, B, r, sc, bf16, Y, U, s);
@@ -362,12 +370,13 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   if (dX || dA) {
     float* bt = (float*)((char*)ws + L.bt);
     float* part = (float*)red;
+    uint16_t* split = (uint16_t*)((char*)ws + L.split);
     if (tc)
       e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, tc_act_pad(tcws), A, w->I, 1, sc,
-                        tc_w_pad(tcws, R), bt, part, tickets);
+                        tc_w_pad(tcws, R), bt, part, tickets, split);
     else
       e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, nullptr, nullptr, 0, 0, 1.0f,
-                        nullptr, bt, part, tickets);
+                        nullptr, bt, part, tickets, split);
   }
   if (e == cudaSuccess && dX) {
     if (tc)
@@ -376,19 +385,20 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
       e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s);
   }
   // dA = s V^T X   [r x I]
+  uint16_t* split = (uint16_t*)((char*)ws + L.split);
   if (e == cudaSuccess && dA)
-    e = launch_coldot(X, bf16, R, w->I, V, r, sc, false, dA, red, s, tickets);
+    e = launch_coldot(X, bf16, R, w->I, V, r, sc, false, dA, red, s, tickets, split);
   // dB = s dY^T U  [O x r]
   if (e == cudaSuccess && dB) {
     const float* U = U_in;
     if (!U) {
       float* Uw = (float*)((char*)ws + L.u);
       e = launch_rowdot(X, bf16, R, w->I, A, false, r, Uw, s, nullptr, nullptr, 0, 0, 1.0f,
-                        nullptr, nullptr, (float*)red, tickets);
+                        nullptr, nullptr, (float*)red, tickets, split);
       U = Uw;
     }
     if (e == cudaSuccess)
-      e = launch_coldot(dY, bf16, R, w->O, U, r, sc, true, dB, red, s, tickets);
+      e = launch_coldot(dY, bf16, R, w->O, U, r, sc, true, dB, red, s, tickets, split);
   }
   return cuda_status(e);
 }

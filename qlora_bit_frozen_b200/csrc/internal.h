@@ -55,15 +55,21 @@ cudaError_t launch_rowdot(const void* P, bool bf16, int64_t R, int64_t K, const 
                           uint16_t* pad = nullptr, const float* side_src = nullptr,
                           int64_t side_extent = 0, int side_mode = 0, float side_mul = 1.0f,
                           uint16_t* side_dst = nullptr, float* lt_ws = nullptr,
-                          float* part_ws = nullptr, unsigned* tickets = nullptr);
+                          float* part_ws = nullptr, unsigned* tickets = nullptr,
+                          uint16_t* split_ws = nullptr);
 // part_ws (rowdot_ws bytes) and tickets (kWsTickets bytes, zero on entry
 // and left zero) let the bf16 tensor-core path split K across blocks.
 size_t rowdot_ws(int64_t R, int64_t K, int32_t r);
+// split_ws (adapter_split_ws(extent, r) bytes, nullable): scratch for the
+// bf16 hi / lo copy of the r-wide operand (factor over K, or U / V over R)
+// that the tensor-core side products read above rank 8.
+size_t adapter_split_ws(int64_t extent, int32_t r);
 size_t coldot_ws(int64_t R, int64_t N, int32_t r);
 // tickets: as for launch_rowdot (nullptr: no row splits on the tensor-core path)
 cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const float* aux,
                           int32_t r, float s, bool out_nr, float* out, void* ws,
-                          cudaStream_t st, unsigned* tickets = nullptr);
+                          cudaStream_t st, unsigned* tickets = nullptr,
+                          uint16_t* split_ws = nullptr);
 // out = scale * sum of the split partials.  pdl: launched with a
 // programmatic dependency on the kernel before it (which must have
 // triggered its dependents); the kernel waits for that grid first.
