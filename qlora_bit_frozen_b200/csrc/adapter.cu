@@ -728,16 +728,43 @@ struct ColMma {
   static constexpr int SMEM = kMmaStages * STAGE + TILE;
 };
 
+// One coldot product: out(j, n) = s sum_m aux[m, j] P[m, n] over column
+// blocks x row splits, with its own partial buffer and ticket counters.
+struct ColJob {
+  const __nv_bfloat16* P;
+  int64_t R, N;
+  const float* aux;
+  int64_t astride;
+  int r, col_blocks, splits, tiles_per_split;
+  float s;
+  int out_nr;
+  float* out;
+  float* part;
+  unsigned* tickets;
+};
+
+// Grid = the blocks of job a, then those of job b (col_blocks = 0: none):
+// the two side products of a backward pass, dA and dB, share one launch.
 template <int NT, int FM>
-__global__ void __launch_bounds__(kThreads) coldot_mma_kernel(
-    const __nv_bfloat16* __restrict__ P, int64_t R, int64_t N, const float* __restrict__ aux,
-    int64_t astride, int r, int col_blocks, int splits, int tiles_per_split, float s, int out_nr,
-    float* __restrict__ out, float* __restrict__ part, unsigned* __restrict__ tickets) {
+__global__ void __launch_bounds__(kThreads) coldot_mma_kernel(const ColJob ja, const ColJob jb) {
   using C = ColMma<NT, FM>;
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;
+  const int na = ja.col_blocks * ja.splits;
+  const bool first = (int)blockIdx.x < na;
+  const ColJob& jo = first ? ja : jb;
+  const int lb = first ? (int)blockIdx.x : (int)blockIdx.x - na;
+  const __nv_bfloat16* __restrict__ P = jo.P;
+  const int64_t R = jo.R, N = jo.N, astride = jo.astride;
+  const float* __restrict__ aux = jo.aux;
+  const int r = jo.r, splits = jo.splits, tiles_per_split = jo.tiles_per_split;
+  const float s = jo.s;
+  const int out_nr = jo.out_nr;
+  float* __restrict__ out = jo.out;
+  float* __restrict__ part = jo.part;
+  unsigned* __restrict__ tickets = jo.tickets;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cb = (int)blockIdx.x, sp = (int)blockIdx.y;
+  const int cb = lb % jo.col_blocks, sp = lb / jo.col_blocks;
   const int64_t n0 = (int64_t)cb * C::NC;
   const int ntiles = (int)((R + C::RT - 1) / C::RT);
   const int t_lo = sp * tiles_per_split, t_hi = min(ntiles, t_lo + tiles_per_split);
@@ -1049,21 +1076,49 @@ cudaError_t split_factor(const float* src, int64_t extent, int r, bool nr, uint1
   return cudaGetLastError();
 }
 
+ColJob col_job(const __nv_bfloat16* P, int64_t R, int64_t N, const float* aux, int64_t astride,
+               int r, const MmaPlan& pl, float s, bool out_nr, float* out, float* part,
+               unsigned* tickets) {
+  ColJob j;
+  j.P = P;
+  j.R = R;
+  j.N = N;
+  j.aux = aux;
+  j.astride = astride;
+  j.r = r;
+  j.col_blocks = pl.blocks;
+  j.splits = pl.splits;
+  j.tiles_per_split = pl.tiles_per_split;
+  j.s = s;
+  j.out_nr = out_nr ? 1 : 0;
+  j.out = out;
+  j.part = part;
+  j.tickets = tickets;
+  return j;
+}
+
 template <int NT, int FM>
-cudaError_t coldot_mma_go(const __nv_bfloat16* P, int64_t R, int64_t N, const float* aux,
-                          int64_t astride, int r, const MmaPlan& pl, float s, bool out_nr,
-                          float* out, float* part, unsigned* tickets, cudaStream_t st) {
+cudaError_t coldot_mma_pair_go(const ColJob& ja, const ColJob& jb, cudaStream_t st) {
   using C = ColMma<NT, FM>;
   static bool attr = false;
   auto kern = coldot_mma_kernel<NT, FM>;
   cudaError_t e = set_smem_once(kern, C::SMEM, attr);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)pl.blocks, (unsigned)pl.splits);
-  kern<<<grid, kThreads, C::SMEM, st>>>(P, R, N, aux, astride, r, pl.blocks, pl.splits,
-                                        pl.tiles_per_split, s, out_nr ? 1 : 0, out, part, tickets);
+  const unsigned grid = (unsigned)(ja.col_blocks * ja.splits + jb.col_blocks * jb.splits);
+  kern<<<grid, kThreads, C::SMEM, st>>>(ja, jb);
   count_launch();
   return cudaGetLastError();
 }
+
+template <int NT, int FM>
+cudaError_t coldot_mma_go(const __nv_bfloat16* P, int64_t R, int64_t N, const float* aux,
+                          int64_t astride, int r, const MmaPlan& pl, float s, bool out_nr,
+                          float* out, float* part, unsigned* tickets, cudaStream_t st) {
+  ColJob none = {};
+  return coldot_mma_pair_go<NT, FM>(
+      col_job(P, R, N, aux, astride, r, pl, s, out_nr, out, part, tickets), none, st);
+}
+
 
 }  // namespace
 
@@ -1187,6 +1242,47 @@ cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const 
     coldot_r<float>(P, R, N, aux, r, c, s, out_nr, part, slice_tickets, out, st);
   count_launch();
   return cudaGetLastError();
+}
+
+cudaError_t launch_coldot_pair(const void* PA, int64_t NA, const float* auxA, bool out_nrA,
+                               float* outA, void* wsA, uint16_t* splitA, const void* PB,
+                               int64_t NB, const float* auxB, bool out_nrB, float* outB, void* wsB,
+                               uint16_t* splitB, int64_t R, int32_t r, float s, cudaStream_t st,
+                               unsigned* tickets, bool* done) {
+  *done = false;
+  if (R <= 0 || NA <= 0 || NB <= 0 || !tickets) return cudaSuccess;
+  if (!coldot_mma_ok(PA, true, R, NA, auxA) || !coldot_mma_ok(PB, true, R, NB, auxB))
+    return cudaSuccess;
+  const MmaPlan pa = coldot_mma_plan(R, NA, r, true), pb = coldot_mma_plan(R, NB, r, true);
+  if (pa.blocks + pb.blocks > kMaxTickets) return cudaSuccess;
+  const __nv_bfloat16* A = (const __nv_bfloat16*)PA;
+  const __nv_bfloat16* B = (const __nv_bfloat16*)PB;
+  *done = true;
+  if (rank_tiles(r) >= 2 && splitA && splitB && ((uintptr_t)splitA % 16) == 0 &&
+      ((uintptr_t)splitB % 16) == 0) {
+    int64_t lda = 0, ldb = 0;
+    cudaError_t e = split_factor(auxA, R, r, true, splitA, &lda, st);
+    if (e == cudaSuccess) e = split_factor(auxB, R, r, true, splitB, &ldb, st);
+    if (e != cudaSuccess) return e;
+    const ColJob ja = col_job(A, R, NA, (const float*)splitA, lda, r, pa, s, out_nrA, outA,
+                              (float*)wsA, tickets);
+    const ColJob jb = col_job(B, R, NB, (const float*)splitB, ldb, r, pb, s, out_nrB, outB,
+                              (float*)wsB, tickets + pa.blocks);
+    switch (rank_tiles(r)) {
+      case 2: return coldot_mma_pair_go<2, 2>(ja, jb, st);
+      case 4: return coldot_mma_pair_go<4, 2>(ja, jb, st);
+      default: return coldot_mma_pair_go<8, 2>(ja, jb, st);
+    }
+  }
+  const ColJob ja = col_job(A, R, NA, auxA, 0, r, pa, s, out_nrA, outA, (float*)wsA, tickets);
+  const ColJob jb = col_job(B, R, NB, auxB, 0, r, pb, s, out_nrB, outB, (float*)wsB,
+                            tickets + pa.blocks);
+  switch (rank_tiles(r)) {
+    case 1: return coldot_mma_pair_go<1, 0>(ja, jb, st);
+    case 2: return coldot_mma_pair_go<2, 0>(ja, jb, st);
+    case 4: return coldot_mma_pair_go<4, 0>(ja, jb, st);
+    default: return coldot_mma_pair_go<8, 0>(ja, jb, st);
+  }
 }
 
 }  // namespace qlora

@@ -144,7 +144,7 @@ struct FwdLayout {
   size_t u = 0, red = 0, split = 0, tc = 0, total = 0;
 };
 struct BwdLayout {
-  size_t u = 0, v = 0, bt = 0, red = 0, split = 0, tc = 0, total = 0;
+  size_t u = 0, v = 0, bt = 0, red = 0, red2 = 0, split = 0, split2 = 0, tc = 0, total = 0;
 };
 
 FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t compute) {
@@ -184,6 +184,10 @@ BwdLayout bwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
   for (size_t m : sps)
     if (m > sp) sp = m;
   off += sp;
+  L.red2 = off;  // dB partials when dA and dB share a launch
+  off += coldot_ws(R, w->O, r);
+  L.split2 = off;  // bf16 hi / lo copy of U for that launch
+  off += adapter_split_ws(R, r);
   L.tc = off;
   if (compute == QLORA_COMPUTE_BF16) off += tc_dx_ws(view_of(w), R);
   L.total = off;
@@ -384,22 +388,25 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
     else
       e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s);
   }
-  // dA = s V^T X   [r x I]
+  // dA = s V^T X [r x I] and dB = s dY^T U [O x r]: one launch when both
+  // are wanted (two independent side products), else one each.
   uint16_t* split = (uint16_t*)((char*)ws + L.split);
-  if (e == cudaSuccess && dA)
-    e = launch_coldot(X, bf16, R, w->I, V, r, sc, false, dA, red, s, tickets, split);
-  // dB = s dY^T U  [O x r]
-  if (e == cudaSuccess && dB) {
-    const float* U = U_in;
-    if (!U) {
-      float* Uw = (float*)((char*)ws + L.u);
-      e = launch_rowdot(X, bf16, R, w->I, A, false, r, Uw, s, nullptr, nullptr, 0, 0, 1.0f,
-                        nullptr, nullptr, (float*)red, tickets, split);
-      U = Uw;
-    }
-    if (e == cudaSuccess)
-      e = launch_coldot(dY, bf16, R, w->O, U, r, sc, true, dB, red, s, tickets, split);
+  const float* U = U_in;
+  if (e == cudaSuccess && dB && !U) {
+    float* Uw = (float*)((char*)ws + L.u);
+    e = launch_rowdot(X, bf16, R, w->I, A, false, r, Uw, s, nullptr, nullptr, 0, 0, 1.0f,
+                      nullptr, nullptr, (float*)red, tickets, split);
+    U = Uw;
   }
+  bool paired = false;
+  if (e == cudaSuccess && dA && dB && bf16)
+    e = launch_coldot_pair(X, w->I, V, false, dA, red, split, dY, w->O, U, true, dB,
+                           (char*)ws + L.red2, (uint16_t*)((char*)ws + L.split2), R, r, sc, s,
+                           tickets, &paired);
+  if (e == cudaSuccess && dA && !paired)
+    e = launch_coldot(X, bf16, R, w->I, V, r, sc, false, dA, red, s, tickets, split);
+  if (e == cudaSuccess && dB && !paired)
+    e = launch_coldot(dY, bf16, R, w->O, U, r, sc, true, dB, red, s, tickets, split);
   return cuda_status(e);
 }
 

@@ -70,6 +70,16 @@ cudaError_t launch_coldot(const void* P, bool bf16, int64_t R, int64_t N, const 
                           int32_t r, float s, bool out_nr, float* out, void* ws,
                           cudaStream_t st, unsigned* tickets = nullptr,
                           uint16_t* split_ws = nullptr);
+// Two coldot products over the same R rows in one launch (the backward's
+// dA = s V^T X and dB = s dY^T U), each with its own partial buffer
+// (coldot_ws) and split scratch; *done = false (nothing launched) when the
+// tensor-core path does not apply to both, and the caller launches them one
+// by one.
+cudaError_t launch_coldot_pair(const void* PA, int64_t NA, const float* auxA, bool out_nrA,
+                               float* outA, void* wsA, uint16_t* splitA, const void* PB,
+                               int64_t NB, const float* auxB, bool out_nrB, float* outB, void* wsB,
+                               uint16_t* splitB, int64_t R, int32_t r, float s, cudaStream_t st,
+                               unsigned* tickets, bool* done);
 // out = scale * sum of the split partials.  pdl: launched with a
 // programmatic dependency on the kernel before it (which must have
 // triggered its dependents); the kernel waits for that grid first.
