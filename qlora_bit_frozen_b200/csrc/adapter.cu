@@ -747,6 +747,8 @@ struct ColJob {
 // the two side products of a backward pass, dA and dB, share one launch.
 template <int NT, int FM>
 __global__ void __launch_bounds__(kThreads) coldot_mma_kernel(const ColJob ja, const ColJob jb) {
+  // the input-gradient GEMM queued next may start its weight stream now
+  if (threadIdx.x == 0) griddep_launch_dependents();
   using C = ColMma<NT, FM>;
   extern __shared__ __align__(16) uint8_t sm[];
   __shared__ int s_last;

@@ -382,12 +382,6 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
       e = launch_rowdot(dY, bf16, R, w->O, B, true, r, V, s, nullptr, nullptr, 0, 0, 1.0f,
                         nullptr, bt, part, tickets, split);
   }
-  if (e == cudaSuccess && dX) {
-    if (tc)
-      e = launch_tc_dx(v, dY, R, V, A, r, sc, dX, tcws, (uint32_t*)ws, s);
-    else
-      e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s);
-  }
   // dA = s V^T X [r x I] and dB = s dY^T U [O x r]: one launch when both
   // are wanted (two independent side products), else one each.
   uint16_t* split = (uint16_t*)((char*)ws + L.split);
@@ -407,6 +401,15 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
     e = launch_coldot(X, bf16, R, w->I, V, r, sc, false, dA, red, s, tickets, split);
   if (e == cudaSuccess && dB && !paired)
     e = launch_coldot(dY, bf16, R, w->O, U, r, sc, true, dB, red, s, tickets, split);
+  // dX last: the tensor-core kernel starts behind the side products
+  // (programmatic dependent launch) and waits for them only before its
+  // adapter step, which reads the padded V written above.
+  if (e == cudaSuccess && dX) {
+    if (tc)
+      e = launch_tc_dx(v, dY, R, V, A, r, sc, dX, tcws, (uint32_t*)ws, s);
+    else
+      e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s);
+  }
   return cuda_status(e);
 }
 
