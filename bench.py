@@ -364,67 +364,75 @@ def run_gpu(args):
 
 def run_small_r(q, torch, peaks, args):
     """Bandwidth-bound regime: R in {1, 16} against W [4096 x 4096] and
-    [12288 x 4096] (NF4, B=64, C=256), forward and dX, GB/s on packed weight
-    bytes.  Cold L2: rotating weight copies totalling >= 4x L2, captured in
+    [12288 x 4096], forward and dX, GB/s on packed weight bytes.  Formats:
+    NF4 (B=64, C=256, tensor-core path) and affine 4/8-bit with G=64 (SIMT
+    path).  Cold L2: rotating weight copies totalling >= 4x L2, captured in
     a CUDA graph."""
     out = {}
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+
+    def clone(w):
+        c = lambda t: None if t is None else t.clone()
+        return q.QuantizedWeight(w.fmt, w.O, w.I, w.block, w.group, w.bits, c(w.codes),
+                                 c(w.scale_codes), c(w.group_absmax), c(w.mean), c(w.scale),
+                                 c(w.bias))
+
     for name in ("bw_sweep_4096", "bw_sweep_12288"):
         wl = synth.workload(name)
         lin = wl.linears[0]
         W = torch.from_numpy(synth.weight(wl, 0)).cuda()
-        base = q.qlora_quantize_nf4(W, 64, 256)
+        formats = [("", q.qlora_quantize_nf4(W, 64, 256))]
+        for bits in (4, 8):
+            formats.append((f"_affine{bits}_G64", q.qlora_quantize_affine(W, bits, 64)))
         del W
-        payload = base.payload_bytes()
-        ncopy = max(2, math.ceil(4 * l2 / payload))
-        copies = [base] + [q.QuantizedWeight(base.fmt, base.O, base.I, base.block, base.group, base.bits,
-                                             base.codes.clone(), base.scale_codes.clone(),
-                                             base.group_absmax.clone(), base.mean.clone())
-                           for _ in range(ncopy - 1)]
         A = torch.from_numpy(synth.adapters(wl, 0)[0]).cuda()
         B = torch.from_numpy(synth.adapters(wl, 0)[1]).cuda()
-        for R in (1, 16):
-            X = torch.randn((R, lin.I), device="cuda").to(torch.bfloat16)
-            dY = torch.randn((R, lin.O), device="cuda").to(torch.bfloat16)
-            Y = torch.empty((R, lin.O), device="cuda", dtype=torch.bfloat16)
-            dX = torch.empty((R, lin.I), device="cuda", dtype=torch.bfloat16)
-            U = torch.empty((R, wl.r), device="cuda")
-            wsf = q.workspace(q.qlora_linear_workspace_bytes(base, R, wl.r, 0, 1))
-            wsb = q.workspace(q.qlora_linear_workspace_bytes(base, R, wl.r, 1, 1))
-            res = {}
-            for op in ("fwd", "dx"):
-                def call(w):
-                    if op == "fwd":
-                        q.qlora_linear_fwd(w, X, A, B, wl.alpha, Y=Y, U_out=U, ws=wsf)
-                    else:
-                        q.qlora_linear_bwd(w, None, dY, A, B, wl.alpha, U=U, want_da=False, want_db=False,
-                                           dX=dX, ws=wsb)
-                for w in copies:
-                    call(w)
-                torch.cuda.synchronize()
-                s = torch.cuda.Stream()
-                s.wait_stream(torch.cuda.current_stream())
-                g = torch.cuda.CUDAGraph()
-                reps = max(64, ncopy)
-                with torch.cuda.graph(g, stream=s):
-                    for k in range(reps):
-                        call(copies[k % ncopy])
-                torch.cuda.synchronize()
-                g.replay()
-                torch.cuda.synchronize()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                g.replay()
-                e1.record()
-                torch.cuda.synchronize()
-                t_call = e0.elapsed_time(e1) / reps
-                gbs = payload / (t_call * 1e-3) / 1e9
-                res[op] = {"us_per_call": round(t_call * 1e3, 3), "packed_GBps": round(gbs, 1),
-                           "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
-                del g
-            out[f"{name}_R{R}"] = {"packed_bytes": int(payload), **res}
-        del copies, base
-        torch.cuda.empty_cache()
+        for tag, base in formats:
+            payload = base.payload_bytes()
+            ncopy = max(2, math.ceil(4 * l2 / payload))
+            copies = [base] + [clone(base) for _ in range(ncopy - 1)]
+            for R in (1, 16):
+                X = torch.randn((R, lin.I), device="cuda").to(torch.bfloat16)
+                dY = torch.randn((R, lin.O), device="cuda").to(torch.bfloat16)
+                Y = torch.empty((R, lin.O), device="cuda", dtype=torch.bfloat16)
+                dX = torch.empty((R, lin.I), device="cuda", dtype=torch.bfloat16)
+                U = torch.empty((R, wl.r), device="cuda")
+                wsf = q.workspace(q.qlora_linear_workspace_bytes(base, R, wl.r, 0, 1))
+                wsb = q.workspace(q.qlora_linear_workspace_bytes(base, R, wl.r, 1, 1))
+                res = {}
+                for op in ("fwd", "dx"):
+                    def call(w):
+                        if op == "fwd":
+                            q.qlora_linear_fwd(w, X, A, B, wl.alpha, Y=Y, U_out=U, ws=wsf)
+                        else:
+                            q.qlora_linear_bwd(w, None, dY, A, B, wl.alpha, U=U, want_da=False,
+                                               want_db=False, dX=dX, ws=wsb)
+                    for w in copies:
+                        call(w)
+                    torch.cuda.synchronize()
+                    st = torch.cuda.Stream()
+                    st.wait_stream(torch.cuda.current_stream())
+                    g = torch.cuda.CUDAGraph()
+                    reps = max(64, ncopy)
+                    with torch.cuda.graph(g, stream=st):
+                        for k in range(reps):
+                            call(copies[k % ncopy])
+                    torch.cuda.synchronize()
+                    g.replay()
+                    torch.cuda.synchronize()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    g.replay()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    t_call = e0.elapsed_time(e1) / reps
+                    gbs = payload / (t_call * 1e-3) / 1e9
+                    res[op] = {"us_per_call": round(t_call * 1e3, 3), "packed_GBps": round(gbs, 1),
+                               "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+                    del g
+                out[f"{name}{tag}_R{R}"] = {"packed_bytes": int(payload), **res}
+            del copies, base
+            torch.cuda.empty_cache()
     out["peak_GBps"] = peaks["hbm_gbs"]
     out["peak_source"] = f"{peaks['source']} HBM copy bandwidth"
     out["timing"] = f"CUDA graph of >= 64 calls rotating weight copies >= 4x L2"
