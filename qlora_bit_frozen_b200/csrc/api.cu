@@ -144,7 +144,8 @@ struct FwdLayout {
   size_t u = 0, red = 0, split = 0, tc = 0, total = 0;
 };
 struct BwdLayout {
-  size_t u = 0, v = 0, bt = 0, red = 0, red2 = 0, split = 0, split2 = 0, tc = 0, total = 0;
+  size_t u = 0, v = 0, bt = 0, red = 0, red2 = 0, split = 0, split2 = 0, gemv = 0, tc = 0,
+         total = 0;
 };
 
 FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t compute) {
@@ -188,6 +189,8 @@ BwdLayout bwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
   off += coldot_ws(R, w->O, r);
   L.split2 = off;  // bf16 hi / lo copy of U for that launch
   off += adapter_split_ws(R, r);
+  L.gemv = off;  // dX partials of the small-R affine path
+  off += gemv_dx_ws(view_of(w), R);
   L.tc = off;
   if (compute == QLORA_COMPUTE_BF16) off += tc_dx_ws(view_of(w), R);
   L.total = off;
@@ -408,7 +411,7 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
     if (tc)
       e = launch_tc_dx(v, dY, R, V, A, r, sc, dX, tcws, (uint32_t*)ws, s);
     else
-      e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s);
+      e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s, (float*)((char*)ws + L.gemv));
   }
   return cuda_status(e);
 }

@@ -39,9 +39,12 @@ cudaError_t launch_dequantize(const WView& w, float* out, cudaStream_t st);
 cudaError_t launch_simt_fwd(const WView& w, const void* X, int64_t R, const float* A,
                             const float* B, int32_t r, float s, bool bf16, void* Y, float* U,
                             cudaStream_t st);
+// gemv_ws (gemv_dx_ws bytes, nullable): split partials of the small-R
+// affine path.
 cudaError_t launch_simt_dx(const WView& w, const void* dY, int64_t R, const float* A,
                            const float* V, int32_t r, float s, bool bf16, void* dX,
-                           cudaStream_t st);
+                           cudaStream_t st, float* gemv_ws = nullptr);
+size_t gemv_dx_ws(const WView& w, int64_t R);
 // adapter side products
 // adapter.cu
 //   out[m, j] = sum_k P[m, k] L(k, j); pad (nullable): its bf16 copy [R x 64].
