@@ -213,7 +213,11 @@ size_t qlora_linear_workspace_bytes(const qlora_weight* w, int64_t R, int32_t r,
  * Every weight is decoded from its nibble and block scale inside the
  * kernels; no full-size floating-point weight is formed.  R = 0 is valid.
  * bf16 mode: W_hat and the adapter operands enter the tensor cores as bf16,
- * accumulation is fp32, Y is rounded to bf16 once.
+ * accumulation is fp32, Y is rounded to bf16 once.  U (and, in the
+ * backward, V, dA and dB) use the bf16 activations exactly and the fp32
+ * factors to 16 significant bits (each split into two bf16 halves).
+ * Deterministic: the same inputs give the same bits (every reduction
+ * across blocks is summed in a fixed order).
  * Requires 1 <= r <= 64 and I % block == 0.
  */
 qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, const float* A,
@@ -267,7 +271,9 @@ uint64_t qlora_kernel_launch_count(void);
  * records a CUDA event pair on the launching stream around each launch of
  * its tensor-core GEMM kernels (up to max_records launches; events are
  * created here, no device memory is allocated); 0 disables and drops
- * pending records.
+ * pending records.  While enabled, those kernels are launched in plain
+ * stream order (no programmatic overlap with the launch before them), so
+ * the recorded durations are the kernels' own.
  */
 qlora_status qlora_kernel_timing_enable(int32_t max_records);
 
