@@ -60,6 +60,10 @@ def _load():
         lib.oracle_linear_fwd.restype = None
         lib.oracle_linear_bwd.argtypes = [P, P, P, i64, P, i64, P, P, i32, f32, P, P, P]
         lib.oracle_linear_bwd.restype = None
+        lib.oracle_merge.argtypes = [P, P, P, i32, f32, P]
+        lib.oracle_merge.restype = None
+        lib.oracle_adam_step.argtypes = [P, P, P, P, i64, i64, f32, f32, f32, f32, P, P, P]
+        lib.oracle_adam_step.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -229,6 +233,33 @@ def linear_bwd(w: QWeight, X, dY, A, Bm, r: int, alpha: float, rows=None,
     _load().oracle_linear_bwd(ctypes.byref(cw), _ptr(X), _ptr(dY), R, _ptr(rows), n, _ptr(A), _ptr(Bm),
                               r, float(alpha), _ptr(dX), _ptr(dA), _ptr(dB))
     return dX, dA, dB
+
+
+def merge(w: QWeight, A, Bm, r: int, alpha: float) -> np.ndarray:
+    """W_hat + (alpha/r) Bm A as an fp64 [O x I] matrix (export)."""
+    A = _c(A, np.float32)
+    Bm = _c(Bm, np.float32)
+    out = np.zeros((w.O, w.I), np.float64)
+    cw = _cweight(w)
+    _load().oracle_merge(ctypes.byref(cw), _ptr(A), _ptr(Bm), r, float(alpha), _ptr(out))
+    return out
+
+
+def adam_step(p, g, m, v, t: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+              eps: float = 1e-8):
+    """One Adam step with bias correction: (p', m', v') in fp64 from fp32 state."""
+    p = _c(p, np.float32).ravel()
+    g = _c(g, np.float32).ravel()
+    m = _c(m, np.float32).ravel()
+    v = _c(v, np.float32).ravel()
+    n = p.size
+    assert g.size == n and m.size == n and v.size == n and t >= 1
+    po = np.zeros(n, np.float64)
+    mo = np.zeros(n, np.float64)
+    vo = np.zeros(n, np.float64)
+    _load().oracle_adam_step(_ptr(p), _ptr(g), _ptr(m), _ptr(v), n, int(t), float(lr), float(beta1),
+                             float(beta2), float(eps), _ptr(po), _ptr(mo), _ptr(vo))
+    return po, mo, vo
 
 
 def nf4_payload_bytes(N: int, B: int, C: int) -> int:

@@ -29,6 +29,12 @@
  *           a normal distribution.  The 16 values are not printed on the
  *           pages; oracle_nf4_codebook() builds them from the normal
  *           quantile construction of the NF4 data type.
+ *   [EXPORT] "QLoRA Fine-Tuning", section "Training lifecycle" (step 5:
+ *           dequantize the packed weights, add the trained LoRA deltas,
+ *           restore an ordinary fp32 matrix).
+ *   [ADAM]  same page, sections "Training lifecycle" (only the adapter
+ *           factors are trained, with Adam) and "Current scope" (paged
+ *           Adam state: pages of at most page_size elements).
  *   [AFF]   "LoRA vs QLoRA on Apple Silicon: memory/quality tradeoffs in
  *           MLX", sections "Method" and "Honest caveats": affine group-wise
  *           integer quantization with fp32 scale and bias (formula not
@@ -39,7 +45,9 @@
  * to the lower index; w/s_b is a true fp32 division; the mean mu sums block
  * scales in fp64 sequentially inside each group of C blocks, then the group
  * partials sequentially; "round" is round-half-away-from-zero; odd N leaves
- * the last high nibble 0; an empty tensor has mu = 0.
+ * the last high nibble 0; an empty tensor has mu = 0; the adapter optimizer
+ * is Adam with bias correction, eps added after the square root and no
+ * weight decay; the merged weight adds s B A to the decoded weight.
  */
 #include <float.h>
 #include <math.h>
@@ -510,6 +518,64 @@ void oracle_linear_bwd(const OracleWeight* w, const float* X, const float* dY, i
   }
   free(V);
   free(U);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Export and the adapter optimizer step.                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * [EXPORT]  W_merged = W_hat + s B A,  s = alpha / r.  A [r x I], Bm [O x r];
+ * out [O x I] in fp64.  The export step of the training lifecycle
+ * dequantizes every packed weight and adds its trained LoRA delta, giving
+ * an ordinary floating-point matrix; the delta of element (o, i) is the
+ * rank-r sum over k of B[o,k] A[k,i], the same product the forward applies
+ * to X (Y = X W_merged^T).  The delta is summed in fp64, in k order.
+ */
+void oracle_merge(const OracleWeight* w, const float* A, const float* Bm, int32_t r, float alpha,
+                  double* out) {
+  ensure_codebook();
+  const int64_t O = w->O, I = w->I;
+  const double s = lora_scale(alpha, r);
+#pragma omp parallel for schedule(static)
+  for (int64_t o = 0; o < O; ++o) {
+    for (int64_t i = 0; i < I; ++i) {
+      double delta = 0.0;
+      for (int32_t k = 0; k < r; ++k) delta += (double)Bm[o * r + k] * (double)A[k * I + i];
+      out[o * I + i] = (double)weight_at(w, o * I + i) + s * delta;
+    }
+  }
+}
+
+/*
+ * [ADAM]  One Adam step on n adapter parameters (the adapter factors are the
+ * only optimizer inputs; the packed base never is).  The pages name Adam but
+ * print no update rule; this is Adam with bias correction, step t >= 1:
+ *   m' = beta1 m + (1 - beta1) g
+ *   v' = beta2 v + (1 - beta2) g^2
+ *   p' = p - lr (m' / (1 - beta1^t)) / (sqrt(v' / (1 - beta2^t)) + eps)
+ * Inputs are the fp32 state; everything is evaluated in fp64 and p', m', v'
+ * are returned in fp64.  Paging the state (pages of at most page_size
+ * elements, one page update at a time) changes when each element is
+ * updated, not what it becomes, so the oracle has no page argument.
+ */
+void oracle_adam_step(const float* p, const float* g, const float* m, const float* v, int64_t n,
+                      int64_t t, float lr, float beta1, float beta2, float eps, double* p_out,
+                      double* m_out, double* v_out) {
+  const double b1 = (double)beta1, b2 = (double)beta2;
+  const double bc1 = 1.0 - pow(b1, (double)t);
+  const double bc2 = 1.0 - pow(b2, (double)t);
+#pragma omp parallel for schedule(static)
+  for (int64_t j = 0; j < n; ++j) {
+    const double gj = (double)g[j];
+    const double mj = b1 * (double)m[j] + (1.0 - b1) * gj;
+    const double vj = b2 * (double)v[j] + (1.0 - b2) * gj * gj;
+    const double mhat = mj / bc1;
+    const double vhat = vj / bc2;
+    p_out[j] = (double)p[j] - (double)lr * mhat / (sqrt(vhat) + (double)eps);
+    m_out[j] = mj;
+    v_out[j] = vj;
+  }
 }
 
 /* Threads OpenMP will use (reported beside the CPU timings). */

@@ -327,3 +327,110 @@ def test_synth_streams_are_stable():
     assert abs(float(a.mean())) < 0.1 and abs(float(a.std()) - 1) < 0.1
     wide, bits = synth.bf16_round(np.array([1.0, 1.00390625, 1.005859375, -2.5], np.float32))
     assert list(wide) == [1.0, 1.0, 1.0078125, -2.5]
+
+
+# ---------------------------------------------------------------- export (merge)
+
+@pytest.mark.parametrize("fmt", ["nf4", "affine"])
+def test_merged_weight_reproduces_the_layer(fmt):
+    """The merged matrix must give the layer's own outputs as a plain dense
+    layer: X W_merged^T equals the forward (which applies the adapter as
+    s (X A^T) B^T) and dY W_merged equals the input gradient (which applies
+    it as s (dY B) A), to fp64 rounding.  O != I, so a transposed operand
+    cannot pass."""
+    w, X, A, Bm, dY, r, alpha = _small_layer(fmt, O=192, I=128, R=5, r=4, alpha=8.0, seed=50)
+    Wm = oracle.merge(w, A, Bm, r, alpha)
+    assert Wm.shape == (192, 128)
+    Y, _ = oracle.linear_fwd(w, X, A, Bm, r, alpha)
+    dX, _, _ = oracle.linear_bwd(w, X, dY, A, Bm, r, alpha, want_da=False, want_db=False)
+    assert np.allclose(Y, X.astype(np.float64) @ Wm.T, rtol=1e-12, atol=1e-12)
+    assert np.allclose(dX, dY.astype(np.float64) @ Wm, rtol=1e-12, atol=1e-12)
+
+
+def test_merge_zero_adapter_and_unit_rank_one():
+    w, X, A, Bm, dY, r, alpha = _small_layer("nf4", O=64, I=128, R=2, r=3, seed=51)
+    Wh = oracle.dequantize(w).astype(np.float64)
+    assert np.array_equal(oracle.merge(w, A, np.zeros_like(Bm), r, alpha), Wh)
+    assert np.array_equal(oracle.merge(w, A, Bm, r, 0.0), Wh)
+    # one unit entry in A (k=1, i=77) and in B (o=9, k=1): the delta is s at
+    # (9, 77) and exactly zero elsewhere.
+    A1 = np.zeros_like(A)
+    B1 = np.zeros_like(Bm)
+    A1[1, 77] = 1.0
+    B1[9, 1] = 1.0
+    s = float(np.float32(alpha) / np.float32(r))
+    D = oracle.merge(w, A1, B1, r, alpha) - Wh
+    expect = np.zeros_like(D)
+    expect[9, 77] = s
+    assert np.allclose(D, expect, rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------- Adam
+
+def test_adam_first_step_is_lr_times_sign():
+    """From a zero state the bias-corrected moments are g and g^2 exactly,
+    so the first step moves each parameter by lr g / (|g| + eps)."""
+    g = synth.normal(60, 257)
+    p = synth.normal(61, 257)
+    z = np.zeros_like(g)
+    lr, eps = 2.0 ** -10, 2.0 ** -27    # exact in fp32, as the oracle takes them
+    po, mo, vo = oracle.adam_step(p, g, z, z, 1, lr, 0.9, 0.999, eps)
+    g64 = g.astype(np.float64)
+    assert np.allclose(po, p - lr * g64 / (np.abs(g64) + eps), rtol=1e-14, atol=1e-15)
+    assert np.allclose(mo, (1 - np.float64(np.float32(0.9))) * g64, rtol=1e-14, atol=0)
+    assert np.allclose(vo, (1 - np.float64(np.float32(0.999))) * g64 * g64, rtol=1e-14, atol=0)
+
+
+def test_adam_constant_gradient_closed_form():
+    """With a constant gradient m_t = (1 - b1^t) g and v_t = (1 - b2^t) g^2,
+    so every bias-corrected step is lr g / (|g| + eps): after T steps
+    p_T = p_0 - T lr g / (|g| + eps).  A wrong bias-correction exponent
+    breaks it at t >= 2."""
+    g = np.array([0.5, -2.0, 3e-3, -7.25], np.float32)
+    p = np.array([1.0, -1.0, 0.25, 4.0], np.float32)
+    m = np.zeros_like(g)
+    v = np.zeros_like(g)
+    b1, b2, lr, eps = 0.9, 0.999, 1e-2, 1e-8
+    b1d, b2d = float(np.float32(b1)), float(np.float32(b2))
+    g64 = g.astype(np.float64)
+    p64 = p.astype(np.float64)
+    T = 6
+    for t in range(1, T + 1):
+        po, mo, vo = oracle.adam_step(p, g, m, v, t, lr, b1, b2, eps)
+        step = lr * g64 / (np.abs(g64) + eps)
+        assert np.allclose(mo, (1 - b1d ** t) * g64, rtol=1e-6)
+        assert np.allclose(vo, (1 - b2d ** t) * g64 * g64, rtol=1e-6)
+        # exact fp64 step from this step's fp32 state
+        assert np.allclose(po, p.astype(np.float64) - step, rtol=1e-6, atol=1e-12)
+        p, m, v = po.astype(np.float32), mo.astype(np.float32), vo.astype(np.float32)
+    assert np.allclose(p.astype(np.float64), p64 - T * lr * g64 / (np.abs(g64) + eps),
+                       rtol=1e-6, atol=1e-7)
+
+
+def test_adam_sign_flip_closed_form():
+    """g = +1 then -1: v_hat stays 1 and m_hat_2 = -(1 - b1)/(1 + b1), so
+    p_2 = p_0 - lr/(1 + eps) + lr (1 - b1)/((1 + b1)(1 + eps))."""
+    b1, b2, lr, eps = 0.9, 0.999, 0.05, 1e-8
+    b1d = float(np.float32(b1))
+    p0 = np.array([0.75], np.float32)
+    z = np.zeros(1, np.float32)
+    p1, m1, v1 = oracle.adam_step(p0, np.ones(1, np.float32), z, z, 1, lr, b1, b2, eps)
+    p2, m2, v2 = oracle.adam_step(p1.astype(np.float32), -np.ones(1, np.float32),
+                                  m1.astype(np.float32), v1.astype(np.float32), 2, lr, b1, b2, eps)
+    assert m2[0] == pytest.approx(-(1 - b1d) ** 2, rel=1e-6)
+    expect = 0.75 - lr / (1 + eps) + lr * (1 - b1d) / ((1 + b1d) * (1 + eps))
+    assert p2[0] == pytest.approx(expect, rel=1e-6)
+
+
+def test_adam_zero_gradient_and_scale_invariance():
+    p = synth.normal(62, 64)
+    z = np.zeros_like(p)
+    po, mo, vo = oracle.adam_step(p, z, z, z, 1, 1e-3)
+    assert np.array_equal(po, p.astype(np.float64)) and not mo.any() and not vo.any()
+    # with eps = 0 the update is invariant to a positive rescaling of g
+    g = synth.normal(63, 64)
+    m = synth.normal(64, 64, std=0.1)
+    v = np.abs(synth.normal(65, 64, std=0.1))
+    a, _, _ = oracle.adam_step(p, g, m, v, 3, 1e-3, eps=0.0)
+    b, _, _ = oracle.adam_step(p, 4 * g, 4 * m, 16 * v, 3, 1e-3, eps=0.0)
+    assert np.allclose(a, b, rtol=1e-13, atol=0)
