@@ -194,6 +194,41 @@ qlora_status qlora_quantize_affine(const float* W, int64_t O, int64_t I, int32_t
  */
 qlora_status qlora_dequantize(const qlora_weight* w, float* W_hat, qlora_stream_t stream);
 
+/*
+ * Export of a trained layer ("QLoRA Fine-Tuning", "Training lifecycle":
+ * at export the packed weights are dequantized and the trained LoRA deltas
+ * added, restoring ordinary fp32 weights).  W_out [O x I] fp32:
+ *   W_out[o,i] = fp32(W_hat[o,i] + fp32(s * delta)),  s = alpha / r (fp32),
+ *   delta = sum_k B[o,k] A[k,i]  (fp32 FMAs in k order),
+ * W_hat decoded exactly as qlora_dequantize does, so B = 0 or alpha = 0
+ * gives the dequantized weight.  A [r x I], B [O x r] fp32, device memory;
+ * W_out must not overlap the inputs.  Any r >= 1 and any O, I.  The result
+ * is a plain fp32 matrix; requantizing it (qlora_quantize_nf4) is a second,
+ * separate approximation.  Never used by the training entry points.
+ */
+qlora_status qlora_merge(const qlora_weight* w, const float* A, const float* B, int32_t r,
+                         float alpha, float* W_out, qlora_stream_t stream);
+
+/*
+ * One Adam step over n fp32 parameters ("QLoRA Fine-Tuning", "Training
+ * lifecycle": only the LoRA factors are optimizer inputs; "Current scope":
+ * paged Adam state).  params, grads, m, v: n floats each, device (or
+ * managed) memory, distinct buffers; params, m and v are updated in place.
+ * With step count t >= 1, bc1 = fp32(1 - beta1^t), bc2 = fp32(1 - beta2^t):
+ *   m = b1 m + fp32(1 - b1) g
+ *   v = b2 v + fp32(1 - b2) g^2
+ *   params -= lr (m / bc1) / (sqrt(v / bc2) + eps)
+ * every fp32 operation rounded once (no contraction).  No weight decay.
+ * page_elems > 0 updates the state in pages of at most page_elems elements,
+ * one launch per page in order (for state kept in managed memory); 0 is one
+ * launch.  The result is the same bits either way.  Requires 0 <= beta < 1,
+ * eps > 0, finite lr.  To update every adapter factor in one call, keep them
+ * in one flat arena (A and B of each layer as views into it).
+ */
+qlora_status qlora_adam_step(float* params, const float* grads, float* m, float* v, int64_t n,
+                             int64_t t, float lr, float beta1, float beta2, float eps,
+                             int64_t page_elems, qlora_stream_t stream);
+
 /* op codes for qlora_linear_workspace_bytes */
 #define QLORA_OP_FWD 0
 #define QLORA_OP_BWD 1

@@ -22,7 +22,7 @@ from ._ffi import (COMPUTE_BF16, COMPUTE_FP32, FMT_AFFINE, FMT_NF4_DQ, OP_BWD, O
 __all__ = [
     "QLoraError", "QuantizedWeight", "qlora_status_string", "qlora_nf4_codebook",
     "qlora_nf4_payload_bytes", "qlora_quantize_nf4", "qlora_quantize_nf4_noalloc", "qlora_quantize_affine",
-    "qlora_dequantize",
+    "qlora_dequantize", "qlora_merge", "qlora_adam_step",
     "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_workspace_status", "qlora_selftest_wait_timeout", "qlora_kernel_launch_count",
     "qlora_kernel_timing_enable", "qlora_kernel_timing_collect",
@@ -173,6 +173,35 @@ def qlora_dequantize(w: QuantizedWeight, out: Optional[torch.Tensor] = None, str
     cw = w.c_struct()
     _check(lib.qlora_dequantize(ctypes.byref(cw), _ptr(out), _stream(stream)), "qlora_dequantize")
     return out
+
+
+def qlora_merge(w: QuantizedWeight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Export: W_hat + (alpha/r) B A as an fp32 [O x I] matrix (A [r x I], B [O x r] fp32)."""
+    lib = _ffi.load()
+    r = A.shape[0]
+    if A.dtype != torch.float32 or B.dtype != torch.float32 or tuple(A.shape) != (r, w.I) \
+            or tuple(B.shape) != (w.O, r) or not A.is_contiguous() or not B.is_contiguous():
+        raise ValueError("A must be contiguous fp32 [r x I] and B contiguous fp32 [O x r]")
+    if out is None:
+        out = torch.empty((w.O, w.I), dtype=torch.float32, device=w.codes.device)
+    cw = w.c_struct()
+    _check(lib.qlora_merge(ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha), _ptr(out), _stream(stream)),
+           "qlora_merge")
+    return out
+
+
+def qlora_adam_step(params: torch.Tensor, grads: torch.Tensor, m: torch.Tensor, v: torch.Tensor, t: int,
+                    lr: float, beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                    page_elems: int = 0, stream=None) -> None:
+    """One in-place Adam step over flat contiguous fp32 tensors (step count t >= 1)."""
+    n = params.numel()
+    for x in (params, grads, m, v):
+        if x.dtype != torch.float32 or not x.is_contiguous() or x.numel() != n:
+            raise ValueError("params, grads, m and v must be contiguous fp32 tensors of one size")
+    st = _ffi.load().qlora_adam_step(_ptr(params), _ptr(grads), _ptr(m), _ptr(v), n, int(t), float(lr),
+                                     float(beta1), float(beta2), float(eps), int(page_elems), _stream(stream))
+    _check(st, "qlora_adam_step")
 
 
 def qlora_linear_workspace_bytes(w: QuantizedWeight, R: int, r: int, op: int, compute: int) -> int:

@@ -59,6 +59,8 @@ SIGNATURES = {
     "qlora_quantize_affine_workspace_bytes": (_sz, [_i64, _i32, _i32]),
     "qlora_quantize_affine": (ctypes.c_int, [_P, _i64, _i64, _i32, _i32, _P, _P, _P, _P, _sz, _P]),
     "qlora_dequantize": (ctypes.c_int, [_W, _P, _P]),
+    "qlora_merge": (ctypes.c_int, [_W, _P, _P, _i32, _f32, _P, _P]),
+    "qlora_adam_step": (ctypes.c_int, [_P, _P, _P, _P, _i64, _i64, _f32, _f32, _f32, _f32, _i64, _P]),
     "qlora_linear_workspace_bytes": (_sz, [_W, _i64, _i32, _i32, _i32]),
     "qlora_linear_fwd": (ctypes.c_int, [_W, _P, _i64, _P, _P, _i32, _f32, _i32, _P, _P, _P, _sz, _P]),
     "qlora_linear_bwd": (ctypes.c_int, [_W, _P, _P, _i64, _P, _P, _i32, _f32, _P, _i32, _P, _P, _P, _P,

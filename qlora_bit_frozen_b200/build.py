@@ -15,12 +15,13 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libqlora.so")
 
-SOURCES = ["api.cu", "quantize.cu", "simt.cu", "adapter.cu", "tc_gemm.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "quantize.cu", "simt.cu", "adapter.cu", "tc_gemm.cu", "noalloc.cu", "merge.cu",
+           "adam.cu"]
 HEADERS = ["common.cuh", "internal.h", "tc_gemm.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I" + INCLUDE, "-I" + CSRC]
-EXTRA = {"quantize.cu": ["--fmad=false"]}
+EXTRA = {"quantize.cu": ["--fmad=false"], "adam.cu": ["--fmad=false"]}
 
 
 def _nvcc():

@@ -1,5 +1,6 @@
 // api.cu -- the extern "C" entry points of libqlora (declared in qlora.h):
 // host-side argument checks, workspace layout and kernel dispatch.
+#include <math.h>
 #include <string.h>
 
 #include <mutex>
@@ -294,6 +295,33 @@ qlora_status qlora_dequantize(const qlora_weight* w, float* W_hat, qlora_stream_
   st = device_ready();
   if (st != QLORA_OK) return st;
   return cuda_status(launch_dequantize(view_of(w), W_hat, (cudaStream_t)stream));
+}
+
+qlora_status qlora_merge(const qlora_weight* w, const float* A, const float* B, int32_t r,
+                         float alpha, float* W_out, qlora_stream_t stream) {
+  qlora_status st = check_weight(w, false);
+  if (st != QLORA_OK) return st;
+  if (r < 1) return QLORA_ERR_SHAPE;
+  if (w->O * w->I > 0 && (!A || !B || !W_out)) return QLORA_ERR_INVALID_ARG;
+  st = device_ready();
+  if (st != QLORA_OK) return st;
+  const float s = alpha / (float)r;
+  return cuda_status(launch_merge(view_of(w), A, B, r, s, W_out, (cudaStream_t)stream));
+}
+
+qlora_status qlora_adam_step(float* params, const float* grads, float* m, float* v, int64_t n,
+                             int64_t t, float lr, float beta1, float beta2, float eps,
+                             int64_t page_elems, qlora_stream_t stream) {
+  if (n < 0 || t < 1 || page_elems < 0) return QLORA_ERR_SHAPE;
+  if (!(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f))
+    return QLORA_ERR_INVALID_ARG;
+  if (!(eps > 0.0f) || !isfinite(eps) || !isfinite(lr)) return QLORA_ERR_INVALID_ARG;
+  if (n == 0) return QLORA_OK;
+  if (!params || !grads || !m || !v) return QLORA_ERR_INVALID_ARG;
+  qlora_status st = device_ready();
+  if (st != QLORA_OK) return st;
+  return cuda_status(launch_adam(params, grads, m, v, n, t, lr, beta1, beta2, eps, page_elems,
+                                 (cudaStream_t)stream));
 }
 
 size_t qlora_linear_workspace_bytes(const qlora_weight* w, int64_t R, int32_t r, int32_t op,

@@ -35,6 +35,16 @@ cudaError_t launch_affine_quantize(const float* W, int64_t N, int32_t bits, int3
                                    cudaStream_t st);
 cudaError_t launch_dequantize(const WView& w, float* out, cudaStream_t st);
 
+// merge.cu -- out [O x I] = W_hat + s B A (B [O x r], A [r x I], fp32)
+cudaError_t launch_merge(const WView& w, const float* A, const float* B, int32_t r, float s,
+                         float* out, cudaStream_t st);
+
+// adam.cu -- one Adam step over n fp32 parameters; page > 0: one launch per
+// page of at most `page` elements, in order
+cudaError_t launch_adam(float* p, const float* g, float* m, float* v, int64_t n, int64_t t,
+                        float lr, float beta1, float beta2, float eps, int64_t page,
+                        cudaStream_t st);
+
 // simt.cu -- generic (SIMT) linear kernels, both compute modes
 cudaError_t launch_simt_fwd(const WView& w, const void* X, int64_t R, const float* A,
                             const float* B, int32_t r, float s, bool bf16, void* Y, float* U,

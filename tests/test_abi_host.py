@@ -82,6 +82,30 @@ def test_bad_arguments_rejected_before_launch(lib):
     assert lib.qlora_dequantize(None, dummy, None) == _ffi.ERR_INVALID_ARG
 
 
+def test_merge_and_adam_arguments_rejected_before_launch(lib):
+    ws = ctypes.create_string_buffer(1024)
+    d = ctypes.c_void_p((ctypes.addressof(ws) + 255) // 256 * 256)
+    w = _ffi.qlora_weight(_ffi.FMT_NF4_DQ, 64, 128, 64, 256, 4, d.value, d.value, d.value, d.value, None, None)
+    P = ctypes.byref(w)
+    assert lib.qlora_merge(P, d, d, 0, 1.0, d, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_merge(P, None, d, 8, 1.0, d, None) == _ffi.ERR_INVALID_ARG
+    assert lib.qlora_merge(P, d, d, 8, 1.0, None, None) == _ffi.ERR_INVALID_ARG
+    assert lib.qlora_merge(None, d, d, 8, 1.0, d, None) == _ffi.ERR_INVALID_ARG
+    w.bits = 8
+    assert lib.qlora_merge(P, d, d, 8, 1.0, d, None) == _ffi.ERR_SHAPE
+    adam = lib.qlora_adam_step
+    assert adam(d, d, d, d, -1, 1, 1e-3, 0.9, 0.999, 1e-8, 0, None) == _ffi.ERR_SHAPE
+    assert adam(d, d, d, d, 16, 0, 1e-3, 0.9, 0.999, 1e-8, 0, None) == _ffi.ERR_SHAPE
+    assert adam(d, d, d, d, 16, 1, 1e-3, 0.9, 0.999, 1e-8, -4, None) == _ffi.ERR_SHAPE
+    assert adam(d, d, d, d, 16, 1, 1e-3, 1.0, 0.999, 1e-8, 0, None) == _ffi.ERR_INVALID_ARG
+    assert adam(d, d, d, d, 16, 1, 1e-3, 0.9, -0.5, 1e-8, 0, None) == _ffi.ERR_INVALID_ARG
+    assert adam(d, d, d, d, 16, 1, 1e-3, 0.9, 0.999, 0.0, 0, None) == _ffi.ERR_INVALID_ARG
+    assert adam(d, d, d, d, 16, 1, float("nan"), 0.9, 0.999, 1e-8, 0, None) == _ffi.ERR_INVALID_ARG
+    assert adam(d, None, d, d, 16, 1, 1e-3, 0.9, 0.999, 1e-8, 0, None) == _ffi.ERR_INVALID_ARG
+    # an empty arena is a valid no-op, even with null pointers
+    assert adam(None, None, None, None, 0, 1, 1e-3, 0.9, 0.999, 1e-8, 0, None) == _ffi.OK
+
+
 def test_workspace_sizes_are_consistent(lib):
     w = _ffi.qlora_weight(_ffi.FMT_NF4_DQ, 2048, 1024, 64, 256, 4, None, None, None, None, None, None)
     P = ctypes.byref(w)
