@@ -332,6 +332,10 @@ def run_gpu(args):
     if world == 1:
         quant = time_quantize(q, torch, wl)
 
+    export = None
+    if world == 1 and args.export:
+        export = time_export(q, torch, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, args.cpu_rows)
@@ -355,7 +359,7 @@ def run_gpu(args):
                     "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ems / args.steps, 5)},
             "clocks": clk, "gpu_launches": int(launches), "kernels_per_step": int(kernels_per_step),
             "timing": "device step captured once in a CUDA graph and replayed; CUDA events around each replay; per-kernel durations from a second pass with events around each tensor-core launch",
-            "small_r": small, "quantize": quant,
+            "small_r": small, "quantize": quant, "export": export,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -454,6 +458,57 @@ def time_quantize(q, torch, wl):
             "note": "host wall clock incl. the flag read-back synchronization"}
 
 
+def time_export(q, torch, peaks):
+    """The two lifecycle kernels around the layer, each timed with CUDA
+    events around single launches, L2 flushed before each (outside the
+    events): the fp32 export of an 8B-class MLP weight (12288 x 4096, r = 32)
+    and one Adam step over the 1,146,880 adapter parameters of the Qwen3-0.6B
+    q/v adapters."""
+    O, I, r = 12288, 4096, 32
+    w = q.qlora_quantize_nf4(torch.randn(O, I, device="cuda") * 0.02)
+    A = torch.randn(r, I, device="cuda") * 0.02
+    B = torch.randn(O, r, device="cuda") * 0.02
+    out = torch.empty(O, I, device="cuda")
+    n = 1146880
+    p = torch.randn(n, device="cuda") * 0.02
+    g = torch.randn(n, device="cuda") * 1e-2
+    m = torch.zeros(n, device="cuda")
+    v = torch.zeros(n, device="cuda")
+    flush = torch.empty(2 * 126 * 2 ** 20 // 4, device="cuda")
+
+    def timed(fn, reps):
+        ms = []
+        for i in range(reps):
+            flush.fill_(float(i))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn(i)
+            e1.record()
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        ms.sort()
+        return ms[len(ms) // 2]
+
+    for i in range(3):
+        q.qlora_merge(w, A, B, 2.0 * r, out=out)
+        q.qlora_adam_step(p, g, m, v, i + 1, 1e-3)
+    torch.cuda.synchronize()
+    mms = timed(lambda i: q.qlora_merge(w, A, B, 2.0 * r, out=out), 10)
+    ams = timed(lambda i: q.qlora_adam_step(p, g, m, v, i + 4, 1e-3), 20)
+    mbytes = w.payload_bytes() + 4 * O * I + 4 * r * (O + I)
+    abytes = 28 * n
+    peak = peaks["hbm_gbs"]
+    mg = mbytes / mms / 1e6
+    ag = abytes / ams / 1e6
+    return {
+        "merge": {"shape": [O, I, r], "ms": round(mms, 4), "bytes": int(mbytes), "GBps": round(mg, 1),
+                  "frac": round(mg / peak, 4)},
+        "adam": {"params": n, "ms": round(ams, 4), "bytes": int(abytes), "GBps": round(ag, 1),
+                 "frac": round(ag / peak, 4)},
+        "peak_GBps": peak, "timing": "median of single launches, CUDA events, L2 flushed before each",
+    }
+
+
 # --------------------------------------------------------------- CPU oracle
 
 def cpu_baseline(wl, rows):
@@ -529,6 +584,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=1024, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-r", dest="small_r", action="store_false")
+    ap.add_argument("--no-export", dest="export", action="store_false",
+                    help="skip timing the fp32 export (merge) and the adapter Adam step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -8,7 +8,8 @@
 // outer product: the CTA stages A[k0.., tile columns] and B[tile rows, k0..]
 // in shared memory, 32 ranks at a time, and each thread accumulates a 4 x 4
 // block of the tile with fp32 FMAs in rank order.  The epilogue decodes the
-// weight of each element exactly as qlora_dequantize does and adds the
+// weight of each element exactly as qlora_dequantize does (levels read from
+// a shared-memory copy of the NF4 table) and adds the
 // scaled delta with one rounding each (__fmul_rn, __fadd_rn), so with B = 0
 // or alpha = 0 the result equals the dequantized weight.  Written with
 // float4 stores when every row starts on a 16-byte boundary; the bound is
@@ -42,15 +43,17 @@ __device__ __forceinline__ uint64_t idiv(uint64_t a, uint32_t d) {
 }
 
 // Weight at flat index n (same arithmetic as the diagnostic dequantization).
+// lut: the 16 NF4 levels in shared memory (lanes that look up different
+// levels read different banks; the constant cache would serialize them).
 template <bool NARROW>
-__device__ __forceinline__ float weight1(const WView& w, uint64_t n) {
+__device__ __forceinline__ float weight1(const WView& w, uint64_t n, const float* lut) {
   if (w.fmt == QLORA_FMT_NF4_DQ) {
     const uint32_t byte = __ldg(w.codes + (n >> 1));
     const uint32_t code = (n & 1) ? (byte >> 4) : (byte & 15u);
     const uint64_t b = idiv<NARROW>(n, (uint32_t)w.block);
     const uint64_t g = idiv<NARROW>(b, (uint32_t)w.group);
     const float sb = decode_block_scale(__ldg(w.qcodes + b), __ldg(w.t + g), __ldg(w.mu));
-    return __fmul_rn(kNF4[code], sb);
+    return __fmul_rn(lut[code], sb);
   }
   uint32_t q;
   if (w.bits == 8) {
@@ -66,17 +69,17 @@ __device__ __forceinline__ float weight1(const WView& w, uint64_t n) {
 // Four consecutive weights n0..n0+3 with n0 % 4 == 0 and block % 4 == 0:
 // one block (group), one scale decode.
 template <bool NARROW>
-__device__ __forceinline__ void weight4(const WView& w, uint64_t n0, float v[4]) {
+__device__ __forceinline__ void weight4(const WView& w, uint64_t n0, const float* lut, float v[4]) {
   if (w.fmt == QLORA_FMT_NF4_DQ) {
     const uint64_t b = idiv<NARROW>(n0, (uint32_t)w.block);
     const uint64_t g = idiv<NARROW>(b, (uint32_t)w.group);
     const float sb = decode_block_scale(__ldg(w.qcodes + b), __ldg(w.t + g), __ldg(w.mu));
     const uint32_t lo = __ldg(w.codes + (n0 >> 1));
     const uint32_t hi = __ldg(w.codes + (n0 >> 1) + 1);
-    v[0] = __fmul_rn(kNF4[lo & 15u], sb);
-    v[1] = __fmul_rn(kNF4[lo >> 4], sb);
-    v[2] = __fmul_rn(kNF4[hi & 15u], sb);
-    v[3] = __fmul_rn(kNF4[hi >> 4], sb);
+    v[0] = __fmul_rn(lut[lo & 15u], sb);
+    v[1] = __fmul_rn(lut[lo >> 4], sb);
+    v[2] = __fmul_rn(lut[hi & 15u], sb);
+    v[3] = __fmul_rn(lut[hi >> 4], sb);
     return;
   }
   const uint64_t g = idiv<NARROW>(n0, (uint32_t)w.block);
@@ -102,6 +105,8 @@ template <bool NARROW, bool VEC>
 __global__ void __launch_bounds__(kThreads) merge_kernel(MergeArgs a) {
   __shared__ __align__(16) float As[kRank][kCols];  // A[k0 + k, i0 + c]
   __shared__ float Bs[kRank][kRows + 1];            // B[o0 + row, k0 + k]
+  __shared__ float lut[16];
+  if (threadIdx.x < 16) lut[threadIdx.x] = kNF4[threadIdx.x];  // visible after the first barrier (r >= 1)
   const int tx = threadIdx.x & 15;
   const int ty = threadIdx.x >> 4;
   const int64_t O = a.w.O, I = a.w.I;
@@ -149,7 +154,7 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(MergeArgs a) {
     const uint64_t n0 = (uint64_t)o * (uint64_t)I + (uint64_t)ib;
     if (VEC) {  // I % 4 == 0: ib < I implies ib + 3 < I
       float v[4];
-      weight4<NARROW>(a.w, n0, v);
+      weight4<NARROW>(a.w, n0, lut, v);
       float4 res;
       res.x = __fadd_rn(v[0], __fmul_rn(a.s, acc[q][0]));
       res.y = __fadd_rn(v[1], __fmul_rn(a.s, acc[q][1]));
@@ -160,7 +165,7 @@ __global__ void __launch_bounds__(kThreads) merge_kernel(MergeArgs a) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         if (ib + j < I)
-          a.out[n0 + j] = __fadd_rn(weight1<NARROW>(a.w, n0 + j), __fmul_rn(a.s, acc[q][j]));
+          a.out[n0 + j] = __fadd_rn(weight1<NARROW>(a.w, n0 + j, lut), __fmul_rn(a.s, acc[q][j]));
       }
     }
   }
