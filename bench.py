@@ -334,7 +334,10 @@ def run_gpu(args):
 
     export = None
     if world == 1 and args.export:
-        export = time_export(q, torch, peaks)
+        try:
+            export = time_export(q, torch, peaks)
+        except (RuntimeError, ValueError) as e:  # reported in the line, not fatal to it
+            export = {"error": str(e)[:300]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
