@@ -17,6 +17,8 @@
  *     Q-LoRA layer" (base + (alpha/r)(x A^T) B^T with fp32 A/B).
  *   "LoRA vs QLoRA on Apple Silicon ... in MLX", "Method" (affine
  *     group-wise 4/8-bit quantization with fp32 scale and bias).
+ *   "QLoRA Fine-Tuning", "Training lifecycle" and "Current scope" (the
+ *     adapter-only Adam step with paged state, and the fp32 export).
  *
  * Conventions for every entry point:
  *   - All array arguments are DEVICE pointers owned by the caller, unless a
@@ -24,6 +26,9 @@
  *   - The library never allocates device memory.  Scratch space is a caller
  *     workspace (`ws`, `ws_bytes`); its required size comes from the
  *     matching *_workspace_bytes() function.  `ws` must be 256-byte aligned.
+ *   - fp32 arrays must be 4-byte aligned and bf16 arrays 2-byte aligned
+ *     (QLORA_ERR_ALIGNMENT otherwise); faster paths that need 16-byte
+ *     alignment are chosen only when the pointers have it.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  Only qlora_quantize_nf4, qlora_quantize_affine and
  *     qlora_workspace_status synchronize `stream` (to read a device flag).

@@ -74,6 +74,8 @@ static void timing_clear_locked() {
 namespace {
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+// Element alignment of fp32 arrays (null counts as aligned).
+bool al4(const void* p) { return aligned(p, 4); }
 
 qlora_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
@@ -108,9 +110,11 @@ qlora_status check_weight(const qlora_weight* w, bool for_linear) {
     if (w->bits != 4 || w->group < 1) return QLORA_ERR_SHAPE;
     if (N > 0 && (!w->codes || !w->scale_codes || !w->group_absmax || !w->mean))
       return QLORA_ERR_INVALID_ARG;
+    if (!al4(w->group_absmax) || !al4(w->mean)) return QLORA_ERR_ALIGNMENT;
   } else if (w->fmt == QLORA_FMT_AFFINE) {
     if (w->bits != 4 && w->bits != 8) return QLORA_ERR_SHAPE;
     if (N > 0 && (!w->codes || !w->scale || !w->bias)) return QLORA_ERR_INVALID_ARG;
+    if (!al4(w->scale) || !al4(w->bias)) return QLORA_ERR_ALIGNMENT;
   } else {
     return QLORA_ERR_INVALID_ARG;
   }
@@ -245,7 +249,7 @@ qlora_status qlora_quantize_nf4(const float* W, int64_t O, int64_t I, int32_t B,
   const int64_t N = O * I;
   if (!mu || !ws) return QLORA_ERR_INVALID_ARG;
   if (N > 0 && (!W || !codes || !scale_codes || !t)) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
+  if (!aligned(ws, 256) || !al4(W) || !al4(t) || !al4(mu)) return QLORA_ERR_ALIGNMENT;
   if (ws_bytes < nf4_quantize_ws(N, B, C)) return QLORA_ERR_WORKSPACE;
   qlora_status st = device_ready();
   if (st != QLORA_OK) return st;
@@ -274,7 +278,7 @@ qlora_status qlora_quantize_affine(const float* W, int64_t O, int64_t I, int32_t
   const int64_t N = O * I;
   if (!ws) return QLORA_ERR_INVALID_ARG;
   if (N > 0 && (!W || !codes || !scale || !bias)) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
+  if (!aligned(ws, 256) || !al4(W) || !al4(scale) || !al4(bias)) return QLORA_ERR_ALIGNMENT;
   if (ws_bytes < kWsHeader) return QLORA_ERR_WORKSPACE;
   qlora_status st = device_ready();
   if (st != QLORA_OK) return st;
@@ -292,6 +296,7 @@ qlora_status qlora_dequantize(const qlora_weight* w, float* W_hat, qlora_stream_
   qlora_status st = check_weight(w, false);
   if (st != QLORA_OK) return st;
   if (w->O * w->I > 0 && !W_hat) return QLORA_ERR_INVALID_ARG;
+  if (!al4(W_hat)) return QLORA_ERR_ALIGNMENT;
   st = device_ready();
   if (st != QLORA_OK) return st;
   return cuda_status(launch_dequantize(view_of(w), W_hat, (cudaStream_t)stream));
@@ -303,6 +308,7 @@ qlora_status qlora_merge(const qlora_weight* w, const float* A, const float* B, 
   if (st != QLORA_OK) return st;
   if (r < 1) return QLORA_ERR_SHAPE;
   if (w->O * w->I > 0 && (!A || !B || !W_out)) return QLORA_ERR_INVALID_ARG;
+  if (!al4(A) || !al4(B) || !al4(W_out)) return QLORA_ERR_ALIGNMENT;
   st = device_ready();
   if (st != QLORA_OK) return st;
   const float s = alpha / (float)r;
@@ -318,6 +324,7 @@ qlora_status qlora_adam_step(float* params, const float* grads, float* m, float*
   if (!(eps > 0.0f) || !isfinite(eps) || !isfinite(lr)) return QLORA_ERR_INVALID_ARG;
   if (n == 0) return QLORA_OK;
   if (!params || !grads || !m || !v) return QLORA_ERR_INVALID_ARG;
+  if (!al4(params) || !al4(grads) || !al4(m) || !al4(v)) return QLORA_ERR_ALIGNMENT;
   qlora_status st = device_ready();
   if (st != QLORA_OK) return st;
   return cuda_status(launch_adam(params, grads, m, v, n, t, lr, beta1, beta2, eps, page_elems,
@@ -342,7 +349,7 @@ static qlora_status check_linear_common(const qlora_weight* w, int64_t R, const 
   if (r > 64) return QLORA_ERR_UNSUPPORTED;
   if (compute != QLORA_COMPUTE_FP32 && compute != QLORA_COMPUTE_BF16) return QLORA_ERR_INVALID_ARG;
   if (!A || !B || !ws) return QLORA_ERR_INVALID_ARG;
-  if (!aligned(ws, 256)) return QLORA_ERR_ALIGNMENT;
+  if (!aligned(ws, 256) || !al4(A) || !al4(B)) return QLORA_ERR_ALIGNMENT;
   return QLORA_OK;
 }
 
@@ -352,6 +359,8 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
   qlora_status st = check_linear_common(w, R, A, B, r, compute, ws);
   if (st != QLORA_OK) return st;
   if (R > 0 && (!X || !Y)) return QLORA_ERR_INVALID_ARG;
+  const size_t esz = compute == QLORA_COMPUTE_BF16 ? 2 : 4;
+  if (!aligned(X, esz) || !aligned(Y, esz) || !al4(U_out)) return QLORA_ERR_ALIGNMENT;
   const FwdLayout L = fwd_layout(w, R, r, compute);
   if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   st = device_ready();
@@ -385,6 +394,10 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   if (st != QLORA_OK) return st;
   if (R > 0 && !dY) return QLORA_ERR_INVALID_ARG;
   if (R > 0 && (dA || (dB && !U_in)) && !X) return QLORA_ERR_INVALID_ARG;
+  const size_t esz = compute == QLORA_COMPUTE_BF16 ? 2 : 4;
+  if (!aligned(X, esz) || !aligned(dY, esz) || !aligned(dX, esz) || !al4(U_in) || !al4(dA) ||
+      !al4(dB))
+    return QLORA_ERR_ALIGNMENT;
   const BwdLayout L = bwd_layout(w, R, r, compute);
   if (ws_bytes < L.total) return QLORA_ERR_WORKSPACE;
   st = device_ready();

@@ -56,6 +56,7 @@ extern "C" qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t O, in
   const int64_t N = O * I;
   if (!mu) return QLORA_ERR_INVALID_ARG;
   if (N > 0 && (!W || !codes || !scale_codes || !t)) return QLORA_ERR_INVALID_ARG;
+  if ((uintptr_t)W % 4 || (uintptr_t)t % 4 || (uintptr_t)mu % 4) return QLORA_ERR_ALIGNMENT;
   if (nf4_quantize_ws(N, B, C) > kNoAllocScratchBytes) return QLORA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) {

@@ -106,6 +106,30 @@ def test_merge_and_adam_arguments_rejected_before_launch(lib):
     assert adam(None, None, None, None, 0, 1, 1e-3, 0.9, 0.999, 1e-8, 0, None) == _ffi.OK
 
 
+def test_misaligned_element_pointers_rejected_before_launch(lib):
+    ws = ctypes.create_string_buffer(4096)
+    d = ctypes.c_void_p((ctypes.addressof(ws) + 255) // 256 * 256)
+    odd = ctypes.c_void_p(d.value + 2)     # 2-byte aligned: fine for bf16, not for fp32
+    byte = ctypes.c_void_p(d.value + 1)
+    assert lib.qlora_quantize_nf4(odd, 4, 64, 64, 256, d, d, d, d, d, 2048, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_quantize_nf4_noalloc(d, 4, 64, 64, 256, d, d, odd, d, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_quantize_affine(d, 4, 64, 4, 64, d, odd, d, d, 2048, None) == _ffi.ERR_ALIGNMENT
+    w = _ffi.qlora_weight(_ffi.FMT_NF4_DQ, 64, 128, 64, 256, 4, d.value, d.value, odd.value, d.value, None, None)
+    P = ctypes.byref(w)
+    assert lib.qlora_dequantize(P, d, None) == _ffi.ERR_ALIGNMENT
+    w.group_absmax = d.value
+    assert lib.qlora_dequantize(P, odd, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_merge(P, d, odd, 8, 1.0, d, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_adam_step(d, d, odd, d, 16, 1, 1e-3, 0.9, 0.999, 1e-8, 0, None) == _ffi.ERR_ALIGNMENT
+    big = 1 << 20
+    # bf16 activations may sit on a 2-byte boundary, fp32 ones may not
+    assert lib.qlora_linear_fwd(P, byte, 4, d, d, 8, 1.0, 1, d, None, d, big, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_linear_fwd(P, odd, 4, d, d, 8, 1.0, 0, d, None, d, big, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_linear_fwd(P, d, 4, odd, d, 8, 1.0, 1, d, None, d, big, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_linear_bwd(P, d, byte, 4, d, d, 8, 1.0, None, 1, d, d, d, d, big, None) == _ffi.ERR_ALIGNMENT
+    assert lib.qlora_linear_bwd(P, d, d, 4, d, d, 8, 1.0, None, 1, d, odd, d, d, big, None) == _ffi.ERR_ALIGNMENT
+
+
 def test_workspace_sizes_are_consistent(lib):
     w = _ffi.qlora_weight(_ffi.FMT_NF4_DQ, 2048, 1024, 64, 256, 4, None, None, None, None, None, None)
     P = ctypes.byref(w)
