@@ -26,6 +26,7 @@ import numpy as np
 from . import build as _build
 
 FMT_NF4_DQ = 0
+FMT_NF4_FP32SCALE = 1
 FMT_AFFINE = 2
 
 OK = 0
@@ -165,6 +166,15 @@ def quantize_nf4(W, B: int = 64, C: int = 256, return_s: bool = False):
         raise ValueError(f"oracle_quantize_nf4 status {st}")
     w = QWeight(FMT_NF4_DQ, O, I, B, C, 4, codes, qcodes, t, float(mu[0]))
     return (w, s[:M]) if return_s else w
+
+
+def quantize_nf4_legacy(W, B: int = 64) -> QWeight:
+    """NF4 codes with the legacy scales: one fp32 block absmax s_b per block
+    (the same codes as the double-quantized format, which encodes with the
+    exact s_b too)."""
+    W = _c(W, np.float32)
+    w, s = quantize_nf4(W, B, 256, return_s=True)
+    return QWeight(FMT_NF4_FP32SCALE, w.O, w.I, B, 0, 4, w.codes, scale=np.ascontiguousarray(s))
 
 
 def decode_scale(q: int, t: float, mu: float) -> np.float32:

@@ -60,6 +60,7 @@
 #define ORACLE_ERR_ARG 2
 
 #define ORACLE_FMT_NF4_DQ 0
+#define ORACLE_FMT_NF4_FP32SCALE 1
 #define ORACLE_FMT_AFFINE 2
 
 /* ------------------------------------------------------------------------ */
@@ -322,7 +323,7 @@ int oracle_quantize_affine(const float* W, int64_t N, int32_t bits, int32_t G, u
 /* ------------------------------------------------------------------------ */
 
 typedef struct {
-  int32_t fmt; /* ORACLE_FMT_NF4_DQ or ORACLE_FMT_AFFINE */
+  int32_t fmt; /* ORACLE_FMT_NF4_DQ, ORACLE_FMT_NF4_FP32SCALE or ORACLE_FMT_AFFINE */
   int64_t O, I;
   int32_t block; /* B (NF4) or G (affine) */
   int32_t group; /* C (NF4) */
@@ -355,6 +356,11 @@ static float weight_at(const OracleWeight* w, int64_t n) {
     int64_t g = b / w->group;
     float s = oracle_decode_scale(w->qcodes[b], w->t[g], w->mu);
     return g_cb[code] * s;
+  } else if (w->fmt == ORACLE_FMT_NF4_FP32SCALE) {
+    /* [NF4] legacy scales: the block absmax s_b itself, one fp32 per block */
+    uint8_t byte = w->codes[n >> 1];
+    int code = (n & 1) ? (byte >> 4) : (byte & 15);
+    return g_cb[code] * w->scale[n / w->block];
   } else {
     int q;
     if (w->bits == 8) {

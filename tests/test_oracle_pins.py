@@ -103,6 +103,50 @@ def test_exact_round_trip_with_common_power_of_two_scale():
     assert np.array_equal(oracle.dequantize(w).view(np.uint32), W.view(np.uint32))
 
 
+def test_legacy_scales_round_trip_payload_and_error_bound():
+    """Legacy format ("NF4 representation": one fp32 scale per block).  A
+    matrix built as c[k] * s_b with a different power-of-two s_b per block
+    comes back bit for bit; the payload is ceil(N/2) + 4 ceil(N/B) bytes;
+    on random weights every error is at most half the widest gap between
+    adjacent levels times s_b, and a block's largest |w| is exact."""
+    _, c32 = oracle.nf4_codebook()
+    rng = np.random.default_rng(3)
+    B, nb = 64, 23
+    k = rng.integers(0, 16, size=(nb, B))
+    k[:, 0] = rng.choice([0, 15], size=nb)
+    sc = (2.0 ** rng.integers(-9, 3, size=nb)).astype(np.float32)
+    W = (c32[k] * sc[:, None]).astype(np.float32).reshape(1, -1)
+    w = oracle.quantize_nf4_legacy(W, B)
+    assert np.array_equal(w.scale, sc)
+    assert np.array_equal(oracle.dequantize(w).view(np.uint32), W.view(np.uint32))
+    W2 = synth.normal(31, (48, 320), std=0.02)
+    w2 = oracle.quantize_nf4_legacy(W2, B)
+    N = W2.size
+    assert w2.codes.size + 4 * w2.scale.size == oracle.legacy_payload_bytes(N, B)
+    Wh = oracle.dequantize(w2).reshape(-1, B).astype(np.float64)
+    Wf = W2.reshape(-1, B).astype(np.float64)
+    half_gap = np.max(np.diff(c32.astype(np.float64))) / 2
+    s = np.abs(Wf).max(axis=1)
+    assert np.all(np.abs(Wh - Wf) <= half_gap * s[:, None] * (1 + 1e-6))
+    j = np.abs(Wf).argmax(axis=1)
+    assert np.array_equal(Wh[np.arange(len(j)), j], Wf[np.arange(len(j)), j])
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "legacy", "affine"])
+def test_forward_on_each_format_equals_dense_gemm(fmt):
+    W = synth.normal(32, (80, 128), std=0.02)
+    w = {"nf4": lambda: oracle.quantize_nf4(W, 64, 3), "legacy": lambda: oracle.quantize_nf4_legacy(W, 64),
+         "affine": lambda: oracle.quantize_affine(W, 8, 32)}[fmt]()
+    X = synth.normal(33, (6, 128))
+    A = synth.normal(34, (4, 128), std=0.02)
+    Bm = synth.normal(35, (80, 4), std=0.02)
+    Wh = oracle.dequantize(w).astype(np.float64)
+    Y, _ = oracle.linear_fwd(w, X, A, Bm, 4, 8.0)
+    X64 = X.astype(np.float64)
+    ref = X64 @ Wh.T + 2.0 * (X64 @ A.astype(np.float64).T) @ Bm.astype(np.float64).T
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-12)
+
+
 def test_double_quant_special_codes_and_error_bound():
     W = synth.normal(77, (64, 1024), std=0.02)
     w, s = oracle.quantize_nf4(W, 64, 256, return_s=True)
