@@ -142,6 +142,50 @@ def test_workspace_sizes_are_consistent(lib):
     assert lib.qlora_linear_workspace_bytes(P, 16, 8, 2, 1) == 0
 
 
+def _a256(x):
+    return -(-x // 256) * 256
+
+
+def _planned_splits(Mw, KB, R, sms=148):
+    """The tensor-core tile plan as the design states it: token tile = the
+    smallest power of two >= R in 16..256, halved (not below 64) while the
+    grid fills under 3/4 of a wave; below one wave of tiles, split K so the
+    grid is one wave (two CTAs per SM below 256-token tiles), keeping at
+    least 4 K steps per split and no empty split."""
+    mt = Mw // 128
+    bn = 16
+    while bn < 256 and bn < R:
+        bn *= 2
+    while bn > 64 and 4 * mt * (-(-R // bn)) < 3 * sms:
+        bn //= 2
+    tiles = mt * (-(-R // bn))
+    splits = 1
+    if 0 < tiles < sms:
+        splits = max(1, min((1 if bn >= 256 else 2) * sms // tiles, max(1, KB // 4)))
+    per = -(-KB // splits)
+    return bn, -(-KB // per)
+
+
+@pytest.mark.parametrize("O,I,R", [(12288, 4096, 1), (12288, 4096, 16), (4096, 4096, 1), (4096, 4096, 16),
+                                   (4096, 4096, 128), (2048, 1024, 4096), (1024, 1024, 4096),
+                                   (12288, 4096, 8192), (5120, 17408, 16384), (128, 128, 3)])
+def test_tensor_core_plan_through_workspace_sizes(lib, O, I, R):
+    """The bf16 workspace exceeds the fp32 one by exactly the tensor-core
+    region: the padded U/V copy (R x 64 bf16), the adapter weight operand
+    (rows x 64 bf16) and, when K is split, one fp32 partial per split.  This
+    checks the host planner (split count, no empty split) without a GPU;
+    the planner sees 148 SMs here (no device)."""
+    w = _ffi.qlora_weight(_ffi.FMT_NF4_DQ, O, I, 64, 256, 4, None, None, None, None, None, None)
+    P = ctypes.byref(w)
+    for op, Mw, KB in ((0, O, I // 64), (1, I, O // 64)):
+        extra = lib.qlora_linear_workspace_bytes(P, R, 8, op, 1) - lib.qlora_linear_workspace_bytes(P, R, 8, op, 0)
+        _, splits = _planned_splits(Mw, KB, R)
+        part = _a256(splits * R * Mw * 4) if splits > 1 else 0
+        assert extra == _a256(R * 128) + _a256(Mw * 128) + part, (op, splits)
+        per = -(-KB // splits)
+        assert 1 <= splits <= max(1, KB) and (splits - 1) * per < KB <= splits * per
+
+
 def test_status_strings(lib):
     for s in range(9):
         assert lib.qlora_status_string(s)
