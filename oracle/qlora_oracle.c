@@ -123,7 +123,7 @@ void oracle_nf4_codebook(double out64[16], float out32[16]) {
 /* ------------------------------------------------------------------------ */
 
 /*
- * [NF4] "the nearest entry in the codebook".  code = number of midpoints
+ * [NF4] each normalized weight takes its closest level.  code = number of midpoints
  * (c_k + c_{k+1})/2 (exact in fp64) strictly below x, which is argmin_k
  * |x - c_k| with the lower index kept on a tie.
  */
