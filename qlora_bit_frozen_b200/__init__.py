@@ -54,6 +54,21 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
+def _need(where: str, name: str, t: Optional[torch.Tensor], dev, shape=None, dtype=None):
+    """Reject (before any launch) a tensor the kernels would misread: not on
+    the weight's CUDA device, not dense, or of the wrong shape or dtype."""
+    if t is None:
+        return
+    if not t.is_cuda or t.device != dev:
+        raise ValueError(f"{where}: {name} must be a CUDA tensor on {dev}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{where}: {name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{where}: {name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{where}: {name} must be contiguous")
+
+
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
     """A 256-byte aligned device workspace of at least nbytes (torch allocates)."""
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
@@ -170,6 +185,7 @@ def qlora_dequantize(w: QuantizedWeight, out: Optional[torch.Tensor] = None, str
     lib = _ffi.load()
     if out is None:
         out = torch.empty((w.O, w.I), dtype=torch.float32, device=w.codes.device)
+    _need("qlora_dequantize", "out", out, w.codes.device, (w.O, w.I), torch.float32)
     cw = w.c_struct()
     _check(lib.qlora_dequantize(ctypes.byref(cw), _ptr(out), _stream(stream)), "qlora_dequantize")
     return out
@@ -185,6 +201,10 @@ def qlora_merge(w: QuantizedWeight, A: torch.Tensor, B: torch.Tensor, alpha: flo
         raise ValueError("A must be contiguous fp32 [r x I] and B contiguous fp32 [O x r]")
     if out is None:
         out = torch.empty((w.O, w.I), dtype=torch.float32, device=w.codes.device)
+    dev = w.codes.device
+    _need("qlora_merge", "A", A, dev)
+    _need("qlora_merge", "B", B, dev)
+    _need("qlora_merge", "out", out, dev, (w.O, w.I), torch.float32)
     cw = w.c_struct()
     _check(lib.qlora_merge(ctypes.byref(cw), _ptr(A), _ptr(B), r, float(alpha), _ptr(out), _stream(stream)),
            "qlora_merge")
@@ -199,6 +219,7 @@ def qlora_adam_step(params: torch.Tensor, grads: torch.Tensor, m: torch.Tensor, 
     for x in (params, grads, m, v):
         if x.dtype != torch.float32 or not x.is_contiguous() or x.numel() != n:
             raise ValueError("params, grads, m and v must be contiguous fp32 tensors of one size")
+        _need("qlora_adam_step", "params/grads/m/v", x, params.device)
     st = _ffi.load().qlora_adam_step(_ptr(params), _ptr(grads), _ptr(m), _ptr(v), n, int(t), float(lr),
                                      float(beta1), float(beta2), float(eps), int(page_elems), _stream(stream))
     _check(st, "qlora_adam_step")
@@ -232,6 +253,13 @@ def qlora_linear_fwd(w: QuantizedWeight, X: torch.Tensor, A: torch.Tensor, B: to
         U_out = torch.empty((R, r), dtype=torch.float32, device=X.device)
     if ws is None:
         ws = workspace(qlora_linear_workspace_bytes(w, R, r, OP_FWD, compute), X.device)
+    dev, f = w.codes.device, "qlora_linear_fwd"
+    _need(f, "X", X, dev, (R, w.I))
+    _need(f, "A", A, dev, (r, w.I), torch.float32)
+    _need(f, "B", B, dev, (w.O, r), torch.float32)
+    _need(f, "Y", Y, dev, (R, w.O), X.dtype)
+    _need(f, "U_out", U_out, dev, (R, r), torch.float32)
+    _need(f, "ws", ws, dev)
     cw = w.c_struct()
     st = lib.qlora_linear_fwd(ctypes.byref(cw), _ptr(X), R, _ptr(A), _ptr(B), r, float(alpha), compute,
                               _ptr(Y), _ptr(U_out), _ptr(ws), ws.numel(), _stream(stream))
@@ -258,6 +286,16 @@ def qlora_linear_bwd(w: QuantizedWeight, X: Optional[torch.Tensor], dY: torch.Te
         dB = torch.empty((w.O, r), dtype=torch.float32, device=dev)
     if ws is None:
         ws = workspace(qlora_linear_workspace_bytes(w, R, r, OP_BWD, compute), dev)
+    wd, f = w.codes.device, "qlora_linear_bwd"
+    _need(f, "dY", dY, wd, (R, w.O))
+    _need(f, "X", X, wd, (R, w.I), dY.dtype)
+    _need(f, "A", A, wd, (r, w.I), torch.float32)
+    _need(f, "B", B, wd, (w.O, r), torch.float32)
+    _need(f, "U", U, wd, (R, r), torch.float32)
+    _need(f, "dX", dX if want_dx else None, wd, (R, w.I), dY.dtype)
+    _need(f, "dA", dA if want_da else None, wd, (r, w.I), torch.float32)
+    _need(f, "dB", dB if want_db else None, wd, (w.O, r), torch.float32)
+    _need(f, "ws", ws, wd)
     cw = w.c_struct()
     st = lib.qlora_linear_bwd(ctypes.byref(cw), _ptr(X), _ptr(dY), R, _ptr(A), _ptr(B), r, float(alpha),
                               _ptr(U), compute, _ptr(dX if want_dx else None), _ptr(dA if want_da else None),

@@ -200,3 +200,34 @@ def test_no_device_means_error_not_fallback(lib):
     d = ctypes.c_void_p(wsp.value)
     st = lib.qlora_quantize_nf4(d, 1, 64, 64, 256, d, d, d, d, wsp, 2048, None)
     assert st == _ffi.ERR_CUDA
+
+
+def test_binding_rejects_host_and_misshapen_tensors(lib):
+    """The Python binding refuses, before any launch, tensors the kernels
+    would misread: host tensors, wrong shapes or dtypes, non-dense views."""
+    import torch
+    import qlora_bit_frozen_b200 as q
+    O, I, r, R = 64, 128, 8, 4
+    w = q.QuantizedWeight(q.FMT_NF4_DQ, O, I, 64, 256, 4, torch.zeros(O * I // 2, dtype=torch.uint8),
+                          torch.zeros(O * I // 64, dtype=torch.uint8), torch.zeros(1), torch.zeros(1))
+    X = torch.zeros(R, I, dtype=torch.bfloat16)
+    A = torch.zeros(r, I)
+    B = torch.zeros(O, r)
+    dY = torch.zeros(R, O, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        q.qlora_linear_fwd(w, X, A, B, 16.0)
+    with pytest.raises(ValueError, match="CUDA"):
+        q.qlora_linear_bwd(w, X, dY, A, B, 16.0)
+    with pytest.raises(ValueError, match="CUDA"):
+        q.qlora_dequantize(w)
+    with pytest.raises(ValueError, match="CUDA"):
+        q.qlora_merge(w, A, B, 16.0)
+    p = torch.zeros(16)
+    with pytest.raises(ValueError, match="CUDA"):
+        q.qlora_adam_step(p, p.clone(), p.clone(), p.clone(), 1, 1e-3)
+    with pytest.raises(ValueError):
+        q.qlora_merge(w, A.t(), B, 16.0)                      # wrong shape
+    with pytest.raises(ValueError):
+        q.qlora_adam_step(p, p[::2].clone(), p.clone(), p.clone(), 1, 1e-3)   # sizes differ
+    with pytest.raises(ValueError):
+        q.qlora_linear_fwd(w, X.to(torch.float16), A, B, 16.0)  # unsupported activation dtype
