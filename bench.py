@@ -434,8 +434,15 @@ def run_small_r(q, torch, peaks, args):
                     torch.cuda.synchronize()
                     t_call = e0.elapsed_time(e1) / reps
                     gbs = payload / (t_call * 1e-3) / 1e9
+                    # every other tensor the call touches, once: activations in
+                    # and out (bf16), A and B (fp32), U written (fwd)
+                    other = 2 * R * (lin.I + lin.O) + 4 * wl.r * (lin.I + lin.O)
+                    if op == "fwd":
+                        other += 4 * R * wl.r
+                    tgbs = (payload + other) / (t_call * 1e-3) / 1e9
                     res[op] = {"us_per_call": round(t_call * 1e3, 3), "packed_GBps": round(gbs, 1),
-                               "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+                               "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
+                               "total_GBps": round(tgbs, 1)}
                     del g
                 out[f"{name}{tag}_R{R}"] = {"packed_bytes": int(payload), **res}
             del copies, base
