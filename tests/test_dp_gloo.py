@@ -1,6 +1,7 @@
 """Data-parallel exchange on CPU: two gloo ranks each compute the adapter
 gradients of their token shard with the oracle, sum them with the same
-all-reduce the benchmark uses, and must reproduce the full-batch gradients.
+all-reduce the benchmark uses, and must reproduce the full-batch gradients;
+after one Adam step on the summed gradients the replicas stay identical.
 Also checks the max-over-ranks timing reduction and the shard split."""
 import os
 import socket
@@ -44,6 +45,12 @@ def _worker(rank, world, port, out_dir):
         gA = torch.from_numpy(dA)
         gB = torch.from_numpy(dB)
         dp.allreduce_adapter_grads([gA, gB])
+        # every replica then takes the same Adam step on the summed gradients
+        params = np.concatenate([A.ravel(), B.ravel()]).astype(np.float32)
+        grads = np.concatenate([gA.numpy().ravel(), gB.numpy().ravel()]).astype(np.float32)
+        zero = np.zeros_like(params)
+        p1, _, _ = oracle.adam_step(params, grads, zero, zero, 1, 1e-3)
+        np.save(os.path.join(out_dir, f"p{rank}.npy"), p1)
         t = dp.max_over_ranks(float(rank + 1))
         np.save(os.path.join(out_dir, f"dA{rank}.npy"), gA.numpy())
         np.save(os.path.join(out_dir, f"dB{rank}.npy"), gB.numpy())
@@ -84,3 +91,12 @@ def test_two_rank_gradient_sum_equals_full_batch(tmp_path):
         assert np.allclose(gA, dA, rtol=1e-12, atol=1e-14)
         assert np.allclose(gB, dB, rtol=1e-12, atol=1e-14)
         assert float(np.load(tmp_path / f"t{r}.npy")[0]) == 2.0
+    # replicas stay identical after the optimizer step, and follow the
+    # full-batch step
+    p0, p1 = np.load(tmp_path / "p0.npy"), np.load(tmp_path / "p1.npy")
+    assert np.array_equal(p0, p1)
+    params = np.concatenate([A.ravel(), B.ravel()]).astype(np.float32)
+    grads = np.concatenate([dA.ravel(), dB.ravel()]).astype(np.float32)
+    zero = np.zeros_like(params)
+    full, _, _ = oracle.adam_step(params, grads, zero, zero, 1, 1e-3)
+    assert np.allclose(p0, full, rtol=1e-9, atol=1e-9)
