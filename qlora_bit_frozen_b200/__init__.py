@@ -96,6 +96,51 @@ class QuantizedWeight:
                               for t in (self.codes, self.scale_codes, self.group_absmax, self.mean,
                                         self.scale, self.bias)))
 
+    _BUFFERS = ("codes", "scale_codes", "group_absmax", "mean", "scale", "bias")
+
+    def expected_sizes(self) -> dict:
+        """Element count and dtype of every buffer the format defines."""
+        N = self.O * self.I
+        if self.fmt == FMT_NF4_DQ:
+            M = -(-N // self.block)
+            S = -(-M // self.group)
+            return {"codes": ((N + 1) // 2, torch.uint8), "scale_codes": (M, torch.uint8),
+                    "group_absmax": (S, torch.float32), "mean": (1, torch.float32)}
+        ng = -(-N // self.block)
+        return {"codes": (N if self.bits == 8 else (N + 1) // 2, torch.uint8),
+                "scale": (ng, torch.float32), "bias": (ng, torch.float32)}
+
+    def state_dict(self) -> dict:
+        """Host copy of the format fields and the packed buffers, byte for
+        byte (the canonical serialization for checkpoints)."""
+        d = {"fmt": self.fmt, "O": self.O, "I": self.I, "block": self.block, "group": self.group,
+             "bits": self.bits}
+        for k in self._BUFFERS:
+            t = getattr(self, k)
+            if t is not None:
+                d[k] = t.detach().cpu().contiguous().numpy().copy()
+        return d
+
+    @classmethod
+    def from_state_dict(cls, d: dict, device="cuda") -> "QuantizedWeight":
+        """Inverse of state_dict(); every buffer is checked against the size
+        and dtype its format fields imply before it reaches the device."""
+        import numpy as np
+        w = cls(int(d["fmt"]), int(d["O"]), int(d["I"]), int(d["block"]), int(d["group"]), int(d["bits"]),
+                codes=torch.empty(0, dtype=torch.uint8))
+        if w.fmt not in (FMT_NF4_DQ, FMT_AFFINE) or w.O < 0 or w.I < 0 or w.block < 1 \
+                or (w.fmt == FMT_NF4_DQ and (w.group < 1 or w.bits != 4)) or (w.fmt == FMT_AFFINE and w.bits not in (4, 8)):
+            raise ValueError("inconsistent format fields")
+        for k, (n, dt) in w.expected_sizes().items():
+            if k not in d or d[k] is None:
+                raise ValueError(f"missing buffer {k}")
+            a = np.ascontiguousarray(d[k])
+            t = torch.from_numpy(a)
+            if t.dtype != dt or t.numel() != n:
+                raise ValueError(f"buffer {k}: expected {n} x {dt}, got {t.numel()} x {t.dtype}")
+            setattr(w, k, t.reshape(-1).to(device))
+        return w
+
     def payload_bytes(self) -> int:
         ts = [self.codes, self.scale_codes, self.group_absmax, self.mean, self.scale, self.bias]
         return sum(t.numel() * t.element_size() for t in ts if t is not None)

@@ -199,3 +199,21 @@ def test_training_loop_keeps_packed_weight_and_exports():
     ref = oracle.merge(ow, hA, hB, r, alpha)
     s = float(np.float32(alpha) / np.float32(r))
     assert np.all(np.abs(got - ref) <= _merge_bound(ref, hA, hB, s, r))
+
+
+def test_checkpoint_round_trip_keeps_outputs_bitwise(tmp_path):
+    """A quantized weight written to a file with state_dict() and read back
+    with from_state_dict() decodes and multiplies to the same bits."""
+    W = synth.normal(450, (256, 512), std=0.02)
+    gw, _ = _weights("nf4", W)
+    path = tmp_path / "w.npz"
+    np.savez(path, **gw.state_dict())
+    with np.load(path) as f:
+        gw2 = q.QuantizedWeight.from_state_dict({k: f[k] for k in f.files})
+    assert torch.equal(q.qlora_dequantize(gw), q.qlora_dequantize(gw2))
+    X = to_dev_f32(synth.normal(451, (64, 512))).to(torch.bfloat16)
+    A = to_dev_f32(synth.normal(452, (8, 512), std=0.02))
+    Bm = to_dev_f32(synth.normal(453, (256, 8), std=0.02))
+    Y1, _ = q.qlora_linear_fwd(gw, X, A, Bm, 16.0)
+    Y2, _ = q.qlora_linear_fwd(gw2, X, A, Bm, 16.0)
+    assert torch.equal(Y1, Y2)
