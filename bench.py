@@ -460,11 +460,17 @@ def time_quantize(q, torch, wl):
         q.qlora_quantize_nf4(W)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    for W in Ws:
-        q.qlora_quantize_nf4(W)  # synchronizes (reads the non-finite flag)
+    qs = [q.qlora_quantize_nf4(W) for W in Ws]  # each synchronizes (reads the non-finite flag)
     dt = time.perf_counter() - t0
     n = sum(W.numel() for W in Ws)
+    parts = {"codes": sum(w.codes.numel() for w in qs),
+             "scale_codes": sum(w.scale_codes.numel() for w in qs),
+             "group_absmax": sum(4 * w.group_absmax.numel() for w in qs),
+             "mean": sum(4 * w.mean.numel() for w in qs)}
+    total = sum(parts.values())
     return {"ms": round(dt * 1e3, 3), "weights": int(n), "GBps_fp32_in": round(n * 4 / dt / 1e9, 1),
+            "payload_bytes": {**{k: int(v) for k, v in parts.items()}, "total": int(total),
+                              "bits_per_weight": round(8 * total / n, 4)},
             "note": "host wall clock incl. the flag read-back synchronization"}
 
 
