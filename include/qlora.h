@@ -110,12 +110,13 @@ const char* qlora_status_string(qlora_status st);
 
 /*
  * HOST.  Writes the library's 16 fp32 NF4 levels (ascending, c[7] = 0) to
- * the host array `out`.  Source: "QLoRA: Fine-Tuning Under Memory
- * Constraints", "Understand what NF4 chooses" (levels follow a normal
- * distribution) and "QLoRA Fine-Tuning", "NF4 representation" (fixed
- * 16-value codebook): normal quantiles at probabilities spaced evenly from
- * delta = ((1-1/30)+(1-1/32))/2 down to 1/2 (8 positive, 7 negative, plus
- * zero), divided by the largest, rounded to fp32.
+ * the host array `out`.  Source: "QLoRA Fine-Tuning", "NF4 representation"
+ * (a fixed 16-value codebook whose constants match the canonical
+ * bitsandbytes mapping) and "QLoRA: Fine-Tuning Under Memory Constraints",
+ * "Understand what NF4 chooses" (levels follow a normal distribution).  The
+ * values are that canonical table bit for bit: normal quantiles at
+ * single-precision probabilities spaced evenly from 0.9677083 down to 1/2
+ * (8 positive, 7 negative, plus zero), divided by the largest.
  */
 qlora_status qlora_nf4_codebook(float out[16]);
 

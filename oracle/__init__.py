@@ -11,8 +11,9 @@ each function follows and the readings taken where the pages are silent.
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against values the pages print, closed forms, special cases, library
 routines (scipy's normal quantile, numpy matmul on the dequantized matrix)
-and finite differences.  Bit-level agreement with bitsandbytes' NF4 table
-and with MLX's affine rounding is parity unpinned (neither is available).
+and finite differences; the NF4 levels equal the published canonical table
+bit for bit.  Bit-level agreement with MLX's affine rounding is parity
+unpinned (MLX is not available).
 """
 from __future__ import annotations
 

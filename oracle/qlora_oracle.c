@@ -27,8 +27,10 @@
  *           "See how a scale can hide small values" (2-bit absmax example).
  *   [NFC]   same page, section "Understand what NF4 chooses": levels follow
  *           a normal distribution.  The 16 values are not printed on the
- *           pages; oracle_nf4_codebook() builds them from the normal
- *           quantile construction of the NF4 data type.
+ *           pages, which fix them as the canonical bitsandbytes mapping
+ *           ("QLoRA Fine-Tuning", "NF4 representation");
+ *           oracle_nf4_codebook() builds that table from the normal
+ *           quantile construction evaluated in single precision.
  *   [EXPORT] "QLoRA Fine-Tuning", section "Training lifecycle" (step 5:
  *           dequantize the packed weights, add the trained LoRA deltas,
  *           restore an ordinary fp32 matrix).
@@ -85,26 +87,48 @@ double oracle_norm_ppf(double p) {
 }
 
 /*
- * [NFC] NF4 levels: normal quantiles at probabilities spaced evenly from an
- * offset delta down to 1/2 -- 8 on the positive side, 7 on the negative side
- * (1/2 itself excluded on both), plus an exact zero; scaled so the largest
- * magnitude is 1; sorted ascending.  delta is the midpoint of 1 - 1/30 and
- * 1 - 1/32.  out64 keeps the fp64 values, out32 their fp32 roundings (the
- * table the quantized format uses).
+ * [NFC] + [NF4] NF4 levels.  The pages fix the table as the canonical
+ * mapping of the bitsandbytes implementation ("NF4 representation") and say
+ * the levels follow a normal distribution ("Understand what NF4 chooses").
+ * That table is the normal-quantile construction evaluated in single
+ * precision:
+ *   - offset delta = 0.9677083 (the midpoint of 1 - 1/30 and 1 - 1/32,
+ *     written to seven decimals), as an fp32 number;
+ *   - n evenly spaced fp32 probabilities from delta to 1/2 (n = 9 for the
+ *     positive side, n = 8 for the negative side), 1/2 itself dropped:
+ *     step = fp32((1/2 - delta) / (n - 1)); the first half of the sequence
+ *     steps up from delta (delta + j step), the second half down from 1/2
+ *     (1/2 - (n - 1 - j) step), every product and sum rounded to fp32;
+ *   - the standard normal quantile of each probability (fp64), rounded to
+ *     fp32: 8 positive levels, 7 negated ones, and an exact zero;
+ *   - sorted ascending and divided (fp32) by the largest.
+ * out32 is the table the quantized format uses; out64 holds the same values
+ * widened to fp64.
  */
+static void nf4_probabilities(int n, float* p) {
+  const float delta = 0.9677083f, half = 0.5f;
+  const float step = (half - delta) / (float)(n - 1);
+  for (int j = 0; j < n; ++j) {
+    if (j < n / 2) {
+      const float t = (float)j * step;
+      p[j] = delta + t;
+    } else {
+      const float t = (float)(n - 1 - j) * step;
+      p[j] = half - t;
+    }
+  }
+}
+
 void oracle_nf4_codebook(double out64[16], float out32[16]) {
-  const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
-  double v[16];
+  float pp[9], pn[8], v[16];
+  nf4_probabilities(9, pp);
+  nf4_probabilities(8, pn);
   int n = 0;
-  for (int j = 0; j < 8; ++j) v[n++] = oracle_norm_ppf(delta + (0.5 - delta) * (double)j / 8.0);
-  v[n++] = 0.0;
-  for (int j = 0; j < 7; ++j) v[n++] = -oracle_norm_ppf(delta + (0.5 - delta) * (double)j / 7.0);
-  double mx = 0.0;
-  for (int k = 0; k < 16; ++k)
-    if (fabs(v[k]) > mx) mx = fabs(v[k]);
-  for (int k = 0; k < 16; ++k) v[k] /= mx;
+  for (int j = 0; j < 8; ++j) v[n++] = (float)oracle_norm_ppf((double)pp[j]);
+  v[n++] = 0.0f;
+  for (int j = 0; j < 7; ++j) v[n++] = (float)(-oracle_norm_ppf((double)pn[j]));
   for (int a = 1; a < 16; ++a) { /* insertion sort, ascending */
-    double key = v[a];
+    float key = v[a];
     int b = a - 1;
     while (b >= 0 && v[b] > key) {
       v[b + 1] = v[b];
@@ -112,9 +136,10 @@ void oracle_nf4_codebook(double out64[16], float out32[16]) {
     }
     v[b + 1] = key;
   }
+  const float mx = v[15];
   for (int k = 0; k < 16; ++k) {
-    out64[k] = v[k];
-    out32[k] = (float)v[k];
+    out32[k] = v[k] / mx;
+    out64[k] = (double)out32[k];
   }
 }
 

@@ -105,6 +105,7 @@ int64_t nf4_blocks(int64_t N, int32_t B) { return (N + B - 1) / B; }
 qlora_status check_weight(const qlora_weight* w, bool for_linear) {
   if (!w) return QLORA_ERR_INVALID_ARG;
   if (w->O < 0 || w->I < 0 || w->block < 1) return QLORA_ERR_SHAPE;
+  if (!weight_count_ok(w->O, w->I)) return QLORA_ERR_SHAPE;
   const int64_t N = w->O * w->I;
   if (w->fmt == QLORA_FMT_NF4_DQ) {
     if (w->bits != 4 || w->group < 1) return QLORA_ERR_SHAPE;
@@ -238,7 +239,7 @@ size_t qlora_nf4_payload_bytes(int64_t N, int32_t B, int32_t C) {
 }
 
 size_t qlora_quantize_nf4_workspace_bytes(int64_t N, int32_t B, int32_t C) {
-  if (N < 0 || B < 1 || C < 1) return 0;
+  if (N < 0 || N > kMaxWeights || B < 1 || C < 1) return 0;
   return nf4_quantize_ws(N, B, C);
 }
 
@@ -246,6 +247,7 @@ qlora_status qlora_quantize_nf4(const float* W, int64_t O, int64_t I, int32_t B,
                                 uint8_t* codes, uint8_t* scale_codes, float* t, float* mu,
                                 void* ws, size_t ws_bytes, qlora_stream_t stream) {
   if (O < 0 || I < 0 || B < 1 || C < 1) return QLORA_ERR_SHAPE;
+  if (!weight_count_ok(O, I)) return QLORA_ERR_SHAPE;
   const int64_t N = O * I;
   if (!mu || !ws) return QLORA_ERR_INVALID_ARG;
   if (N > 0 && (!W || !codes || !scale_codes || !t)) return QLORA_ERR_INVALID_ARG;
@@ -275,6 +277,7 @@ qlora_status qlora_quantize_affine(const float* W, int64_t O, int64_t I, int32_t
                                    size_t ws_bytes, qlora_stream_t stream) {
   if (O < 0 || I < 0 || G < 1) return QLORA_ERR_SHAPE;
   if (bits != 4 && bits != 8) return QLORA_ERR_SHAPE;
+  if (!weight_count_ok(O, I)) return QLORA_ERR_SHAPE;
   const int64_t N = O * I;
   if (!ws) return QLORA_ERR_INVALID_ARG;
   if (N > 0 && (!W || !codes || !scale || !bias)) return QLORA_ERR_INVALID_ARG;

@@ -10,18 +10,20 @@
 namespace qlora {
 
 // ---------------------------------------------------------------------------
-// NF4 levels, fp32.  Normal quantiles at probabilities spaced evenly from
-// delta = ((1-1/30)+(1-1/32))/2 down to 1/2 (8 positive, 7 negative, 1/2
-// excluded), plus 0, divided by the largest and rounded to fp32
-// ("QLoRA: Fine-Tuning Under Memory Constraints", "Understand what NF4
-// chooses"; "QLoRA Fine-Tuning", "NF4 representation").  Every value sits at
-// least 0.02 ulp away from an fp32 rounding boundary, so the rounding is
-// unambiguous.
+// NF4 levels, fp32: the canonical table of the NF4 data type ("QLoRA
+// Fine-Tuning", "NF4 representation": the fixed 16-value codebook matches
+// the canonical bitsandbytes mapping; "QLoRA: Fine-Tuning Under Memory
+// Constraints", "Understand what NF4 chooses": the levels follow a normal
+// distribution).  These are the values printed for the NormalFloat 4-bit
+// type in the QLoRA paper's appendix, written as exact hex floats: normal
+// quantiles at single-precision probabilities spaced evenly from 0.9677083
+// down to 1/2 (8 positive, 7 negative, 1/2 excluded), plus 0, divided by
+// the largest.
 // ---------------------------------------------------------------------------
 #define QLORA_NF4_LEVELS                                                                   \
-  {-0x1.000000p+0f, -0x1.647362p-1f, -0x1.0cd65cp-1f, -0x1.94653cp-2f, -0x1.234496p-2f,    \
-   -0x1.7a6a7ap-3f, -0x1.74f0d2p-4f, 0.0f,           0x1.45f602p-4f,  0x1.4995bep-3f,     \
-   0x1.f809b4p-3f,  0x1.5a066cp-2f,  0x1.c3496ap-2f, 0x1.200f52p-1f,  0x1.722760p-1f,     \
+  {-0x1.000000p+0f, -0x1.647362p-1f, -0x1.0cd660p-1f, -0x1.946540p-2f, -0x1.23449ap-2f,    \
+   -0x1.7a6a7ep-3f, -0x1.74f0e2p-4f, 0.0f,           0x1.45f5fep-4f,  0x1.4995c6p-3f,     \
+   0x1.f809bap-3f,  0x1.5a0674p-2f,  0x1.c34970p-2f, 0x1.200f56p-1f,  0x1.722766p-1f,     \
    0x1.000000p+0f}
 
 static __device__ __constant__ float kNF4[16] = QLORA_NF4_LEVELS;

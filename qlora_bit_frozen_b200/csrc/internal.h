@@ -18,6 +18,16 @@ inline void count_launch(uint64_t n = 1) { g_launches.fetch_add(n, std::memory_o
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Largest weight count any entry point accepts (2^40, far beyond one GPU's
+// memory).  Checked before any size arithmetic, so that O * I and the byte
+// counts derived from it cannot overflow.
+constexpr int64_t kMaxWeights = (int64_t)1 << 40;
+inline bool weight_count_ok(int64_t O, int64_t I) {
+  if (O < 0 || I < 0) return false;
+  if (O == 0 || I == 0) return true;
+  return O <= kMaxWeights / I;
+}
+
 // Zeroed ticket counters after the workspace status header (1024 x u32):
 // zeroed with the header at the start of every linear call; kernels that
 // take one leave it zero again.

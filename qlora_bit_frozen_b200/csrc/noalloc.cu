@@ -53,6 +53,9 @@ extern "C" qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t O, in
                                                    uint8_t* scale_codes, float* t, float* mu,
                                                    qlora_stream_t stream) {
   if (O < 0 || I < 0 || B < 1 || C < 1) return QLORA_ERR_SHAPE;
+  // O * I (and the scratch size derived from it) is computed only once it
+  // is known not to overflow; the size check then bounds every write.
+  if (!weight_count_ok(O, I)) return QLORA_ERR_SHAPE;
   const int64_t N = O * I;
   if (!mu) return QLORA_ERR_INVALID_ARG;
   if (N > 0 && (!W || !codes || !scale_codes || !t)) return QLORA_ERR_INVALID_ARG;

@@ -50,6 +50,20 @@ def test_payload_bytes_match_oracle(lib, N, B, C):
     assert lib.qlora_nf4_payload_bytes(N, B, C) == oracle.nf4_payload_bytes(N, B, C)
 
 
+def test_overflowing_shapes_rejected_before_any_size_arithmetic(lib):
+    """O * I beyond 2^40 weights is refused with a shape error before the
+    library computes any size from it (2^31 x 2^31 would wrap a signed
+    product, and a wrapped scratch size could pass the no-alloc size check).
+    Pointers are never dereferenced: the check comes first."""
+    d = ctypes.c_void_p(256)
+    big = 1 << 31
+    assert lib.qlora_quantize_nf4_noalloc(d, big, big, 1, 1, d, d, d, d, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_quantize_nf4(d, big, big, 1, 1, d, d, d, d, d, 1 << 20, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_quantize_affine(d, big, big, 4, 64, d, d, d, d, 1 << 20, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_quantize_nf4_workspace_bytes((1 << 40) + 1, 64, 256) == 0
+    assert lib.qlora_quantize_nf4_noalloc(d, (1 << 40) + 1, 1, 64, 256, d, d, d, d, None) == _ffi.ERR_SHAPE
+
+
 def test_bad_arguments_rejected_before_launch(lib):
     ws = ctypes.create_string_buffer(1024)
     wsp = ctypes.c_void_p((ctypes.addressof(ws) + 255) // 256 * 256)

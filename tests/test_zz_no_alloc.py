@@ -4,14 +4,16 @@ It exists for callers that cannot allocate device memory themselves -- e.g.
 a plugin inside a framework whose caching allocator owns the GPU memory, or
 a C caller with no allocator -- and therefore cannot hand the library a
 workspace.  Checked here through the C ABI against qlora_quantize_nf4 (which
-uses a caller workspace): two calls in a row must both give bit-identical
-packed codes, scale codes, t_g and mu, since the shared scratch keeps the
-previous call's contents.  This file is collected last on purpose."""
+uses a caller workspace) and against the CPU oracle: two calls in a row must
+both give bit-identical packed codes, scale codes, t_g and mu, since the
+shared scratch keeps the previous call's contents.  This file is collected
+last on purpose."""
 import ctypes
 
 import numpy as np
 import pytest
 
+import oracle
 import synth
 
 torch = pytest.importorskip("torch")
@@ -46,12 +48,16 @@ def test_noalloc_matches_workspace_entry_point_twice():
         ws = torch.empty(lib.qlora_quantize_nf4_workspace_bytes(O * I, B, C), dtype=torch.uint8, device=W.device)
         st = lib.qlora_quantize_nf4(_ptr(W), O, I, B, C, *map(_ptr, ref), _ptr(ws), ws.numel(), stream)
         assert st == _ffi.OK
+        ow = oracle.quantize_nf4(W_host, B, C)
+        want = (ow.codes, ow.qcodes, np.asarray(ow.t, np.float32), np.array([ow.mu], np.float32))
         for _ in range(2):  # the second call runs on scratch holding the first call's contents
             out = _outputs(O, I, B, C, W.device)
             st = lib.qlora_quantize_nf4_noalloc(_ptr(W), O, I, B, C, *map(_ptr, out), stream)
             assert st == _ffi.OK, lib.qlora_status_string(st)
-            for a, b in zip(out, ref):
-                assert np.array_equal(a.cpu().numpy().view(np.uint8), b.cpu().numpy().view(np.uint8))
+            for a, b, o in zip(out, ref, want):
+                got = a.cpu().numpy().view(np.uint8)
+                assert np.array_equal(got, b.cpu().numpy().view(np.uint8))
+                assert np.array_equal(got, np.ascontiguousarray(o).view(np.uint8))
 
 
 def test_noalloc_rejects_inputs_beyond_its_scratch():
