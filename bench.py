@@ -36,7 +36,8 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "QLoRA linear fwd+bwd TFLOP/s (large R) & packed-weight HBM GB/s (small R), % roofline"
-DEFAULT_WORKLOAD = "qwen3_0.6b_attn_qv"
+DEFAULT_WORKLOAD = "14b_layer"
+OTHER_WORKLOADS = ["qwen3_0.6b_attn_qv", "8b_mlp"]
 
 
 def algorithmic_flops(wl: synth.Workload, R: int) -> float:
@@ -107,9 +108,10 @@ class ClockSampler:
 
 class Layer:
     """Device buffers of one linear: quantized weight, adapters, inputs,
-    outputs and workspaces (all allocated before timing)."""
+    outputs and workspaces (all allocated before timing).  dA and dB are
+    views into the caller's flat gradient arena (one all-reduce per step)."""
 
-    def __init__(self, q, torch, wl, li, R, rank_seed):
+    def __init__(self, q, torch, wl, li, R, rank_seed, dA, dB, host_outputs):
         lin = wl.linears[li]
         dev = "cuda"
         W = synth.weight(wl, li)
@@ -124,17 +126,21 @@ class Layer:
         ds = synth.normal(wl.seed(li, "dY") + 7919 * rank_seed, (R, lin.O))
         _, xb = synth.bf16_round(xs)
         _, db = synth.bf16_round(ds)
-        self.x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
-        self.dy_host = torch.from_numpy(db.view(np.int16)).view(torch.bfloat16).pin_memory()
-        self.X = self.x_host.to(dev)
-        self.dY = self.dy_host.to(dev)
+        del xs, ds
+        xh = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
+        dh = torch.from_numpy(db.view(np.int16)).view(torch.bfloat16)
+        self.X = xh.to(dev)
+        self.dY = dh.to(dev)
+        self.x_host = xh.pin_memory() if host_outputs else None
+        self.dy_host = dh.pin_memory() if host_outputs else None
         self.Y = torch.empty((R, lin.O), dtype=torch.bfloat16, device=dev)
         self.U = torch.empty((R, wl.r), dtype=torch.float32, device=dev)
         self.dX = torch.empty((R, lin.I), dtype=torch.bfloat16, device=dev)
-        self.dA = torch.empty((wl.r, lin.I), dtype=torch.float32, device=dev)
-        self.dB = torch.empty((lin.O, wl.r), dtype=torch.float32, device=dev)
-        self.dA_host = torch.empty_like(self.dA, device="cpu").pin_memory()
-        self.dB_host = torch.empty_like(self.dB, device="cpu").pin_memory()
+        self.dA = dA
+        self.dB = dB
+        if host_outputs:  # the step's results, read back by the end-to-end pass
+            self.y_host = torch.empty_like(self.Y, device="cpu").pin_memory()
+            self.dx_host = torch.empty_like(self.dX, device="cpu").pin_memory()
         self.ws_f = q.workspace(q.qlora_linear_workspace_bytes(self.w, R, wl.r, 0, q.COMPUTE_BF16))
         self.ws_b = q.workspace(q.qlora_linear_workspace_bytes(self.w, R, wl.r, 1, q.COMPUTE_BF16))
         self.alpha = wl.alpha
@@ -145,6 +151,31 @@ class Layer:
         q.qlora_linear_fwd(self.w, X, self.A, self.B, self.alpha, Y=self.Y, U_out=self.U, ws=self.ws_f)
         q.qlora_linear_bwd(self.w, X, dY, self.A, self.B, self.alpha, U=self.U, dX=self.dX, dA=self.dA,
                            dB=self.dB, ws=self.ws_b)
+
+
+class Model:
+    """Every linear of a workload on this rank, with the adapter gradients
+    of all of them in one flat fp32 arena."""
+
+    def __init__(self, q, torch, wl, rank, host_outputs=False):
+        R = wl.R
+        sizes = [(wl.r * l.I, l.O * wl.r) for l in wl.linears]
+        self.grads = torch.empty(sum(a + b for a, b in sizes), dtype=torch.float32, device="cuda")
+        self.layers = []
+        off = 0
+        for li, (na, nb) in enumerate(sizes):
+            lin = wl.linears[li]
+            dA = self.grads[off:off + na].view(wl.r, lin.I)
+            dB = self.grads[off + na:off + na + nb].view(lin.O, wl.r)
+            off += na + nb
+            self.layers.append(Layer(q, torch, wl, li, R, rank, dA, dB, host_outputs))
+        if host_outputs:
+            self.grads_host = torch.empty_like(self.grads, device="cpu").pin_memory()
+
+    def step(self, q, dp, xs=None, dys=None):
+        for i, L in enumerate(self.layers):
+            L.step(q, None if xs is None else xs[i], None if dys is None else dys[i])
+        dp.allreduce_flat(self.grads)
 
 
 def measured_traffic(workload, kernel):
@@ -167,47 +198,31 @@ def measured_traffic(workload, kernel):
     return int(k["dram_bytes_per_launch"]) if k else None
 
 
-def run_gpu(args):
-    import torch
-    import torch.distributed as dist
+def choose_peak(peaks, ms_per_step):
+    """Roofline denominator: the measured burst bf16 figure for kernels in a
+    short step, the sustained (seconds-long, power-capped) one when the
+    kernels are timed inside a long step (>= 1 ms per step, repeated)."""
+    if ms_per_step >= 1.0:
+        return peaks["bf16_tflops_sustained"], f"{peaks['source']} bf16 dense (sustained: kernels timed inside a {ms_per_step:.1f} ms step)"
+    return peaks["bf16_tflops"], f"{peaks['source']} bf16 dense (burst: kernels timed inside a {ms_per_step:.3f} ms step)"
 
-    import qlora_bit_frozen_b200 as q
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    wl = synth.workload(args.workload)
-    R = wl.R
-    layers = [Layer(q, torch, wl, li, R, rank) for li in range(len(wl.linears))]
-    l2 = torch.cuda.get_device_properties(local).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device="cuda")
+def measure_step(q, torch, dist, dp, model, wl, world, steps, warmup, flush, peaks, sample_clocks=None):
+    """Device-timed step of `model` (graph replays between CUDA events, L2
+    flushed outside the events, max over ranks) plus the per-kernel pass.
+    Returns the metrics of one workload."""
     stream = torch.cuda.current_stream()
-
-    from qlora_bit_frozen_b200 import dp
-
-    def allreduce_grads():
-        dp.allreduce_adapter_grads([g for L in layers for g in (L.dA, L.dB)])
-
-    def step():
-        for L in layers:
-            L.step(q)
-        allreduce_grads()
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
-        step()
+        model.step(q, dp)
     barrier()
 
-    # ------------------------------------------------ timed region (device)
     # One step is captured once in a CUDA graph (no host launch gaps in the
     # device timing) and replayed K times between CUDA events.  A second
     # graph of the same step, with the library's event pair around each
@@ -220,39 +235,38 @@ def run_gpu(args):
         cap = torch.cuda.Stream()
         cap.wait_stream(torch.cuda.current_stream())
         with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
-            step()
+            model.step(q, dp)
         torch.cuda.synchronize()
         return g
 
     n_before = q.qlora_kernel_launch_count()
     graph = capture()
     kernels_per_step = q.qlora_kernel_launch_count() - n_before
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.zero_()
         graph.replay()
     barrier()
-    clocks = ClockSampler(local)
-    clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if sample_clocks is not None:
+        sample_clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
         graph.replay()
         ev[i][1].record(stream)
     barrier()
-    clk = clocks.stop()
-    launches = kernels_per_step * args.steps
+    clk = sample_clocks.stop() if sample_clocks is not None else None
     ms = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), device="cuda")
     del graph
 
-    nrec = 16 * len(layers)
+    nrec = 16 * len(model.layers)
     q.qlora_kernel_timing_enable(nrec)
     tgraph = capture()
     tgraph.replay()  # warm-up; each replay re-records the same event pairs
     torch.cuda.synchronize()
     recs = []
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         tgraph.replay()
         torch.cuda.synchronize()
@@ -262,15 +276,85 @@ def run_gpu(args):
             print(f"kernel timing unavailable: {e}", file=sys.stderr)
     del tgraph
     q.qlora_kernel_timing_enable(0)
-    for L in layers:
+    for L in model.layers:
         assert q.qlora_workspace_status(L.ws_f) == 0 and q.qlora_workspace_status(L.ws_b) == 0
-    ms_per_step = ms / args.steps
-    flops_step = algorithmic_flops(wl, R)
+    ms_per_step = ms / steps
+    flops_step = algorithmic_flops(wl, wl.R)
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
 
+    by_kind = {}
+    for kind, kms, kfl in recs:
+        d = by_kind.setdefault(kind, [0.0, 0.0, 0])
+        d[0] += kms
+        d[1] += kfl
+        d[2] += 1
+    kernels = {}
+    for kind, (kms, kfl, n) in sorted(by_kind.items()):
+        name = "tc_qlinear_fwd" if kind == 0 else "tc_qlinear_dx"
+        kernels[name] = {"launches": n, "ms_total": round(kms, 4),
+                         "tflops": round(kfl / (kms * 1e-3) / 1e12, 2) if kms > 0 else None,
+                         "share_of_step": round(kms / ms, 4) if ms > 0 else None}
+    roofline = None
+    if by_kind:
+        kind, (kms, kfl, n) = max(by_kind.items(), key=lambda kv: kv[1][0])
+        achieved = kfl / (kms * 1e-3) / 1e12
+        peak, src = choose_peak(peaks, ms_per_step)
+        kname = "tc_qlinear_fwd" if kind == 0 else "tc_qlinear_dx"
+        roofline = {"bound": "tensor", "kernel": kname,
+                    "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / peak, 4), "traffic": measured_traffic(wl.name, kname),
+                    "peak_source": src, "frac_of_burst_peak": round(achieved / peaks["bf16_tflops"], 4),
+                    "flops_per_launch": kfl / n, "avg_launch_ms": kms / n}
+    step_peak, step_src = choose_peak(peaks, ms_per_step)
+    return {"ms_per_step": ms_per_step, "value": value, "kernels": kernels, "roofline": roofline,
+            "kernels_per_step": int(kernels_per_step), "clocks": clk,
+            "step_frac_of_peak": round(value / world / step_peak, 4),
+            "step_frac_of_burst_peak": round(value / world / peaks["bf16_tflops"], 4),
+            "step_peak_source": step_src}
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import qlora_bit_frozen_b200 as q
+    from qlora_bit_frozen_b200 import dp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    peaks = load_peaks()
+    wl = synth.workload(args.workload)
+    R = wl.R
+    model = Model(q, torch, wl, rank, host_outputs=True)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    main = measure_step(q, torch, dist, dp, model, wl, world, args.steps, args.warmup, flush, peaks,
+                        sample_clocks=clocks)
+    launches = main["kernels_per_step"] * args.steps
+    ms_per_step = main["ms_per_step"]
+    flops_step = algorithmic_flops(wl, R)
+    value = main["value"]
+
     # ---------------------------------------- end to end through the API
+    # Every step copies its inputs X, dY in from pinned host memory and its
+    # results back out: Y, dX of every linear and the summed adapter
+    # gradients (the flat dA/dB arena).
+    layers = model.layers
     h2d = sum(L.x_host.numel() * 2 + L.dy_host.numel() * 2 for L in layers)
-    d2h = sum(L.dA.numel() * 4 + L.dB.numel() * 4 for L in layers)
+    d2h = sum(L.Y.numel() * 2 + L.dX.numel() * 2 for L in layers) + model.grads.numel() * 4
     xs = [torch.empty_like(L.X) for L in layers]
     dys = [torch.empty_like(L.dY) for L in layers]
 
@@ -278,51 +362,46 @@ def run_gpu(args):
         for L, X, dY in zip(layers, xs, dys):
             X.copy_(L.x_host, non_blocking=True)
             dY.copy_(L.dy_host, non_blocking=True)
-            L.step(q, X, dY)
-        allreduce_grads()
+        model.step(q, dp, xs, dys)
         for L in layers:
-            L.dA_host.copy_(L.dA, non_blocking=True)
-            L.dB_host.copy_(L.dB, non_blocking=True)
+            L.y_host.copy_(L.Y, non_blocking=True)
+            L.dx_host.copy_(L.dX, non_blocking=True)
+        model.grads_host.copy_(model.grads, non_blocking=True)
 
+    e2e_steps = max(3, min(args.steps, 10))
     for _ in range(max(1, min(args.warmup, 3))):
         e2e_step()
     barrier()
-    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for i in range(args.steps):
+    ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    for i in range(e2e_steps):
         flush.zero_()
         ee[i][0].record(stream)
         e2e_step()
         ee[i][1].record(stream)
     barrier()
     ems = dp.max_over_ranks(sum(a.elapsed_time(b) for a, b in ee), device="cuda")
-    e2e_value = flops_step * world / (ems / args.steps * 1e-3) / 1e12
+    e2e_value = flops_step * world / (ems / e2e_steps * 1e-3) / 1e12
+    del xs, dys, model
+    torch.cuda.empty_cache()
 
-    # ------------------------------------------------------------- roofline
-    peaks = load_peaks()
-    by_kind = {}
-    for kind, kms, kfl in recs:
-        d = by_kind.setdefault(kind, [0.0, 0.0, 0])
-        d[0] += kms
-        d[1] += kfl
-        d[2] += 1
-    dom = max(by_kind.items(), key=lambda kv: kv[1][0]) if by_kind else None
-    roofline = None
-    kernels = {}
-    for kind, (kms, kfl, n) in sorted(by_kind.items()):
-        name = "tc_qlinear_fwd" if kind == 0 else "tc_qlinear_dx"
-        kernels[name] = {"launches": n, "ms_total": round(kms, 4),
-                         "tflops": round(kfl / (kms * 1e-3) / 1e12, 2) if kms > 0 else None,
-                         "share_of_step": round(kms / ms, 4) if ms > 0 else None}
-    if dom is not None:
-        kind, (kms, kfl, n) = dom
-        achieved = kfl / (kms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
-        kname = "tc_qlinear_fwd" if kind == 0 else "tc_qlinear_dx"
-        roofline = {"bound": "tensor", "kernel": kname,
-                    "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                    "frac": round(achieved / peak, 4), "traffic": measured_traffic(wl.name, kname),
-                    "peak_source": f"{peaks['source']} bf16 dense (burst)",
-                    "flops_per_launch": kfl / n, "avg_launch_ms": kms / n}
+    # --------------------------- the other large-R configurations, same rules
+    others = {}
+    for name in args.also:
+        if name == wl.name:
+            continue
+        owl = synth.workload(name)
+        om = Model(q, torch, owl, rank)
+        r = measure_step(q, torch, dist, dp, om, owl, world, args.steps, args.warmup, flush, peaks)
+        others[name] = {"value": round(r["value"], 3), "unit": "TFLOP/s", "ms_per_step": round(r["ms_per_step"], 5),
+                        "tokens_per_gpu": owl.R, "r": owl.r,
+                        "step_frac_of_peak": r["step_frac_of_peak"],
+                        "step_frac_of_burst_peak": r["step_frac_of_burst_peak"],
+                        "step_peak_source": r["step_peak_source"],
+                        "roofline": r["roofline"], "kernels": r["kernels"],
+                        "kernels_per_step": r["kernels_per_step"]}
+        launches += r["kernels_per_step"] * args.steps
+        del om
+        torch.cuda.empty_cache()
 
     small = None
     if args.small_r and world == 1:
@@ -341,7 +420,7 @@ def run_gpu(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, args.cpu_rows)
+        cpu = cpu_baseline(wl, args.cpu_rows if args.cpu_rows > 0 else default_sample_rows(wl))
 
     if world > 1:
         dist.barrier()
@@ -356,12 +435,19 @@ def run_gpu(args):
                        "nf4_block": wl.block, "dq_group": wl.group, "compute": "bf16, fp32 accumulate",
                        "parallelism": f"dp{world}" if world > 1 else "single GPU",
                        "l2": "flushed between timed steps (2x L2 write, outside the events)"},
-            "roofline": roofline, "kernels": kernels,
+            "step_frac_of_peak": main["step_frac_of_peak"],
+            "step_frac_of_burst_peak": main["step_frac_of_burst_peak"],
+            "step_peak_source": main["step_peak_source"],
+            "roofline": main["roofline"], "kernels": main["kernels"],
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d),
-                    "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ems / args.steps, 5)},
-            "clocks": clk, "gpu_launches": int(launches), "kernels_per_step": int(kernels_per_step),
+                    "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ems / e2e_steps, 5),
+                    "steps": e2e_steps,
+                    "copies": "X, dY in; Y, dX and the all-reduced dA/dB arena out, every step"},
+            "clocks": main["clocks"], "gpu_launches": int(launches),
+            "kernels_per_step": main["kernels_per_step"],
             "timing": "device step captured once in a CUDA graph and replayed; CUDA events around each replay; per-kernel durations from a second pass with events around each tensor-core launch",
+            "other_configs": others,
             "small_r": small, "quantize": quant, "export": export,
         }
         print(json.dumps(line), flush=True)
@@ -370,11 +456,12 @@ def run_gpu(args):
 
 
 def run_small_r(q, torch, peaks, args):
-    """Bandwidth-bound regime: R in {1, 16} against W [4096 x 4096] and
+    """Bandwidth-bound regime: R in {1, 16, 128} against W [4096 x 4096] and
     [12288 x 4096], forward and dX, GB/s on packed weight bytes.  Formats:
-    NF4 (B=64, C=256, tensor-core path) and affine 4/8-bit with G=64 (SIMT
-    path).  Cold L2: rotating weight copies totalling >= 4x L2, captured in
-    a CUDA graph."""
+    NF4 (B=64, C=256) and affine 4/8-bit with G in {32, 64, 128}.  Cold L2:
+    rotating weight copies totalling >= 4x L2, captured in a CUDA graph.
+    At 128 tokens the call is above the ridge point, so TFLOP/s (2 R O I
+    per call) is reported beside GB/s."""
     out = {}
     l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
 
@@ -388,17 +475,18 @@ def run_small_r(q, torch, peaks, args):
         wl = synth.workload(name)
         lin = wl.linears[0]
         W = torch.from_numpy(synth.weight(wl, 0)).cuda()
-        formats = [("", q.qlora_quantize_nf4(W, 64, 256))]
+        formats = [("", lambda: q.qlora_quantize_nf4(W, 64, 256))]
         for bits in (4, 8):
-            formats.append((f"_affine{bits}_G64", q.qlora_quantize_affine(W, bits, 64)))
-        del W
+            for G in (32, 64, 128):
+                formats.append((f"_affine{bits}_G{G}", lambda bits=bits, G=G: q.qlora_quantize_affine(W, bits, G)))
         A = torch.from_numpy(synth.adapters(wl, 0)[0]).cuda()
         B = torch.from_numpy(synth.adapters(wl, 0)[1]).cuda()
-        for tag, base in formats:
+        for tag, make in formats:
+            base = make()
             payload = base.payload_bytes()
             ncopy = max(2, math.ceil(4 * l2 / payload))
             copies = [base] + [clone(base) for _ in range(ncopy - 1)]
-            for R in (1, 16):
+            for R in (1, 16, 128):
                 X = torch.randn((R, lin.I), device="cuda").to(torch.bfloat16)
                 dY = torch.randn((R, lin.O), device="cuda").to(torch.bfloat16)
                 Y = torch.empty((R, lin.O), device="cuda", dtype=torch.bfloat16)
@@ -442,11 +530,13 @@ def run_small_r(q, torch, peaks, args):
                     tgbs = (payload + other) / (t_call * 1e-3) / 1e9
                     res[op] = {"us_per_call": round(t_call * 1e3, 3), "packed_GBps": round(gbs, 1),
                                "frac_hbm": round(gbs / peaks["hbm_gbs"], 4),
-                               "total_GBps": round(tgbs, 1)}
+                               "total_GBps": round(tgbs, 1),
+                               "tflops": round(2.0 * R * lin.O * lin.I / (t_call * 1e-3) / 1e12, 3)}
                     del g
                 out[f"{name}{tag}_R{R}"] = {"packed_bytes": int(payload), **res}
             del copies, base
             torch.cuda.empty_cache()
+        del W
     out["peak_GBps"] = peaks["hbm_gbs"]
     out["peak_source"] = f"{peaks['source']} HBM copy bandwidth"
     out["timing"] = f"CUDA graph of >= 64 calls rotating weight copies >= 4x L2"
@@ -527,6 +617,16 @@ def time_export(q, torch, peaks):
 
 # --------------------------------------------------------------- CPU oracle
 
+def default_sample_rows(wl) -> int:
+    """Tokens of the oracle's bounded sample: about 1e11 algorithmic flops
+    (tens of seconds of fp64 work on a few host cores), 16..1024 tokens,
+    never more than the workload has."""
+    per_token = algorithmic_flops(wl, 1)
+    rows = int(1e11 // per_token)
+    rows = max(16, min(1024, rows))
+    return min(rows, wl.R)
+
+
 def cpu_baseline(wl, rows):
     """The oracle (plain C, fp64, OpenMP) on the first `rows` tokens of every
     linear: Y, U, dX, dA, dB.  TFLOP/s on the algorithmic flops of the sample."""
@@ -545,7 +645,8 @@ def cpu_baseline(wl, rows):
     fl = algorithmic_flops(wl, R)
     return {"value": round(fl / t_total / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
             "kind": "oracle", "seconds": round(t_total, 3),
-            "sample": f"first {R} of {wl.R} tokens of every linear of {wl.name}; Y, U, dX, dA, dB in fp64"}
+            "sample": f"first {R} of {wl.R} tokens of every linear of {wl.name}; Y, U, dX, dA, dB in fp64 "
+                      f"(the rate is per algorithmic flop of the sample; the oracle's cost is linear in tokens)"}
 
 
 def run_reference(args):
@@ -555,7 +656,7 @@ def run_reference(args):
         return
     import oracle
     wl = synth.workload(args.workload)
-    R = min(args.ref_rows, wl.R)
+    R = min(args.ref_rows if args.ref_rows > 0 else default_sample_rows(wl), wl.R)
     prep = []
     for li in range(len(wl.linears)):
         W = synth.weight(wl, li)
@@ -588,23 +689,53 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def main():
+def launch_ranks(args, argv):
+    """--gpus N > 1 outside a torchrun launch: start N ranks on this node
+    (one per GPU) with torch.distributed.run on 127.0.0.1 and return its
+    exit status."""
+    import socket
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd, cwd=ROOT)
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOADS[1:])
-    ap.add_argument("--cpu-rows", type=int, default=1 << 30,
-                    help="tokens of the CPU-baseline sample (default: the whole workload)")
-    ap.add_argument("--ref-rows", type=int, default=1024, help="tokens per step of the reference arm")
+    ap.add_argument("--also", nargs="*", default=None,
+                    help="other large-R workloads timed the same way into other_configs "
+                         "(default: the Qwen3-0.6B q/v and 8B MLP configurations)")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="tokens of the CPU-baseline sample (0: a bounded sample of about 1e11 flops)")
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="tokens per step of the reference arm (0: the same bounded sample size)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-small-r", dest="small_r", action="store_false")
     ap.add_argument("--no-export", dest="export", action="store_false",
                     help="skip timing the fp32 export (merge) and the adapter Adam step")
-    args = ap.parse_args()
+    ap.add_argument("--print-ranks", action="store_true",
+                    help="each rank prints its RANK/WORLD_SIZE as JSON and exits (checks the launcher)")
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.also is None:
+        args.also = list(OTHER_WORKLOADS)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args, argv))
+    if args.print_ranks:
+        print(json.dumps({"rank": int(os.environ.get("RANK", "0")),
+                          "world": int(os.environ.get("WORLD_SIZE", "1")),
+                          "local_rank": int(os.environ.get("LOCAL_RANK", "0"))}), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

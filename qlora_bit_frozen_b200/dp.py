@@ -26,6 +26,17 @@ def allreduce_adapter_grads(grads: Iterable[torch.Tensor], group=None) -> None:
         dist.all_reduce(g, op=dist.ReduceOp.SUM, group=group)
 
 
+def allreduce_flat(grads: torch.Tensor, group=None) -> None:
+    """Sum one flat gradient arena (every dA and dB of the model laid out
+    back to back) in place over all ranks: one collective per step instead
+    of one per tensor."""
+    if not dist.is_available() or not dist.is_initialized():
+        return
+    if dist.get_world_size(group) == 1:
+        return
+    dist.all_reduce(grads, op=dist.ReduceOp.SUM, group=group)
+
+
 def max_over_ranks(value: float, device="cpu", group=None) -> float:
     """The maximum of a per-rank scalar (step time) over all ranks."""
     if not dist.is_available() or not dist.is_initialized() or dist.get_world_size(group) == 1:

@@ -9,10 +9,10 @@ import sys
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _run(env_extra):
+def _run(env_extra, extra_args=("--impl", "reference", "--workload", "qwen3_0.6b_attn_qv",
+                                 "--steps", "1", "--warmup", "3", "--ref-rows", "16")):
     env = dict(os.environ, **env_extra)
-    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                          "--steps", "1", "--warmup", "3", "--ref-rows", "16"],
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *extra_args],
                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
     return [l for l in out.stdout.splitlines() if l.startswith("{")]
@@ -37,3 +37,30 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_other_ranks_exit_quietly():
     assert _run({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_default_workload_is_the_largest_single_gpu_config():
+    import bench
+    assert bench.DEFAULT_WORKLOAD == "14b_layer"
+    assert set(bench.OTHER_WORKLOADS) == {"qwen3_0.6b_attn_qv", "8b_mlp"}
+
+
+def test_gpus_flag_starts_one_rank_per_gpu():
+    """--gpus 2 outside torchrun re-launches itself with torch.distributed.run:
+    two ranks start, each sees its own RANK / LOCAL_RANK and WORLD_SIZE 2."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--print-ranks"],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    ranks = sorted((json.loads(l)["rank"], json.loads(l)["local_rank"], json.loads(l)["world"])
+                   for l in out.stdout.splitlines() if l.startswith("{"))
+    assert ranks == [(0, 0, 2), (1, 1, 2)]
+
+
+def test_default_sample_is_bounded():
+    import bench
+    import synth
+    for name in ("qwen3_0.6b_attn_qv", "8b_mlp", "14b_layer"):
+        wl = synth.workload(name)
+        rows = bench.default_sample_rows(wl)
+        assert 16 <= rows <= 1024 and bench.algorithmic_flops(wl, rows) <= 1.5e11

@@ -42,9 +42,13 @@ def _worker(rank, world, port, out_dir):
         w = oracle.quantize_nf4(W)
         lo, hi = dp.shard_rows(wl.R, world, rank)
         _, dA, dB = oracle.linear_bwd(w, X[lo:hi], dY[lo:hi], A, B, wl.r, wl.alpha, want_dx=False)
-        gA = torch.from_numpy(dA)
-        gB = torch.from_numpy(dB)
+        gA = torch.from_numpy(dA.copy())
+        gB = torch.from_numpy(dB.copy())
         dp.allreduce_adapter_grads([gA, gB])
+        # the benchmark's form: every gradient in one flat arena, one collective
+        flat = torch.from_numpy(np.concatenate([dA.ravel(), dB.ravel()]))
+        dp.allreduce_flat(flat)
+        np.save(os.path.join(out_dir, f"flat{rank}.npy"), flat.numpy())
         # every replica then takes the same Adam step on the summed gradients
         params = np.concatenate([A.ravel(), B.ravel()]).astype(np.float32)
         grads = np.concatenate([gA.numpy().ravel(), gB.numpy().ravel()]).astype(np.float32)
@@ -91,6 +95,8 @@ def test_two_rank_gradient_sum_equals_full_batch(tmp_path):
         assert np.allclose(gA, dA, rtol=1e-12, atol=1e-14)
         assert np.allclose(gB, dB, rtol=1e-12, atol=1e-14)
         assert float(np.load(tmp_path / f"t{r}.npy")[0]) == 2.0
+        flat = np.load(tmp_path / f"flat{r}.npy")
+        assert np.array_equal(flat, np.concatenate([gA.ravel(), gB.ravel()]))
     # replicas stay identical after the optimizer step, and follow the
     # full-batch step
     p0, p1 = np.load(tmp_path / "p0.npy"), np.load(tmp_path / "p1.npy")

@@ -232,16 +232,23 @@ def test_bf16_adapter_only_and_zero_alpha():
 
 
 @pytest.mark.parametrize("name", ["bw_sweep_4096", "bw_sweep_12288"])
-@pytest.mark.parametrize("R", [1, 16, 128])
+@pytest.mark.parametrize("R", [1, 2, 4, 8, 13, 16, 128])
 def test_bf16_small_row_sweep_nf4(name, R):
     wl = synth.workload(name, R=R)
     _check(_run_layer(wl, 0, want=("Y", "dX")), TOL["bf16"])
 
 
+@pytest.mark.parametrize("name", ["bw_sweep_4096", "bw_sweep_12288"])
+@pytest.mark.parametrize("R", [1, 16, 128])
 @pytest.mark.parametrize("bits,G", [(4, 32), (4, 64), (4, 128), (8, 32), (8, 64), (8, 128)])
-def test_bf16_small_row_sweep_affine(bits, G):
-    wl = synth.workload("bw_sweep_4096", R=16)
-    _check(_run_layer(wl, 0, want=("Y", "dX"), fmt="affine", bits=bits, G=G), TOL["bf16"])
+def test_bf16_small_row_sweep_affine(name, R, bits, G):
+    """Affine weights at 1, 16 and 128 tokens against both sweep matrices:
+    the single-token, the up-to-16-token and the many-token paths, for
+    every (bits, G) of the sweep.  The 128-token case on the larger matrix
+    compares 32 sampled rows (the oracle computes them one by one)."""
+    wl = synth.workload(name, R=R)
+    rows = synth.sample_rows(R, 32, seed=R + bits + G) if (R == 128 and name.endswith("12288")) else None
+    _check(_run_layer(wl, 0, rows=rows, want=("Y", "dX"), fmt="affine", bits=bits, G=G), TOL["bf16"])
 
 
 @pytest.mark.parametrize("name,li", [("8b_mlp", 0), ("8b_mlp", 2), ("14b_layer", 1), ("14b_layer", 6)])
