@@ -66,8 +66,9 @@ typedef enum {
 } qlora_status;
 
 typedef enum {
-  QLORA_FMT_NF4_DQ = 0, /* NF4 codes + u8 scale codes + fp32 t_g + fp32 mu */
-  QLORA_FMT_AFFINE = 2  /* 4/8-bit codes + fp32 scale and bias per group   */
+  QLORA_FMT_NF4_DQ = 0,        /* NF4 codes + u8 scale codes + fp32 t_g + fp32 mu */
+  QLORA_FMT_NF4_FP32SCALE = 1, /* NF4 codes + one fp32 absmax per block (legacy) */
+  QLORA_FMT_AFFINE = 2         /* 4/8-bit codes + fp32 scale and bias per group   */
 } qlora_format;
 
 typedef enum {
@@ -86,6 +87,12 @@ typedef enum {
  *            scale_codes  M = ceil(N/B) bytes q_b
  *            group_absmax S = ceil(M/C) floats t_g
  *            mean         1 float mu
+ *   NF4_FP32SCALE (legacy scale storage):  block = B, group ignored,
+ *            bits = 4.
+ *            codes        ceil(N/2) bytes, as for NF4_DQ
+ *            scale        M = ceil(N/B) floats: the block absmax s_b itself
+ *            (ceil(N/2) + 4M payload bytes, about 4.5 bits per weight at
+ *            B = 64; w_hat = c[code] * s_b)
  *   AFFINE:  block = G (weights per group), group ignored, bits = 4 or 8.
  *            codes        ceil(N*bits/8) bytes (4-bit: low nibble first)
  *            scale, bias  ceil(N/G) floats each
@@ -172,6 +179,30 @@ qlora_status qlora_quantize_nf4_noalloc(const float* W, int64_t O, int64_t I, in
                                         uint8_t* codes, uint8_t* scale_codes, float* t, float* mu,
                                         qlora_stream_t stream);
 
+/*
+ * HOST.  Payload bytes of the legacy format: ceil(N/2) + 4 ceil(N/B)
+ * ("QLoRA Fine-Tuning", "NF4 representation": one fp32 scale per block,
+ * about 4.5 bits per weight at B = 64).  0 on bad arguments.
+ */
+size_t qlora_nf4_fp32scale_payload_bytes(int64_t N, int32_t B);
+
+/* HOST.  Workspace bytes qlora_quantize_nf4_fp32scale needs (the status header). */
+size_t qlora_quantize_nf4_fp32scale_workspace_bytes(int64_t N, int32_t B);
+
+/*
+ * Quantize W [O x I] fp32 to NF4 with the legacy scale storage ("QLoRA
+ * Fine-Tuning", "NF4 representation": each block's absmax kept as an fp32
+ * number).  Codes exactly as qlora_quantize_nf4 (nearest level to
+ * fp32(w / s_b), ties to the lower level, low nibble first, an all-zero
+ * block gets s_b = 0 and code 7); scale[b] = s_b.
+ * Outputs (device): codes [ceil(N/2)], scale [M].  Bit-exact and
+ * deterministic.  Synchronizes `stream` to read the non-finite flag
+ * (QLORA_ERR_NONFINITE on NaN/Inf).  N = 0 is valid.
+ */
+qlora_status qlora_quantize_nf4_fp32scale(const float* W, int64_t O, int64_t I, int32_t B,
+                                          uint8_t* codes, float* scale, void* ws, size_t ws_bytes,
+                                          qlora_stream_t stream);
+
 /* HOST.  Workspace bytes qlora_quantize_affine needs. */
 size_t qlora_quantize_affine_workspace_bytes(int64_t N, int32_t bits, int32_t G);
 
@@ -195,6 +226,7 @@ qlora_status qlora_quantize_affine(const float* W, int64_t O, int64_t I, int32_t
  * kernels never call).  W_hat [O x I] fp32:
  *   NF4_DQ: c[code] * s_hat_b,  s_hat_b = clamp(mu + fp32(fp32(t_g (q_b -
  *           128)) / 127), 0, FLT_MAX);
+ *   NF4_FP32SCALE: c[code] * s_b;
  *   AFFINE: fp32(scale_g * code) + bias_g.
  * Bit-exact.  Never used by qlora_linear_fwd / qlora_linear_bwd.
  */

@@ -16,17 +16,18 @@ from typing import Optional, Tuple
 import torch
 
 from . import _ffi
-from ._ffi import (COMPUTE_BF16, COMPUTE_FP32, FMT_AFFINE, FMT_NF4_DQ, OP_BWD, OP_FWD,
-                   qlora_weight)
+from ._ffi import (COMPUTE_BF16, COMPUTE_FP32, FMT_AFFINE, FMT_NF4_DQ, FMT_NF4_FP32SCALE, OP_BWD,
+                   OP_FWD, qlora_weight)
 
 __all__ = [
     "QLoraError", "QuantizedWeight", "qlora_status_string", "qlora_nf4_codebook",
     "qlora_nf4_payload_bytes", "qlora_quantize_nf4", "qlora_quantize_nf4_noalloc", "qlora_quantize_affine",
+    "qlora_nf4_fp32scale_payload_bytes", "qlora_quantize_nf4_fp32scale",
     "qlora_dequantize", "qlora_merge", "qlora_adam_step",
     "qlora_linear_workspace_bytes", "qlora_linear_fwd", "qlora_linear_bwd",
     "qlora_workspace_status", "qlora_selftest_wait_timeout", "qlora_kernel_launch_count",
     "qlora_kernel_timing_enable", "qlora_kernel_timing_collect",
-    "COMPUTE_FP32", "COMPUTE_BF16", "FMT_NF4_DQ", "FMT_AFFINE", "workspace",
+    "COMPUTE_FP32", "COMPUTE_BF16", "FMT_NF4_DQ", "FMT_NF4_FP32SCALE", "FMT_AFFINE", "workspace",
 ]
 
 
@@ -106,6 +107,8 @@ class QuantizedWeight:
             S = -(-M // self.group)
             return {"codes": ((N + 1) // 2, torch.uint8), "scale_codes": (M, torch.uint8),
                     "group_absmax": (S, torch.float32), "mean": (1, torch.float32)}
+        if self.fmt == FMT_NF4_FP32SCALE:
+            return {"codes": ((N + 1) // 2, torch.uint8), "scale": (-(-N // self.block), torch.float32)}
         ng = -(-N // self.block)
         return {"codes": (N if self.bits == 8 else (N + 1) // 2, torch.uint8),
                 "scale": (ng, torch.float32), "bias": (ng, torch.float32)}
@@ -128,8 +131,9 @@ class QuantizedWeight:
         import numpy as np
         w = cls(int(d["fmt"]), int(d["O"]), int(d["I"]), int(d["block"]), int(d["group"]), int(d["bits"]),
                 codes=torch.empty(0, dtype=torch.uint8))
-        if w.fmt not in (FMT_NF4_DQ, FMT_AFFINE) or w.O < 0 or w.I < 0 or w.block < 1 \
-                or (w.fmt == FMT_NF4_DQ and (w.group < 1 or w.bits != 4)) or (w.fmt == FMT_AFFINE and w.bits not in (4, 8)):
+        if w.fmt not in (FMT_NF4_DQ, FMT_NF4_FP32SCALE, FMT_AFFINE) or w.O < 0 or w.I < 0 or w.block < 1 \
+                or (w.fmt == FMT_NF4_DQ and (w.group < 1 or w.bits != 4)) \
+                or (w.fmt == FMT_NF4_FP32SCALE and w.bits != 4) or (w.fmt == FMT_AFFINE and w.bits not in (4, 8)):
             raise ValueError("inconsistent format fields")
         for k, (n, dt) in w.expected_sizes().items():
             if k not in d or d[k] is None:
@@ -203,6 +207,30 @@ def qlora_quantize_nf4_noalloc(W: torch.Tensor, B: int = 64, C: int = 256, strea
                                         _stream(stream))
     _check(st, "qlora_quantize_nf4_noalloc")
     return QuantizedWeight(FMT_NF4_DQ, O, I, B, C, 4, codes, q, t, mu)
+
+
+def qlora_nf4_fp32scale_payload_bytes(N: int, B: int = 64) -> int:
+    return int(_ffi.load().qlora_nf4_fp32scale_payload_bytes(N, B))
+
+
+def qlora_quantize_nf4_fp32scale(W: torch.Tensor, B: int = 64, stream=None) -> QuantizedWeight:
+    """NF4 codes with the legacy scale storage (one fp32 absmax per block) of
+    a CUDA fp32 [O x I] matrix (synchronizes the stream)."""
+    lib = _ffi.load()
+    if W.dim() != 2 or W.dtype != torch.float32 or not W.is_cuda:
+        raise ValueError("W must be a CUDA float32 matrix")
+    W = W.contiguous()
+    O, I = W.shape
+    N = O * I
+    M = -(-N // B)
+    dev = W.device
+    codes = torch.empty((N + 1) // 2, dtype=torch.uint8, device=dev)
+    scale = torch.empty(M, dtype=torch.float32, device=dev)
+    ws = workspace(lib.qlora_quantize_nf4_fp32scale_workspace_bytes(N, B), dev)
+    st = lib.qlora_quantize_nf4_fp32scale(_ptr(W), O, I, B, _ptr(codes), _ptr(scale), _ptr(ws), ws.numel(),
+                                          _stream(stream))
+    _check(st, "qlora_quantize_nf4_fp32scale")
+    return QuantizedWeight(FMT_NF4_FP32SCALE, O, I, B, 0, 4, codes, scale=scale)
 
 
 def qlora_quantize_affine(W: torch.Tensor, bits: int = 4, G: int = 64, stream=None) -> QuantizedWeight:

@@ -21,6 +21,7 @@ ERR_TIMEOUT = 7
 ERR_WORKSPACE = 8
 
 FMT_NF4_DQ = 0
+FMT_NF4_FP32SCALE = 1
 FMT_AFFINE = 2
 COMPUTE_FP32 = 0
 COMPUTE_BF16 = 1
@@ -56,6 +57,9 @@ SIGNATURES = {
     "qlora_quantize_nf4_workspace_bytes": (_sz, [_i64, _i32, _i32]),
     "qlora_quantize_nf4": (ctypes.c_int, [_P, _i64, _i64, _i32, _i32, _P, _P, _P, _P, _P, _sz, _P]),
     "qlora_quantize_nf4_noalloc": (ctypes.c_int, [_P, _i64, _i64, _i32, _i32, _P, _P, _P, _P, _P]),
+    "qlora_nf4_fp32scale_payload_bytes": (_sz, [_i64, _i32]),
+    "qlora_quantize_nf4_fp32scale_workspace_bytes": (_sz, [_i64, _i32]),
+    "qlora_quantize_nf4_fp32scale": (ctypes.c_int, [_P, _i64, _i64, _i32, _P, _P, _P, _sz, _P]),
     "qlora_quantize_affine_workspace_bytes": (_sz, [_i64, _i32, _i32]),
     "qlora_quantize_affine": (ctypes.c_int, [_P, _i64, _i64, _i32, _i32, _P, _P, _P, _P, _sz, _P]),
     "qlora_dequantize": (ctypes.c_int, [_W, _P, _P]),

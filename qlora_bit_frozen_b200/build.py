@@ -15,9 +15,9 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libqlora.so")
 
-SOURCES = ["api.cu", "quantize.cu", "simt.cu", "adapter.cu", "tc_gemm.cu", "noalloc.cu", "merge.cu",
-           "adam.cu"]
-HEADERS = ["common.cuh", "internal.h", "tc_gemm.h"]
+SOURCES = ["api.cu", "quantize.cu", "simt.cu", "adapter.cu", "tc_gemm.cu", "smallr.cu", "noalloc.cu",
+           "merge.cu", "adam.cu"]
+HEADERS = ["common.cuh", "internal.h", "tc_gemm.h", "smallr.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I" + INCLUDE, "-I" + CSRC]
@@ -41,7 +41,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     nvcc = _nvcc()
-    objs = []
+    objs, cmds = [], []
     for src in SOURCES:
         obj = os.path.join(BUILD, src.replace(".cu", ".o"))
         cmd = [nvcc, *ARCH, *FLAGS, *EXTRA.get(src, []), "-c", os.path.join(CSRC, src), "-o", obj]
@@ -49,8 +49,13 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
             cmd.insert(1, "-Xptxas=-v")
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.check_call(cmd)
+        cmds.append(cmd)
         objs.append(obj)
+    # translation units compile independently: run them side by side
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+        for _ in ex.map(subprocess.check_call, cmds):
+            pass
     cmd = [nvcc, *ARCH, "-shared", "-cudart", "static", "-o", LIB, *objs]
     if verbose:
         print(" ".join(cmd), flush=True)

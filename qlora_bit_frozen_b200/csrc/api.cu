@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "smallr.h"
 #include "tc_gemm.h"
 
 namespace qlora {
@@ -112,6 +113,10 @@ qlora_status check_weight(const qlora_weight* w, bool for_linear) {
     if (N > 0 && (!w->codes || !w->scale_codes || !w->group_absmax || !w->mean))
       return QLORA_ERR_INVALID_ARG;
     if (!al4(w->group_absmax) || !al4(w->mean)) return QLORA_ERR_ALIGNMENT;
+  } else if (w->fmt == QLORA_FMT_NF4_FP32SCALE) {
+    if (w->bits != 4) return QLORA_ERR_SHAPE;
+    if (N > 0 && (!w->codes || !w->scale)) return QLORA_ERR_INVALID_ARG;
+    if (!al4(w->scale)) return QLORA_ERR_ALIGNMENT;
   } else if (w->fmt == QLORA_FMT_AFFINE) {
     if (w->bits != 4 && w->bits != 8) return QLORA_ERR_SHAPE;
     if (N > 0 && (!w->codes || !w->scale || !w->bias)) return QLORA_ERR_INVALID_ARG;
@@ -147,10 +152,10 @@ WView view_of(const qlora_weight* w) {
 constexpr size_t kWsZeroed = kWsHeader + kWsTickets;
 
 struct FwdLayout {
-  size_t u = 0, red = 0, split = 0, tc = 0, total = 0;
+  size_t u = 0, red = 0, split = 0, sr = 0, tc = 0, total = 0;
 };
 struct BwdLayout {
-  size_t u = 0, v = 0, bt = 0, red = 0, red2 = 0, split = 0, split2 = 0, gemv = 0, tc = 0,
+  size_t u = 0, v = 0, bt = 0, red = 0, red2 = 0, split = 0, split2 = 0, gemv = 0, sr = 0, tc = 0,
          total = 0;
 };
 
@@ -163,6 +168,8 @@ FwdLayout fwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
   off += rowdot_ws(R, w->I, r);
   L.split = off;  // bf16 hi / lo copy of A (above rank 8)
   off += adapter_split_ws(w->I, r);
+  L.sr = off;  // split-K partials of the few-token path
+  if (compute == QLORA_COMPUTE_BF16) off += smallr_ws(false, view_of(w), R);
   L.tc = off;
   if (compute == QLORA_COMPUTE_BF16) off += tc_fwd_ws(view_of(w), R);
   L.total = off;
@@ -197,6 +204,8 @@ BwdLayout bwd_layout(const qlora_weight* w, int64_t R, int32_t r, int32_t comput
   off += adapter_split_ws(R, r);
   L.gemv = off;  // dX partials of the small-R affine path
   off += gemv_dx_ws(view_of(w), R);
+  L.sr = off;  // split-K partials of the few-token path
+  if (compute == QLORA_COMPUTE_BF16) off += smallr_ws(true, view_of(w), R);
   L.tc = off;
   if (compute == QLORA_COMPUTE_BF16) off += tc_dx_ws(view_of(w), R);
   L.total = off;
@@ -257,6 +266,38 @@ qlora_status qlora_quantize_nf4(const float* W, int64_t O, int64_t I, int32_t B,
   if (st != QLORA_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   st = cuda_status(launch_nf4_quantize(W, N, B, C, codes, scale_codes, t, mu, ws, s));
+  if (st != QLORA_OK) return st;
+  uint32_t h[3];
+  st = read_header(ws, s, h);
+  if (st != QLORA_OK) return st;
+  if (h[2]) return QLORA_ERR_NONFINITE;
+  return h[0] ? (qlora_status)h[0] : QLORA_OK;
+}
+
+size_t qlora_nf4_fp32scale_payload_bytes(int64_t N, int32_t B) {
+  if (N < 0 || N > kMaxWeights || B < 1) return 0;
+  return (size_t)((N + 1) / 2) + 4 * (size_t)((N + B - 1) / B);
+}
+
+size_t qlora_quantize_nf4_fp32scale_workspace_bytes(int64_t N, int32_t B) {
+  if (N < 0 || N > kMaxWeights || B < 1) return 0;
+  return kWsHeader;
+}
+
+qlora_status qlora_quantize_nf4_fp32scale(const float* W, int64_t O, int64_t I, int32_t B,
+                                          uint8_t* codes, float* scale, void* ws, size_t ws_bytes,
+                                          qlora_stream_t stream) {
+  if (O < 0 || I < 0 || B < 1) return QLORA_ERR_SHAPE;
+  if (!weight_count_ok(O, I)) return QLORA_ERR_SHAPE;
+  const int64_t N = O * I;
+  if (!ws) return QLORA_ERR_INVALID_ARG;
+  if (N > 0 && (!W || !codes || !scale)) return QLORA_ERR_INVALID_ARG;
+  if (!aligned(ws, 256) || !al4(W) || !al4(scale)) return QLORA_ERR_ALIGNMENT;
+  if (ws_bytes < kWsHeader) return QLORA_ERR_WORKSPACE;
+  qlora_status st = device_ready();
+  if (st != QLORA_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  st = cuda_status(launch_nf4_fp32scale_quantize(W, N, B, codes, scale, ws, s));
   if (st != QLORA_OK) return st;
   uint32_t h[3];
   st = read_header(ws, s, h);
@@ -378,7 +419,14 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
   float* U = U_out ? U_out : (float*)((char*)ws + L.u);
   const WView v = view_of(w);
   const bool bf16 = compute == QLORA_COMPUTE_BF16;
-  if (bf16 && tc_fwd_supported(v, X, Y, R)) {
+  if (bf16 && smallr_supported(v, R, X, Y)) {
+    // 1..16 tokens: U = X A^T, then the bandwidth-bound GEMV, which starts
+    // its weight stream at once and waits for U only in its epilogue
+    e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, nullptr, nullptr, 0, 0, 1.0f, nullptr,
+                      nullptr, red, tickets, (uint16_t*)((char*)ws + L.split));
+    if (e == cudaSuccess)
+      e = launch_smallr_fwd(v, X, R, U, B, r, sc, Y, (char*)ws + L.sr, (uint32_t*)ws, tickets, s);
+  } else if (bf16 && tc_fwd_supported(v, X, Y, R)) {
     void* tcws = (char*)ws + L.tc;
     e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws), B, w->O, 0, sc,
                       tc_w_pad(tcws, R), nullptr, red, tickets, (uint16_t*)((char*)ws + L.split));
@@ -416,7 +464,8 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   void* red = (char*)ws + L.red;
   // V = dY B  (B is [O x r]: L(k = o, j) = B[o*r + j]); its padded bf16 copy
   // feeds the tensor-core kernel's adapter step
-  const bool tc = dX && bf16 && tc_dx_supported(v, dY, dX, R);
+  const bool sr = dX && bf16 && smallr_supported(v, R, dY, dX);
+  const bool tc = !sr && dX && bf16 && tc_dx_supported(v, dY, dX, R);
   void* tcws = (char*)ws + L.tc;
   if (dX || dA) {
     float* bt = (float*)((char*)ws + L.bt);
@@ -452,7 +501,9 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   // (programmatic dependent launch) and waits for them only before its
   // adapter step, which reads the padded V written above.
   if (e == cudaSuccess && dX) {
-    if (tc)
+    if (sr)
+      e = launch_smallr_dx(v, dY, R, V, A, r, sc, dX, (char*)ws + L.sr, (uint32_t*)ws, tickets, s);
+    else if (tc)
       e = launch_tc_dx(v, dY, R, V, A, r, sc, dX, tcws, (uint32_t*)ws, s);
     else
       e = launch_simt_dx(v, dY, R, A, V, r, sc, bf16, dX, s, (float*)((char*)ws + L.gemv));

@@ -106,16 +106,21 @@ __device__ __forceinline__ float decode_block_scale(uint32_t q, float t, float m
   return s;
 }
 
+// Scale of NF4 block b: the double-quantized s_hat_b, or the stored fp32
+// absmax of the legacy format ("NF4 representation": legacy scale storage).
+__device__ __forceinline__ float nf4_block_scale(const WView& w, int64_t b) {
+  if (w.fmt == QLORA_FMT_NF4_FP32SCALE) return __ldg(w.scale + b);
+  const int64_t g = b / w.group;
+  return decode_block_scale(__ldg(w.qcodes + b), __ldg(w.t + g), __ldg(w.mu));
+}
+
 // w_hat at flat index n (per-element decode; used by the SIMT and
 // diagnostic kernels).
 __device__ __forceinline__ float decode_weight(const WView& w, int64_t n) {
-  if (w.fmt == QLORA_FMT_NF4_DQ) {
+  if (w.fmt != QLORA_FMT_AFFINE) {
     uint32_t byte = __ldg(w.codes + (n >> 1));
     uint32_t code = (n & 1) ? (byte >> 4) : (byte & 15u);
-    int64_t b = n / w.block;
-    int64_t g = b / w.group;
-    float s = decode_block_scale(__ldg(w.qcodes + b), __ldg(w.t + g), __ldg(w.mu));
-    return __fmul_rn(kNF4[code], s);
+    return __fmul_rn(kNF4[code], nf4_block_scale(w, n / w.block));
   } else {
     uint32_t q;
     if (w.bits == 8) {

@@ -40,6 +40,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 cudaError_t launch_nf4_quantize(const float* W, int64_t N, int32_t B, int32_t C, uint8_t* codes,
                                 uint8_t* qcodes, float* t, float* mu, void* ws, cudaStream_t st);
 size_t nf4_quantize_ws(int64_t N, int32_t B, int32_t C);
+// legacy scale storage: codes and the fp32 block absmax (ws: the status header)
+cudaError_t launch_nf4_fp32scale_quantize(const float* W, int64_t N, int32_t B, uint8_t* codes,
+                                          float* scale, void* ws, cudaStream_t st);
 cudaError_t launch_affine_quantize(const float* W, int64_t N, int32_t bits, int32_t G,
                                    uint8_t* codes, float* scale, float* bias, void* ws,
                                    cudaStream_t st);

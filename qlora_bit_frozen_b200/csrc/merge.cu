@@ -47,12 +47,17 @@ __device__ __forceinline__ uint64_t idiv(uint64_t a, uint32_t d) {
 // levels read different banks; the constant cache would serialize them).
 template <bool NARROW>
 __device__ __forceinline__ float weight1(const WView& w, uint64_t n, const float* lut) {
-  if (w.fmt == QLORA_FMT_NF4_DQ) {
+  if (w.fmt != QLORA_FMT_AFFINE) {
     const uint32_t byte = __ldg(w.codes + (n >> 1));
     const uint32_t code = (n & 1) ? (byte >> 4) : (byte & 15u);
     const uint64_t b = idiv<NARROW>(n, (uint32_t)w.block);
-    const uint64_t g = idiv<NARROW>(b, (uint32_t)w.group);
-    const float sb = decode_block_scale(__ldg(w.qcodes + b), __ldg(w.t + g), __ldg(w.mu));
+    float sb;
+    if (w.fmt == QLORA_FMT_NF4_FP32SCALE) {
+      sb = __ldg(w.scale + b);
+    } else {
+      const uint64_t g = idiv<NARROW>(b, (uint32_t)w.group);
+      sb = decode_block_scale(__ldg(w.qcodes + b), __ldg(w.t + g), __ldg(w.mu));
+    }
     return __fmul_rn(lut[code], sb);
   }
   uint32_t q;
@@ -70,10 +75,15 @@ __device__ __forceinline__ float weight1(const WView& w, uint64_t n, const float
 // one block (group), one scale decode.
 template <bool NARROW>
 __device__ __forceinline__ void weight4(const WView& w, uint64_t n0, const float* lut, float v[4]) {
-  if (w.fmt == QLORA_FMT_NF4_DQ) {
+  if (w.fmt != QLORA_FMT_AFFINE) {
     const uint64_t b = idiv<NARROW>(n0, (uint32_t)w.block);
-    const uint64_t g = idiv<NARROW>(b, (uint32_t)w.group);
-    const float sb = decode_block_scale(__ldg(w.qcodes + b), __ldg(w.t + g), __ldg(w.mu));
+    float sb;
+    if (w.fmt == QLORA_FMT_NF4_FP32SCALE) {
+      sb = __ldg(w.scale + b);
+    } else {
+      const uint64_t g = idiv<NARROW>(b, (uint32_t)w.group);
+      sb = decode_block_scale(__ldg(w.qcodes + b), __ldg(w.t + g), __ldg(w.mu));
+    }
     const uint32_t lo = __ldg(w.codes + (n0 >> 1));
     const uint32_t hi = __ldg(w.codes + (n0 >> 1) + 1);
     v[0] = __fmul_rn(lut[lo & 15u], sb);

@@ -1,4 +1,5 @@
-// quantize.cu -- NF4 double-quant and affine quantizers, diagnostic dequantize.
+// quantize.cu -- NF4 quantizers (double-quantized and legacy fp32 scales),
+// the affine quantizer, diagnostic dequantize.
 //
 // "QLoRA Fine-Tuning" (Riftco Transformer how-to), section "NF4
 // representation": blockwise absmax s_b, nearest of the 16 NF4 levels to
@@ -217,6 +218,21 @@ cudaError_t launch_nf4_quantize(const float* W, int64_t N, int32_t B, int32_t C,
   if (S > 0) {
     nf4_dq_kernel<<<grid_for(S * 32, kThreads), kThreads, 0, st>>>(s, M, C, S, mu, t, qcodes);
     count_launch(1);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_nf4_fp32scale_quantize(const float* W, int64_t N, int32_t B, uint8_t* codes,
+                                          float* scale, void* ws, cudaStream_t st) {
+  const int64_t M = (N + B - 1) / B;
+  uint32_t* hdr = (uint32_t*)ws;
+  cudaError_t e = cudaMemsetAsync(ws, 0, kWsHeader, st);
+  if (e != cudaSuccess) return e;
+  if (M > 0) {
+    // the absmax is the stored scale itself; codes as in the double-quantized format
+    nf4_absmax_kernel<<<grid_for(M * 32, kThreads), kThreads, 0, st>>>(W, N, B, M, scale, hdr);
+    nf4_encode_kernel<<<grid_for((N + 1) / 2, kThreads), kThreads, 0, st>>>(W, N, B, scale, codes);
+    count_launch(2);
   }
   return cudaGetLastError();
 }

@@ -1,0 +1,954 @@
+// smallr.cu -- the QLoRA linear layer at a handful of tokens (1..16).
+//
+// Forward  Y  = X W_hat^T + s U B^T     ("QLoRA Fine-Tuning", "Forward and
+// Input    dX = dY W_hat + s V A         backward": every weight decoded from
+// gradient                               its code and block scale inside the
+//                                        sums; "LoRA vs QLoRA on Apple
+//                                        Silicon", "Results": the 4-bit base
+//                                        reads 4x fewer weight bytes)
+//
+// With 1..16 tokens the layer streams the packed weight once and does a few
+// multiply-adds per weight: it is bound by HBM bandwidth on the packed
+// bytes, and the work per byte is the decode.  The kernels here are a
+// split-K GEMV shaped for that:
+//
+//  * the weight is the M side of mma.sync.m16n8k16 (bf16 in, fp32
+//    accumulate); the tokens are N (one or two 8-token tiles), so a single
+//    token wastes MMA columns, not decode work;
+//  * codes are decoded two weights at a time through a 256-entry byte table
+//    in shared memory: entry[byte] = (v[byte & 15], v[byte >> 4]) as a bf16
+//    pair, one copy per lane at stride 256 bytes, so a lookup is one byte
+//    permute (which builds the address) and one conflict-free 32-bit shared
+//    load, and the result is an MMA operand register as it stands;
+//  * the tables hold UNSCALED values (the 16 NF4 levels, or the integers
+//    0..15 of affine codes), so the block or group scale is applied once per
+//    block: in the forward pass to the block's fp32 partial sums
+//    (acc += s_b * D_b; the affine bias adds bias_g * sum(x) over the group),
+//    in the input gradient to the dY operand (dY[o] * s(o, b) is the same for
+//    every column of a 64-column block);
+//  * 8-bit affine codes are split into their two nibbles: a code byte looks
+//    up (lo, hi) in the same integer table and meets the activation pair
+//    (x, 16 x), so x q = x lo + 16 x hi with the K dimension doubled;
+//  * affine groups of 32 (two per 64-column block) run two passes with the
+//    other group's operand lanes zeroed;
+//  * K is split across the CTAs of a one-wave grid; partial sums go to the
+//    workspace and the last CTA of each output tile (a ticket counter) adds
+//    them in split order, so the result is deterministic, and adds the
+//    adapter term s U B^T (or s V A) from U / V computed by the launch just
+//    before (programmatic dependent launch: the weight stream starts at
+//    once, the wait comes only before U / V are read).
+//
+// No floating-point copy of the weight exists anywhere: codes go from HBM to
+// registers and from registers, through the table, into the MMA.
+#include "common.cuh"
+#include "internal.h"
+#include "smallr.h"
+
+namespace qlora {
+
+namespace {
+
+constexpr int kSrThreads = 256;       // 8 warps
+constexpr int kTableBytes = 256 * 256;  // 256 entries x 64 words (32 lane copies used)
+constexpr int kTicketBase = 512;      // ticket counters [512, 1024) of the workspace
+
+enum SrFmt { kFmtNF4 = 0, kFmtA4 = 1, kFmtA8 = 2 };
+
+struct SrParams {
+  const uint8_t* codes;
+  const uint8_t* qcodes;  // NF4: scale codes q_b
+  const float* t;         // NF4: t_g
+  const float* mu;        // NF4: mu
+  const float* scale;     // affine scale, or the legacy format's fp32 s_b
+  const float* bias;      // affine
+  int32_t legacy;         // NF4 with fp32 block scales
+  int32_t G;              // affine group size
+  uint32_t C;             // NF4 scale-group size (blocks)
+  int32_t c_shift;        // log2(C) or -1
+  const __nv_bfloat16* act;  // X [R x I] (forward) or dY [R x O] (input gradient)
+  int32_t R;
+  int64_t O, I;
+  const float* aux;   // U [R x r] (forward) or V [R x r] (input gradient)
+  const float* lora;  // B [O x r] (forward) or A [r x I] (input gradient)
+  int32_t r;
+  float s;
+  __nv_bfloat16* out;  // Y [R x O] or dX [R x I]
+  float* part;         // split partials [splits][R][extent]
+  unsigned* tickets;   // one counter per output tile, zero on entry, left zero
+  int32_t splits;
+  int32_t per_split;   // K blocks (forward) or 16-row steps (input gradient) per split
+  uint32_t* err;
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Streamed once: bypass L1 and let L2 evict these lines first.
+__device__ __forceinline__ uint2 ld_stream_u2(const uint8_t* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+               : "=r"(v.x), "=r"(v.y)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_stream_u4(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_stream_u1(const uint8_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// The lane's copy of table entry `byte k of w`: address byte * 256 + lane * 4
+// (laneoff holds lane * 4 in its low byte, zeros above), built by one permute.
+__device__ __forceinline__ uint32_t tbl(const uint32_t* table, uint32_t w, uint32_t laneoff,
+                                        int k) {
+  const uint32_t addr = prmt(w, laneoff, 0x5504u | ((uint32_t)k << 4));
+  return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(table) + addr);
+}
+
+// Fill the byte table: NF4 levels, or the integers 0..15 (affine codes).
+template <int FMT>
+__device__ __forceinline__ void fill_table(uint32_t* table) {
+  for (int e = threadIdx.x; e < 256 * 8; e += kSrThreads) {
+    const int entry = e >> 3, q4 = e & 7;  // 8 x uint4 = 32 lane copies
+    float lo, hi;
+    if (FMT == kFmtNF4) {
+      lo = kNF4[entry & 15];
+      hi = kNF4[entry >> 4];
+    } else {
+      lo = (float)(entry & 15);
+      hi = (float)(entry >> 4);
+    }
+    const uint32_t v = pack_bf16x2(lo, hi);
+    reinterpret_cast<uint4*>(table)[entry * 16 + q4] = make_uint4(v, v, v, v);
+  }
+}
+
+// NF4 block scale of flat block index b: the double-quantized s_hat_b, or
+// the stored fp32 absmax of the legacy format.
+__device__ __forceinline__ float nf4_scale(const SrParams& p, uint32_t b, float mu) {
+  if (p.legacy) return __ldg(p.scale + b);
+  const uint32_t g = p.c_shift >= 0 ? (b >> p.c_shift) : b / p.C;
+  return decode_block_scale(__ldg(p.qcodes + b), __ldg(p.t + g), mu);
+}
+
+// ------------------------------------------------------------------ forward
+//
+// CTA: 128 weight rows x one K range (split blockIdx.y).  Warp (wr, wk):
+// rows 64 wr .. +63 (four 16-row m-tiles), K blocks kb = lo + wk, lo + wk + 4,
+// ... of the range.  Per block the lane holds, for rows g and g + 8 of each
+// m-tile, the 16 columns 16 t .. 16 t + 15 (t = lane % 4, g = lane / 4):
+// 8 code bytes (4-bit) or 16 (8-bit).  MMA j of the block pairs K index
+// (2t, 2t+1) with columns 16t + 4j + {0,1} and (2t+8, 2t+9) with
+// 16t + 4j + {2,3} (4-bit; 8-bit: one column per K pair, 16t + 2j and
+// 16t + 2j + 1), and the activation operand is loaded in the same order.
+template <int FMT>
+struct FwdShape {
+  static constexpr int kChunkU32 = FMT == kFmtA8 ? 4 : 2;  // code words per row per block
+  static constexpr int kMmas = FMT == kFmtA8 ? 8 : 4;      // MMAs per m-tile per block
+};
+
+template <int NT, int FMT, bool G32>
+__global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd_kernel(const SrParams p) {
+  using S = FwdShape<FMT>;
+  constexpr int CW = S::kChunkU32;
+  extern __shared__ __align__(1024) uint8_t sr_smem[];
+  uint32_t* table = reinterpret_cast<uint32_t*>(sr_smem);
+  fill_table<FMT>(table);
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int wr = warp & 1, wk = warp >> 1;
+  const int64_t I = p.I, O = p.O;
+  const int64_t rbase = (int64_t)blockIdx.x * 128 + 64 * wr;
+  const int KB = (int)(I / 64);
+  const int kb_lo = (int)blockIdx.y * p.per_split;
+  const int kb_hi = min(KB, kb_lo + p.per_split);
+  const uint32_t laneoff = (uint32_t)lane * 4u;
+  const int64_t row_bytes = FMT == kFmtA8 ? I : I / 2;
+  const int bbytes = FMT == kFmtA8 ? 64 : 32;  // code bytes per row per block
+  const float mu = (FMT == kFmtNF4 && !p.legacy) ? __ldg(p.mu) : 0.0f;
+  constexpr int NP = G32 ? 2 : 1;  // group passes per block
+
+  float acc[4][NT][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][n][c] = 0.0f;
+
+  // code chunks of this lane: [m-tile][row g / g + 8][words]; each m-tile's
+  // registers are refilled with the next block's codes as soon as they are
+  // decoded, so one block is always in flight without a second buffer
+  uint32_t cur[4][2][CW];
+  const uint8_t* cbase = p.codes + (rbase + g) * row_bytes + (FMT == kFmtA8 ? 16 : 8) * t;
+  auto load_mtile = [&](uint32_t (&dst)[2][CW], int mt, int kb) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint8_t* src = cbase + (int64_t)(16 * mt + 8 * h) * row_bytes + (int64_t)kb * bbytes;
+      if (CW == 2) {
+        const uint2 v = ld_stream_u2(src);
+        dst[h][0] = v.x;
+        dst[h][CW - 1] = v.y;
+      } else {
+        const uint4 v = ld_stream_u4(src);
+        dst[h][0] = v.x;
+        dst[h][1 % CW] = v.y;
+        dst[h][2 % CW] = v.z;
+        dst[h][3 % CW] = v.w;
+      }
+    }
+  };
+  // Per-row block (or group) parameters of rows rbase + lane and
+  // rbase + 32 + lane, loaded one block ahead.
+  //   NF4: q_b and t_g (decoded per block); affine: scale and bias per pass.
+  float pa[2][NP], pb[2][NP], na[2][NP], nb[2][NP];
+  auto load_params = [&](float (&sa)[2][NP], float (&sb)[2][NP], int kb) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t row = rbase + 32 * h + lane;
+      if (FMT == kFmtNF4) {
+        sa[h][0] = nf4_scale(p, (uint32_t)(row * KB + kb), mu);
+        sb[h][0] = 0.0f;
+      } else {
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+          const int64_t gi = (row * I + (int64_t)kb * 64 + 32 * q) / p.G;
+          sa[h][q] = __ldg(p.scale + gi);
+          sb[h][q] = __ldg(p.bias + gi);
+        }
+      }
+    }
+  };
+
+  int kb = kb_lo + wk;
+  if (kb < kb_hi) {
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) load_mtile(cur[mt], mt, kb);
+    load_params(pa, pb, kb);
+  }
+  const bool tok_ok0 = g < p.R, tok_ok1 = (8 + g) < p.R;
+  for (; kb < kb_hi; kb += 4) {
+    const int kbn = kb + 4;
+    const bool more = kbn < kb_hi;
+    if (more) load_params(na, nb, kbn);
+    // activation operand: columns 64 kb + 16 t + 4 m .. + 3 of tokens g and 8 + g
+    uint2 xw[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const bool ok = n == 0 ? tok_ok0 : tok_ok1;
+      const __nv_bfloat16* xr = p.act + (int64_t)(8 * n + g) * I + (int64_t)kb * 64 + 16 * t;
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        xw[n][m] = ok ? __ldg(reinterpret_cast<const uint2*>(xr + 4 * m)) : make_uint2(0u, 0u);
+    }
+    // B operand registers per MMA j: 4-bit (x[c], x[c+1]) pairs as loaded;
+    // 8-bit (x[c], 16 x[c]) pairs.
+    uint32_t bx[NT][S::kMmas][2];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      if (FMT == kFmtA8) {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const uint32_t w0 = xw[n][m].x, w1 = xw[n][m].y;
+          const uint32_t s0 = hmul2_bf16(w0, 0x41804180u), s1 = hmul2_bf16(w1, 0x41804180u);  // 16.0
+          bx[n][2 * m][0] = prmt(w0, s0, 0x5410u);
+          bx[n][2 * m][1] = prmt(w0, s0, 0x7632u);
+          bx[n][2 * m + 1][0] = prmt(w1, s1, 0x5410u);
+          bx[n][2 * m + 1][1] = prmt(w1, s1, 0x7632u);
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          bx[n][m][0] = xw[n][m].x;
+          bx[n][m][1] = xw[n][m].y;
+        }
+      }
+    }
+    // affine: sum of the activations over each group pass (ones-operand MMA)
+    float xs[NP][NT][4];
+    if (FMT != kFmtNF4) {
+      // the ones operand: (1, 1) pairs for 4-bit, (1, 0) for 8-bit (only the x half)
+      const uint32_t one = FMT == kFmtA8 ? 0x00003F80u : 0x3F803F80u;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        const uint32_t a = (!G32 || (t >> 1) == q) ? one : 0u;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) xs[q][n][c] = 0.0f;
+#pragma unroll
+          for (int j = 0; j < S::kMmas; ++j)
+            mma_bf16_16816(xs[q][n], a, a, a, a, bx[n][j][0], bx[n][j][1]);
+        }
+      }
+    }
+    // rows of this lane's accumulators: 16 mt + g (c0, c1) and 16 mt + g + 8 (c2, c3)
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+      const int srcA = 16 * (mt & 1) + g, srcB = srcA + 8;
+      const int hsel = mt >> 1;  // rows 0..31 from the first parameter set, 32..63 the second
+      float sA[NP], sB[NP], bA[NP], bB[NP];
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        const float va = hsel ? pa[1][q] : pa[0][q];
+        const float vb = hsel ? pb[1][q] : pb[0][q];
+        sA[q] = __shfl_sync(0xffffffffu, va, srcA);
+        sB[q] = __shfl_sync(0xffffffffu, va, srcB);
+        bA[q] = __shfl_sync(0xffffffffu, vb, srcA);
+        bB[q] = __shfl_sync(0xffffffffu, vb, srcB);
+      }
+      // decoded pairs of rows g (pA) and g + 8 (pB): one per code byte
+      uint32_t pA[4 * CW], pB[4 * CW];
+#pragma unroll
+      for (int w = 0; w < CW; ++w)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          pA[4 * w + k] = tbl(table, cur[mt][0][w], laneoff, k);
+          pB[4 * w + k] = tbl(table, cur[mt][1][w], laneoff, k);
+        }
+      if (more) load_mtile(cur[mt], mt, kbn);
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        const bool keep = !G32 || (t >> 1) == q;
+        float D[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) D[n][c] = 0.0f;
+#pragma unroll
+        for (int j = 0; j < S::kMmas; ++j) {
+          const uint32_t a0 = keep ? pA[2 * j] : 0u, a1 = keep ? pB[2 * j] : 0u;
+          const uint32_t a2 = keep ? pA[2 * j + 1] : 0u, a3 = keep ? pB[2 * j + 1] : 0u;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) mma_bf16_16816(D[n], a0, a1, a2, a3, bx[n][j][0], bx[n][j][1]);
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          if (FMT == kFmtNF4) {
+            acc[mt][n][0] = fmaf(sA[q], D[n][0], acc[mt][n][0]);
+            acc[mt][n][1] = fmaf(sA[q], D[n][1], acc[mt][n][1]);
+            acc[mt][n][2] = fmaf(sB[q], D[n][2], acc[mt][n][2]);
+            acc[mt][n][3] = fmaf(sB[q], D[n][3], acc[mt][n][3]);
+          } else {
+            acc[mt][n][0] = fmaf(sA[q], D[n][0], fmaf(bA[q], xs[q][n][0], acc[mt][n][0]));
+            acc[mt][n][1] = fmaf(sA[q], D[n][1], fmaf(bA[q], xs[q][n][1], acc[mt][n][1]));
+            acc[mt][n][2] = fmaf(sB[q], D[n][2], fmaf(bB[q], xs[q][n][2], acc[mt][n][2]));
+            acc[mt][n][3] = fmaf(sB[q], D[n][3], fmaf(bB[q], xs[q][n][3], acc[mt][n][3]));
+          }
+        }
+      }
+    }
+    if (more) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+          pa[h][q] = na[h][q];
+          pb[h][q] = nb[h][q];
+        }
+    }
+  }
+
+  // ---- combine the four K warps of each row half (fixed order wk = 0..3)
+  __syncthreads();  // every warp is done with the table: reuse its memory
+  float* red = reinterpret_cast<float*>(sr_smem);  // [wr][wk 1..3][mt][n][c][lane]
+  constexpr int kSlab = 4 * NT * 4 * 32;
+  if (wk > 0) {
+    float* dst = red + ((size_t)(wr * 3 + wk - 1)) * kSlab;
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[((mt * NT + n) * 4 + c) * 32 + lane] = acc[mt][n][c];
+  }
+  __syncthreads();
+  const bool single = p.splits == 1;
+  if (wk == 0) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      const float* src = red + ((size_t)(wr * 3 + k)) * kSlab;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[mt][n][c] += src[((mt * NT + n) * 4 + c) * 32 + lane];
+    }
+    if (single) griddep_wait();  // U comes from the launch before this one
+    // lane outputs: row rbase + 16 mt + g (+ 8 for c2, c3), token 8 n + 2 t (+1)
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int64_t row = rbase + 16 * mt + g + 8 * (c >> 1);
+          const int tok = 8 * n + 2 * t + (c & 1);
+          if (tok >= p.R) continue;
+          if (single) {
+            float ad = 0.0f;
+            for (int j = 0; j < p.r; ++j)
+              ad = fmaf(__ldg(p.aux + (int64_t)tok * p.r + j), __ldg(p.lora + row * p.r + j), ad);
+            p.out[(int64_t)tok * O + row] = __float2bfloat16_rn(fmaf(p.s, ad, acc[mt][n][c]));
+          } else {
+            p.part[((int64_t)blockIdx.y * p.R + tok) * O + row] = acc[mt][n][c];
+          }
+        }
+  }
+  if (single) {
+    if (threadIdx.x == 0) griddep_wait();
+    return;
+  }
+  // ---- split-K: the last CTA of this 128-row tile sums the partials in order
+  __shared__ unsigned s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    s_last = atomicAdd(&p.tickets[blockIdx.x], 1u) == (unsigned)(p.splits - 1) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) {
+    if (threadIdx.x == 0) griddep_wait();
+    return;
+  }
+  __threadfence();
+  griddep_wait();
+  const int64_t r0 = (int64_t)blockIdx.x * 128;
+  for (int e = threadIdx.x; e < 128 * p.R; e += kSrThreads) {
+    const int tok = e >> 7;
+    const int64_t row = r0 + (e & 127);
+    float v = 0.0f;
+    for (int sp = 0; sp < p.splits; ++sp) v += __ldcg(p.part + ((int64_t)sp * p.R + tok) * O + row);
+    float ad = 0.0f;
+    for (int j = 0; j < p.r; ++j)
+      ad = fmaf(__ldg(p.aux + (int64_t)tok * p.r + j), __ldg(p.lora + row * p.r + j), ad);
+    p.out[(int64_t)tok * O + row] = __float2bfloat16_rn(fmaf(p.s, ad, v));
+  }
+  if (threadIdx.x == 0) p.tickets[blockIdx.x] = 0u;  // ready for the next call
+}
+
+// ------------------------------------------------------------ input gradient
+//
+// CTA: one 64-column block cb of W (the M side: 64 outputs of dX) x one
+// range of W rows (split blockIdx.y), the rows split evenly over the 8
+// warps.  A K step is 16 rows (4-bit) or 8 rows (8-bit).
+//   4-bit: lane (g, t) reads bytes 4 g .. 4 g + 3 of the block (columns
+//     8 g .. 8 g + 7) of rows o + 2t, o + 2t + 1, o + 2t + 8, o + 2t + 9; the
+//     nibbles of two consecutive rows are interleaved into bytes
+//     (w[o][c], w[o+1][c]) and looked up, giving the MMA pairs along K.
+//   8-bit: bytes 8 g .. 8 g + 7 (columns 8 g .. 8 g + 7) of rows o + t and
+//     o + t + 4; a byte's (lo, hi) pair is the K pair, met by (v, 16 v).
+// M mapping (both): m-tile mt row g <-> column 8 g + 2 mt, row g + 8 <->
+// column 8 g + 2 mt + 1.  The B operand is dY[token][row] times the row's
+// scale for this block (NF4 s_hat, affine scale), rounded to bf16; the
+// affine bias enters through a ones-operand MMA with dY * bias.
+template <int FMT>
+struct DxShape {
+  static constexpr int kStepRows = FMT == kFmtA8 ? 8 : 16;
+  static constexpr int kSteps = 4;  // K steps per loop iteration (loaded one iteration ahead)
+};
+
+template <int NT, int FMT, bool G32>
+__global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_kernel(const SrParams p) {
+  using S = DxShape<FMT>;
+  constexpr int SR = S::kStepRows, NS = S::kSteps;
+  extern __shared__ __align__(1024) uint8_t sr_smem[];
+  uint32_t* table = reinterpret_cast<uint32_t*>(sr_smem);
+  fill_table<FMT>(table);
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int64_t I = p.I, O = p.O;
+  const int cb = blockIdx.x;  // 64-column block
+  const int KB = (int)(I / 64);
+  const int64_t row_bytes = FMT == kFmtA8 ? I : I / 2;
+  const uint32_t laneoff = (uint32_t)lane * 4u;
+  const float mu = (FMT == kFmtNF4 && !p.legacy) ? __ldg(p.mu) : 0.0f;
+  constexpr int NP = G32 ? 2 : 1;
+
+  // rows of this CTA, then of this warp, in K steps
+  const int64_t nsteps_all = O / SR;
+  const int64_t st_lo = (int64_t)blockIdx.y * p.per_split;
+  const int64_t st_hi = min(nsteps_all, st_lo + (int64_t)p.per_split);
+  const int64_t cnt = st_hi > st_lo ? st_hi - st_lo : 0;
+  const int64_t w_lo = st_lo + cnt * warp / 8, w_hi = st_lo + cnt * (warp + 1) / 8;
+
+  float acc[4][NT][4];
+  float accb[NP][NT][4];  // affine bias term (same for every M row of a pass)
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[a][n][c] = 0.0f;
+#pragma unroll
+  for (int q = 0; q < NP; ++q)
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) accb[q][n][c] = 0.0f;
+
+  // rows of lane (g, t) within a step
+  auto step_row = [&](int i) -> int {  // i = 0..3 (4-bit) or 0..1 (8-bit)
+    if (FMT == kFmtA8) return t + 4 * i;
+    return 2 * t + (i & 1) + 8 * (i >> 1);
+  };
+  constexpr int RPL = FMT == kFmtA8 ? 2 : 4;  // rows per lane per step
+  constexpr int WPR = FMT == kFmtA8 ? 2 : 1;  // code words per row
+  // code words of this lane: [step of the iteration][row][word]; a step's
+  // registers are refilled with the next iteration's codes once decoded
+  uint32_t cur[NS][RPL][WPR];
+  const uint8_t* cbase = p.codes + (int64_t)cb * (FMT == kFmtA8 ? 64 : 32) + (FMT == kFmtA8 ? 8 : 4) * g;
+  auto load_step = [&](uint32_t (&dst)[RPL][WPR], int64_t st) {
+#pragma unroll
+    for (int i = 0; i < RPL; ++i) {
+      if (st < w_hi) {
+        const uint8_t* src = cbase + (st * SR + step_row(i)) * row_bytes;
+        if (WPR == 1) {
+          dst[i][0] = ld_stream_u1(src);
+        } else {
+          const uint2 v = ld_stream_u2(src);
+          dst[i][0] = v.x;
+          dst[i][WPR - 1] = v.y;
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < WPR; ++w) dst[i][w] = 0u;
+      }
+    }
+  };
+  // Per-row scale (and bias) for this column block: lane L holds row
+  // st0 * SR + L of the iteration's NS * SR rows (<= 64: two rows per lane
+  // for 4-bit).
+  constexpr int PRL = NS * SR / 32;  // parameter rows per lane
+  float ps[PRL][NP], pbv[PRL][NP], ns_[PRL][NP], nbv[PRL][NP];
+  auto load_params = [&](float (&sv)[PRL][NP], float (&bv)[PRL][NP], int64_t st0) {
+#pragma unroll
+    for (int k = 0; k < PRL; ++k) {
+      const int64_t row = st0 * SR + 32 * k + lane;
+      const bool ok = row < w_hi * SR;
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        if (!ok) {
+          sv[k][q] = 0.0f;
+          bv[k][q] = 0.0f;
+        } else if (FMT == kFmtNF4) {
+          sv[k][q] = nf4_scale(p, (uint32_t)(row * KB + cb), mu);
+          bv[k][q] = 0.0f;
+        } else {
+          const int64_t gi = (row * I + (int64_t)cb * 64 + 32 * q) / p.G;
+          sv[k][q] = __ldg(p.scale + gi);
+          bv[k][q] = __ldg(p.bias + gi);
+        }
+      }
+    }
+  };
+
+  int64_t st0 = w_lo;
+  if (st0 < w_hi) {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) load_step(cur[s], st0 + s);
+    load_params(ps, pbv, st0);
+  }
+  for (; st0 < w_hi; st0 += NS) {
+    const int64_t stn = st0 + NS;
+    if (stn < w_hi) load_params(ns_, nbv, stn);
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const int64_t st = st0 + s;
+      if (st >= w_hi) break;
+      const int64_t o0 = st * SR;
+      // B operand: bf16 (dY * scale) for the lane's K rows, tokens g, 8 + g
+      // 4-bit: pairs of rows (2t, 2t+1) -> b0, (2t+8, 2t+9) -> b1
+      // 8-bit: (v, 16 v) of row t -> b0, of row t + 4 -> b1
+      uint32_t bq[NP][NT][2], bb[NP][NT][2];
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          // scale / bias of the rows this register covers, from the lanes
+          // that loaded them (lane = row within the iteration mod 32)
+          float sv0, sv1, bv0, bv1;
+          const int rr0 = s * SR + (FMT == kFmtA8 ? (t + 4 * hh) : (2 * t + 8 * hh));
+          {
+            const int k0 = rr0 >> 5;
+            const float vs = k0 == 0 ? ps[0][q] : ps[PRL - 1][q];
+            const float vb = k0 == 0 ? pbv[0][q] : pbv[PRL - 1][q];
+            sv0 = __shfl_sync(0xffffffffu, vs, rr0 & 31);
+            bv0 = __shfl_sync(0xffffffffu, vb, rr0 & 31);
+          }
+          if (FMT != kFmtA8) {
+            const int rr1 = rr0 + 1;
+            const int k1 = rr1 >> 5;
+            const float vs = k1 == 0 ? ps[0][q] : ps[PRL - 1][q];
+            const float vb = k1 == 0 ? pbv[0][q] : pbv[PRL - 1][q];
+            sv1 = __shfl_sync(0xffffffffu, vs, rr1 & 31);
+            bv1 = __shfl_sync(0xffffffffu, vb, rr1 & 31);
+          } else {
+            sv1 = 0.0f;
+            bv1 = 0.0f;
+          }
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const int tok = 8 * n + g;
+            const bool ok = tok < p.R;
+            const int64_t orow = o0 + (FMT == kFmtA8 ? (t + 4 * hh) : (2 * t + 8 * hh));
+            float d0 = 0.0f, d1 = 0.0f;
+            if (ok) {
+              if (FMT == kFmtA8) {
+                d0 = __bfloat162float(p.act[(int64_t)tok * O + orow]);
+              } else {
+                const uint32_t pr = __ldg(reinterpret_cast<const uint32_t*>(p.act + (int64_t)tok * O + orow));
+                d0 = __uint_as_float(pr << 16);
+                d1 = __uint_as_float(pr & 0xFFFF0000u);
+              }
+            }
+            if (FMT == kFmtA8) {
+              const float v = d0 * sv0;
+              bq[q][n][hh] = pack_bf16x2(v, 16.0f * __bfloat162float(__float2bfloat16_rn(v)));
+              bb[q][n][hh] = pack_bf16x2(d0 * bv0, 0.0f);
+            } else {
+              bq[q][n][hh] = pack_bf16x2(d0 * sv0, d1 * sv1);
+              bb[q][n][hh] = pack_bf16x2(d0 * bv0, d1 * bv1);
+            }
+          }
+        }
+      }
+      // A operand pairs: [m-tile][a0..a3]; then refill this step's code
+      // registers with the next iteration's
+      uint32_t A[4][4];
+      if (FMT == kFmtA8) {
+        // rows t (a0: M row g, a1: M row g + 8) and t + 4 (a2, a3); column
+        // 8 g + 2 mt (+1 for M row g + 8) is byte 2 mt (+1) of the 8 bytes
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const int w = mt >> 1, k = 2 * (mt & 1);
+          A[mt][0] = tbl(table, cur[s][0][w], laneoff, k);
+          A[mt][1] = tbl(table, cur[s][0][w], laneoff, k + 1);
+          A[mt][2] = tbl(table, cur[s][1][w], laneoff, k);
+          A[mt][3] = tbl(table, cur[s][1][w], laneoff, k + 1);
+        }
+      } else {
+        // rows (2t, 2t+1) -> P1, (2t+8, 2t+9) -> P2; zip the nibbles so that
+        // byte m of ze is (w[o][8g+2m], w[o+1][8g+2m]) and of zo the odd column
+        uint32_t ze[2], zo[2];
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+          const uint32_t wa = cur[s][2 * pp][0], wb = cur[s][2 * pp + 1][0];
+          ze[pp] = (wa & 0x0F0F0F0Fu) | ((wb << 4) & 0xF0F0F0F0u);
+          zo[pp] = ((wa >> 4) & 0x0F0F0F0Fu) | (wb & 0xF0F0F0F0u);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          A[mt][0] = tbl(table, ze[0], laneoff, mt);
+          A[mt][1] = tbl(table, zo[0], laneoff, mt);
+          A[mt][2] = tbl(table, ze[1], laneoff, mt);
+          A[mt][3] = tbl(table, zo[1], laneoff, mt);
+        }
+      }
+      if (stn + s < w_hi) load_step(cur[s], stn + s);
+#pragma unroll
+      for (int q = 0; q < NP; ++q) {
+        const bool keep = !G32 || (g >> 2) == q;
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const uint32_t a0 = keep ? A[mt][0] : 0u, a1 = keep ? A[mt][1] : 0u;
+          const uint32_t a2 = keep ? A[mt][2] : 0u, a3 = keep ? A[mt][3] : 0u;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) mma_bf16_16816(acc[mt][n], a0, a1, a2, a3, bq[q][n][0], bq[q][n][1]);
+        }
+        if (FMT != kFmtNF4) {
+          const uint32_t one = keep ? 0x3F803F80u : 0u;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) mma_bf16_16816(accb[q][n], one, one, one, one, bb[q][n][0], bb[q][n][1]);
+        }
+      }
+    }
+    if (stn < w_hi) {
+#pragma unroll
+      for (int k = 0; k < PRL; ++k)
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+          ps[k][q] = ns_[k][q];
+          pbv[k][q] = nbv[k][q];
+        }
+    }
+  }
+  if (FMT != kFmtNF4) {  // the bias term belongs to every M row of its pass
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+      const bool mine = !G32 || (g >> 2) == q;
+      if (!mine) continue;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[mt][n][c] += accb[q][n][c];
+    }
+  }
+
+  // ---- combine the 8 warps (fixed order)
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(sr_smem);  // [warp 1..7][mt][n][c][lane]
+  constexpr int kSlab = 4 * NT * 4 * 32;
+  if (warp > 0) {
+    float* dst = red + (size_t)(warp - 1) * kSlab;
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[((mt * NT + n) * 4 + c) * 32 + lane] = acc[mt][n][c];
+  }
+  __syncthreads();
+  const bool single = p.splits == 1;
+  if (warp == 0) {
+    for (int k = 0; k < 7; ++k) {
+      const float* src = red + (size_t)k * kSlab;
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[mt][n][c] += src[((mt * NT + n) * 4 + c) * 32 + lane];
+    }
+    if (single) griddep_wait();  // V comes from the launches before this one
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int64_t col = (int64_t)cb * 64 + 8 * g + 2 * mt + (c >> 1);
+          const int tok = 8 * n + 2 * t + (c & 1);
+          if (tok >= p.R) continue;
+          if (single) {
+            float ad = 0.0f;
+            for (int j = 0; j < p.r; ++j)
+              ad = fmaf(__ldg(p.aux + (int64_t)tok * p.r + j), __ldg(p.lora + (int64_t)j * I + col), ad);
+            p.out[(int64_t)tok * I + col] = __float2bfloat16_rn(fmaf(p.s, ad, acc[mt][n][c]));
+          } else {
+            p.part[((int64_t)blockIdx.y * p.R + tok) * I + col] = acc[mt][n][c];
+          }
+        }
+  }
+  if (single) {
+    if (threadIdx.x == 0) griddep_wait();
+    return;
+  }
+  __shared__ unsigned s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0)
+    s_last = atomicAdd(&p.tickets[blockIdx.x], 1u) == (unsigned)(p.splits - 1) ? 1u : 0u;
+  __syncthreads();
+  if (!s_last) {
+    if (threadIdx.x == 0) griddep_wait();
+    return;
+  }
+  __threadfence();
+  griddep_wait();
+  const int64_t c0 = (int64_t)cb * 64;
+  for (int e = threadIdx.x; e < 64 * p.R; e += kSrThreads) {
+    const int tok = e >> 6;
+    const int64_t col = c0 + (e & 63);
+    float v = 0.0f;
+    for (int sp = 0; sp < p.splits; ++sp) v += __ldcg(p.part + ((int64_t)sp * p.R + tok) * I + col);
+    float ad = 0.0f;
+    for (int j = 0; j < p.r; ++j)
+      ad = fmaf(__ldg(p.aux + (int64_t)tok * p.r + j), __ldg(p.lora + (int64_t)j * I + col), ad);
+    p.out[(int64_t)tok * I + col] = __float2bfloat16_rn(fmaf(p.s, ad, v));
+  }
+  if (threadIdx.x == 0) p.tickets[blockIdx.x] = 0u;
+}
+
+// ------------------------------------------------------------------ host
+
+int sr_fmt(const WView& w) {
+  if (w.fmt != QLORA_FMT_AFFINE) return kFmtNF4;
+  return w.bits == 8 ? kFmtA8 : kFmtA4;
+}
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+struct SrPlan {
+  int tiles;      // 128-row tiles (forward) or 64-column blocks (input gradient)
+  int splits;
+  int per_split;  // K blocks or K steps per split
+};
+
+// One wave at two CTAs per SM: tiles x splits ~ 2 x SMs.
+SrPlan sr_plan(bool dx, const WView& w) {
+  SrPlan pl;
+  const int target = 2 * num_sms();
+  if (!dx) {
+    pl.tiles = (int)(w.O / 128);
+    const int KB = (int)(w.I / 64);
+    int sp = (target + pl.tiles / 2) / pl.tiles;
+    if (sp < 1) sp = 1;
+    if (sp > KB / 4) sp = KB / 4 > 0 ? KB / 4 : 1;  // at least one block per K warp
+    pl.per_split = (KB + sp - 1) / sp;
+    pl.splits = (KB + pl.per_split - 1) / pl.per_split;
+  } else {
+    pl.tiles = (int)(w.I / 64);
+    const int step = sr_fmt(w) == kFmtA8 ? 8 : 16;
+    const int nst = (int)(w.O / step);
+    int sp = (target + pl.tiles / 2) / pl.tiles;
+    if (sp < 1) sp = 1;
+    if (sp > nst / 8) sp = nst / 8 > 0 ? nst / 8 : 1;  // at least one step per warp
+    pl.per_split = (nst + sp - 1) / sp;
+    pl.splits = (nst + pl.per_split - 1) / pl.per_split;
+  }
+  return pl;
+}
+
+template <int NT, int FMT, bool G32>
+cudaError_t sr_launch(bool dx, const SrPlan& pl, const SrParams& p, cudaStream_t st) {
+  auto kern = dx ? smallr_dx_kernel<NT, FMT, G32> : smallr_fwd_kernel<NT, FMT, G32>;
+  static bool attr_fwd = false, attr_dx = false;
+  bool& attr = dx ? attr_dx : attr_fwd;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTableBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)pl.tiles, (unsigned)pl.splits);
+  cfg.blockDim = dim3(kSrThreads);
+  cfg.dynamicSmemBytes = kTableBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr1[1];
+  attr1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr1[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr1;
+  cfg.numAttrs = timing_enabled() ? 0 : 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
+  count_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+template <int FMT, bool G32>
+cudaError_t sr_launch_nt(bool dx, const SrPlan& pl, const SrParams& p, cudaStream_t st) {
+  if (p.R <= 8) return sr_launch<1, FMT, G32>(dx, pl, p, st);
+  return sr_launch<2, FMT, G32>(dx, pl, p, st);
+}
+
+cudaError_t sr_dispatch(bool dx, const WView& w, const SrParams& p, const SrPlan& pl,
+                        cudaStream_t st) {
+  const int f = sr_fmt(w);
+  if (f == kFmtNF4) return sr_launch_nt<kFmtNF4, false>(dx, pl, p, st);
+  const bool g32 = w.block == 32;
+  if (f == kFmtA4) return g32 ? sr_launch_nt<kFmtA4, true>(dx, pl, p, st) : sr_launch_nt<kFmtA4, false>(dx, pl, p, st);
+  return g32 ? sr_launch_nt<kFmtA8, true>(dx, pl, p, st) : sr_launch_nt<kFmtA8, false>(dx, pl, p, st);
+}
+
+SrParams sr_params(const WView& w, const void* act, int64_t R, const float* aux,
+                   const float* lora, int32_t r, float s, void* out, void* ws, uint32_t* hdr,
+                   unsigned* tickets, const SrPlan& pl) {
+  SrParams p;
+  p.codes = w.codes;
+  p.qcodes = w.qcodes;
+  p.t = w.t;
+  p.mu = w.mu;
+  p.scale = w.scale;
+  p.bias = w.bias;
+  p.legacy = w.fmt == QLORA_FMT_NF4_FP32SCALE ? 1 : 0;
+  p.G = w.block;
+  p.C = (uint32_t)(w.group < 1 ? 1 : w.group);
+  p.c_shift = ((p.C & (p.C - 1)) == 0) ? __builtin_ctz(p.C) : -1;
+  p.act = (const __nv_bfloat16*)act;
+  p.R = (int32_t)R;
+  p.O = w.O;
+  p.I = w.I;
+  p.aux = aux;
+  p.lora = lora;
+  p.r = r;
+  p.s = s;
+  p.out = (__nv_bfloat16*)out;
+  p.part = (float*)ws;
+  p.tickets = tickets + kTicketBase;
+  p.splits = pl.splits;
+  p.per_split = pl.per_split;
+  p.err = hdr;
+  return p;
+}
+
+}  // namespace
+
+bool smallr_supported(const WView& w, int64_t R, const void* act, const void* out) {
+  if (R < 1 || R > 16) return false;
+  if (w.O < 128 || w.I < 64 || w.O % 128 != 0 || w.I % 64 != 0) return false;
+  if (w.O > 65536 || w.I > 32768) return false;  // ticket ranges (see kTicketBase)
+  if (((uintptr_t)w.codes % 16) != 0 || ((uintptr_t)act % 16) != 0 || ((uintptr_t)out % 4) != 0)
+    return false;
+  if (w.fmt == QLORA_FMT_NF4_DQ) return w.block == 64 && w.group >= 1;
+  if (w.fmt == QLORA_FMT_NF4_FP32SCALE) return w.block == 64;
+  if (w.fmt == QLORA_FMT_AFFINE)
+    return (w.bits == 4 || w.bits == 8) && (w.block == 32 || w.block == 64 || w.block == 128);
+  return false;
+}
+
+size_t smallr_ws(bool dx, const WView& w, int64_t R) {
+  if (!smallr_supported(w, R, (const void*)16, (const void*)16)) return 0;
+  const SrPlan pl = sr_plan(dx, w);
+  if (pl.splits <= 1) return 0;
+  const int64_t extent = dx ? w.I : w.O;
+  return align_up((size_t)pl.splits * (size_t)R * (size_t)extent * 4, 256);
+}
+
+cudaError_t launch_smallr_fwd(const WView& w, const void* X, int64_t R, const float* U,
+                              const float* B, int32_t r, float s, void* Y, void* ws,
+                              uint32_t* hdr, unsigned* tickets, cudaStream_t st) {
+  const SrPlan pl = sr_plan(false, w);
+  const SrParams p = sr_params(w, X, R, U, B, r, s, Y, ws, hdr, tickets, pl);
+  return sr_dispatch(false, w, p, pl, st);
+}
+
+cudaError_t launch_smallr_dx(const WView& w, const void* dY, int64_t R, const float* V,
+                             const float* A, int32_t r, float s, void* dX, void* ws,
+                             uint32_t* hdr, unsigned* tickets, cudaStream_t st) {
+  const SrPlan pl = sr_plan(true, w);
+  const SrParams p = sr_params(w, dY, R, V, A, r, s, dX, ws, hdr, tickets, pl);
+  return sr_dispatch(true, w, p, pl, st);
+}
+
+}  // namespace qlora

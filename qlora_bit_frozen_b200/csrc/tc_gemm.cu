@@ -66,6 +66,7 @@ struct TcParams {
   const uint8_t* qcodes;
   const float* t;
   const float* mu;
+  const float* sb;   // legacy format: the fp32 block absmax s_b (else null)
   void* out;         // bf16 [R x Mw], or fp32 partials [splits][R][Mw]
   int32_t partial;
   uint32_t* err;
@@ -472,7 +473,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     const int group = (warp - 2) >> 2;
     const int quad = warp & 3;
     const int u = DX ? (int)threadIdx.x - 64 - 128 * group : 32 * quad + lane;
-    const float mu = __ldg(p.mu);
+    const bool legacy = p.sb != nullptr;  // fp32 block scales stored as they are
+    const float mu = legacy ? 0.0f : __ldg(p.mu);
     const uint32_t bpr = (uint32_t)(p.I / kBK);  // blocks per W row
     auto block_of = [&](int kb) -> uint32_t {
       if (!DX) return (uint32_t)(m0 + u) * bpr + (uint32_t)kb;
@@ -513,8 +515,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       tw[j] = 0.0f;
       if (itj < nk) {
         const uint32_t b = block_of(kb_lo + itj);
-        qw[j] = __ldg(p.qcodes + b);
-        tw[j] = __ldg(p.t + group_of(b));
+        if (legacy) {
+          tw[j] = __ldg(p.sb + b);
+        } else {
+          qw[j] = __ldg(p.qcodes + b);
+          tw[j] = __ldg(p.t + group_of(b));
+        }
       }
     }
     bool ok = true;
@@ -522,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     int s = group % NIN, d = group % NDEC;
     uint32_t ph_in = 0;
     for (int it = group; it < nk; it += kDecGroups) {
-      const float sc = decode_block_scale(qw[0], tw[0], mu);
+      const float sc = legacy ? tw[0] : decode_block_scale(qw[0], tw[0], mu);
 #pragma unroll
       for (int j = 0; j + 1 < kPf; ++j) {
         qw[j] = qw[j + 1];
@@ -532,8 +538,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
         const int itn = it + kPf * kDecGroups;
         if (itn < nk) {
           const uint32_t b = block_of(kb_lo + itn);
-          qw[kPf - 1] = __ldg(p.qcodes + b);
-          tw[kPf - 1] = __ldg(p.t + group_of(b));
+          if (legacy) {
+            tw[kPf - 1] = __ldg(p.sb + b);
+          } else {
+            qw[kPf - 1] = __ldg(p.qcodes + b);
+            tw[kPf - 1] = __ldg(p.t + group_of(b));
+          }
         }
       }
       if (((it >> 1) & 3) == 0 && __any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
@@ -751,7 +761,13 @@ int group_cols(int bn) { return bn >= 64 ? bn / kDecGroups : bn; }
 bool ptr_aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 bool common_supported(const WView& w, int64_t R) {
-  if (w.fmt != QLORA_FMT_NF4_DQ || w.block != kBK || w.group < 1) return false;
+  if (w.fmt == QLORA_FMT_NF4_DQ) {
+    if (w.block != kBK || w.group < 1) return false;
+  } else if (w.fmt == QLORA_FMT_NF4_FP32SCALE) {
+    if (w.block != kBK) return false;
+  } else {
+    return false;
+  }
   if (R <= 0 || R > (int64_t)INT32_MAX - 256) return false;
   if (w.I % 128 != 0 || w.O % 128 != 0) return false;
   if (w.O > INT32_MAX || w.I > INT32_MAX) return false;
@@ -848,11 +864,12 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   p.kb_per_split = pl.kb_per_split;
   p.r_slices = (r + 15) / 16;
   p.rank = r;
-  p.C = (uint32_t)w.group;
-  p.c_shift = ((w.group & (w.group - 1)) == 0) ? __builtin_ctz((unsigned)w.group) : -1;
+  p.C = (uint32_t)(w.group < 1 ? 1 : w.group);
+  p.c_shift = ((p.C & (p.C - 1)) == 0) ? __builtin_ctz(p.C) : -1;
   p.qcodes = w.qcodes;
   p.t = w.t;
   p.mu = w.mu;
+  p.sb = w.fmt == QLORA_FMT_NF4_FP32SCALE ? w.scale : nullptr;
   p.partial = pl.splits > 1;
   p.out = pl.splits > 1 ? (void*)part : Y;
   p.err = hdr;
@@ -900,11 +917,12 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   p.kb_per_split = pl.kb_per_split;
   p.r_slices = (r + 15) / 16;
   p.rank = r;
-  p.C = (uint32_t)w.group;
-  p.c_shift = ((w.group & (w.group - 1)) == 0) ? __builtin_ctz((unsigned)w.group) : -1;
+  p.C = (uint32_t)(w.group < 1 ? 1 : w.group);
+  p.c_shift = ((p.C & (p.C - 1)) == 0) ? __builtin_ctz(p.C) : -1;
   p.qcodes = w.qcodes;
   p.t = w.t;
   p.mu = w.mu;
+  p.sb = w.fmt == QLORA_FMT_NF4_FP32SCALE ? w.scale : nullptr;
   p.partial = pl.splits > 1;
   p.out = pl.splits > 1 ? (void*)part : dX;
   p.err = hdr;

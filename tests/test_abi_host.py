@@ -50,6 +50,25 @@ def test_payload_bytes_match_oracle(lib, N, B, C):
     assert lib.qlora_nf4_payload_bytes(N, B, C) == oracle.nf4_payload_bytes(N, B, C)
 
 
+@pytest.mark.parametrize("N,B", [(0, 64), (1, 64), (101, 64), (65536, 64), (89128960, 64), (231, 16)])
+def test_legacy_payload_bytes_match_oracle(lib, N, B):
+    assert lib.qlora_nf4_fp32scale_payload_bytes(N, B) == oracle.legacy_payload_bytes(N, B)
+
+
+def test_legacy_quantizer_arguments_rejected_before_launch(lib):
+    ws = ctypes.create_string_buffer(1024)
+    wsp = ctypes.c_void_p((ctypes.addressof(ws) + 255) // 256 * 256)
+    d = ctypes.c_void_p(256)
+    f = lib.qlora_quantize_nf4_fp32scale
+    assert f(None, -1, 4, 64, None, None, wsp, 512, None) == _ffi.ERR_SHAPE
+    assert f(None, 4, 4, 0, None, None, wsp, 512, None) == _ffi.ERR_SHAPE
+    assert f(None, 4, 64, 64, None, None, wsp, 512, None) == _ffi.ERR_INVALID_ARG
+    assert f(d, 4, 64, 64, d, d, ctypes.c_void_p(wsp.value + 8), 512, None) == _ffi.ERR_ALIGNMENT
+    assert f(d, 4, 64, 64, d, d, wsp, 16, None) == _ffi.ERR_WORKSPACE
+    assert f(d, 1 << 31, 1 << 31, 64, d, d, wsp, 512, None) == _ffi.ERR_SHAPE
+    assert lib.qlora_quantize_nf4_fp32scale_workspace_bytes(1000, 64) >= 256
+
+
 def test_overflowing_shapes_rejected_before_any_size_arithmetic(lib):
     """O * I beyond 2^40 weights is refused with a shape error before the
     library computes any size from it (2^31 x 2^31 would wrap a signed
@@ -180,22 +199,44 @@ def _planned_splits(Mw, KB, R, sms=148):
     return bn, -(-KB // per)
 
 
+def _smallr_splits(dx, O, I, R, sms=148):
+    """The few-token plan as the design states it (1..16 tokens, O % 128 == 0,
+    I % 64 == 0): 128-row tiles (forward) or 64-column blocks (input
+    gradient) times K splits filling one wave at two CTAs per SM, at least
+    one 64-column block per K warp (4) or one 16-row step per warp (8), no
+    empty split.  0 when the path does not apply."""
+    if not (1 <= R <= 16 and O % 128 == 0 and I % 64 == 0 and O <= 65536 and I <= 32768):
+        return 0
+    target = 2 * sms
+    if not dx:
+        tiles, n, per_min = O // 128, I // 64, 4
+    else:
+        tiles, n, per_min = I // 64, O // 16, 8
+    sp = max(1, (target + tiles // 2) // tiles)
+    sp = min(sp, max(1, n // per_min))
+    per = -(-n // sp)
+    return -(-n // per)
+
+
 @pytest.mark.parametrize("O,I,R", [(12288, 4096, 1), (12288, 4096, 16), (4096, 4096, 1), (4096, 4096, 16),
                                    (4096, 4096, 128), (2048, 1024, 4096), (1024, 1024, 4096),
                                    (12288, 4096, 8192), (5120, 17408, 16384), (128, 128, 3)])
 def test_tensor_core_plan_through_workspace_sizes(lib, O, I, R):
     """The bf16 workspace exceeds the fp32 one by exactly the tensor-core
     region: the padded U/V copy (R x 64 bf16), the adapter weight operand
-    (rows x 64 bf16) and, when K is split, one fp32 partial per split.  This
-    checks the host planner (split count, no empty split) without a GPU;
-    the planner sees 148 SMs here (no device)."""
+    (rows x 64 bf16) and, when K is split, one fp32 partial per split; at
+    1..16 tokens also the few-token path's split partials.  This checks the
+    host planners (split count, no empty split) without a GPU; the planners
+    see 148 SMs here (no device)."""
     w = _ffi.qlora_weight(_ffi.FMT_NF4_DQ, O, I, 64, 256, 4, None, None, None, None, None, None)
     P = ctypes.byref(w)
     for op, Mw, KB in ((0, O, I // 64), (1, I, O // 64)):
         extra = lib.qlora_linear_workspace_bytes(P, R, 8, op, 1) - lib.qlora_linear_workspace_bytes(P, R, 8, op, 0)
         _, splits = _planned_splits(Mw, KB, R)
         part = _a256(splits * R * Mw * 4) if splits > 1 else 0
-        assert extra == _a256(R * 128) + _a256(Mw * 128) + part, (op, splits)
+        srs = _smallr_splits(op == 1, O, I, R)
+        sr = _a256(srs * R * (I if op == 1 else O) * 4) if srs > 1 else 0
+        assert extra == _a256(R * 128) + _a256(Mw * 128) + part + sr, (op, splits, srs)
         per = -(-KB // splits)
         assert 1 <= splits <= max(1, KB) and (splits - 1) * per < KB <= splits * per
 

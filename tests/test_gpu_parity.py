@@ -93,6 +93,22 @@ def test_quantize_affine_bit_exact(bits, G):
     assert np.array_equal(Wh.view(np.uint32), oracle.dequantize(ow).view(np.uint32))
 
 
+@pytest.mark.parametrize("name,li,B", [("fp32_single_256", 0, 64), ("qwen3_0.6b_attn_qv", 0, 64),
+                                       ("raw_odd", (1, 101), 64), ("raw_odd", (7, 33), 16)])
+def test_quantize_nf4_fp32scale_bit_exact(name, li, B):
+    """Legacy scale storage ("NF4 representation": one fp32 absmax per
+    block): codes and s_b bit-exact against the oracle, and the dequantized
+    weight c[code] * s_b too."""
+    W = _case_weight(name, li)
+    ow = oracle.quantize_nf4_legacy(W, B)
+    gw = q.qlora_quantize_nf4_fp32scale(to_dev_f32(W), B)
+    assert np.array_equal(gw.codes.cpu().numpy(), ow.codes)
+    assert np.array_equal(gw.scale.cpu().numpy().view(np.uint32), ow.scale.view(np.uint32))
+    assert gw.payload_bytes() == oracle.legacy_payload_bytes(W.size, B)
+    Wh = q.qlora_dequantize(gw).cpu().numpy()
+    assert np.array_equal(Wh.view(np.uint32), oracle.dequantize(ow).view(np.uint32))
+
+
 # ------------------------------------------------------------ forward/backward
 
 def _run_layer(wl, li, rows=None, want=("Y", "dX", "dA", "dB"), fmt="nf4", bits=4, G=64, R=None):
@@ -102,6 +118,11 @@ def _run_layer(wl, li, rows=None, want=("Y", "dX", "dA", "dB"), fmt="nf4", bits=
         gw = q.qlora_quantize_nf4(Wd, wl.block, wl.group)
         ow = oracle.quantize_nf4(d["W"], wl.block, wl.group)
         _assert_same_nf4(gw, ow)
+    elif fmt == "nf4_fp32scale":
+        gw = q.qlora_quantize_nf4_fp32scale(Wd, wl.block)
+        ow = oracle.quantize_nf4_legacy(d["W"], wl.block)
+        assert np.array_equal(gw.codes.cpu().numpy(), ow.codes)
+        assert np.array_equal(gw.scale.cpu().numpy().view(np.uint32), ow.scale.view(np.uint32))
     else:
         gw = q.qlora_quantize_affine(Wd, bits, G)
         ow = oracle.quantize_affine(d["W"], bits, G)
@@ -249,6 +270,30 @@ def test_bf16_small_row_sweep_affine(name, R, bits, G):
     wl = synth.workload(name, R=R)
     rows = synth.sample_rows(R, 32, seed=R + bits + G) if (R == 128 and name.endswith("12288")) else None
     _check(_run_layer(wl, 0, rows=rows, want=("Y", "dX"), fmt="affine", bits=bits, G=G), TOL["bf16"])
+
+
+@pytest.mark.parametrize("R", [1, 16, 64, 4096])
+def test_bf16_fp32scale_format(R):
+    """The legacy fp32-scale format through every bf16 path: the few-token
+    GEMV (1, 16), the tensor-core kernel with split-K (64) and without (4096)."""
+    wl = synth.workload("qwen3_0.6b_attn_qv", R=R)
+    _check(_run_layer(wl, 0, fmt="nf4_fp32scale"), TOL["bf16"])
+
+
+def test_fp32_fp32scale_format():
+    wl = synth.workload("fp32_single_256")
+    _check(_run_layer(wl, 0, fmt="nf4_fp32scale"), TOL["fp32"])
+
+
+def test_merge_fp32scale_format():
+    """Export of a legacy-format weight: B = 0 gives the dequantized matrix."""
+    W = synth.normal(77, (256, 512), std=0.02)
+    gw = q.qlora_quantize_nf4_fp32scale(to_dev_f32(W), 64)
+    A = torch.randn((8, 512), device="cuda")
+    Bz = torch.zeros((256, 8), device="cuda")
+    out = q.qlora_merge(gw, A, Bz, 16.0)
+    ref = oracle.dequantize(oracle.quantize_nf4_legacy(W, 64))
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), ref.view(np.uint32))
 
 
 @pytest.mark.parametrize("name,li", [("8b_mlp", 0), ("8b_mlp", 2), ("14b_layer", 1), ("14b_layer", 6)])
