@@ -5,9 +5,11 @@
 // gradient                               "Design / Q-LoRA layer")
 //
 // The frozen weight never exists as a floating-point matrix in HBM: packed
-// NF4 nibbles arrive in shared memory by TMA, decoder warps turn each
-// 64-weight block into bf16 (codebook level times the double-quant block
-// scale rebuilt from q_b, t_g and mu) in registers and write it where the
+// 4-bit codes arrive in shared memory by TMA, decoder warps turn each
+// 64-weight block into bf16 in registers -- NF4: codebook level times the
+// block scale (double-quantized, rebuilt from q_b, t_g and mu, or the
+// legacy fp32 absmax); affine 4-bit: scale * code + bias of the code's group
+// ("LoRA vs QLoRA on Apple Silicon", "Method") -- and write it where the
 // tensor core reads it (TMEM rows, or 128-byte-swizzled shared-memory rows),
 // and tcgen05.mma accumulates in TMEM.
 //
@@ -28,9 +30,11 @@
 // the launch that computed them has finished (programmatic dependent
 // launch: the K loop before it overlaps that launch).
 //
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM allocator and
-// MMA issuer, warps 2..9 decoders in two groups of four (alternate K
-// steps), then epilogue (TMEM -> registers -> shared memory -> TMA store).
+// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer,
+// then the decoders in two groups (alternate K steps) of four warps (a
+// whole 64-weight row per thread; 320 threads) or, at 256-token tiles, of
+// eight warps (half a row per thread; 576 threads); the decoder warps then
+// run the epilogue (TMEM -> registers -> shared memory -> TMA store).
 // Every mbarrier wait is bounded (%globaltimer); on expiry the CTA records
 // QLORA_ERR_TIMEOUT in the workspace header, stops issuing work, waits
 // (bounded) for its copies in flight, frees TMEM and exits.
@@ -48,8 +52,14 @@ namespace {
 constexpr int kBM = 128;             // weight-side rows per CTA (MMA M)
 constexpr int kBK = 64;              // reduction step (one NF4 block)
 constexpr int kDecGroups = 2;        // decoder groups (alternate K steps)
-constexpr int kDecWarps = 4 * kDecGroups;  // decoder / epilogue warps
-constexpr int kThreads = 32 * (2 + kDecWarps);
+// Decoder warps per group: at 256-token tiles (one CTA per SM) eight, each
+// thread decoding half a 64-weight row, so that twice as many warps hide
+// the decode's dependency latency; four (a whole row per thread) at smaller
+// tiles, which keep two CTAs per SM.
+constexpr int dec_warps(int bn) { return bn >= 256 ? 8 : 4; }
+constexpr int threads_of(int bn) { return 32 * (2 + kDecGroups * dec_warps(bn)); }
+// epilogue groups: four warps each, one per TMEM lane quarter
+constexpr int epi_groups(int bn) { return kDecGroups * dec_warps(bn) / 4; }
 constexpr int kWTile = kBM * kBK * 2;  // decoded weight tile bytes (16 KB)
 constexpr int kPkTile = kBM * kBK / 2; // packed nibbles per step (4 KB)
 
@@ -67,6 +77,9 @@ struct TcParams {
   const float* t;
   const float* mu;
   const float* sb;   // legacy format: the fp32 block absmax s_b (else null)
+  const float* asc;  // affine 4-bit: per-group scale (else null)
+  const float* abi;  // affine 4-bit: per-group bias
+  int32_t g_shift;   // affine: log2(G / 32), G in {32, 64, 128}
   void* out;         // bf16 [R x Mw], or fp32 partials [splits][R][Mw]
   int32_t partial;
   uint32_t* err;
@@ -168,6 +181,24 @@ __device__ __forceinline__ Nf4Planes nf4_planes(float s) {
   return t;
 }
 
+// The same two byte planes for an affine group: the 16 values
+// bf16(fp32(fp32(scale * k) + bias)), k = 0..15 ("LoRA vs QLoRA on Apple
+// Silicon", "Method": w_hat = scale * code + bias, fp32, one rounding per
+// step, as the diagnostic dequantization computes it).
+__device__ __forceinline__ Nf4Planes affine_planes(float sc, float bi) {
+  uint32_t P[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    P[j] = pack_bf16x2(__fadd_rn(__fmul_rn(sc, (float)(2 * j)), bi),
+                       __fadd_rn(__fmul_rn(sc, (float)(2 * j + 1)), bi));
+  Nf4Planes t;
+  t.L0 = __byte_perm(P[0], P[1], 0x6420); t.H0 = __byte_perm(P[0], P[1], 0x7531);
+  t.L1 = __byte_perm(P[2], P[3], 0x6420); t.H1 = __byte_perm(P[2], P[3], 0x7531);
+  t.L2 = __byte_perm(P[4], P[5], 0x6420); t.H2 = __byte_perm(P[4], P[5], 0x7531);
+  t.L3 = __byte_perm(P[6], P[7], 0x6420); t.H3 = __byte_perm(P[6], P[7], 0x7531);
+  return t;
+}
+
 // 8 nibbles (weights 8j .. 8j+7, low nibble first) -> 4 bf16 pairs
 // o[q] = (weight 2q, weight 2q+1) of the 8, low half first.
 // A byte permute reads only the low 16 bits of its selector, so the
@@ -189,33 +220,65 @@ __device__ __forceinline__ void nf4_word(const Nf4Planes& t, uint32_t w, uint32_
 
 // Block (packed bytes 0..15 at pk_lo, 16..31 at pk_hi) -> one 128-byte
 // swizzled shared-memory row at row_addr (row index within its 8-row atom
-// = sw).
-__device__ __forceinline__ void decode_row_smem(const uint8_t* pk_lo, const uint8_t* pk_hi, float s,
+// = sw).  Weights 0..31 decode through table tA, 32..63 through tB (the
+// same table unless an affine group of 32 splits the block).
+__device__ __forceinline__ void decode_row_smem(const uint8_t* pk_lo, const uint8_t* pk_hi,
+                                                const Nf4Planes& tA, const Nf4Planes& tB,
                                                 uint32_t row_addr, uint32_t sw) {
-  const Nf4Planes t = nf4_planes(s);
   const uint4 p0 = *reinterpret_cast<const uint4*>(pk_lo);
   const uint4 p1 = *reinterpret_cast<const uint4*>(pk_hi);
   const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     uint32_t o[4];
-    nf4_word(t, w[j], o);
+    nf4_word(j < 4 ? tA : tB, w[j], o);
     st_shared_v4(row_addr + ((j ^ sw) << 4), o[0], o[1], o[2], o[3]);
   }
 }
 
+// Half block (weights 32 h .. 32 h + 31 from the 16 packed bytes at pk) ->
+// shared-memory chunks 4 h .. 4 h + 3 of the swizzled row at row_addr.
+__device__ __forceinline__ void decode_half_smem(const uint8_t* pk, const Nf4Planes& t,
+                                                 uint32_t row_addr, uint32_t sw, int h) {
+  const uint4 p = *reinterpret_cast<const uint4*>(pk);
+  const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t o[4];
+    nf4_word(t, w[j], o);
+    st_shared_v4(row_addr + ((((uint32_t)(4 * h + j)) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Half block -> 16 registers, v[c] = (weight 32 h + 2c, 32 h + 2c + 1):
+// TMEM columns 16 h .. 16 h + 15 of the row.
+__device__ __forceinline__ void decode_half_regs(const uint8_t* pk, const Nf4Planes& t,
+                                                 uint32_t (&v)[16]) {
+  const uint4 p = *reinterpret_cast<const uint4*>(pk);
+  const uint32_t w[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t o[4];
+    nf4_word(t, w[j], o);
+    v[4 * j] = o[0];
+    v[4 * j + 1] = o[1];
+    v[4 * j + 2] = o[2];
+    v[4 * j + 3] = o[3];
+  }
+}
+
 // Block -> 32 registers, v[c] = (weight 2c, weight 2c+1): one TMEM row of
-// the A operand (32 columns of two bf16 each).
-__device__ __forceinline__ void decode_row_regs(const uint8_t* pk_lo, const uint8_t* pk_hi, float s,
+// the A operand (32 columns of two bf16 each); tables as decode_row_smem.
+__device__ __forceinline__ void decode_row_regs(const uint8_t* pk_lo, const uint8_t* pk_hi,
+                                                const Nf4Planes& tA, const Nf4Planes& tB,
                                                 uint32_t (&v)[32]) {
-  const Nf4Planes t = nf4_planes(s);
   const uint4 p0 = *reinterpret_cast<const uint4*>(pk_lo);
   const uint4 p1 = *reinterpret_cast<const uint4*>(pk_hi);
   const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     uint32_t o[4];
-    nf4_word(t, w[j], o);
+    nf4_word(j < 4 ? tA : tB, w[j], o);
     v[4 * j] = o[0];
     v[4 * j + 1] = o[1];
     v[4 * j + 2] = o[2];
@@ -269,14 +332,14 @@ __device__ __forceinline__ void epilogue_stage(uint32_t tmem, int quad, int lane
   }
 }
 
-// Columns of the token tile each decoder group stores in the epilogue.
+// Columns of the token tile each epilogue group stores.
 template <int BN>
 constexpr int cols_per_group() {
-  return BN >= 64 ? BN / kDecGroups : BN;
+  return BN >= 64 ? BN / epi_groups(BN) : BN;
 }
 
 template <bool DX, int BN>
-__global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
+__global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN>::kMinCtas)
     tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_pk,
                       const __grid_constant__ CUtensorMap tm_aact,
@@ -285,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
   using C = Cfg<DX, BN>;
   constexpr int NIN = C::NIN, NDEC = C::NDEC;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, BN, DX);
-  static_assert((BN >= 64 ? 2 : 1) * 2 * cols_per_group<BN>() * 64 * 4 <= C::kRing,
+  constexpr int DW = dec_warps(BN);
+  static_assert((BN >= 64 ? epi_groups(BN) : 1) * 2 * cols_per_group<BN>() * 64 * 4 <= C::kRing,
                 "epilogue staging must fit in the ring buffers");
 
   extern __shared__ uint8_t smem_raw[];
@@ -322,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       mbar_init(smem_u32(&in_empty[s]), 1);
     }
     for (int d = 0; d < NDEC; ++d) {
-      mbar_init(smem_u32(&dec_full[d]), 4);  // the 4 warps of one decoder group
+      mbar_init(smem_u32(&dec_full[d]), DW);  // the warps of one decoder group
     }
     mbar_init(smem_u32(acc_full), 1);
     mbar_init(smem_u32(ad_full), 1);
@@ -470,11 +534,16 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     // TMEM lane, and stores the block's 32 bf16 pairs with one tcgen05.st.
     // Input gradient: unit u writes one swizzled 128-byte row of the
     // MN-major shared-memory tile (64 weights of W row kb*64 + u%64).
-    const int group = (warp - 2) >> 2;
+    // With eight warps per group, warps wi and wi + 4 of the group share the
+    // rows (units) and take the low (half 0) and high (half 1) 32 weights.
+    const int group = (warp - 2) / DW;
+    const int wi = (warp - 2) % DW;
+    const int half = wi >> 2;  // always 0 with four warps per group
     const int quad = warp & 3;
-    const int u = DX ? (int)threadIdx.x - 64 - 128 * group : 32 * quad + lane;
-    const bool legacy = p.sb != nullptr;  // fp32 block scales stored as they are
-    const float mu = legacy ? 0.0f : __ldg(p.mu);
+    const int u = DX ? (((int)threadIdx.x - 64 - 32 * DW * group) & 127) : 32 * quad + lane;
+    const bool legacy = p.sb != nullptr;   // fp32 block scales stored as they are
+    const bool affine = p.asc != nullptr;  // 4-bit affine groups: (scale, bias)
+    const float mu = (legacy || affine) ? 0.0f : __ldg(p.mu);
     const uint32_t bpr = (uint32_t)(p.I / kBK);  // blocks per W row
     auto block_of = [&](int kb) -> uint32_t {
       if (!DX) return (uint32_t)(m0 + u) * bpr + (uint32_t)kb;
@@ -483,6 +552,22 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
     // scale group of block b (a shift when the group size is a power of two)
     auto group_of = [&](uint32_t b) -> uint32_t {
       return p.c_shift >= 0 ? (b >> p.c_shift) : b / p.C;
+    };
+    // affine group of the first weight this thread decodes in block b (32
+    // weights per half block: group (2 b + half) >> log2(G / 32))
+    auto agroup_of = [&](uint32_t b) -> uint32_t { return (2u * b + (uint32_t)half) >> p.g_shift; };
+    // Per step: NF4 (q_b, t_g); legacy (-, s_b); affine (scale bits, bias).
+    auto load_scale = [&](uint32_t b, uint32_t& q, float& t) {
+      if (affine) {
+        const uint32_t gi = agroup_of(b);
+        q = __float_as_uint(__ldg(p.asc + gi));
+        t = __ldg(p.abi + gi);
+      } else if (legacy) {
+        t = __ldg(p.sb + b);
+      } else {
+        q = __ldg(p.qcodes + b);
+        t = __ldg(p.t + group_of(b));
+      }
     };
     const uint32_t row_off = (uint32_t)((u >> 6) * (kWTile / 2) + (u & 63) * 128);
     const uint32_t sw = (uint32_t)(u & 7);
@@ -513,22 +598,16 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       const int itj = group + j * kDecGroups;
       qw[j] = 128u;
       tw[j] = 0.0f;
-      if (itj < nk) {
-        const uint32_t b = block_of(kb_lo + itj);
-        if (legacy) {
-          tw[j] = __ldg(p.sb + b);
-        } else {
-          qw[j] = __ldg(p.qcodes + b);
-          tw[j] = __ldg(p.t + group_of(b));
-        }
-      }
+      if (itj < nk) load_scale(block_of(kb_lo + itj), qw[j], tw[j]);
     }
     bool ok = true;
     // running ring positions of this group's steps (it = group, group + 2, ...)
     int s = group % NIN, d = group % NDEC;
     uint32_t ph_in = 0;
     for (int it = group; it < nk; it += kDecGroups) {
-      const float sc = legacy ? tw[0] : decode_block_scale(qw[0], tw[0], mu);
+      const float sc = affine ? __uint_as_float(qw[0]) : legacy ? tw[0] : decode_block_scale(qw[0], tw[0], mu);
+      const float bi = tw[0];  // affine bias
+      const uint32_t bcur = block_of(kb_lo + it);
 #pragma unroll
       for (int j = 0; j + 1 < kPf; ++j) {
         qw[j] = qw[j + 1];
@@ -536,15 +615,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
       }
       {
         const int itn = it + kPf * kDecGroups;
-        if (itn < nk) {
-          const uint32_t b = block_of(kb_lo + itn);
-          if (legacy) {
-            tw[kPf - 1] = __ldg(p.sb + b);
-          } else {
-            qw[kPf - 1] = __ldg(p.qcodes + b);
-            tw[kPf - 1] = __ldg(p.t + group_of(b));
-          }
-        }
+        if (itn < nk) load_scale(block_of(kb_lo + itn), qw[kPf - 1], tw[kPf - 1]);
       }
       if (((it >> 1) & 3) == 0 && __any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
       // Decoded slot d was last used by step it - NDEC; the MMA releases a
@@ -563,15 +634,33 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
                mbar_wait(fb, ph_in, p.wait_ns, p.err, 0x302);
       if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
       const uint8_t* src = pk + s * kPkTile;
+      // decode tables: one per block, or (whole-row threads, affine groups
+      // of 32) one per half block, the second group's scale and bias read here
+      const Nf4Planes tA = affine ? affine_planes(sc, bi) : nf4_planes(sc);
+      Nf4Planes tB = tA;
+      if (DW == 4 && affine && p.g_shift == 0) {
+        const uint32_t g2 = 2u * bcur + 1u;
+        tB = affine_planes(__ldg(p.asc + g2), __ldg(p.abi + g2));
+      }
       if (!DX) {
         tc_fence_after();
-        uint32_t v[32];
-        decode_row_regs(src + pk_lo, src + pk_hi, sc, v);
-        tmem_st_32x32b_x32(tm_row + (uint32_t)(d * 32), v);
+        if (DW == 4) {
+          uint32_t v[32];
+          decode_row_regs(src + pk_lo, src + pk_hi, tA, tB, v);
+          tmem_st_32x32b_x32(tm_row + (uint32_t)(d * 32), v);
+        } else {
+          uint32_t v[16];
+          decode_half_regs(src + (half ? pk_hi : pk_lo), tA, v);
+          tmem_st_32x32b_x16(tm_row + (uint32_t)(d * 32 + 16 * half), v);
+        }
         tmem_st_wait();
         tc_fence_before();
       } else {
-        decode_row_smem(src + pk_lo, src + pk_hi, sc, smem_u32(wdec + d * kWTile) + row_off, sw);
+        if (DW == 4)
+          decode_row_smem(src + pk_lo, src + pk_hi, tA, tB, smem_u32(wdec + d * kWTile) + row_off, sw);
+        else
+          decode_half_smem(src + (half ? pk_hi : pk_lo), tA, smem_u32(wdec + d * kWTile) + row_off,
+                           sw, half);
         fence_proxy_async_smem();
       }
       __syncwarp();
@@ -592,10 +681,11 @@ __global__ void __launch_bounds__(kThreads, Cfg<DX, BN>::kMinCtas)
   tc_fence_after();
   if (warp >= 2 && *abort_flag == 0) {
     // ---------------------------------------------------------- epilogue
-    // Warp w reads TMEM lanes 32*(w%4) .. +31; the two decoder groups split
-    // the token columns (group 0 alone when the tile is narrower than 64).
-    // Each group stages its columns in the freed ring buffers and one
-    // thread writes them with two TMA stores (weight-side rows 0..63, 64..127).
+    // Warp w reads TMEM lanes 32*(w%4) .. +31; the epilogue groups (four
+    // warps each) split the token columns (group 0 alone when the tile is
+    // narrower than 64).  Each group stages its columns in the freed ring
+    // buffers and one thread writes them with two TMA stores (weight-side
+    // rows 0..63, 64..127).
     const int group = (warp - 2) >> 2;
     constexpr int kColsPerGroup = cols_per_group<BN>();
     const int c_begin = BN >= 64 ? group * kColsPerGroup : 0;
@@ -728,7 +818,7 @@ cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, con
   const int slot = timing_begin(st, DX ? 1 : 0, flops);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(threads_of(BN));
   cfg.dynamicSmemBytes = (size_t)Cf::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -756,7 +846,7 @@ cudaError_t launch_plan(const TcPlan& pl, dim3 grid, const CUtensorMap& a, const
   }
 }
 
-int group_cols(int bn) { return bn >= 64 ? bn / kDecGroups : bn; }
+int group_cols(int bn) { return bn >= 64 ? bn / epi_groups(bn) : bn; }
 
 bool ptr_aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
@@ -765,6 +855,8 @@ bool common_supported(const WView& w, int64_t R) {
     if (w.block != kBK || w.group < 1) return false;
   } else if (w.fmt == QLORA_FMT_NF4_FP32SCALE) {
     if (w.block != kBK) return false;
+  } else if (w.fmt == QLORA_FMT_AFFINE) {
+    if (w.bits != 4 || (w.block != 32 && w.block != 64 && w.block != 128)) return false;
   } else {
     return false;
   }
@@ -870,6 +962,9 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   p.t = w.t;
   p.mu = w.mu;
   p.sb = w.fmt == QLORA_FMT_NF4_FP32SCALE ? w.scale : nullptr;
+  p.asc = w.fmt == QLORA_FMT_AFFINE ? w.scale : nullptr;
+  p.abi = w.fmt == QLORA_FMT_AFFINE ? w.bias : nullptr;
+  p.g_shift = w.block == 128 ? 2 : w.block == 64 ? 1 : 0;
   p.partial = pl.splits > 1;
   p.out = pl.splits > 1 ? (void*)part : Y;
   p.err = hdr;
@@ -923,6 +1018,9 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   p.t = w.t;
   p.mu = w.mu;
   p.sb = w.fmt == QLORA_FMT_NF4_FP32SCALE ? w.scale : nullptr;
+  p.asc = w.fmt == QLORA_FMT_AFFINE ? w.scale : nullptr;
+  p.abi = w.fmt == QLORA_FMT_AFFINE ? w.bias : nullptr;
+  p.g_shift = w.block == 128 ? 2 : w.block == 64 ? 1 : 0;
   p.partial = pl.splits > 1;
   p.out = pl.splits > 1 ? (void*)part : dX;
   p.err = hdr;

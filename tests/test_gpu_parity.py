@@ -232,6 +232,37 @@ def test_bf16_identity_input_recovers_decoded_weight_bitwise():
     assert np.array_equal(bf16_bits_of(dX), bf16_bits_of(ref))
 
 
+@pytest.mark.parametrize("G", [32, 64, 128])
+def test_bf16_identity_input_recovers_affine_weight_bitwise(G):
+    """4-bit affine weights in the tensor-core kernel: X = I (R = I) and B = 0
+    give Y = bf16(W_hat)^T exactly, dY = I gives dX = bf16(W_hat); every
+    decoded weight (scale * code + bias of its group) checked bit for bit."""
+    O, I = 256, 512
+    W = synth.normal(5 + G, (O, I), std=0.02)
+    gw = q.qlora_quantize_affine(to_dev_f32(W), 4, G)
+    ow = oracle.quantize_affine(W, 4, G)
+    ref = torch.from_numpy(oracle.dequantize(ow)).to(torch.bfloat16)
+    r = 8
+    A = torch.zeros((r, I), device="cuda")
+    Bz = torch.zeros((O, r), device="cuda")
+    Xi = torch.eye(I, device="cuda", dtype=torch.bfloat16)
+    Y, _ = q.qlora_linear_fwd(gw, Xi, A, Bz, 16.0)
+    assert np.array_equal(bf16_bits_of(Y), bf16_bits_of(ref.t()))
+    dYi = torch.eye(O, device="cuda", dtype=torch.bfloat16)
+    dX, _, _ = q.qlora_linear_bwd(gw, None, dYi, A, Bz, 16.0, want_da=False, want_db=False)
+    assert np.array_equal(bf16_bits_of(dX), bf16_bits_of(ref))
+
+
+@pytest.mark.parametrize("G", [32, 64, 128])
+@pytest.mark.parametrize("R", [100, 4096])
+def test_bf16_affine4_tensor_core_path(G, R):
+    """4-bit affine weights at many tokens run on the tensor-core kernel
+    (split-K at 100 tokens, 256-token tiles at 4096); 64 sampled rows."""
+    wl = synth.workload("qwen3_0.6b_attn_qv", R=R)
+    rows = synth.sample_rows(R, 64, seed=G + R)
+    _check(_run_layer(wl, 0, rows=rows, fmt="affine", bits=4, G=G), TOL["bf16"])
+
+
 def test_bf16_adapter_only_and_zero_alpha():
     wl = synth.workload("qwen3_0.6b_attn_qv", R=256)
     d = layer_inputs(wl, 1)
