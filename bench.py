@@ -328,7 +328,7 @@ def run_gpu(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     peaks = load_peaks()
-    wl = synth.workload(args.workload)
+    wl = synth.workload(args.workload, R=args.tokens if args.tokens > 0 else None)
     R = wl.R
     model = Model(q, torch, wl, rank, host_outputs=True)
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
@@ -711,6 +711,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.WORKLOADS[1:])
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the workload's token count per GPU (0: the workload's own)")
     ap.add_argument("--also", nargs="*", default=None,
                     help="other large-R workloads timed the same way into other_configs "
                          "(default: the Qwen3-0.6B q/v and 8B MLP configurations)")

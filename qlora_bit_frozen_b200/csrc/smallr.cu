@@ -102,26 +102,6 @@ __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
   return d;
 }
 
-// Streamed once: bypass L1 and let L2 evict these lines first.
-__device__ __forceinline__ uint2 ld_stream_u2(const uint8_t* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint4 ld_stream_u4(const uint8_t* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-__device__ __forceinline__ uint32_t ld_stream_u1(const uint8_t* p) {
-  uint32_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
 
 // The lane's copy of table entry `byte k of w`: address byte * 256 + lane * 4
 // (laneoff holds lane * 4 in its low byte, zeros above), built by one permute.
@@ -149,13 +129,38 @@ __device__ __forceinline__ void fill_table(uint32_t* table) {
   }
 }
 
-// NF4 block scale of flat block index b: the double-quantized s_hat_b, or
-// the stored fp32 absmax of the legacy format.
-__device__ __forceinline__ float nf4_scale(const SrParams& p, uint32_t b, float mu) {
-  if (p.legacy) return __ldg(p.scale + b);
-  const uint32_t g = p.c_shift >= 0 ? (b >> p.c_shift) : b / p.C;
-  return decode_block_scale(__ldg(p.qcodes + b), __ldg(p.t + g), mu);
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Raw inputs of a block scale, loaded ahead of their use: NF4 (q_b, t_g),
+// or the legacy format's stored s_b (in t, with q = 0xFFFFFFFF).
+__device__ __forceinline__ void nf4_scale_load(const SrParams& p, uint32_t b, uint32_t& q, float& t) {
+  if (p.legacy) {
+    q = 0xFFFFFFFFu;
+    t = __ldg(p.scale + b);
+    return;
+  }
+  const uint32_t g = p.c_shift >= 0 ? (b >> p.c_shift) : b / p.C;
+  q = __ldg(p.qcodes + b);
+  t = __ldg(p.t + g);
+}
+// The block scale as the GEMM uses it: mu + t_g (q_b - 128) / 127 with the
+// division replaced by a multiply (within an ulp of the stored-format
+// decode; the GEMM rounds its operands to bf16 anyway).
+__device__ __forceinline__ float nf4_scale_decode(uint32_t q, float t, float mu) {
+  if (q == 0xFFFFFFFFu) return t;
+  const float s = fmaf(t * (float)((int)q - 128), 1.0f / 127.0f, mu);
+  return fmaxf(s, 0.0f);
+}
+
 
 // ------------------------------------------------------------------ forward
 //
@@ -174,13 +179,16 @@ struct FwdShape {
 };
 
 template <int NT, int FMT, bool G32>
-__global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd_kernel(const SrParams p) {
+__global__ void __launch_bounds__(kSrThreads, FMT == kFmtA8 ? 1 : 2) smallr_fwd_kernel(const SrParams p) {
   using S = FwdShape<FMT>;
   constexpr int CW = S::kChunkU32;
+  constexpr int NSTG = FMT == kFmtA8 ? 2 : 3;          // blocks per warp ring
+  constexpr int RB = FMT == kFmtA8 ? 64 : 32;          // code bytes per row per block
+  constexpr int STG = 64 * RB;                          // one block of the warp's 64 rows
+  constexpr int NP = G32 ? 2 : 1;                       // group passes per block
   extern __shared__ __align__(1024) uint8_t sr_smem[];
   uint32_t* table = reinterpret_cast<uint32_t*>(sr_smem);
   fill_table<FMT>(table);
-  __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -192,9 +200,32 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd
   const int kb_hi = min(KB, kb_lo + p.per_split);
   const uint32_t laneoff = (uint32_t)lane * 4u;
   const int64_t row_bytes = FMT == kFmtA8 ? I : I / 2;
-  const int bbytes = FMT == kFmtA8 ? 64 : 32;  // code bytes per row per block
   const float mu = (FMT == kFmtNF4 && !p.legacy) ? __ldg(p.mu) : 0.0f;
-  constexpr int NP = G32 ? 2 : 1;  // group passes per block
+  // this warp's ring of code blocks, after the table
+  uint8_t* ring = sr_smem + kTableBytes + warp * NSTG * STG;
+  const uint32_t ring_s = smem_u32(ring);
+  // The warp's blocks: kb = kb_lo + wk + 4 i, i < nblk.
+  const int first = kb_lo + wk;
+  const int nblk = first < kb_hi ? (kb_hi - first + 3) / 4 : 0;
+
+  // Copy block i of the warp (64 rows x RB bytes) into ring slot i % NSTG:
+  // 16-byte chunks, row-major, lane-strided (every instruction moves 512
+  // contiguous-by-row bytes).
+  auto issue = [&](int i) {
+    if (i < nblk) {
+      const int kb = first + 4 * i;
+      const uint32_t dst = ring_s + (uint32_t)((i % NSTG) * STG);
+      constexpr int CPR = RB / 16;  // chunks per row
+#pragma unroll
+      for (int j = 0; j < 64 * CPR / 32; ++j) {
+        const int c = lane + 32 * j;
+        const int row = c / CPR, ch = c % CPR;
+        cp_async16(dst + (uint32_t)(row * RB + ch * 16),
+                   p.codes + (rbase + row) * row_bytes + (int64_t)kb * RB + ch * 16);
+      }
+    }
+    cp_async_commit();  // one group per block (empty past the end: uniform counting)
+  };
 
   float acc[4][NT][4];
 #pragma unroll
@@ -204,39 +235,21 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd
 #pragma unroll
       for (int c = 0; c < 4; ++c) acc[a][n][c] = 0.0f;
 
-  // code chunks of this lane: [m-tile][row g / g + 8][words]; each m-tile's
-  // registers are refilled with the next block's codes as soon as they are
-  // decoded, so one block is always in flight without a second buffer
-  uint32_t cur[4][2][CW];
-  const uint8_t* cbase = p.codes + (rbase + g) * row_bytes + (FMT == kFmtA8 ? 16 : 8) * t;
-  auto load_mtile = [&](uint32_t (&dst)[2][CW], int mt, int kb) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint8_t* src = cbase + (int64_t)(16 * mt + 8 * h) * row_bytes + (int64_t)kb * bbytes;
-      if (CW == 2) {
-        const uint2 v = ld_stream_u2(src);
-        dst[h][0] = v.x;
-        dst[h][CW - 1] = v.y;
-      } else {
-        const uint4 v = ld_stream_u4(src);
-        dst[h][0] = v.x;
-        dst[h][1 % CW] = v.y;
-        dst[h][2 % CW] = v.z;
-        dst[h][3 % CW] = v.w;
-      }
-    }
-  };
   // Per-row block (or group) parameters of rows rbase + lane and
-  // rbase + 32 + lane, loaded one block ahead.
-  //   NF4: q_b and t_g (decoded per block); affine: scale and bias per pass.
+  // rbase + 32 + lane, loaded one block ahead as raw values (the loads
+  // complete while the current block is decoded).  NF4: q_b (as float bits)
+  // and t_g, decoded at use; affine: scale and bias per pass.
   float pa[2][NP], pb[2][NP], na[2][NP], nb[2][NP];
   auto load_params = [&](float (&sa)[2][NP], float (&sb)[2][NP], int kb) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int64_t row = rbase + 32 * h + lane;
       if (FMT == kFmtNF4) {
-        sa[h][0] = nf4_scale(p, (uint32_t)(row * KB + kb), mu);
-        sb[h][0] = 0.0f;
+        uint32_t q;
+        float tt;
+        nf4_scale_load(p, (uint32_t)(row * KB + kb), q, tt);
+        sa[h][0] = __uint_as_float(q);
+        sb[h][0] = tt;
       } else {
 #pragma unroll
         for (int q = 0; q < NP; ++q) {
@@ -247,28 +260,40 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd
       }
     }
   };
-
-  int kb = kb_lo + wk;
-  if (kb < kb_hi) {
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt) load_mtile(cur[mt], mt, kb);
-    load_params(pa, pb, kb);
-  }
+  // activation operand: columns 64 kb + 16 t + 4 m .. + 3 of tokens g, 8 + g
   const bool tok_ok0 = g < p.R, tok_ok1 = (8 + g) < p.R;
-  for (; kb < kb_hi; kb += 4) {
-    const int kbn = kb + 4;
-    const bool more = kbn < kb_hi;
-    if (more) load_params(na, nb, kbn);
-    // activation operand: columns 64 kb + 16 t + 4 m .. + 3 of tokens g and 8 + g
-    uint2 xw[NT][4];
+  uint2 xw[NT][4], xn[NT][4];
+  auto load_x = [&](uint2 (&dst)[NT][4], int kb) {
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       const bool ok = n == 0 ? tok_ok0 : tok_ok1;
       const __nv_bfloat16* xr = p.act + (int64_t)(8 * n + g) * I + (int64_t)kb * 64 + 16 * t;
 #pragma unroll
       for (int m = 0; m < 4; ++m)
-        xw[n][m] = ok ? __ldg(reinterpret_cast<const uint2*>(xr + 4 * m)) : make_uint2(0u, 0u);
+        dst[n][m] = ok ? __ldg(reinterpret_cast<const uint2*>(xr + 4 * m)) : make_uint2(0u, 0u);
     }
+  };
+
+  // prologue: NSTG - 1 blocks in flight, parameters and activations of block 0
+#pragma unroll
+  for (int i = 0; i < NSTG - 1; ++i) issue(i);
+  if (nblk > 0) {
+    load_params(pa, pb, first);
+    load_x(xw, first);
+  }
+  __syncthreads();  // the table is complete
+
+  for (int i = 0; i < nblk; ++i) {
+    const int kb = first + 4 * i;
+    const bool more = i + 1 < nblk;
+    issue(i + NSTG - 1);
+    if (more) {
+      load_params(na, nb, kb + 4);
+      load_x(xn, kb + 4);
+    }
+    cp_async_wait<NSTG - 1>();  // block i has landed (this lane's copies)
+    __syncwarp();               // ... and every lane's
+    const uint8_t* blk = ring + (i % NSTG) * STG;
     // B operand registers per MMA j: 4-bit (x[c], x[c+1]) pairs as loaded;
     // 8-bit (x[c], 16 x[c]) pairs.
     uint32_t bx[NT][S::kMmas][2];
@@ -310,6 +335,12 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd
         }
       }
     }
+    // NF4: decode the two block scales this lane loaded (rows lane, 32 + lane)
+    float sdec[2];
+    if (FMT == kFmtNF4) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) sdec[h] = nf4_scale_decode(__float_as_uint(pa[h][0]), pb[h][0], mu);
+    }
     // rows of this lane's accumulators: 16 mt + g (c0, c1) and 16 mt + g + 8 (c2, c3)
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
@@ -318,23 +349,43 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd
       float sA[NP], sB[NP], bA[NP], bB[NP];
 #pragma unroll
       for (int q = 0; q < NP; ++q) {
-        const float va = hsel ? pa[1][q] : pa[0][q];
-        const float vb = hsel ? pb[1][q] : pb[0][q];
+        const float va = FMT == kFmtNF4 ? (hsel ? sdec[1] : sdec[0]) : (hsel ? pa[1][q] : pa[0][q]);
         sA[q] = __shfl_sync(0xffffffffu, va, srcA);
         sB[q] = __shfl_sync(0xffffffffu, va, srcB);
-        bA[q] = __shfl_sync(0xffffffffu, vb, srcA);
-        bB[q] = __shfl_sync(0xffffffffu, vb, srcB);
+        if (FMT != kFmtNF4) {
+          const float vb = hsel ? pb[1][q] : pb[0][q];
+          bA[q] = __shfl_sync(0xffffffffu, vb, srcA);
+          bB[q] = __shfl_sync(0xffffffffu, vb, srcB);
+        } else {
+          bA[q] = 0.0f;
+          bB[q] = 0.0f;
+        }
       }
       // decoded pairs of rows g (pA) and g + 8 (pB): one per code byte
       uint32_t pA[4 * CW], pB[4 * CW];
-#pragma unroll
-      for (int w = 0; w < CW; ++w)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          pA[4 * w + k] = tbl(table, cur[mt][0][w], laneoff, k);
-          pB[4 * w + k] = tbl(table, cur[mt][1][w], laneoff, k);
+      {
+        const uint8_t* ra = blk + (16 * mt + g) * RB + (FMT == kFmtA8 ? 16 : 8) * t;
+        const uint8_t* rb = ra + 8 * RB;
+        uint32_t wa[CW], wb[CW];
+        if (CW == 2) {
+          const uint2 va = *reinterpret_cast<const uint2*>(ra);
+          const uint2 vb = *reinterpret_cast<const uint2*>(rb);
+          wa[0] = va.x; wa[CW - 1] = va.y;
+          wb[0] = vb.x; wb[CW - 1] = vb.y;
+        } else {
+          const uint4 va = *reinterpret_cast<const uint4*>(ra);
+          const uint4 vb = *reinterpret_cast<const uint4*>(rb);
+          wa[0] = va.x; wa[1 % CW] = va.y; wa[2 % CW] = va.z; wa[3 % CW] = va.w;
+          wb[0] = vb.x; wb[1 % CW] = vb.y; wb[2 % CW] = vb.z; wb[3 % CW] = vb.w;
         }
-      if (more) load_mtile(cur[mt], mt, kbn);
+#pragma unroll
+        for (int w = 0; w < CW; ++w)
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            pA[4 * w + k] = tbl(table, wa[w], laneoff, k);
+            pB[4 * w + k] = tbl(table, wb[w], laneoff, k);
+          }
+      }
 #pragma unroll
       for (int q = 0; q < NP; ++q) {
         const bool keep = !G32 || (t >> 1) == q;
@@ -366,6 +417,7 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd
         }
       }
     }
+    __syncwarp();  // every lane is done with this slot before it is refilled
     if (more) {
 #pragma unroll
       for (int h = 0; h < 2; ++h)
@@ -374,8 +426,13 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_fwd
           pa[h][q] = na[h][q];
           pb[h][q] = nb[h][q];
         }
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int m = 0; m < 4; ++m) xw[n][m] = xn[n][m];
     }
   }
+  cp_async_wait<0>();
 
   // ---- combine the four K warps of each row half (fixed order wk = 0..3)
   __syncthreads();  // every warp is done with the table: reuse its memory
@@ -480,10 +537,12 @@ template <int NT, int FMT, bool G32>
 __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_kernel(const SrParams p) {
   using S = DxShape<FMT>;
   constexpr int SR = S::kStepRows, NS = S::kSteps;
+  constexpr int RB = FMT == kFmtA8 ? 64 : 32;  // code bytes per row of the column block
+  constexpr int STG = NS * SR * RB;            // one iteration: 2 KB
+  constexpr int NSTG = 3;                      // iterations per warp ring
   extern __shared__ __align__(1024) uint8_t sr_smem[];
   uint32_t* table = reinterpret_cast<uint32_t*>(sr_smem);
   fill_table<FMT>(table);
-  __syncthreads();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -494,6 +553,8 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
   const uint32_t laneoff = (uint32_t)lane * 4u;
   const float mu = (FMT == kFmtNF4 && !p.legacy) ? __ldg(p.mu) : 0.0f;
   constexpr int NP = G32 ? 2 : 1;
+  uint8_t* ring = sr_smem + kTableBytes + warp * NSTG * STG;
+  const uint32_t ring_s = smem_u32(ring);
 
   // rows of this CTA, then of this warp, in K steps
   const int64_t nsteps_all = O / SR;
@@ -501,6 +562,27 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
   const int64_t st_hi = min(nsteps_all, st_lo + (int64_t)p.per_split);
   const int64_t cnt = st_hi > st_lo ? st_hi - st_lo : 0;
   const int64_t w_lo = st_lo + cnt * warp / 8, w_hi = st_lo + cnt * (warp + 1) / 8;
+  const int nit = (int)((w_hi - w_lo + NS - 1) / NS);  // iterations of NS steps
+
+  // Copy iteration i (NS steps x SR rows x RB bytes of column block cb)
+  // into ring slot i % NSTG; rows past the warp's range are not copied.
+  auto issue = [&](int i) {
+    if (i < nit) {
+      const int64_t r0 = (w_lo + (int64_t)i * NS) * SR;
+      const int64_t rend = w_hi * SR;
+      const uint32_t dst = ring_s + (uint32_t)((i % NSTG) * STG);
+      constexpr int CPR = RB / 16;
+#pragma unroll
+      for (int j = 0; j < NS * SR * CPR / 32; ++j) {
+        const int c = lane + 32 * j;
+        const int row = c / CPR, ch = c % CPR;
+        if (r0 + row < rend)
+          cp_async16(dst + (uint32_t)(row * RB + ch * 16),
+                     p.codes + (r0 + row) * row_bytes + (int64_t)cb * RB + ch * 16);
+      }
+    }
+    cp_async_commit();
+  };
 
   float acc[4][NT][4];
   float accb[NP][NT][4];  // affine bias term (same for every M row of a pass)
@@ -517,38 +599,14 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
 #pragma unroll
       for (int c = 0; c < 4; ++c) accb[q][n][c] = 0.0f;
 
-  // rows of lane (g, t) within a step
-  auto step_row = [&](int i) -> int {  // i = 0..3 (4-bit) or 0..1 (8-bit)
+  // rows of lane (g, t) within a step: 4-bit (2t, 2t+1) and (2t+8, 2t+9);
+  // 8-bit t and t + 4
+  auto step_row = [&](int i) -> int {
     if (FMT == kFmtA8) return t + 4 * i;
     return 2 * t + (i & 1) + 8 * (i >> 1);
   };
-  constexpr int RPL = FMT == kFmtA8 ? 2 : 4;  // rows per lane per step
-  constexpr int WPR = FMT == kFmtA8 ? 2 : 1;  // code words per row
-  // code words of this lane: [step of the iteration][row][word]; a step's
-  // registers are refilled with the next iteration's codes once decoded
-  uint32_t cur[NS][RPL][WPR];
-  const uint8_t* cbase = p.codes + (int64_t)cb * (FMT == kFmtA8 ? 64 : 32) + (FMT == kFmtA8 ? 8 : 4) * g;
-  auto load_step = [&](uint32_t (&dst)[RPL][WPR], int64_t st) {
-#pragma unroll
-    for (int i = 0; i < RPL; ++i) {
-      if (st < w_hi) {
-        const uint8_t* src = cbase + (st * SR + step_row(i)) * row_bytes;
-        if (WPR == 1) {
-          dst[i][0] = ld_stream_u1(src);
-        } else {
-          const uint2 v = ld_stream_u2(src);
-          dst[i][0] = v.x;
-          dst[i][WPR - 1] = v.y;
-        }
-      } else {
-#pragma unroll
-        for (int w = 0; w < WPR; ++w) dst[i][w] = 0u;
-      }
-    }
-  };
   // Per-row scale (and bias) for this column block: lane L holds row
-  // st0 * SR + L of the iteration's NS * SR rows (<= 64: two rows per lane
-  // for 4-bit).
+  // st0 * SR + 32 k + L of the iteration's NS * SR rows.
   constexpr int PRL = NS * SR / 32;  // parameter rows per lane
   float ps[PRL][NP], pbv[PRL][NP], ns_[PRL][NP], nbv[PRL][NP];
   auto load_params = [&](float (&sv)[PRL][NP], float (&bv)[PRL][NP], int64_t st0) {
@@ -561,9 +619,12 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
         if (!ok) {
           sv[k][q] = 0.0f;
           bv[k][q] = 0.0f;
-        } else if (FMT == kFmtNF4) {
-          sv[k][q] = nf4_scale(p, (uint32_t)(row * KB + cb), mu);
-          bv[k][q] = 0.0f;
+        } else if (FMT == kFmtNF4) {  // raw (q_b bits, t_g), decoded at use
+          uint32_t qq;
+          float tt;
+          nf4_scale_load(p, (uint32_t)(row * KB + cb), qq, tt);
+          sv[k][q] = __uint_as_float(qq);
+          bv[k][q] = tt;
         } else {
           const int64_t gi = (row * I + (int64_t)cb * 64 + 32 * q) / p.G;
           sv[k][q] = __ldg(p.scale + gi);
@@ -572,21 +633,60 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
       }
     }
   };
-
-  int64_t st0 = w_lo;
-  if (st0 < w_hi) {
+  // dY of the lane's K rows, tokens g and 8 + g, one iteration ahead:
+  // 4-bit: the bf16 pair (row, row + 1); 8-bit: the row's bf16 in the low half
+  uint32_t dy[NS][NT][2], dyn[NS][NT][2];
+  auto load_dy = [&](uint32_t (&dst)[NS][NT][2], int64_t st0) {
 #pragma unroll
-    for (int s = 0; s < NS; ++s) load_step(cur[s], st0 + s);
-    load_params(ps, pbv, st0);
+    for (int s = 0; s < NS; ++s)
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int tok = 8 * n + g;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int64_t st = st0 + s;
+          const int64_t orow = st * SR + (FMT == kFmtA8 ? (t + 4 * hh) : (2 * t + 8 * hh));
+          uint32_t v = 0u;
+          if (tok < p.R && st < w_hi) {
+            if (FMT == kFmtA8)
+              v = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p.act + (int64_t)tok * O + orow));
+            else
+              v = __ldg(reinterpret_cast<const uint32_t*>(p.act + (int64_t)tok * O + orow));
+          }
+          dst[s][n][hh] = v;
+        }
+      }
+  };
+
+#pragma unroll
+  for (int i = 0; i < NSTG - 1; ++i) issue(i);
+  if (nit > 0) {
+    load_params(ps, pbv, w_lo);
+    load_dy(dy, w_lo);
   }
-  for (; st0 < w_hi; st0 += NS) {
+  __syncthreads();  // the table is complete
+
+  for (int it = 0; it < nit; ++it) {
+    const int64_t st0 = w_lo + (int64_t)it * NS;
     const int64_t stn = st0 + NS;
-    if (stn < w_hi) load_params(ns_, nbv, stn);
+    issue(it + NSTG - 1);
+    if (stn < w_hi) {
+      load_params(ns_, nbv, stn);
+      load_dy(dyn, stn);
+    }
+    cp_async_wait<NSTG - 1>();
+    __syncwarp();
+    const uint8_t* stg = ring + (it % NSTG) * STG;
+    // NF4: decode the block scales of the rows this lane loaded
+    float sdec[PRL];
+    if (FMT == kFmtNF4) {
+#pragma unroll
+      for (int k = 0; k < PRL; ++k) sdec[k] = nf4_scale_decode(__float_as_uint(ps[k][0]), pbv[k][0], mu);
+    }
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
       const int64_t st = st0 + s;
       if (st >= w_hi) break;
-      const int64_t o0 = st * SR;
       // B operand: bf16 (dY * scale) for the lane's K rows, tokens g, 8 + g
       // 4-bit: pairs of rows (2t, 2t+1) -> b0, (2t+8, 2t+9) -> b1
       // 8-bit: (v, 16 v) of row t -> b0, of row t + 4 -> b1
@@ -597,65 +697,67 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
         for (int hh = 0; hh < 2; ++hh) {
           // scale / bias of the rows this register covers, from the lanes
           // that loaded them (lane = row within the iteration mod 32)
-          float sv0, sv1, bv0, bv1;
+          float sv0, sv1, bv0 = 0.0f, bv1 = 0.0f;
           const int rr0 = s * SR + (FMT == kFmtA8 ? (t + 4 * hh) : (2 * t + 8 * hh));
           {
             const int k0 = rr0 >> 5;
-            const float vs = k0 == 0 ? ps[0][q] : ps[PRL - 1][q];
-            const float vb = k0 == 0 ? pbv[0][q] : pbv[PRL - 1][q];
+            const float vs = FMT == kFmtNF4 ? (k0 == 0 ? sdec[0] : sdec[PRL - 1])
+                                            : (k0 == 0 ? ps[0][q] : ps[PRL - 1][q]);
             sv0 = __shfl_sync(0xffffffffu, vs, rr0 & 31);
-            bv0 = __shfl_sync(0xffffffffu, vb, rr0 & 31);
+            if (FMT != kFmtNF4) {
+              const float vb = k0 == 0 ? pbv[0][q] : pbv[PRL - 1][q];
+              bv0 = __shfl_sync(0xffffffffu, vb, rr0 & 31);
+            }
           }
           if (FMT != kFmtA8) {
             const int rr1 = rr0 + 1;
             const int k1 = rr1 >> 5;
-            const float vs = k1 == 0 ? ps[0][q] : ps[PRL - 1][q];
-            const float vb = k1 == 0 ? pbv[0][q] : pbv[PRL - 1][q];
+            const float vs = FMT == kFmtNF4 ? (k1 == 0 ? sdec[0] : sdec[PRL - 1])
+                                            : (k1 == 0 ? ps[0][q] : ps[PRL - 1][q]);
             sv1 = __shfl_sync(0xffffffffu, vs, rr1 & 31);
-            bv1 = __shfl_sync(0xffffffffu, vb, rr1 & 31);
+            if (FMT != kFmtNF4) {
+              const float vb = k1 == 0 ? pbv[0][q] : pbv[PRL - 1][q];
+              bv1 = __shfl_sync(0xffffffffu, vb, rr1 & 31);
+            }
           } else {
             sv1 = 0.0f;
-            bv1 = 0.0f;
           }
 #pragma unroll
           for (int n = 0; n < NT; ++n) {
-            const int tok = 8 * n + g;
-            const bool ok = tok < p.R;
-            const int64_t orow = o0 + (FMT == kFmtA8 ? (t + 4 * hh) : (2 * t + 8 * hh));
-            float d0 = 0.0f, d1 = 0.0f;
-            if (ok) {
-              if (FMT == kFmtA8) {
-                d0 = __bfloat162float(p.act[(int64_t)tok * O + orow]);
-              } else {
-                const uint32_t pr = __ldg(reinterpret_cast<const uint32_t*>(p.act + (int64_t)tok * O + orow));
-                d0 = __uint_as_float(pr << 16);
-                d1 = __uint_as_float(pr & 0xFFFF0000u);
-              }
-            }
+            const uint32_t pr = dy[s][n][hh];
+            const float d0 = __uint_as_float(pr << 16);
+            const float d1 = __uint_as_float(pr & 0xFFFF0000u);
             if (FMT == kFmtA8) {
               const float v = d0 * sv0;
               bq[q][n][hh] = pack_bf16x2(v, 16.0f * __bfloat162float(__float2bfloat16_rn(v)));
               bb[q][n][hh] = pack_bf16x2(d0 * bv0, 0.0f);
             } else {
               bq[q][n][hh] = pack_bf16x2(d0 * sv0, d1 * sv1);
-              bb[q][n][hh] = pack_bf16x2(d0 * bv0, d1 * bv1);
+              bb[q][n][hh] = FMT == kFmtNF4 ? 0u : pack_bf16x2(d0 * bv0, d1 * bv1);
             }
           }
         }
       }
-      // A operand pairs: [m-tile][a0..a3]; then refill this step's code
-      // registers with the next iteration's
+      // A operand pairs: [m-tile][a0..a3] from the staged rows
       uint32_t A[4][4];
+      const uint8_t* sbase = stg + s * SR * RB;
       if (FMT == kFmtA8) {
         // rows t (a0: M row g, a1: M row g + 8) and t + 4 (a2, a3); column
         // 8 g + 2 mt (+1 for M row g + 8) is byte 2 mt (+1) of the 8 bytes
+        uint32_t w[2][2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const uint2 v = *reinterpret_cast<const uint2*>(sbase + step_row(i) * RB + 8 * g);
+          w[i][0] = v.x;
+          w[i][1] = v.y;
+        }
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
-          const int w = mt >> 1, k = 2 * (mt & 1);
-          A[mt][0] = tbl(table, cur[s][0][w], laneoff, k);
-          A[mt][1] = tbl(table, cur[s][0][w], laneoff, k + 1);
-          A[mt][2] = tbl(table, cur[s][1][w], laneoff, k);
-          A[mt][3] = tbl(table, cur[s][1][w], laneoff, k + 1);
+          const int wi = mt >> 1, k = 2 * (mt & 1);
+          A[mt][0] = tbl(table, w[0][wi], laneoff, k);
+          A[mt][1] = tbl(table, w[0][wi], laneoff, k + 1);
+          A[mt][2] = tbl(table, w[1][wi], laneoff, k);
+          A[mt][3] = tbl(table, w[1][wi], laneoff, k + 1);
         }
       } else {
         // rows (2t, 2t+1) -> P1, (2t+8, 2t+9) -> P2; zip the nibbles so that
@@ -663,7 +765,8 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
         uint32_t ze[2], zo[2];
 #pragma unroll
         for (int pp = 0; pp < 2; ++pp) {
-          const uint32_t wa = cur[s][2 * pp][0], wb = cur[s][2 * pp + 1][0];
+          const uint32_t wa = *reinterpret_cast<const uint32_t*>(sbase + step_row(2 * pp) * RB + 4 * g);
+          const uint32_t wb = *reinterpret_cast<const uint32_t*>(sbase + step_row(2 * pp + 1) * RB + 4 * g);
           ze[pp] = (wa & 0x0F0F0F0Fu) | ((wb << 4) & 0xF0F0F0F0u);
           zo[pp] = ((wa >> 4) & 0x0F0F0F0Fu) | (wb & 0xF0F0F0F0u);
         }
@@ -675,7 +778,6 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
           A[mt][3] = tbl(table, zo[1], laneoff, mt);
         }
       }
-      if (stn + s < w_hi) load_step(cur[s], stn + s);
 #pragma unroll
       for (int q = 0; q < NP; ++q) {
         const bool keep = !G32 || (g >> 2) == q;
@@ -693,6 +795,7 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
         }
       }
     }
+    __syncwarp();  // every lane is done with this slot before it is refilled
     if (stn < w_hi) {
 #pragma unroll
       for (int k = 0; k < PRL; ++k)
@@ -701,8 +804,16 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtNF4 ? 2 : 1) smallr_dx_
           ps[k][q] = ns_[k][q];
           pbv[k][q] = nbv[k][q];
         }
+#pragma unroll
+      for (int s = 0; s < NS; ++s)
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          dy[s][n][0] = dyn[s][n][0];
+          dy[s][n][1] = dyn[s][n][1];
+        }
     }
   }
+  cp_async_wait<0>();
   if (FMT != kFmtNF4) {  // the bias term belongs to every M row of its pass
 #pragma unroll
     for (int q = 0; q < NP; ++q) {
@@ -816,14 +927,17 @@ struct SrPlan {
   int per_split;  // K blocks or K steps per split
 };
 
-// One wave at two CTAs per SM: tiles x splits ~ 2 x SMs.
+// One wave: tiles x splits <= CTAs per SM x SMs (two CTAs per SM for NF4,
+// one for the affine variants, which take more registers); never a second,
+// partial wave.
 SrPlan sr_plan(bool dx, const WView& w) {
   SrPlan pl;
-  const int target = 2 * num_sms();
+  const int per_sm = sr_fmt(w) == kFmtNF4 ? 2 : 1;
+  const int target = per_sm * num_sms();
   if (!dx) {
     pl.tiles = (int)(w.O / 128);
     const int KB = (int)(w.I / 64);
-    int sp = (target + pl.tiles / 2) / pl.tiles;
+    int sp = target / pl.tiles;
     if (sp < 1) sp = 1;
     if (sp > KB / 4) sp = KB / 4 > 0 ? KB / 4 : 1;  // at least one block per K warp
     pl.per_split = (KB + sp - 1) / sp;
@@ -832,7 +946,7 @@ SrPlan sr_plan(bool dx, const WView& w) {
     pl.tiles = (int)(w.I / 64);
     const int step = sr_fmt(w) == kFmtA8 ? 8 : 16;
     const int nst = (int)(w.O / step);
-    int sp = (target + pl.tiles / 2) / pl.tiles;
+    int sp = target / pl.tiles;
     if (sp < 1) sp = 1;
     if (sp > nst / 8) sp = nst / 8 > 0 ? nst / 8 : 1;  // at least one step per warp
     pl.per_split = (nst + sp - 1) / sp;
@@ -841,20 +955,28 @@ SrPlan sr_plan(bool dx, const WView& w) {
   return pl;
 }
 
+// Dynamic shared memory: the byte table plus the eight warps' rings of code
+// blocks (forward: 3 blocks of 64 rows, 2 for 8-bit codes; input gradient: 3
+// iterations of 64 rows (4-bit) or 32 rows (8-bit)).
+constexpr int sr_smem_bytes(bool dx, int fmt) {
+  return kTableBytes + 8 * (dx ? 3 * 2048 : (fmt == kFmtA8 ? 2 * 4096 : 3 * 2048));
+}
+
 template <int NT, int FMT, bool G32>
 cudaError_t sr_launch(bool dx, const SrPlan& pl, const SrParams& p, cudaStream_t st) {
   auto kern = dx ? smallr_dx_kernel<NT, FMT, G32> : smallr_fwd_kernel<NT, FMT, G32>;
+  const int smem = sr_smem_bytes(dx, FMT);
   static bool attr_fwd = false, attr_dx = false;
   bool& attr = dx ? attr_dx : attr_fwd;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kTableBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)pl.tiles, (unsigned)pl.splits);
   cfg.blockDim = dim3(kSrThreads);
-  cfg.dynamicSmemBytes = kTableBytes;
+  cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = st;
   cudaLaunchAttribute attr1[1];
   attr1[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

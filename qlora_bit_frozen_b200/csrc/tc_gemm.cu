@@ -56,7 +56,12 @@ constexpr int kDecGroups = 2;        // decoder groups (alternate K steps)
 // thread decoding half a 64-weight row, so that twice as many warps hide
 // the decode's dependency latency; four (a whole row per thread) at smaller
 // tiles, which keep two CTAs per SM.
-constexpr int dec_warps(int bn) { return bn >= 256 ? 8 : 4; }
+// (eight per group at 256-token tiles measured no faster than four on the
+// 8B / 14B / Qwen steps, so four is the default)
+#ifndef QLORA_TC_DEC_WARPS_256
+#define QLORA_TC_DEC_WARPS_256 4
+#endif
+constexpr int dec_warps(int bn) { return bn >= 256 ? QLORA_TC_DEC_WARPS_256 : 4; }
 constexpr int threads_of(int bn) { return 32 * (2 + kDecGroups * dec_warps(bn)); }
 // epilogue groups: four warps each, one per TMEM lane quarter
 constexpr int epi_groups(int bn) { return kDecGroups * dec_warps(bn) / 4; }
@@ -338,7 +343,9 @@ constexpr int cols_per_group() {
   return BN >= 64 ? BN / epi_groups(BN) : BN;
 }
 
-template <bool DX, int BN>
+// WF: weight format, a template parameter so the decoder loop carries no
+// format branches (0 NF4 double-quant, 1 NF4 legacy fp32 scales, 2 affine 4-bit)
+template <bool DX, int BN, int WF>
 __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN>::kMinCtas)
     tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_pk,
@@ -541,8 +548,8 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN>::kMinCtas)
     const int half = wi >> 2;  // always 0 with four warps per group
     const int quad = warp & 3;
     const int u = DX ? (((int)threadIdx.x - 64 - 32 * DW * group) & 127) : 32 * quad + lane;
-    const bool legacy = p.sb != nullptr;   // fp32 block scales stored as they are
-    const bool affine = p.asc != nullptr;  // 4-bit affine groups: (scale, bias)
+    constexpr bool legacy = WF == 1;  // fp32 block scales stored as they are
+    constexpr bool affine = WF == 2;  // 4-bit affine groups: (scale, bias)
     const float mu = (legacy || affine) ? 0.0f : __ldg(p.mu);
     const uint32_t bpr = (uint32_t)(p.I / kBK);  // blocks per W row
     auto block_of = [&](int kb) -> uint32_t {
@@ -801,12 +808,12 @@ int num_sms_cached() {
 // The launch waits for the kernel before it in the stream only where the
 // adapter step needs that kernel's output (programmatic dependent launch):
 // the weight stream starts while U / V are still being computed.
-template <bool DX, int BN>
+template <bool DX, int BN, int WF>
 cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                       const CUtensorMap& d, const CUtensorMap& o, const TcParams& p,
                       cudaStream_t st) {
   using Cf = Cfg<DX, BN>;
-  auto kern = tc_qlinear_kernel<DX, BN>;
+  auto kern = tc_qlinear_kernel<DX, BN, WF>;
   static bool attr_set = false;  // once per instantiation (keeps graph capture free of it)
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cf::kSmem);
@@ -833,17 +840,26 @@ cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, con
   return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+template <bool DX, int WF>
+cudaError_t launch_plan_wf(const TcPlan& pl, dim3 grid, const CUtensorMap& a, const CUtensorMap& b,
+                           const CUtensorMap& c, const CUtensorMap& d, const CUtensorMap& o,
+                           const TcParams& p, cudaStream_t st) {
+  switch (pl.bn) {
+    case 16: return launch_bn<DX, 16, WF>(grid, a, b, c, d, o, p, st);
+    case 32: return launch_bn<DX, 32, WF>(grid, a, b, c, d, o, p, st);
+    case 64: return launch_bn<DX, 64, WF>(grid, a, b, c, d, o, p, st);
+    case 128: return launch_bn<DX, 128, WF>(grid, a, b, c, d, o, p, st);
+    default: return launch_bn<DX, 256, WF>(grid, a, b, c, d, o, p, st);
+  }
+}
+
 template <bool DX>
 cudaError_t launch_plan(const TcPlan& pl, dim3 grid, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& c, const CUtensorMap& d, const CUtensorMap& o,
                         const TcParams& p, cudaStream_t st) {
-  switch (pl.bn) {
-    case 16: return launch_bn<DX, 16>(grid, a, b, c, d, o, p, st);
-    case 32: return launch_bn<DX, 32>(grid, a, b, c, d, o, p, st);
-    case 64: return launch_bn<DX, 64>(grid, a, b, c, d, o, p, st);
-    case 128: return launch_bn<DX, 128>(grid, a, b, c, d, o, p, st);
-    default: return launch_bn<DX, 256>(grid, a, b, c, d, o, p, st);
-  }
+  if (p.asc) return launch_plan_wf<DX, 2>(pl, grid, a, b, c, d, o, p, st);
+  if (p.sb) return launch_plan_wf<DX, 1>(pl, grid, a, b, c, d, o, p, st);
+  return launch_plan_wf<DX, 0>(pl, grid, a, b, c, d, o, p, st);
 }
 
 int group_cols(int bn) { return bn >= 64 ? bn / epi_groups(bn) : bn; }

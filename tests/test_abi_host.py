@@ -202,17 +202,17 @@ def _planned_splits(Mw, KB, R, sms=148):
 def _smallr_splits(dx, O, I, R, sms=148):
     """The few-token plan as the design states it (1..16 tokens, O % 128 == 0,
     I % 64 == 0): 128-row tiles (forward) or 64-column blocks (input
-    gradient) times K splits filling one wave at two CTAs per SM, at least
+    gradient) times K splits filling at most one wave at two CTAs per SM, at least
     one 64-column block per K warp (4) or one 16-row step per warp (8), no
     empty split.  0 when the path does not apply."""
     if not (1 <= R <= 16 and O % 128 == 0 and I % 64 == 0 and O <= 65536 and I <= 32768):
         return 0
-    target = 2 * sms
+    target = 2 * sms  # NF4: two CTAs per SM
     if not dx:
         tiles, n, per_min = O // 128, I // 64, 4
     else:
         tiles, n, per_min = I // 64, O // 16, 8
-    sp = max(1, (target + tiles // 2) // tiles)
+    sp = max(1, target // tiles)
     sp = min(sp, max(1, n // per_min))
     per = -(-n // sp)
     return -(-n // per)
