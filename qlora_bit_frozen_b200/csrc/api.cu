@@ -419,14 +419,18 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
   float* U = U_out ? U_out : (float*)((char*)ws + L.u);
   const WView v = view_of(w);
   const bool bf16 = compute == QLORA_COMPUTE_BF16;
-  if (bf16 && smallr_supported(v, R, X, Y)) {
+  // bf16: the few-token kernels where they are measured faster (or the only
+  // fast path), else the tensor-core kernel, else the SIMT tiles
+  const bool fwd_tc = bf16 && tc_fwd_supported(v, X, Y, R);
+  const bool fwd_sr = bf16 && smallr_supported(v, R, X, Y) && (!fwd_tc || smallr_preferred(false, v, R));
+  if (fwd_sr) {
     // 1..16 tokens: U = X A^T, then the bandwidth-bound GEMV, which starts
     // its weight stream at once and waits for U only in its epilogue
     e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, nullptr, nullptr, 0, 0, 1.0f, nullptr,
                       nullptr, red, tickets, (uint16_t*)((char*)ws + L.split));
     if (e == cudaSuccess)
       e = launch_smallr_fwd(v, X, R, U, B, r, sc, Y, (char*)ws + L.sr, (uint32_t*)ws, tickets, s);
-  } else if (bf16 && tc_fwd_supported(v, X, Y, R)) {
+  } else if (fwd_tc) {
     void* tcws = (char*)ws + L.tc;
     e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws), B, w->O, 0, sc,
                       tc_w_pad(tcws, R), nullptr, red, tickets, (uint16_t*)((char*)ws + L.split));
@@ -464,8 +468,9 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   void* red = (char*)ws + L.red;
   // V = dY B  (B is [O x r]: L(k = o, j) = B[o*r + j]); its padded bf16 copy
   // feeds the tensor-core kernel's adapter step
-  const bool sr = dX && bf16 && smallr_supported(v, R, dY, dX);
-  const bool tc = !sr && dX && bf16 && tc_dx_supported(v, dY, dX, R);
+  const bool dx_tc = dX && bf16 && tc_dx_supported(v, dY, dX, R);
+  const bool sr = dX && bf16 && smallr_supported(v, R, dY, dX) && (!dx_tc || smallr_preferred(true, v, R));
+  const bool tc = !sr && dx_tc;
   void* tcws = (char*)ws + L.tc;
   if (dX || dA) {
     float* bt = (float*)((char*)ws + L.bt);

@@ -1036,6 +1036,18 @@ SrParams sr_params(const WView& w, const void* act, int64_t R, const float* aux,
 
 }  // namespace
 
+// Measured on one B200 (W 12288 x 4096 and 4096 x 4096, CUDA graph, cold L2):
+// these kernels beat the tensor-core kernel for NF4 at one token (12288 x
+// 4096: forward 19.3 vs 27.5 us, input gradient 24.7 vs 29.0 us) but not at
+// 16 (32.5 vs 28.4, 38.8 vs 30.3 us), nor for 4-bit affine codes at any
+// token count; 8-bit affine codes have no tensor-core path.  NF4 takes this
+// path while one 8-token MMA tile covers the tokens.
+bool smallr_preferred(bool dx, const WView& w, int64_t R) {
+  (void)dx;
+  if (w.fmt == QLORA_FMT_AFFINE) return w.bits == 8;
+  return R <= 8;
+}
+
 bool smallr_supported(const WView& w, int64_t R, const void* act, const void* out) {
   if (R < 1 || R > 16) return false;
   if (w.O < 128 || w.I < 64 || w.O % 128 != 0 || w.I % 64 != 0) return false;

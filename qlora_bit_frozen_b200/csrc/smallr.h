@@ -11,6 +11,9 @@ struct WView;
 // NF4 (B = 64) or affine (4/8-bit, G = 32/64/128) weight, 1 <= R <= 16 tokens,
 // O % 128 == 0, I % 64 == 0, codes and activations 16-byte aligned.
 bool smallr_supported(const WView& w, int64_t R, const void* act, const void* out);
+// Whether the few-token kernels are the faster choice for this op, format and
+// token count where the tensor-core kernel also applies (measured).
+bool smallr_preferred(bool dx, const WView& w, int64_t R);
 // Workspace bytes of the split-K partial sums (0 when the plan has one split).
 size_t smallr_ws(bool dx, const WView& w, int64_t R);
 
