@@ -164,217 +164,223 @@ __device__ __forceinline__ float nf4_scale_decode(uint32_t q, float t, float mu)
 
 // ------------------------------------------------------------------ forward
 //
-// CTA: 128 weight rows x one K range (split blockIdx.y).  Warp (wr, wk):
-// rows 64 wr .. +63 (four 16-row m-tiles), K blocks kb = lo + wk, lo + wk + 4,
-// ... of the range.  Per block the lane holds, for rows g and g + 8 of each
-// m-tile, the 16 columns 16 t .. 16 t + 15 (t = lane % 4, g = lane / 4):
-// 8 code bytes (4-bit) or 16 (8-bit).  MMA j of the block pairs K index
-// (2t, 2t+1) with columns 16t + 4j + {0,1} and (2t+8, 2t+9) with
-// 16t + 4j + {2,3} (4-bit; 8-bit: one column per K pair, 16t + 2j and
-// 16t + 2j + 1), and the activation operand is loaded in the same order.
+// CTA: 128 weight rows x one K range (split blockIdx.y).  Warp w owns the
+// 16 rows 16 w .. 16 w + 15 of the tile (one m16 MMA tile) over the CTA's
+// whole K range, so no two warps share an output and nothing is reduced
+// inside the CTA.  Per 64-column block the lane holds, for rows g and g + 8
+// (t = lane % 4, g = lane / 4), the 16 columns 16 t .. 16 t + 15: 8 code
+// bytes (4-bit) or 16 (8-bit).  MMA j of the block pairs K index (2t, 2t+1)
+// with columns 16t + 4j + {0,1} and (2t+8, 2t+9) with 16t + 4j + {2,3}
+// (4-bit; 8-bit: one column per K pair, 16t + 2j and 16t + 2j + 1), and the
+// activation operand is loaded in the same order.
+//
+// Codes stream through a ring of kStages stages per warp, a stage being
+// 128 contiguous bytes of each of the warp's 16 rows (4 blocks of 4-bit
+// codes, 2 of 8-bit): whole 128-byte lines, so that DRAM serves long runs of
+// each row rather than 32-byte pieces of thousands of rows.  In shared
+// memory the 16-byte chunk c of row y sits at c ^ swz(y), which keeps the
+// lanes' reads conflict-free.  Per stage lane l loads the scale inputs of
+// row l % 16 (blocks l / 16, l / 16 + 2, ...; groups of 32: group half
+// l / 16 of every block), and rows g and g + 8 take theirs by shuffles.
 template <int FMT>
 struct FwdShape {
   static constexpr int kChunkU32 = FMT == kFmtA8 ? 4 : 2;  // code words per row per block
-  static constexpr int kMmas = FMT == kFmtA8 ? 8 : 4;      // MMAs per m-tile per block
+  static constexpr int kMmas = FMT == kFmtA8 ? 8 : 4;      // MMAs per block
+  static constexpr int kRowBytes = FMT == kFmtA8 ? 64 : 32;
+  static constexpr int kStageBlocks = 128 / kRowBytes;     // blocks per stage
+  static constexpr int kStages = 3;
 };
+// chunk position swizzle of stage row y (see above)
+template <int FMT>
+__device__ __forceinline__ uint32_t fwd_swz(uint32_t y) {
+  return FMT == kFmtA8 ? ((y & 1u) << 2) : ((y & 3u) << 1);
+}
+
+__device__ __forceinline__ void mma_bf16_16816_zc(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                  uint32_t a2, uint32_t a3, uint32_t b0,
+                                                  uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
+__device__ __forceinline__ void mma_bf16_16816_acc(float (&d)[4], uint32_t a0, uint32_t a1,
+                                                   uint32_t a2, uint32_t a3, uint32_t b0,
+                                                   uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 template <int NT, int FMT, bool G32>
-__global__ void __launch_bounds__(kSrThreads, FMT == kFmtA8 ? 1 : 2) smallr_fwd_kernel(const SrParams p) {
+__global__ void __launch_bounds__(kSrThreads, 2) smallr_fwd_kernel(const SrParams p) {
   using S = FwdShape<FMT>;
   constexpr int CW = S::kChunkU32;
-  constexpr int NSTG = FMT == kFmtA8 ? 2 : 3;          // blocks per warp ring
-  constexpr int RB = FMT == kFmtA8 ? 64 : 32;          // code bytes per row per block
-  constexpr int STG = 64 * RB;                          // one block of the warp's 64 rows
-  constexpr int NP = G32 ? 2 : 1;                       // group passes per block
+  constexpr int KM = S::kMmas;
+  constexpr int RB = S::kRowBytes;
+  constexpr int SB = S::kStageBlocks;
+  constexpr int STG = 16 * 128;      // one stage: 16 rows x 128 bytes
+  constexpr int NSTG = S::kStages;
+  constexpr int NP = G32 ? 2 : 1;    // group passes per block
+  constexpr int NE = G32 ? SB : SB / 2;  // scale entries a lane loads per stage
   extern __shared__ __align__(1024) uint8_t sr_smem[];
   uint32_t* table = reinterpret_cast<uint32_t*>(sr_smem);
   fill_table<FMT>(table);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int wr = warp & 1, wk = warp >> 1;
   const int64_t I = p.I, O = p.O;
-  const int64_t rbase = (int64_t)blockIdx.x * 128 + 64 * wr;
+  const int64_t row0 = (int64_t)blockIdx.x * 128 + 16 * warp;
   const int KB = (int)(I / 64);
   const int kb_lo = (int)blockIdx.y * p.per_split;
   const int kb_hi = min(KB, kb_lo + p.per_split);
+  const int nblk = kb_hi > kb_lo ? kb_hi - kb_lo : 0;
+  const int nstage = (nblk + SB - 1) / SB;
   const uint32_t laneoff = (uint32_t)lane * 4u;
   const int64_t row_bytes = FMT == kFmtA8 ? I : I / 2;
   const float mu = (FMT == kFmtNF4 && !p.legacy) ? __ldg(p.mu) : 0.0f;
-  // this warp's ring of code blocks, after the table
-  uint8_t* ring = sr_smem + kTableBytes + warp * NSTG * STG;
+  const int glog = FMT == kFmtNF4 ? 0 : 31 - __clz(p.G);
+  const uint8_t* ring = sr_smem + kTableBytes + warp * NSTG * STG;
   const uint32_t ring_s = smem_u32(ring);
-  // The warp's blocks: kb = kb_lo + wk + 4 i, i < nblk.
-  const int first = kb_lo + wk;
-  const int nblk = first < kb_hi ? (kb_hi - first + 3) / 4 : 0;
 
-  // Copy block i of the warp (64 rows x RB bytes) into ring slot i % NSTG:
-  // 16-byte chunks, row-major, lane-strided (every instruction moves 512
-  // contiguous-by-row bytes).
-  auto issue = [&](int i) {
-    if (i < nblk) {
-      const int kb = first + 4 * i;
-      const uint32_t dst = ring_s + (uint32_t)((i % NSTG) * STG);
-      constexpr int CPR = RB / 16;  // chunks per row
+  // This lane's copies of a stage: chunk c = lane % 8 of rows lane / 8 + 4 j
+  // (block c * 16 / RB of the stage), stored at chunk c ^ swz(row).
+  const int cch = lane & 7;
+  const int cblk = cch * 16 / RB;
+  const uint8_t* gsrc = p.codes + (row0 + (lane >> 3)) * row_bytes + (int64_t)kb_lo * RB + cch * 16;
+  auto issue = [&](int st) {
+    if (st < nstage && st * SB + cblk < nblk) {
+      const uint32_t dst = ring_s + (uint32_t)((st % NSTG) * STG);
 #pragma unroll
-      for (int j = 0; j < 64 * CPR / 32; ++j) {
-        const int c = lane + 32 * j;
-        const int row = c / CPR, ch = c % CPR;
-        cp_async16(dst + (uint32_t)(row * RB + ch * 16),
-                   p.codes + (rbase + row) * row_bytes + (int64_t)kb * RB + ch * 16);
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t y = (uint32_t)((lane >> 3) + 4 * j);
+        cp_async16(dst + y * 128u + ((((uint32_t)cch) ^ fwd_swz<FMT>(y)) << 4),
+                   gsrc + (int64_t)st * 128 + (int64_t)(4 * j) * row_bytes);
       }
     }
-    cp_async_commit();  // one group per block (empty past the end: uniform counting)
+    cp_async_commit();  // one group per stage (empty past the end: uniform counting)
   };
 
-  float acc[4][NT][4];
+  // Raw scale inputs of stage st: NF4 (q_b as float bits, t_g) of row
+  // l % 16, blocks l / 16 + 2 e; affine (scale, bias), groups of 32: half
+  // l / 16 of block e.
+  const int64_t prow = row0 + (lane & 15);
+  const int phalf = lane >> 4;
+  auto load_params = [&](int st, float (&ra)[NE], float (&rb)[NE]) {
 #pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc[a][n][c] = 0.0f;
-
-  // Per-row block (or group) parameters of rows rbase + lane and
-  // rbase + 32 + lane, loaded one block ahead as raw values (the loads
-  // complete while the current block is decoded).  NF4: q_b (as float bits)
-  // and t_g, decoded at use; affine: scale and bias per pass.
-  float pa[2][NP], pb[2][NP], na[2][NP], nb[2][NP];
-  auto load_params = [&](float (&sa)[2][NP], float (&sb)[2][NP], int kb) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int64_t row = rbase + 32 * h + lane;
+    for (int e = 0; e < NE; ++e) {
+      const int blk = st * SB + (G32 ? e : phalf + 2 * e);
+      const bool ok = blk < nblk;
       if (FMT == kFmtNF4) {
-        uint32_t q;
-        float tt;
-        nf4_scale_load(p, (uint32_t)(row * KB + kb), q, tt);
-        sa[h][0] = __uint_as_float(q);
-        sb[h][0] = tt;
+        uint32_t q = 0xFFFFFFFFu;
+        float tt = 0.0f;
+        if (ok) nf4_scale_load(p, (uint32_t)(prow * KB + kb_lo + blk), q, tt);
+        ra[e] = __uint_as_float(q);
+        rb[e] = tt;
       } else {
-#pragma unroll
-        for (int q = 0; q < NP; ++q) {
-          const int64_t gi = (row * I + (int64_t)kb * 64 + 32 * q) / p.G;
-          sa[h][q] = __ldg(p.scale + gi);
-          sb[h][q] = __ldg(p.bias + gi);
+        ra[e] = 0.0f;
+        rb[e] = 0.0f;
+        if (ok) {
+          const int64_t gi = (prow * I + (int64_t)(kb_lo + blk) * 64 + (G32 ? 32 * phalf : 0)) >> glog;
+          ra[e] = __ldg(p.scale + gi);
+          rb[e] = __ldg(p.bias + gi);
         }
       }
     }
   };
-  // activation operand: columns 64 kb + 16 t + 4 m .. + 3 of tokens g, 8 + g
+  // activation rows of this lane: tokens g (n = 0) and 8 + g (n = 1)
   const bool tok_ok0 = g < p.R, tok_ok1 = (8 + g) < p.R;
-  uint2 xw[NT][4], xn[NT][4];
-  auto load_x = [&](uint2 (&dst)[NT][4], int kb) {
+  const __nv_bfloat16* xrow[NT];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const bool ok = n == 0 ? tok_ok0 : tok_ok1;
-      const __nv_bfloat16* xr = p.act + (int64_t)(8 * n + g) * I + (int64_t)kb * 64 + 16 * t;
-#pragma unroll
-      for (int m = 0; m < 4; ++m)
-        dst[n][m] = ok ? __ldg(reinterpret_cast<const uint2*>(xr + 4 * m)) : make_uint2(0u, 0u);
-    }
-  };
+  for (int n = 0; n < NT; ++n)
+    xrow[n] = p.act + (int64_t)(8 * n + g) * I + (int64_t)kb_lo * 64 + 16 * t;
 
-  // prologue: NSTG - 1 blocks in flight, parameters and activations of block 0
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[n][c] = 0.0f;
+
+  // prologue: NSTG - 1 stages in flight, the first stage's scale inputs
 #pragma unroll
   for (int i = 0; i < NSTG - 1; ++i) issue(i);
-  if (nblk > 0) {
-    load_params(pa, pb, first);
-    load_x(xw, first);
-  }
+  float ca[NE], cb[NE], na[NE], nb[NE];
+  load_params(0, ca, cb);
   __syncthreads();  // the table is complete
 
-  for (int i = 0; i < nblk; ++i) {
-    const int kb = first + 4 * i;
-    const bool more = i + 1 < nblk;
-    issue(i + NSTG - 1);
-    if (more) {
-      load_params(na, nb, kb + 4);
-      load_x(xn, kb + 4);
+  for (int st = 0; st < nstage; ++st) {
+    issue(st + NSTG - 1);
+    if (st + 1 < nstage) load_params(st + 1, na, nb);
+    // activation lines two stages ahead into L1
+#pragma unroll
+    for (int jb = 0; jb < SB; ++jb) {
+      const int bp = (st + 2) * SB + jb;
+      if (bp < nblk) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+          if (n == 0 ? tok_ok0 : tok_ok1)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(xrow[n] + (int64_t)bp * 64));
+      }
     }
-    cp_async_wait<NSTG - 1>();  // block i has landed (this lane's copies)
+    cp_async_wait<NSTG - 1>();  // stage st has landed (this lane's copies)
     __syncwarp();               // ... and every lane's
-    const uint8_t* blk = ring + (i % NSTG) * STG;
-    // B operand registers per MMA j: 4-bit (x[c], x[c+1]) pairs as loaded;
-    // 8-bit (x[c], 16 x[c]) pairs.
-    uint32_t bx[NT][S::kMmas][2];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      if (FMT == kFmtA8) {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t w0 = xw[n][m].x, w1 = xw[n][m].y;
-          const uint32_t s0 = hmul2_bf16(w0, 0x41804180u), s1 = hmul2_bf16(w1, 0x41804180u);  // 16.0
-          bx[n][2 * m][0] = prmt(w0, s0, 0x5410u);
-          bx[n][2 * m][1] = prmt(w0, s0, 0x7632u);
-          bx[n][2 * m + 1][0] = prmt(w1, s1, 0x5410u);
-          bx[n][2 * m + 1][1] = prmt(w1, s1, 0x7632u);
-        }
-      } else {
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          bx[n][m][0] = xw[n][m].x;
-          bx[n][m][1] = xw[n][m].y;
-        }
-      }
-    }
-    // affine: sum of the activations over each group pass (ones-operand MMA)
-    float xs[NP][NT][4];
-    if (FMT != kFmtNF4) {
-      // the ones operand: (1, 1) pairs for 4-bit, (1, 0) for 8-bit (only the x half)
-      const uint32_t one = FMT == kFmtA8 ? 0x00003F80u : 0x3F803F80u;
-#pragma unroll
-      for (int q = 0; q < NP; ++q) {
-        const uint32_t a = (!G32 || (t >> 1) == q) ? one : 0u;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c) xs[q][n][c] = 0.0f;
-#pragma unroll
-          for (int j = 0; j < S::kMmas; ++j)
-            mma_bf16_16816(xs[q][n], a, a, a, a, bx[n][j][0], bx[n][j][1]);
-        }
-      }
-    }
-    // NF4: decode the two block scales this lane loaded (rows lane, 32 + lane)
-    float sdec[2];
+    float sdec[NE];
     if (FMT == kFmtNF4) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) sdec[h] = nf4_scale_decode(__float_as_uint(pa[h][0]), pb[h][0], mu);
+      for (int e = 0; e < NE; ++e) sdec[e] = nf4_scale_decode(__float_as_uint(ca[e]), cb[e], mu);
     }
-    // rows of this lane's accumulators: 16 mt + g (c0, c1) and 16 mt + g + 8 (c2, c3)
+    const uint8_t* stg = ring + (st % NSTG) * STG;
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
-      const int srcA = 16 * (mt & 1) + g, srcB = srcA + 8;
-      const int hsel = mt >> 1;  // rows 0..31 from the first parameter set, 32..63 the second
-      float sA[NP], sB[NP], bA[NP], bB[NP];
+    for (int jb = 0; jb < SB; ++jb) {
+      const int blkn = st * SB + jb;
+      if (blkn >= nblk) break;
+      // activation operand: 16 columns of tokens g, 8 + g as pairs
+      uint32_t bx[NT][KM][2];
 #pragma unroll
-      for (int q = 0; q < NP; ++q) {
-        const float va = FMT == kFmtNF4 ? (hsel ? sdec[1] : sdec[0]) : (hsel ? pa[1][q] : pa[0][q]);
-        sA[q] = __shfl_sync(0xffffffffu, va, srcA);
-        sB[q] = __shfl_sync(0xffffffffu, va, srcB);
-        if (FMT != kFmtNF4) {
-          const float vb = hsel ? pb[1][q] : pb[0][q];
-          bA[q] = __shfl_sync(0xffffffffu, vb, srcA);
-          bB[q] = __shfl_sync(0xffffffffu, vb, srcB);
+      for (int n = 0; n < NT; ++n) {
+        uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+        if (n == 0 ? tok_ok0 : tok_ok1) {
+          const uint4* xp = reinterpret_cast<const uint4*>(xrow[n] + (int64_t)blkn * 64);
+          v0 = __ldg(xp);
+          v1 = __ldg(xp + 1);
+        }
+        const uint32_t xw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        if (FMT == kFmtA8) {
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t w0 = xw[2 * m], w1 = xw[2 * m + 1];
+            const uint32_t s0 = hmul2_bf16(w0, 0x41804180u), s1 = hmul2_bf16(w1, 0x41804180u);  // 16.0
+            bx[n][2 * m][0] = prmt(w0, s0, 0x5410u);
+            bx[n][2 * m][1] = prmt(w0, s0, 0x7632u);
+            bx[n][2 * m + 1][0] = prmt(w1, s1, 0x5410u);
+            bx[n][2 * m + 1][1] = prmt(w1, s1, 0x7632u);
+          }
         } else {
-          bA[q] = 0.0f;
-          bB[q] = 0.0f;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            bx[n][m][0] = xw[2 * m];
+            bx[n][m][1] = xw[2 * m + 1];
+          }
         }
       }
       // decoded pairs of rows g (pA) and g + 8 (pB): one per code byte
       uint32_t pA[4 * CW], pB[4 * CW];
       {
-        const uint8_t* ra = blk + (16 * mt + g) * RB + (FMT == kFmtA8 ? 16 : 8) * t;
-        const uint8_t* rb = ra + 8 * RB;
         uint32_t wa[CW], wb[CW];
         if (CW == 2) {
-          const uint2 va = *reinterpret_cast<const uint2*>(ra);
-          const uint2 vb = *reinterpret_cast<const uint2*>(rb);
+          // 8 bytes: block jb, columns 16 t .. (chunk 2 jb + t / 2, half t % 2)
+          const uint32_t c = (uint32_t)(2 * jb + (t >> 1));
+          const uint32_t off = (uint32_t)(t & 1) * 8u;
+          const uint2 va = *reinterpret_cast<const uint2*>(stg + g * 128 + ((c ^ fwd_swz<FMT>(g)) << 4) + off);
+          const uint2 vb = *reinterpret_cast<const uint2*>(stg + (g + 8) * 128 + ((c ^ fwd_swz<FMT>(g + 8)) << 4) + off);
           wa[0] = va.x; wa[CW - 1] = va.y;
           wb[0] = vb.x; wb[CW - 1] = vb.y;
         } else {
-          const uint4 va = *reinterpret_cast<const uint4*>(ra);
-          const uint4 vb = *reinterpret_cast<const uint4*>(rb);
+          // 16 bytes: block jb, columns 16 t .. (chunk 4 jb + t)
+          const uint32_t c = (uint32_t)(4 * jb + t);
+          const uint4 va = *reinterpret_cast<const uint4*>(stg + g * 128 + ((c ^ fwd_swz<FMT>(g)) << 4));
+          const uint4 vb = *reinterpret_cast<const uint4*>(stg + (g + 8) * 128 + ((c ^ fwd_swz<FMT>(g + 8)) << 4));
           wa[0] = va.x; wa[1 % CW] = va.y; wa[2 % CW] = va.z; wa[3 % CW] = va.w;
           wb[0] = vb.x; wb[1 % CW] = vb.y; wb[2 % CW] = vb.z; wb[3 % CW] = vb.w;
         }
@@ -388,103 +394,94 @@ __global__ void __launch_bounds__(kSrThreads, FMT == kFmtA8 ? 1 : 2) smallr_fwd_
       }
 #pragma unroll
       for (int q = 0; q < NP; ++q) {
+        // scale (and bias) of rows g and g + 8 for this block / group half:
+        // from lane 16 q + row, entry jb (groups of 32), else lane
+        // 16 (jb % 2) + row, entry jb / 2
+        const int src = G32 ? 16 * q : 16 * (jb & 1);
+        const int ent = G32 ? jb : (jb >> 1);
+        float sA, sB, bA = 0.0f, bB = 0.0f;
+        if (FMT == kFmtNF4) {
+          sA = __shfl_sync(0xffffffffu, sdec[ent], src + g);
+          sB = __shfl_sync(0xffffffffu, sdec[ent], src + 8 + g);
+        } else {
+          sA = __shfl_sync(0xffffffffu, ca[ent], src + g);
+          sB = __shfl_sync(0xffffffffu, ca[ent], src + 8 + g);
+          bA = __shfl_sync(0xffffffffu, cb[ent], src + g);
+          bB = __shfl_sync(0xffffffffu, cb[ent], src + 8 + g);
+        }
         const bool keep = !G32 || (t >> 1) == q;
         float D[NT][4];
 #pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) D[n][c] = 0.0f;
-#pragma unroll
-        for (int j = 0; j < S::kMmas; ++j) {
-          const uint32_t a0 = keep ? pA[2 * j] : 0u, a1 = keep ? pB[2 * j] : 0u;
-          const uint32_t a2 = keep ? pA[2 * j + 1] : 0u, a3 = keep ? pB[2 * j + 1] : 0u;
-#pragma unroll
-          for (int n = 0; n < NT; ++n) mma_bf16_16816(D[n], a0, a1, a2, a3, bx[n][j][0], bx[n][j][1]);
-        }
-#pragma unroll
         for (int n = 0; n < NT; ++n) {
-          if (FMT == kFmtNF4) {
-            acc[mt][n][0] = fmaf(sA[q], D[n][0], acc[mt][n][0]);
-            acc[mt][n][1] = fmaf(sA[q], D[n][1], acc[mt][n][1]);
-            acc[mt][n][2] = fmaf(sB[q], D[n][2], acc[mt][n][2]);
-            acc[mt][n][3] = fmaf(sB[q], D[n][3], acc[mt][n][3]);
-          } else {
-            acc[mt][n][0] = fmaf(sA[q], D[n][0], fmaf(bA[q], xs[q][n][0], acc[mt][n][0]));
-            acc[mt][n][1] = fmaf(sA[q], D[n][1], fmaf(bA[q], xs[q][n][1], acc[mt][n][1]));
-            acc[mt][n][2] = fmaf(sB[q], D[n][2], fmaf(bB[q], xs[q][n][2], acc[mt][n][2]));
-            acc[mt][n][3] = fmaf(sB[q], D[n][3], fmaf(bB[q], xs[q][n][3], acc[mt][n][3]));
+#pragma unroll
+          for (int j = 0; j < KM; ++j) {
+            const uint32_t a0 = keep ? pA[2 * j] : 0u, a1 = keep ? pB[2 * j] : 0u;
+            const uint32_t a2 = keep ? pA[2 * j + 1] : 0u, a3 = keep ? pB[2 * j + 1] : 0u;
+            if (j == 0)
+              mma_bf16_16816_zc(D[n], a0, a1, a2, a3, bx[n][j][0], bx[n][j][1]);
+            else
+              mma_bf16_16816_acc(D[n], a0, a1, a2, a3, bx[n][j][0], bx[n][j][1]);
+          }
+        }
+        if (FMT == kFmtNF4) {
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            acc[n][0] = fmaf(sA, D[n][0], acc[n][0]);
+            acc[n][1] = fmaf(sA, D[n][1], acc[n][1]);
+            acc[n][2] = fmaf(sB, D[n][2], acc[n][2]);
+            acc[n][3] = fmaf(sB, D[n][3], acc[n][3]);
+          }
+        } else {
+          // sum of the activations over the group (ones operand: (1, 1)
+          // pairs for 4-bit, (1, 0) for 8-bit, the x half only)
+          const uint32_t one = keep ? (FMT == kFmtA8 ? 0x00003F80u : 0x3F803F80u) : 0u;
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            float xs[4];
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+              if (j == 0)
+                mma_bf16_16816_zc(xs, one, one, one, one, bx[n][j][0], bx[n][j][1]);
+              else
+                mma_bf16_16816_acc(xs, one, one, one, one, bx[n][j][0], bx[n][j][1]);
+            }
+            acc[n][0] = fmaf(sA, D[n][0], fmaf(bA, xs[0], acc[n][0]));
+            acc[n][1] = fmaf(sA, D[n][1], fmaf(bA, xs[1], acc[n][1]));
+            acc[n][2] = fmaf(sB, D[n][2], fmaf(bB, xs[2], acc[n][2]));
+            acc[n][3] = fmaf(sB, D[n][3], fmaf(bB, xs[3], acc[n][3]));
           }
         }
       }
     }
     __syncwarp();  // every lane is done with this slot before it is refilled
-    if (more) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll
-        for (int q = 0; q < NP; ++q) {
-          pa[h][q] = na[h][q];
-          pb[h][q] = nb[h][q];
-        }
-#pragma unroll
-      for (int n = 0; n < NT; ++n)
-#pragma unroll
-        for (int m = 0; m < 4; ++m) xw[n][m] = xn[n][m];
+    for (int e = 0; e < NE; ++e) {
+      ca[e] = na[e];
+      cb[e] = nb[e];
     }
   }
   cp_async_wait<0>();
 
-  // ---- combine the four K warps of each row half (fixed order wk = 0..3)
-  __syncthreads();  // every warp is done with the table: reuse its memory
-  float* red = reinterpret_cast<float*>(sr_smem);  // [wr][wk 1..3][mt][n][c][lane]
-  constexpr int kSlab = 4 * NT * 4 * 32;
-  if (wk > 0) {
-    float* dst = red + ((size_t)(wr * 3 + wk - 1)) * kSlab;
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-      for (int n = 0; n < NT; ++n)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) dst[((mt * NT + n) * 4 + c) * 32 + lane] = acc[mt][n][c];
-  }
-  __syncthreads();
+  // ---- outputs of this warp: rows row0 + g (+ 8 for c2, c3), tokens 8 n + 2 t (+ 1)
   const bool single = p.splits == 1;
-  if (wk == 0) {
+  if (single) griddep_wait();  // U comes from the launch before this one
 #pragma unroll
-    for (int k = 0; k < 3; ++k) {
-      const float* src = red + ((size_t)(wr * 3 + k)) * kSlab;
+  for (int n = 0; n < NT; ++n)
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[mt][n][c] += src[((mt * NT + n) * 4 + c) * 32 + lane];
+    for (int c = 0; c < 4; ++c) {
+      const int64_t row = row0 + g + 8 * (c >> 1);
+      const int tok = 8 * n + 2 * t + (c & 1);
+      if (tok >= p.R) continue;
+      if (single) {
+        float ad = 0.0f;
+        for (int j = 0; j < p.r; ++j)
+          ad = fmaf(__ldg(p.aux + (int64_t)tok * p.r + j), __ldg(p.lora + row * p.r + j), ad);
+        p.out[(int64_t)tok * O + row] = __float2bfloat16_rn(fmaf(p.s, ad, acc[n][c]));
+      } else {
+        p.part[((int64_t)blockIdx.y * p.R + tok) * O + row] = acc[n][c];
+      }
     }
-    if (single) griddep_wait();  // U comes from the launch before this one
-    // lane outputs: row rbase + 16 mt + g (+ 8 for c2, c3), token 8 n + 2 t (+1)
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-      for (int n = 0; n < NT; ++n)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int64_t row = rbase + 16 * mt + g + 8 * (c >> 1);
-          const int tok = 8 * n + 2 * t + (c & 1);
-          if (tok >= p.R) continue;
-          if (single) {
-            float ad = 0.0f;
-            for (int j = 0; j < p.r; ++j)
-              ad = fmaf(__ldg(p.aux + (int64_t)tok * p.r + j), __ldg(p.lora + row * p.r + j), ad);
-            p.out[(int64_t)tok * O + row] = __float2bfloat16_rn(fmaf(p.s, ad, acc[mt][n][c]));
-          } else {
-            p.part[((int64_t)blockIdx.y * p.R + tok) * O + row] = acc[mt][n][c];
-          }
-        }
-  }
-  if (single) {
-    if (threadIdx.x == 0) griddep_wait();
-    return;
-  }
+  if (single) return;
   // ---- split-K: the last CTA of this 128-row tile sums the partials in order
   __shared__ unsigned s_last;
   __threadfence();
@@ -927,12 +924,12 @@ struct SrPlan {
   int per_split;  // K blocks or K steps per split
 };
 
-// One wave: tiles x splits <= CTAs per SM x SMs (two CTAs per SM for NF4,
-// one for the affine variants, which take more registers); never a second,
-// partial wave.
+// One wave: tiles x splits <= CTAs per SM x SMs (two CTAs per SM; one for
+// the affine input-gradient variants, which take more registers); never a
+// second, partial wave.
 SrPlan sr_plan(bool dx, const WView& w) {
   SrPlan pl;
-  const int per_sm = sr_fmt(w) == kFmtNF4 ? 2 : 1;
+  const int per_sm = (!dx || sr_fmt(w) == kFmtNF4) ? 2 : 1;
   const int target = per_sm * num_sms();
   if (!dx) {
     pl.tiles = (int)(w.O / 128);
@@ -956,10 +953,11 @@ SrPlan sr_plan(bool dx, const WView& w) {
 }
 
 // Dynamic shared memory: the byte table plus the eight warps' rings of code
-// blocks (forward: 3 blocks of 64 rows, 2 for 8-bit codes; input gradient: 3
-// iterations of 64 rows (4-bit) or 32 rows (8-bit)).
+// (forward: 3 stages of 16 rows x 128 bytes; input gradient: 3 iterations
+// of 64 rows (4-bit) or 32 rows (8-bit)).
 constexpr int sr_smem_bytes(bool dx, int fmt) {
-  return kTableBytes + 8 * (dx ? 3 * 2048 : (fmt == kFmtA8 ? 2 * 4096 : 3 * 2048));
+  (void)fmt;
+  return kTableBytes + 8 * 3 * 2048;
 }
 
 template <int NT, int FMT, bool G32>
@@ -1037,15 +1035,18 @@ SrParams sr_params(const WView& w, const void* act, int64_t R, const float* aux,
 }  // namespace
 
 // Measured on one B200 (W 12288 x 4096 and 4096 x 4096, CUDA graph, cold L2):
-// these kernels beat the tensor-core kernel for NF4 at one token (12288 x
-// 4096: forward 19.3 vs 27.5 us, input gradient 24.7 vs 29.0 us) but not at
-// 16 (32.5 vs 28.4, 38.8 vs 30.3 us), nor for 4-bit affine codes at any
-// token count; 8-bit affine codes have no tensor-core path.  NF4 takes this
-// path while one 8-token MMA tile covers the tokens.
+// at one token these kernels beat the tensor-core kernel for NF4 (12288 x
+// 4096: forward 19.3 vs 27.5 us, input gradient 24.7 vs 29.0 us) and, in the
+// forward, for 8-bit affine codes (30.3 vs 31.5 us); at 16 tokens the
+// tensor-core kernel wins (NF4 forward 32.5 vs 28.4 us, input gradient 38.8
+// vs 30.3; 8-bit affine 46.1 vs 32.2 and 59.7 vs 34.8), and for 4-bit affine
+// codes at every token count; the 8-bit affine input gradient at one token
+// as well (46.8 vs 34.5 us).  This path is taken while one 8-token MMA tile
+// covers the tokens, for NF4 and the 8-bit affine forward.
 bool smallr_preferred(bool dx, const WView& w, int64_t R) {
-  (void)dx;
-  if (w.fmt == QLORA_FMT_AFFINE) return w.bits == 8;
-  return R <= 8;
+  if (R > 8) return false;
+  if (w.fmt == QLORA_FMT_AFFINE) return !dx && w.bits == 8;
+  return true;
 }
 
 bool smallr_supported(const WView& w, int64_t R, const void* act, const void* out) {

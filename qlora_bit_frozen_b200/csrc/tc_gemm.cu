@@ -66,7 +66,6 @@ constexpr int threads_of(int bn) { return 32 * (2 + kDecGroups * dec_warps(bn));
 // epilogue groups: four warps each, one per TMEM lane quarter
 constexpr int epi_groups(int bn) { return kDecGroups * dec_warps(bn) / 4; }
 constexpr int kWTile = kBM * kBK * 2;  // decoded weight tile bytes (16 KB)
-constexpr int kPkTile = kBM * kBK / 2; // packed nibbles per step (4 KB)
 
 struct TcParams {
   int64_t R;         // tokens
@@ -85,6 +84,7 @@ struct TcParams {
   const float* asc;  // affine 4-bit: per-group scale (else null)
   const float* abi;  // affine 4-bit: per-group bias
   int32_t g_shift;   // affine: log2(G / 32), G in {32, 64, 128}
+  int32_t pbits;     // code bits: 4, or 8 (affine)
   void* out;         // bf16 [R x Mw], or fp32 partials [splits][R][Mw]
   int32_t partial;
   uint32_t* err;
@@ -114,19 +114,26 @@ constexpr int pow2_at_least(int x) {
 //              producer thread issues a few large copies, not many small ones)
 //   adx      : with G > 1, the adapter step's token tile (U / V), outside
 //              the ring
-template <bool DX, int BN>
+template <bool DX, int BN, int PB = 4>
 struct Cfg {
   static constexpr int kAct = BN * kBK * 2;
+  static constexpr int kPk = kBM * kBK * PB / 8;  // packed codes per step: 4 KB (4-bit), 8 KB (8-bit)
   static constexpr int G = tma_group(BN);
-  static constexpr int NIN = DX ? (BN >= 256 ? 4 : BN >= 128 ? 3 : BN >= 64 ? 5 : BN >= 32 ? 6 : 8)
-                                : (BN >= 256 ? 5 : BN >= 128 ? 4 : BN >= 64 ? 6 : BN >= 32 ? 8 : 12);
+  // 8-bit codes double the packed tile: shallower rings keep the same
+  // occupancy (two CTAs per SM below 256-token tiles)
+  static constexpr int NIN = PB == 4
+      ? (DX ? (BN >= 256 ? 4 : BN >= 128 ? 3 : BN >= 64 ? 5 : BN >= 32 ? 6 : 8)
+            : (BN >= 256 ? 5 : BN >= 128 ? 4 : BN >= 64 ? 6 : BN >= 32 ? 8 : 12))
+      : (DX ? (BN >= 256 ? 4 : BN >= 128 ? 2 : BN >= 64 ? 3 : 4)
+            : (BN >= 256 ? 5 : BN >= 128 ? 3 : BN >= 64 ? 5 : BN >= 32 ? 6 : 8));
   static_assert(NIN % G == 0, "a TMA group fills whole ring slots");
-  static constexpr int NDEC = DX ? (BN >= 256 ? 3 : 2) : (BN >= 128 ? 4 : 6);
+  static constexpr int NDEC4 = DX ? (BN >= 256 ? 3 : 2) : (BN >= 128 ? 4 : 6);
+  static constexpr int NDEC = NDEC4 < NIN ? NDEC4 : NIN;
   static_assert(NDEC <= NIN, "decoded slots are released through the in-ring barriers");
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr int kTmemCols = pow2_at_least(DX ? kAccCols : kAccCols + NDEC * 32);
   static constexpr int kWdec = DX ? NDEC * kWTile : 0;
-  static constexpr int kRing = NIN * (kAct + kPkTile) + kWdec;  // also the epilogue staging
+  static constexpr int kRing = NIN * (kAct + kPk) + kWdec;  // also the epilogue staging
   static constexpr int kAdx = G > 1 ? (kAct + 1023) / 1024 * 1024 : 0;
   static constexpr int kBars = 8 * (2 * NIN + NDEC + 2) + 16;
   static constexpr int kSmem = 1024 + kRing + kWTile + kAdx + kBars;
@@ -291,6 +298,59 @@ __device__ __forceinline__ void decode_row_regs(const uint8_t* pk_lo, const uint
   }
 }
 
+// 8-bit affine codes: weight = fp32(fp32(scale * q) + bias) ("LoRA vs QLoRA
+// on Apple Silicon", "Method"; the diagnostic dequantization's arithmetic),
+// the code byte placed in the mantissa of 2^23 and the 2^23 subtracted
+// (exact), two weights packed per bf16 pair.
+__device__ __forceinline__ float aff8_weight(uint32_t w, int k, float sc, float bi) {
+  uint32_t m;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m) : "r"(w), "r"(0x4B000000u), "r"(0x7540u | (uint32_t)k));
+  const float q = __fsub_rn(__uint_as_float(m), 8388608.0f);
+  return __fadd_rn(__fmul_rn(sc, q), bi);
+}
+// 16 code bytes (weights 16 c .. 16 c + 15) -> 8 bf16 pairs
+__device__ __forceinline__ void aff8_chunk(uint4 c, float sc, float bi, uint32_t (&o)[8]) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    o[2 * j] = pack_bf16x2(aff8_weight(w[j], 0, sc, bi), aff8_weight(w[j], 1, sc, bi));
+    o[2 * j + 1] = pack_bf16x2(aff8_weight(w[j], 2, sc, bi), aff8_weight(w[j], 3, sc, bi));
+  }
+}
+// Forward, 8-bit: the row's 64 bytes as TMA wrote them (64-byte swizzle:
+// chunk c at c ^ x), chunks c0 .. c0 + nc - 1 -> v[8 (c - c0) ..], weights
+// 0..31 with (sc0, bi0), 32..63 with (sc1, bi1).
+template <int NC>
+__device__ __forceinline__ void aff8_regs(const uint8_t* row, uint32_t x, int c0, float sc0, float bi0,
+                                          float sc1, float bi1, uint32_t (&v)[8 * NC]) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const int cc = c0 + c;
+    const uint4 p = *reinterpret_cast<const uint4*>(row + ((((uint32_t)cc) ^ x) << 4));
+    uint32_t o[8];
+    aff8_chunk(p, cc < 2 ? sc0 : sc1, cc < 2 ? bi0 : bi1, o);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[8 * c + j] = o[j];
+  }
+}
+// Input gradient, 8-bit: the unit's 64 bytes are chunks 4 h .. 4 h + 3 of a
+// 128-byte row (128-byte swizzle: chunk c at c ^ y7); chunks cl .. cl + nc - 1
+// of the unit decode into output chunks 2 cl .. of the swizzled decoded row.
+template <int NC>
+__device__ __forceinline__ void aff8_smem(const uint8_t* row, uint32_t y7, int h, int cl, float sc0,
+                                          float bi0, float sc1, float bi1, uint32_t row_addr,
+                                          uint32_t sw) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    const int cc = cl + c;  // 0..3 within the unit
+    const uint4 p = *reinterpret_cast<const uint4*>(row + ((((uint32_t)(4 * h + cc)) ^ y7) << 4));
+    uint32_t o[8];
+    aff8_chunk(p, cc < 2 ? sc0 : sc1, cc < 2 ? bi0 : bi1, o);
+    st_shared_v4(row_addr + ((((uint32_t)(2 * cc)) ^ sw) << 4), o[0], o[1], o[2], o[3]);
+    st_shared_v4(row_addr + ((((uint32_t)(2 * cc + 1)) ^ sw) << 4), o[4], o[5], o[6], o[7]);
+  }
+}
+
 // TMA bulk tensor store of a shared-memory box (3D map: weight-side
 // column, token, split); coordinates past the tensor edge are not written.
 __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int32_t x, int32_t y,
@@ -344,15 +404,16 @@ constexpr int cols_per_group() {
 }
 
 // WF: weight format, a template parameter so the decoder loop carries no
-// format branches (0 NF4 double-quant, 1 NF4 legacy fp32 scales, 2 affine 4-bit)
+// format branches (0 NF4 double-quant, 1 NF4 legacy fp32 scales, 2 affine
+// 4-bit, 3 affine 8-bit)
 template <bool DX, int BN, int WF>
-__global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN>::kMinCtas)
+__global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::kMinCtas)
     tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_pk,
                       const __grid_constant__ CUtensorMap tm_aact,
                       const __grid_constant__ CUtensorMap tm_aw,
                       const __grid_constant__ CUtensorMap tm_out, const TcParams p) {
-  using C = Cfg<DX, BN>;
+  using C = Cfg<DX, BN, WF == 3 ? 8 : 4>;
   constexpr int NIN = C::NIN, NDEC = C::NDEC;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, BN, DX);
   constexpr int DW = dec_warps(BN);
@@ -362,8 +423,8 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN>::kMinCtas)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* act = smem;                        // NIN x BN*128
-  uint8_t* pk = act + NIN * C::kAct;          // NIN x 4 KB
-  uint8_t* wdec = pk + NIN * kPkTile;         // input gradient: NDEC x 16 KB
+  uint8_t* pk = act + NIN * C::kAct;          // NIN x 4 KB (4-bit) or 8 KB (8-bit)
+  uint8_t* wdec = pk + NIN * C::kPk;          // input gradient: NDEC x 16 KB
   uint8_t* adw = wdec + C::kWdec;             // 16 KB
   uint8_t* adx = adw + kWTile;                // G > 1: adapter token tile
   uint64_t* bars = (uint64_t*)(adx + C::kAdx);
@@ -428,12 +489,12 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN>::kMinCtas)
         }
         const uint32_t fb = smem_u32(&full_in[s0]);
         const int kb = kb_lo + it0;
-        mbar_arrive_expect_tx(fb, G * (C::kAct + kPkTile));
+        mbar_arrive_expect_tx(fb, G * (C::kAct + C::kPk));
         tma_load_3d(smem_u32(act + s0 * C::kAct), &tm_act, fb, 0, (int32_t)n0, kb);
         if (!DX)
-          tma_load_3d(smem_u32(pk + s0 * kPkTile), &tm_pk, fb, 0, m0, kb);
+          tma_load_3d(smem_u32(pk + s0 * C::kPk), &tm_pk, fb, 0, m0, kb);
         else
-          tma_load_3d(smem_u32(pk + s0 * kPkTile), &tm_pk, fb, m0 / 2, 0, kb);
+          tma_load_3d(smem_u32(pk + s0 * C::kPk), &tm_pk, fb, WF == 3 ? m0 : m0 / 2, 0, kb);
         issued = it0 + G;
         s0 += G;
         if (s0 == NIN) { s0 = 0; ph ^= 1u; }
@@ -549,7 +610,7 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN>::kMinCtas)
     const int quad = warp & 3;
     const int u = DX ? (((int)threadIdx.x - 64 - 32 * DW * group) & 127) : 32 * quad + lane;
     constexpr bool legacy = WF == 1;  // fp32 block scales stored as they are
-    constexpr bool affine = WF == 2;  // 4-bit affine groups: (scale, bias)
+    constexpr bool affine = WF >= 2;  // affine groups: (scale, bias); WF 3: 8-bit codes
     const float mu = (legacy || affine) ? 0.0f : __ldg(p.mu);
     const uint32_t bpr = (uint32_t)(p.I / kBK);  // blocks per W row
     auto block_of = [&](int kb) -> uint32_t {
@@ -640,7 +701,49 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN>::kMinCtas)
         w_ok = (eb == 0 || mbar_wait(eb, ep, p.wait_ns, p.err, 0x301)) &&
                mbar_wait(fb, ph_in, p.wait_ns, p.err, 0x302);
       if (!__all_sync(0xffffffffu, w_ok)) { *abort_flag = 1; ok = false; break; }
-      const uint8_t* src = pk + s * kPkTile;
+      const uint8_t* src = pk + s * C::kPk;
+      if (WF == 3) {
+        // 8-bit codes: per-weight arithmetic; a whole-row thread with groups
+        // of 32 reads the second group's scale and bias here
+        float sc1 = sc, bi1 = bi;
+        if (DW == 4 && p.g_shift == 0) {
+          const uint32_t g2 = 2u * bcur + 1u;
+          sc1 = __ldg(p.asc + g2);
+          bi1 = __ldg(p.abi + g2);
+        }
+        if (!DX) {
+          tc_fence_after();
+          const uint8_t* row = src + (uint32_t)u * 64;
+          const uint32_t x = ((uint32_t)u >> 1) & 3u;
+          if (DW == 4) {
+            uint32_t v[32];
+            aff8_regs<4>(row, x, 0, sc, bi, sc1, bi1, v);
+            tmem_st_32x32b_x32(tm_row + (uint32_t)(d * 32), v);
+          } else {
+            uint32_t v[16];
+            aff8_regs<2>(row, x, 2 * half, sc, bi, sc, bi, v);
+            tmem_st_32x32b_x16(tm_row + (uint32_t)(d * 32 + 16 * half), v);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+        } else {
+          const uint32_t o = (uint32_t)(u & 63), hh = (uint32_t)(u >> 6);
+          const uint8_t* row = src + o * 128;
+          const uint32_t daddr = smem_u32(wdec + d * kWTile) + row_off;
+          if (DW == 4)
+            aff8_smem<4>(row, o & 7u, (int)hh, 0, sc, bi, sc1, bi1, daddr, sw);
+          else
+            aff8_smem<2>(row, o & 7u, (int)hh, 2 * half, sc, bi, sc, bi, daddr, sw);
+          fence_proxy_async_smem();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&dec_full[d]));
+        s += kDecGroups;
+        if (s >= NIN) { s -= NIN; ph_in ^= 1u; }
+        d += kDecGroups;
+        if (d >= NDEC) d -= NDEC;
+        continue;
+      }
       // decode tables: one per block, or (whole-row threads, affine groups
       // of 32) one per half block, the second group's scale and bias read here
       const Nf4Planes tA = affine ? affine_planes(sc, bi) : nf4_planes(sc);
@@ -812,7 +915,7 @@ template <bool DX, int BN, int WF>
 cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                       const CUtensorMap& d, const CUtensorMap& o, const TcParams& p,
                       cudaStream_t st) {
-  using Cf = Cfg<DX, BN>;
+  using Cf = Cfg<DX, BN, WF == 3 ? 8 : 4>;
   auto kern = tc_qlinear_kernel<DX, BN, WF>;
   static bool attr_set = false;  // once per instantiation (keeps graph capture free of it)
   if (!attr_set) {
@@ -857,7 +960,8 @@ template <bool DX>
 cudaError_t launch_plan(const TcPlan& pl, dim3 grid, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& c, const CUtensorMap& d, const CUtensorMap& o,
                         const TcParams& p, cudaStream_t st) {
-  if (p.asc) return launch_plan_wf<DX, 2>(pl, grid, a, b, c, d, o, p, st);
+  if (p.asc) return p.pbits == 8 ? launch_plan_wf<DX, 3>(pl, grid, a, b, c, d, o, p, st)
+                                 : launch_plan_wf<DX, 2>(pl, grid, a, b, c, d, o, p, st);
   if (p.sb) return launch_plan_wf<DX, 1>(pl, grid, a, b, c, d, o, p, st);
   return launch_plan_wf<DX, 0>(pl, grid, a, b, c, d, o, p, st);
 }
@@ -872,7 +976,8 @@ bool common_supported(const WView& w, int64_t R) {
   } else if (w.fmt == QLORA_FMT_NF4_FP32SCALE) {
     if (w.block != kBK) return false;
   } else if (w.fmt == QLORA_FMT_AFFINE) {
-    if (w.bits != 4 || (w.block != 32 && w.block != 64 && w.block != 128)) return false;
+    if ((w.bits != 4 && w.bits != 8) || (w.block != 32 && w.block != 64 && w.block != 128))
+      return false;
   } else {
     return false;
   }
@@ -959,8 +1064,12 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   const uint32_t g = (uint32_t)tma_group(pl.bn);
   if (!make_map3(&m_act, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, (uint64_t)R, (uint64_t)(I / 64),
                  (uint64_t)I * 2, 128, 64, bn, g, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 32, (uint64_t)O, (uint64_t)(I / 64),
-                 (uint64_t)(I / 2), 32, 32, 128, g, CU_TENSOR_MAP_SWIZZLE_32B) ||
+      !(w.bits == 8
+            ? make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, (uint64_t)O,
+                        (uint64_t)(I / 64), (uint64_t)I, 64, 64, 128, g, CU_TENSOR_MAP_SWIZZLE_64B)
+            : make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 32, (uint64_t)O,
+                        (uint64_t)(I / 64), (uint64_t)(I / 2), 32, 32, 128, g,
+                        CU_TENSOR_MAP_SWIZZLE_32B)) ||
       !make_map(&m_aact, upad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&m_aw, bpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, O, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
@@ -981,6 +1090,7 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   p.asc = w.fmt == QLORA_FMT_AFFINE ? w.scale : nullptr;
   p.abi = w.fmt == QLORA_FMT_AFFINE ? w.bias : nullptr;
   p.g_shift = w.block == 128 ? 2 : w.block == 64 ? 1 : 0;
+  p.pbits = w.bits;
   p.partial = pl.splits > 1;
   p.out = pl.splits > 1 ? (void*)part : Y;
   p.err = hdr;
@@ -1014,9 +1124,13 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   const uint32_t g = (uint32_t)tma_group(pl.bn);
   if (!make_map3(&m_act, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, (uint64_t)R, (uint64_t)(O / 64),
                  (uint64_t)O * 2, 128, 64, bn, g, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(I / 2), 64,
-                 (uint64_t)(O / 64), (uint64_t)(I / 2), (uint64_t)64 * (I / 2), 64, 64, g,
-                 CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !(w.bits == 8
+            ? make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)I, 64,
+                        (uint64_t)(O / 64), (uint64_t)I, (uint64_t)64 * I, 128, 64, g,
+                        CU_TENSOR_MAP_SWIZZLE_128B)
+            : make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(I / 2), 64,
+                        (uint64_t)(O / 64), (uint64_t)(I / 2), (uint64_t)64 * (I / 2), 64, 64, g,
+                        CU_TENSOR_MAP_SWIZZLE_64B)) ||
       !make_map(&m_aact, vpad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 64, R, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&m_aw, apad, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, 64, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
@@ -1037,6 +1151,7 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   p.asc = w.fmt == QLORA_FMT_AFFINE ? w.scale : nullptr;
   p.abi = w.fmt == QLORA_FMT_AFFINE ? w.bias : nullptr;
   p.g_shift = w.block == 128 ? 2 : w.block == 64 ? 1 : 0;
+  p.pbits = w.bits;
   p.partial = pl.splits > 1;
   p.out = pl.splits > 1 ? (void*)part : dX;
   p.err = hdr;

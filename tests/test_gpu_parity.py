@@ -233,14 +233,16 @@ def test_bf16_identity_input_recovers_decoded_weight_bitwise():
 
 
 @pytest.mark.parametrize("G", [32, 64, 128])
-def test_bf16_identity_input_recovers_affine_weight_bitwise(G):
-    """4-bit affine weights in the tensor-core kernel: X = I (R = I) and B = 0
-    give Y = bf16(W_hat)^T exactly, dY = I gives dX = bf16(W_hat); every
-    decoded weight (scale * code + bias of its group) checked bit for bit."""
+@pytest.mark.parametrize("bits", [4, 8])
+def test_bf16_identity_input_recovers_affine_weight_bitwise(bits, G):
+    """4- and 8-bit affine weights in the tensor-core kernel: X = I (R = I)
+    and B = 0 give Y = bf16(W_hat)^T exactly, dY = I gives dX = bf16(W_hat);
+    every decoded weight (scale * code + bias of its group) checked bit for
+    bit."""
     O, I = 256, 512
-    W = synth.normal(5 + G, (O, I), std=0.02)
-    gw = q.qlora_quantize_affine(to_dev_f32(W), 4, G)
-    ow = oracle.quantize_affine(W, 4, G)
+    W = synth.normal(5 + G + bits, (O, I), std=0.02)
+    gw = q.qlora_quantize_affine(to_dev_f32(W), bits, G)
+    ow = oracle.quantize_affine(W, bits, G)
     ref = torch.from_numpy(oracle.dequantize(ow)).to(torch.bfloat16)
     r = 8
     A = torch.zeros((r, I), device="cuda")
@@ -254,13 +256,15 @@ def test_bf16_identity_input_recovers_affine_weight_bitwise(G):
 
 
 @pytest.mark.parametrize("G", [32, 64, 128])
-@pytest.mark.parametrize("R", [100, 4096])
-def test_bf16_affine4_tensor_core_path(G, R):
-    """4-bit affine weights at many tokens run on the tensor-core kernel
-    (split-K at 100 tokens, 256-token tiles at 4096); 64 sampled rows."""
+@pytest.mark.parametrize("R", [40, 100, 300, 4096])
+@pytest.mark.parametrize("bits", [4, 8])
+def test_bf16_affine_tensor_core_path(bits, G, R):
+    """4- and 8-bit affine weights at many tokens run on the tensor-core
+    kernel (split-K at 40 and 100 tokens, a ragged 300 over 128- and
+    64-token tiles, 256-token tiles at 4096); 64 sampled rows."""
     wl = synth.workload("qwen3_0.6b_attn_qv", R=R)
-    rows = synth.sample_rows(R, 64, seed=G + R)
-    _check(_run_layer(wl, 0, rows=rows, fmt="affine", bits=4, G=G), TOL["bf16"])
+    rows = synth.sample_rows(R, 64, seed=G + R + bits)
+    _check(_run_layer(wl, 0, rows=rows, fmt="affine", bits=bits, G=G), TOL["bf16"])
 
 
 def test_bf16_adapter_only_and_zero_alpha():
