@@ -1034,18 +1034,18 @@ SrParams sr_params(const WView& w, const void* act, int64_t R, const float* aux,
 
 }  // namespace
 
-// Measured on one B200 (W 12288 x 4096 and 4096 x 4096, CUDA graph, cold L2):
-// at one token these kernels beat the tensor-core kernel for NF4 (12288 x
-// 4096: forward 19.3 vs 27.5 us, input gradient 24.7 vs 29.0 us) and, in the
-// forward, for 8-bit affine codes (30.3 vs 31.5 us); at 16 tokens the
-// tensor-core kernel wins (NF4 forward 32.5 vs 28.4 us, input gradient 38.8
-// vs 30.3; 8-bit affine 46.1 vs 32.2 and 59.7 vs 34.8), and for 4-bit affine
-// codes at every token count; the 8-bit affine input gradient at one token
-// as well (46.8 vs 34.5 us).  This path is taken while one 8-token MMA tile
-// covers the tokens, for NF4 and the 8-bit affine forward.
+// Measured on one B200 (W 12288 x 4096 and 4096 x 4096, whole call in a
+// CUDA graph, cold L2), against the tensor-core kernel: at one token the
+// forward here is faster for NF4 (12288 x 4096: 17.1 vs 28.9 us), 4-bit
+// affine codes (G = 64: 23.3 vs 30.0 us) and 8-bit codes in groups of 64
+// or 128 (31.1 vs 31.4 us), the input gradient only for NF4 (23.9 vs
+// 30.0 us; 4-bit affine G = 64: 36.3 vs 33.9 us); at 16 tokens the
+// tensor-core kernel wins every case (NF4 forward 31.4 vs 29.6 us, input
+// gradient 38.9 vs 31.4 us).  So this path is taken while one 8-token MMA
+// tile covers the tokens, in those cases.
 bool smallr_preferred(bool dx, const WView& w, int64_t R) {
   if (R > 8) return false;
-  if (w.fmt == QLORA_FMT_AFFINE) return !dx && w.bits == 8;
+  if (w.fmt == QLORA_FMT_AFFINE) return !dx && (w.bits == 4 || w.block >= 64);
   return true;
 }
 
