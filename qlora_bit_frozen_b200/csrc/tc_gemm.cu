@@ -31,10 +31,10 @@
 // launch: the K loop before it overlaps that launch).
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer,
-// then the decoders in two groups (alternate K steps) of four warps (a
-// whole 64-weight row per thread; 320 threads) or, at 256-token tiles, of
-// eight warps (half a row per thread; 576 threads); the decoder warps then
-// run the epilogue (TMEM -> registers -> shared memory -> TMA store).
+// then the decoders in groups of four warps (a whole 64-weight row per
+// thread) that take K steps in turn: two groups (320 threads) up to
+// 128-token tiles, four (576 threads) at 256-token tiles; the decoder warps
+// then run the epilogue (TMEM -> registers -> shared memory -> TMA store).
 // Every mbarrier wait is bounded (%globaltimer); on expiry the CTA records
 // QLORA_ERR_TIMEOUT in the workspace header, stops issuing work, waits
 // (bounded) for its copies in flight, frees TMEM and exits.
@@ -51,20 +51,28 @@ namespace {
 
 constexpr int kBM = 128;             // weight-side rows per CTA (MMA M)
 constexpr int kBK = 64;              // reduction step (one NF4 block)
-constexpr int kDecGroups = 2;        // decoder groups (alternate K steps)
-// Decoder warps per group: at 256-token tiles (one CTA per SM) eight, each
-// thread decoding half a 64-weight row, so that twice as many warps hide
-// the decode's dependency latency; four (a whole row per thread) at smaller
-// tiles, which keep two CTAs per SM.
-// (eight per group at 256-token tiles measured no faster than four on the
-// 8B / 14B / Qwen steps, so four is the default)
+// Decoder groups (group g decodes the K steps g, g + groups, ...): four at
+// 256-token tiles (one CTA per SM), so that each group has four MMA steps'
+// time for its tile decode (the decode is a dependent chain of ~200
+// instructions per thread; with two groups it set the pace of the tensor
+// pipe), except for the 8-bit input gradient, whose rings leave no room for
+// the fourth decoded slot; two at smaller tiles, which keep two CTAs per SM.
+#ifndef QLORA_TC_DEC_GROUPS_256
+#define QLORA_TC_DEC_GROUPS_256 4
+#endif
+constexpr int dec_groups(bool dx, int bn, int pb) {
+  return (bn >= 256 && !(dx && pb == 8)) ? QLORA_TC_DEC_GROUPS_256 : 2;
+}
+// Decoder warps per group: four, a whole 64-weight row per thread (a
+// compile-time option gives eight at 256-token tiles, each thread decoding
+// half a row; it measured no faster on the 8B / 14B / Qwen steps).
 #ifndef QLORA_TC_DEC_WARPS_256
 #define QLORA_TC_DEC_WARPS_256 4
 #endif
 constexpr int dec_warps(int bn) { return bn >= 256 ? QLORA_TC_DEC_WARPS_256 : 4; }
-constexpr int threads_of(int bn) { return 32 * (2 + kDecGroups * dec_warps(bn)); }
-// epilogue groups: four warps each, one per TMEM lane quarter
-constexpr int epi_groups(int bn) { return kDecGroups * dec_warps(bn) / 4; }
+// epilogue groups: four warps each, one per TMEM lane quarter (the warps of
+// the first two decoder groups)
+constexpr int epi_groups(int bn) { return 2 * dec_warps(bn) / 4; }
 constexpr int kWTile = kBM * kBK * 2;  // decoded weight tile bytes (16 KB)
 
 struct TcParams {
@@ -127,9 +135,12 @@ struct Cfg {
       : (DX ? (BN >= 256 ? 4 : BN >= 128 ? 2 : BN >= 64 ? 3 : 4)
             : (BN >= 256 ? 5 : BN >= 128 ? 3 : BN >= 64 ? 5 : BN >= 32 ? 6 : 8));
   static_assert(NIN % G == 0, "a TMA group fills whole ring slots");
-  static constexpr int NDEC4 = DX ? (BN >= 256 ? 3 : 2) : (BN >= 128 ? 4 : 6);
+  static constexpr int DG = dec_groups(DX, BN, PB);
+  static constexpr int kThreads = 32 * (2 + DG * dec_warps(BN));
+  static constexpr int NDEC4 = DX ? (BN >= 256 ? (DG > 3 ? DG : 3) : 2) : (BN >= 128 ? 4 : 6);
   static constexpr int NDEC = NDEC4 < NIN ? NDEC4 : NIN;
   static_assert(NDEC <= NIN, "decoded slots are released through the in-ring barriers");
+  static_assert(DG <= NDEC && DG <= NIN, "one group's next step is at most one ring cycle on");
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
   static constexpr int kTmemCols = pow2_at_least(DX ? kAccCols : kAccCols + NDEC * 32);
   static constexpr int kWdec = DX ? NDEC * kWTile : 0;
@@ -407,7 +418,8 @@ constexpr int cols_per_group() {
 // format branches (0 NF4 double-quant, 1 NF4 legacy fp32 scales, 2 affine
 // 4-bit, 3 affine 8-bit)
 template <bool DX, int BN, int WF>
-__global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::kMinCtas)
+__global__ void __launch_bounds__(Cfg<DX, BN, WF == 3 ? 8 : 4>::kThreads,
+                                  Cfg<DX, BN, WF == 3 ? 8 : 4>::kMinCtas)
     tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_pk,
                       const __grid_constant__ CUtensorMap tm_aact,
@@ -417,6 +429,7 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::
   constexpr int NIN = C::NIN, NDEC = C::NDEC;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, BN, DX);
   constexpr int DW = dec_warps(BN);
+  constexpr int DG = C::DG;
   static_assert((BN >= 64 ? epi_groups(BN) : 1) * 2 * cols_per_group<BN>() * 64 * 4 <= C::kRing,
                 "epilogue staging must fit in the ring buffers");
 
@@ -597,7 +610,7 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::
     __syncwarp();
   } else {
     // ------------------------------------------------------------ decoders
-    // Two groups of 4 warps; group g decodes the steps it = g, g+2, ...
+    // DG groups of DW warps; group g decodes the steps it = g, g + DG, ...
     // Forward: the thread decodes weight row 32*(warp%4) + lane, its own
     // TMEM lane, and stores the block's 32 bf16 pairs with one tcgen05.st.
     // Input gradient: unit u writes one swizzled 128-byte row of the
@@ -663,16 +676,16 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::
     float tw[kPf];
 #pragma unroll
     for (int j = 0; j < kPf; ++j) {
-      const int itj = group + j * kDecGroups;
+      const int itj = group + j * DG;
       qw[j] = 128u;
       tw[j] = 0.0f;
       if (itj < nk) load_scale(block_of(kb_lo + itj), qw[j], tw[j]);
     }
     bool ok = true;
-    // running ring positions of this group's steps (it = group, group + 2, ...)
+    // running ring positions of this group's steps (it = group, group + DG, ...)
     int s = group % NIN, d = group % NDEC;
     uint32_t ph_in = 0;
-    for (int it = group; it < nk; it += kDecGroups) {
+    for (int it = group; it < nk; it += DG) {
       const float sc = affine ? __uint_as_float(qw[0]) : legacy ? tw[0] : decode_block_scale(qw[0], tw[0], mu);
       const float bi = tw[0];  // affine bias
       const uint32_t bcur = block_of(kb_lo + it);
@@ -682,7 +695,7 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::
         tw[j] = tw[j + 1];
       }
       {
-        const int itn = it + kPf * kDecGroups;
+        const int itn = it + kPf * DG;
         if (itn < nk) load_scale(block_of(kb_lo + itn), qw[kPf - 1], tw[kPf - 1]);
       }
       if (((it >> 1) & 3) == 0 && __any_sync(0xffffffffu, *abort_flag != 0)) { ok = false; break; }
@@ -738,9 +751,9 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&dec_full[d]));
-        s += kDecGroups;
+        s += DG;
         if (s >= NIN) { s -= NIN; ph_in ^= 1u; }
-        d += kDecGroups;
+        d += DG;
         if (d >= NDEC) d -= NDEC;
         continue;
       }
@@ -775,9 +788,9 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&dec_full[d]));
-      s += kDecGroups;
+      s += DG;
       if (s >= NIN) { s -= NIN; ph_in ^= 1u; }
-      d += kDecGroups;
+      d += DG;
       if (d >= NDEC) d -= NDEC;
     }
     // the accumulator is complete once acc_full fires
@@ -800,7 +813,7 @@ __global__ void __launch_bounds__(threads_of(BN), Cfg<DX, BN, WF == 3 ? 8 : 4>::
     constexpr int kColsPerGroup = cols_per_group<BN>();
     const int c_begin = BN >= 64 ? group * kColsPerGroup : 0;
     const int c_end = BN >= 64 ? c_begin + kColsPerGroup : (group == 0 ? BN : 0);
-    if (c_end > c_begin) {
+    if (group < epi_groups(BN) && c_end > c_begin) {
       const int es = p.partial ? 4 : 2;
       uint8_t* ep = smem + (size_t)group * 2 * kColsPerGroup * 64 * es;
       if (p.partial)
@@ -928,7 +941,7 @@ cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, con
   const int slot = timing_begin(st, DX ? 1 : 0, flops);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(threads_of(BN));
+  cfg.blockDim = dim3(Cf::kThreads);
   cfg.dynamicSmemBytes = (size_t)Cf::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
