@@ -134,21 +134,30 @@ namespace {
 constexpr int kGemvKC = 256;            // K columns staged per chunk (8 per lane)
 constexpr int kGemvWR = 4;              // weight rows per warp
 constexpr int kGemvRows = 8 * kGemvWR;  // weight rows per block
-constexpr int kDxCols = 256;            // dX columns per block (one per thread)
+// dX: each thread owns kDxCP(RM) adjacent columns (8 up to 4 tokens, 4
+// above, to bound the RM x CP accumulators)
+constexpr int dx_cp(int rm) { return rm <= 4 ? 8 : 4; }
 constexpr int kDxChunk = 256;           // W rows of dY staged per chunk
 
-// Affine weight at flat index n: scale_g * q + bias_g, one rounding each
-// (the same arithmetic as decode_weight).
-__device__ __forceinline__ float affine_at(const WView& w, int64_t n) {
-  uint32_t q;
-  if (w.bits == 8) {
-    q = __ldg(w.codes + n);
-  } else {
-    const uint32_t byte = __ldg(w.codes + (n >> 1));
-    q = (n & 1) ? (byte >> 4) : (byte & 15u);
-  }
+// Affine weights are scale_g * q + bias_g, one rounding each (the same
+// arithmetic as decode_weight).
+// 4 consecutive affine weights from flat index n (n % 4 == 0; the group size
+// is a multiple of 8, so they share one scale and bias): one code load.
+__device__ __forceinline__ void affine_decode4(const WView& w, int64_t n, float (&v)[4]) {
   const int64_t g = n / w.block;
-  return __fadd_rn(__fmul_rn(__ldg(w.scale + g), (float)q), __ldg(w.bias + g));
+  const float sc = __ldg(w.scale + g), bi = __ldg(w.bias + g);
+  uint32_t q[4];
+  if (w.bits == 8) {
+    const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(w.codes + n));
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q[e] = (b >> (8 * e)) & 255u;
+  } else {
+    const uint32_t b = __ldg(reinterpret_cast<const unsigned short*>(w.codes + (n >> 1)));
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q[e] = (b >> (4 * e)) & 15u;  // low nibble first
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] = __fadd_rn(__fmul_rn(sc, (float)q[e]), bi);
 }
 
 // 8 consecutive affine weights from flat index n (n % 8 == 0; the group size
@@ -242,17 +251,23 @@ __global__ void __launch_bounds__(256) gemv_fwd_kernel(WView w, int R, const T* 
 }
 
 // dX partial over W rows [oa, oa + orange): part[split][m][i] =
-// sum_o dY[m, o] W_hat[o, i]; one thread per column i, dY staged per chunk.
+// sum_o dY[m, o] W_hat[o, i].  Each thread owns CP adjacent columns: per W
+// row one vector load of their codes and one scale / bias pair (the CP
+// columns lie in one affine group), CP x RM multiply-adds; a warp reads a
+// contiguous run of the row.  dY is staged per chunk in shared memory.
 template <typename T, int RM>
 __global__ void __launch_bounds__(256) gemv_dx_kernel(WView w, int R, const T* __restrict__ dY,
                                                       int64_t orange, float* __restrict__ part) {
+  constexpr int CP = dx_cp(RM);
   __shared__ float ys[RM][kDxChunk];
   const int64_t I = w.I, O = w.O;
-  const int64_t i = (int64_t)blockIdx.x * kDxCols + threadIdx.x;
+  const int64_t i0 = ((int64_t)blockIdx.x * 256 + threadIdx.x) * CP;
   const int64_t oa = (int64_t)blockIdx.y * orange, ob = min(O, oa + orange);
-  float acc[RM];
+  float acc[RM][CP];
 #pragma unroll
-  for (int m = 0; m < RM; ++m) acc[m] = 0.0f;
+  for (int m = 0; m < RM; ++m)
+#pragma unroll
+    for (int e = 0; e < CP; ++e) acc[m][e] = 0.0f;
   for (int64_t c0 = oa; c0 < ob; c0 += kDxChunk) {
     __syncthreads();
     for (int e = threadIdx.x; e < RM * kDxChunk; e += 256) {
@@ -261,18 +276,31 @@ __global__ void __launch_bounds__(256) gemv_dx_kernel(WView w, int R, const T* _
       ys[m][c] = (m < R && o < ob) ? to_f32<T>(dY[(int64_t)m * O + o]) : 0.0f;
     }
     __syncthreads();
-    if (i >= I) continue;
+    if (i0 >= I) continue;
     const int nc = (int)min((int64_t)kDxChunk, ob - c0);
+#pragma unroll 4
     for (int c = 0; c < nc; ++c) {
-      const float wv = affine_at(w, (c0 + c) * I + i);
+      float v[CP];
+      if constexpr (CP == 8)
+        affine_decode8(w, (c0 + c) * I + i0, v);
+      else
+        affine_decode4(w, (c0 + c) * I + i0, v);
 #pragma unroll
-      for (int m = 0; m < RM; ++m) acc[m] = fmaf(wv, ys[m][c], acc[m]);
+      for (int m = 0; m < RM; ++m) {
+        const float y = ys[m][c];
+#pragma unroll
+        for (int e = 0; e < CP; ++e) acc[m][e] = fmaf(v[e], y, acc[m][e]);
+      }
     }
   }
-  if (i >= I) return;
+  if (i0 >= I) return;
 #pragma unroll
   for (int m = 0; m < RM; ++m)
-    if (m < R) part[((int64_t)blockIdx.y * R + m) * I + i] = acc[m];
+    if (m < R) {
+      float* dst = part + ((int64_t)blockIdx.y * R + m) * I + i0;
+#pragma unroll
+      for (int e = 0; e < CP; ++e) dst[e] = acc[m][e];
+    }
 }
 
 // dX[m, i] = sum over splits (in order) + s sum_j V[m, j] A[j, i].
@@ -296,14 +324,19 @@ struct DxPlan {
   int64_t orange;
 };
 
-DxPlan dx_plan(const WView& w) {
+// Columns per block: 256 threads x the columns each owns at this token count.
+int dx_cols(int64_t R) { return 256 * (R <= 4 ? 8 : 4); }
+
+// Row splits: about two CTAs per SM in all, each at least 64 W rows (a
+// multiple of 64; the last chunk of a range may be partial).
+DxPlan dx_plan(const WView& w, int64_t R) {
   DxPlan p;
-  p.col_blocks = (int)cdiv(w.I, kDxCols);
+  p.col_blocks = (int)cdiv(w.I, dx_cols(R));
   int64_t splits = (2 * 148 + p.col_blocks - 1) / p.col_blocks;
-  const int64_t max_splits = cdiv(w.O, kDxChunk);
+  const int64_t max_splits = cdiv(w.O, 64);
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
-  p.orange = (cdiv(w.O, splits) + kDxChunk - 1) / kDxChunk * kDxChunk;
+  p.orange = (cdiv(w.O, splits) + 63) / 64 * 64;
   p.splits = (int)cdiv(w.O, p.orange);
   return p;
 }
@@ -352,7 +385,7 @@ bool gemv_ok(const WView& w, int64_t R) {
 
 size_t gemv_dx_ws(const WView& w, int64_t R) {
   if (!gemv_ok(w, R)) return 0;
-  return align_up((size_t)dx_plan(w).splits * (size_t)R * (size_t)w.I * 4, 256);
+  return align_up((size_t)dx_plan(w, R).splits * (size_t)R * (size_t)w.I * 4, 256);
 }
 
 cudaError_t launch_simt_fwd(const WView& w, const void* X, int64_t R, const float* A,
@@ -385,7 +418,7 @@ cudaError_t launch_simt_dx(const WView& w, const void* dY, int64_t R, const floa
                            cudaStream_t st, float* gemv_ws) {
   if (R == 0) return cudaSuccess;
   if (gemv_ws && gemv_ok(w, R)) {
-    const DxPlan p = dx_plan(w);
+    const DxPlan p = dx_plan(w, R);
     if (bf16)
       gemv_dx_r<__nv_bfloat16>(w, (int)R, dY, p, gemv_ws, st);
     else

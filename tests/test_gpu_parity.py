@@ -255,6 +255,36 @@ def test_bf16_identity_input_recovers_affine_weight_bitwise(bits, G):
     assert np.array_equal(bf16_bits_of(dX), bf16_bits_of(ref))
 
 
+@pytest.mark.parametrize("fmt,bits,G", [("nf4", 4, 64), ("nf4_fp32scale", 4, 64), ("affine", 4, 32),
+                                        ("affine", 8, 128)])
+def test_bf16_identity_input_pre_decoded_bitwise(fmt, bits, G):
+    """From 2048 tokens on 256-token tiles the weight is decoded to bf16 once
+    per call and the GEMM reads that copy: X = I (4096 tokens, W 1024 x 4096)
+    gives Y = bf16(W_hat)^T and dY = I (4096 tokens, W 4096 x 1024) gives
+    dX = bf16(W_hat), bit for bit, for every weight format."""
+    def quant(W):
+        if fmt == "nf4":
+            return q.qlora_quantize_nf4(to_dev_f32(W)), oracle.quantize_nf4(W)
+        if fmt == "nf4_fp32scale":
+            return q.qlora_quantize_nf4_fp32scale(to_dev_f32(W), 64), oracle.quantize_nf4_legacy(W, 64)
+        return q.qlora_quantize_affine(to_dev_f32(W), bits, G), oracle.quantize_affine(W, bits, G)
+    r = 8
+    for O, I, fwd in ((1024, 4096, True), (4096, 1024, False)):
+        W = synth.normal(40 + bits + G + O, (O, I), std=0.02)
+        gw, ow = quant(W)
+        ref = torch.from_numpy(oracle.dequantize(ow)).to(torch.bfloat16)
+        A = torch.zeros((r, I), device="cuda")
+        Bz = torch.zeros((O, r), device="cuda")
+        if fwd:
+            Xi = torch.eye(I, device="cuda", dtype=torch.bfloat16)
+            Y, _ = q.qlora_linear_fwd(gw, Xi, A, Bz, 16.0)
+            assert np.array_equal(bf16_bits_of(Y), bf16_bits_of(ref.t()))
+        else:
+            dYi = torch.eye(O, device="cuda", dtype=torch.bfloat16)
+            dX, _, _ = q.qlora_linear_bwd(gw, None, dYi, A, Bz, 16.0, want_da=False, want_db=False)
+            assert np.array_equal(bf16_bits_of(dX), bf16_bits_of(ref))
+
+
 @pytest.mark.parametrize("G", [32, 64, 128])
 @pytest.mark.parametrize("R", [40, 100, 300, 4096])
 @pytest.mark.parametrize("bits", [4, 8])
@@ -305,6 +335,18 @@ def test_bf16_small_row_sweep_affine(name, R, bits, G):
     wl = synth.workload(name, R=R)
     rows = synth.sample_rows(R, 32, seed=R + bits + G) if (R == 128 and name.endswith("12288")) else None
     _check(_run_layer(wl, 0, rows=rows, want=("Y", "dX"), fmt="affine", bits=bits, G=G), TOL["bf16"])
+
+
+@pytest.mark.parametrize("R", [1, 5, 16])
+@pytest.mark.parametrize("bits,G", [(4, 32), (4, 128), (8, 64)])
+def test_fp32_small_row_affine(R, bits, G):
+    """fp32 compute mode with affine weights at 1..16 tokens on W 4096x4096:
+    the CUDA-core forward GEMV and the input-gradient GEMV (8 adjacent
+    columns per thread up to 4 tokens, 4 above; 16 row splits summed in
+    order)."""
+    wl = synth.workload("bw_sweep_4096", R=R)
+    wl.compute = "fp32"
+    _check(_run_layer(wl, 0, want=("Y", "dX"), fmt="affine", bits=bits, G=G), TOL["fp32"])
 
 
 @pytest.mark.parametrize("R", [1, 16, 64, 4096])
