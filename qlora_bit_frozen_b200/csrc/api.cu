@@ -432,7 +432,9 @@ qlora_status qlora_linear_fwd(const qlora_weight* w, const void* X, int64_t R, c
       e = launch_smallr_fwd(v, X, R, U, B, r, sc, Y, (char*)ws + L.sr, (uint32_t*)ws, tickets, s);
   } else if (fwd_tc) {
     void* tcws = (char*)ws + L.tc;
-    e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws), B, w->O, 0, sc,
+    e = tc_prepare(false, v, R, tcws, s);
+    if (e == cudaSuccess)
+      e = launch_rowdot(X, true, R, w->I, A, false, r, U, s, tc_act_pad(tcws), B, w->O, 0, sc,
                       tc_w_pad(tcws, R), nullptr, red, tickets, (uint16_t*)((char*)ws + L.split));
     if (e == cudaSuccess) e = launch_tc_fwd(v, X, R, U, B, r, sc, Y, tcws, (uint32_t*)ws, s);
   } else {
@@ -472,7 +474,8 @@ qlora_status qlora_linear_bwd(const qlora_weight* w, const void* X, const void* 
   const bool sr = dX && bf16 && smallr_supported(v, R, dY, dX) && (!dx_tc || smallr_preferred(true, v, R));
   const bool tc = !sr && dx_tc;
   void* tcws = (char*)ws + L.tc;
-  if (dX || dA) {
+  if (tc) e = tc_prepare(true, v, R, tcws, s);
+  if (e == cudaSuccess && (dX || dA)) {
     float* bt = (float*)((char*)ws + L.bt);
     float* part = (float*)red;
     uint16_t* split = (uint16_t*)((char*)ws + L.split);

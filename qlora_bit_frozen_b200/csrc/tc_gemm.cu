@@ -61,7 +61,7 @@ constexpr int kBK = 64;              // reduction step (one NF4 block)
 #define QLORA_TC_DEC_GROUPS_256 4
 #endif
 constexpr int dec_groups(bool dx, int bn, int pb) {
-  return (bn >= 256 && !(dx && pb == 8)) ? QLORA_TC_DEC_GROUPS_256 : 2;
+  return (bn >= 256 && !(dx && pb == 8) && pb != 16) ? QLORA_TC_DEC_GROUPS_256 : 2;
 }
 // Decoder warps per group: four, a whole 64-weight row per thread (a
 // compile-time option gives eight at 256-token tiles, each thread decoding
@@ -93,6 +93,7 @@ struct TcParams {
   const float* abi;  // affine 4-bit: per-group bias
   int32_t g_shift;   // affine: log2(G / 32), G in {32, 64, 128}
   int32_t pbits;     // code bits: 4, or 8 (affine)
+  int32_t pre;       // the weight was decoded to bf16 before the launch (256-token tiles)
   void* out;         // bf16 [R x Mw], or fp32 partials [splits][R][Mw]
   int32_t partial;
   uint32_t* err;
@@ -122,6 +123,9 @@ constexpr int pow2_at_least(int x) {
 //              producer thread issues a few large copies, not many small ones)
 //   adx      : with G > 1, the adapter step's token tile (U / V), outside
 //              the ring
+// bits per weight of a format's packed tile (WF 4: bf16, already decoded)
+constexpr int wf_bits(int wf) { return wf == 4 ? 16 : wf == 3 ? 8 : 4; }
+
 template <bool DX, int BN, int PB = 4>
 struct Cfg {
   static constexpr int kAct = BN * kBK * 2;
@@ -129,7 +133,11 @@ struct Cfg {
   static constexpr int G = tma_group(BN);
   // 8-bit codes double the packed tile: shallower rings keep the same
   // occupancy (two CTAs per SM below 256-token tiles)
-  static constexpr int NIN = PB == 4
+  // PB 16: the weight tile is bf16 already (decoded once per call into the
+  // workspace), 16 KB per step, no decoded-tile slots; 256-token tiles only
+  static constexpr bool kPre = PB == 16;
+  static constexpr int NIN = kPre ? 4
+      : PB == 4
       ? (DX ? (BN >= 256 ? 4 : BN >= 128 ? 3 : BN >= 64 ? 5 : BN >= 32 ? 6 : 8)
             : (BN >= 256 ? 5 : BN >= 128 ? 4 : BN >= 64 ? 6 : BN >= 32 ? 8 : 12))
       : (DX ? (BN >= 256 ? 4 : BN >= 128 ? 2 : BN >= 64 ? 3 : 4)
@@ -142,8 +150,8 @@ struct Cfg {
   static_assert(NDEC <= NIN, "decoded slots are released through the in-ring barriers");
   static_assert(DG <= NDEC && DG <= NIN, "one group's next step is at most one ring cycle on");
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
-  static constexpr int kTmemCols = pow2_at_least(DX ? kAccCols : kAccCols + NDEC * 32);
-  static constexpr int kWdec = DX ? NDEC * kWTile : 0;
+  static constexpr int kTmemCols = pow2_at_least((DX || kPre) ? kAccCols : kAccCols + NDEC * 32);
+  static constexpr int kWdec = (DX && !kPre) ? NDEC * kWTile : 0;
   static constexpr int kRing = NIN * (kAct + kPk) + kWdec;  // also the epilogue staging
   static constexpr int kAdx = G > 1 ? (kAct + 1023) / 1024 * 1024 : 0;
   static constexpr int kBars = 8 * (2 * NIN + NDEC + 2) + 16;
@@ -362,6 +370,44 @@ __device__ __forceinline__ void aff8_smem(const uint8_t* row, uint32_t y7, int h
   }
 }
 
+// The whole weight decoded to bf16 once per call, for the 256-token path:
+// thread b decodes 64-weight block b with the same tables and arithmetic as
+// the in-GEMM decoders (bit-identical values), 32 or 64 code bytes in, 128
+// bytes out.
+template <int WF>
+__global__ void __launch_bounds__(256) expand_bf16_kernel(const TcParams p, const uint8_t* codes,
+                                                          int64_t nblocks, uint4* out) {
+  const int64_t b = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (b >= nblocks) return;
+  uint32_t v[32];
+  if (WF == 3) {
+    const uint32_t g0 = (uint32_t)((2 * b) >> p.g_shift), g1 = (uint32_t)((2 * b + 1) >> p.g_shift);
+    aff8_regs<4>(codes + 64 * b, 0u, 0, __ldg(p.asc + g0), __ldg(p.abi + g0), __ldg(p.asc + g1),
+                 __ldg(p.abi + g1), v);
+  } else {
+    Nf4Planes tA, tB;
+    if (WF == 2) {
+      const uint32_t g0 = (uint32_t)((2 * b) >> p.g_shift), g1 = (uint32_t)((2 * b + 1) >> p.g_shift);
+      tA = affine_planes(__ldg(p.asc + g0), __ldg(p.abi + g0));
+      tB = g1 == g0 ? tA : affine_planes(__ldg(p.asc + g1), __ldg(p.abi + g1));
+    } else {
+      float sc;
+      if (WF == 1) {
+        sc = __ldg(p.sb + b);
+      } else {
+        const uint32_t g = p.c_shift >= 0 ? (uint32_t)(b >> p.c_shift) : (uint32_t)(b / p.C);
+        sc = decode_block_scale(__ldg(p.qcodes + b), __ldg(p.t + g), __ldg(p.mu));
+      }
+      tA = nf4_planes(sc);
+      tB = tA;
+    }
+    decode_row_regs(codes + 32 * b, codes + 32 * b + 16, tA, tB, v);
+  }
+  uint4* dst = out + 8 * b;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) dst[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+}
+
 // TMA bulk tensor store of a shared-memory box (3D map: weight-side
 // column, token, split); coordinates past the tensor edge are not written.
 __device__ __forceinline__ void tma_store_3d(const void* tmap, uint32_t src, int32_t x, int32_t y,
@@ -416,16 +462,16 @@ constexpr int cols_per_group() {
 
 // WF: weight format, a template parameter so the decoder loop carries no
 // format branches (0 NF4 double-quant, 1 NF4 legacy fp32 scales, 2 affine
-// 4-bit, 3 affine 8-bit)
+// 4-bit, 3 affine 8-bit, 4 weights decoded to bf16 before the launch)
 template <bool DX, int BN, int WF>
-__global__ void __launch_bounds__(Cfg<DX, BN, WF == 3 ? 8 : 4>::kThreads,
-                                  Cfg<DX, BN, WF == 3 ? 8 : 4>::kMinCtas)
+__global__ void __launch_bounds__(Cfg<DX, BN, wf_bits(WF)>::kThreads,
+                                  Cfg<DX, BN, wf_bits(WF)>::kMinCtas)
     tc_qlinear_kernel(const __grid_constant__ CUtensorMap tm_act,
                       const __grid_constant__ CUtensorMap tm_pk,
                       const __grid_constant__ CUtensorMap tm_aact,
                       const __grid_constant__ CUtensorMap tm_aw,
                       const __grid_constant__ CUtensorMap tm_out, const TcParams p) {
-  using C = Cfg<DX, BN, WF == 3 ? 8 : 4>;
+  using C = Cfg<DX, BN, wf_bits(WF)>;
   constexpr int NIN = C::NIN, NDEC = C::NDEC;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, BN, DX);
   constexpr int DW = dec_warps(BN);
@@ -504,10 +550,14 @@ __global__ void __launch_bounds__(Cfg<DX, BN, WF == 3 ? 8 : 4>::kThreads,
         const int kb = kb_lo + it0;
         mbar_arrive_expect_tx(fb, G * (C::kAct + C::kPk));
         tma_load_3d(smem_u32(act + s0 * C::kAct), &tm_act, fb, 0, (int32_t)n0, kb);
-        if (!DX)
+        if (!DX) {
           tma_load_3d(smem_u32(pk + s0 * C::kPk), &tm_pk, fb, 0, m0, kb);
-        else
+        } else if (WF == 4) {  // W^T tile, MN-major: two 64-column boxes
+          tma_load_3d(smem_u32(pk + s0 * C::kPk), &tm_pk, fb, m0, 0, kb);
+          tma_load_3d(smem_u32(pk + s0 * C::kPk + kWTile / 2), &tm_pk, fb, m0 + 64, 0, kb);
+        } else {
           tma_load_3d(smem_u32(pk + s0 * C::kPk), &tm_pk, fb, WF == 3 ? m0 : m0 / 2, 0, kb);
+        }
         issued = it0 + G;
         s0 += G;
         if (s0 == NIN) { s0 = 0; ph ^= 1u; }
@@ -561,6 +611,7 @@ __global__ void __launch_bounds__(Cfg<DX, BN, WF == 3 ? 8 : 4>::kThreads,
       const uint32_t act0 = smem_u32(act);
       const uint64_t bdesc0 = sdesc(act0, 16, 1024);
       const uint64_t adesc0 = sdesc(smem_u32(wdec), 8192, 1024);
+      const uint32_t pk_s0 = smem_u32(pk);
       int s = 0, d = 0;
       uint32_t ph_in = 0, ph_dec = 0;
       bool ok = true;
@@ -569,8 +620,10 @@ __global__ void __launch_bounds__(Cfg<DX, BN, WF == 3 ? 8 : 4>::kThreads,
         // The decoders waited for this step's TMA group (token and packed
         // tiles land on the same barrier) before they arrived on dec_full,
         // so dec_full alone orders the MMA after both copies.
-        const uint32_t db = smem_u32(&dec_full[d]);
-        if (!mbar_wait(db, ph_dec, p.wait_ns, p.err, 0x202)) {
+        // pre-decoded weights: the step's TMA group (both operands) is
+        // all the MMA waits for; otherwise the decoded tile
+        const uint32_t db = WF == 4 ? smem_u32(&full_in[s - s % G]) : smem_u32(&dec_full[d]);
+        if (!mbar_wait(db, WF == 4 ? ph_in : ph_dec, p.wait_ns, p.err, 0x202)) {
           *abort_flag = 1;
           ok = false;
           break;
@@ -580,12 +633,20 @@ __global__ void __launch_bounds__(Cfg<DX, BN, WF == 3 ? 8 : 4>::kThreads,
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          if (!DX)
+          if (WF == 4) {
+            const uint32_t a_s = pk_s0 + (uint32_t)(s * C::kPk);
+            if (!DX)  // W tile K-major (128-byte rows, 128-byte swizzle)
+              umma_bf16(tmem, sdesc(a_s, 16, 1024) + 2 * kk, bd + 2 * kk, kIdesc, acc);
+            else      // W^T tile MN-major, as the decoded tile below
+              umma_bf16(tmem, sdesc(a_s, 8192, 1024) + (uint64_t)((uint32_t)(kk * 2048) >> 4),
+                        bd + 2 * kk, kIdesc, acc);
+          } else if (!DX) {
             umma_bf16_ta(tmem, tmem + (uint32_t)(C::kAccCols + d * 32 + kk * 8), bd + 2 * kk,
                          kIdesc, acc);
-          else
+          } else {
             umma_bf16(tmem, adesc0 + (uint64_t)((uint32_t)(d * kWTile + kk * 2048) >> 4),
                       bd + 2 * kk, kIdesc, acc);
+          }
         }
         umma_commit(smem_u32(&in_empty[s]));  // frees the in-ring stage and, NDEC steps on, the decoded slot
         if (++s == NIN) { s = 0; ph_in ^= 1u; }
@@ -608,6 +669,10 @@ __global__ void __launch_bounds__(Cfg<DX, BN, WF == 3 ? 8 : 4>::kThreads,
       umma_commit(smem_u32(acc_full));
     }
     __syncwarp();
+  } else if (WF == 4) {
+    // weights decoded before the launch: the decoder warps only run the
+    // epilogue, once the accumulator is complete
+    if (!mbar_wait(smem_u32(acc_full), 0, p.wait_ns, p.err, 0x401)) *abort_flag = 1;
   } else {
     // ------------------------------------------------------------ decoders
     // DG groups of DW warps; group g decodes the steps it = g, g + DG, ...
@@ -928,7 +993,7 @@ template <bool DX, int BN, int WF>
 cudaError_t launch_bn(dim3 grid, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                       const CUtensorMap& d, const CUtensorMap& o, const TcParams& p,
                       cudaStream_t st) {
-  using Cf = Cfg<DX, BN, WF == 3 ? 8 : 4>;
+  using Cf = Cfg<DX, BN, wf_bits(WF)>;
   auto kern = tc_qlinear_kernel<DX, BN, WF>;
   static bool attr_set = false;  // once per instantiation (keeps graph capture free of it)
   if (!attr_set) {
@@ -973,6 +1038,7 @@ template <bool DX>
 cudaError_t launch_plan(const TcPlan& pl, dim3 grid, const CUtensorMap& a, const CUtensorMap& b,
                         const CUtensorMap& c, const CUtensorMap& d, const CUtensorMap& o,
                         const TcParams& p, cudaStream_t st) {
+  if (p.pre) return launch_bn<DX, 256, 4>(grid, a, b, c, d, o, p, st);
   if (p.asc) return p.pbits == 8 ? launch_plan_wf<DX, 3>(pl, grid, a, b, c, d, o, p, st)
                                  : launch_plan_wf<DX, 2>(pl, grid, a, b, c, d, o, p, st);
   if (p.sb) return launch_plan_wf<DX, 1>(pl, grid, a, b, c, d, o, p, st);
@@ -1044,18 +1110,87 @@ bool tc_dx_supported(const WView& w, const void* dY, const void* dX, int64_t R) 
   return common_supported(w, R) && ptr_aligned(dY, 16) && ptr_aligned(dX, 16);
 }
 
+// From this many tokens on (with 256-token tiles and no K split) the input
+// gradient decodes the weight to bf16 once per call and the GEMM reads it
+// with TMA: the decode and its shared-memory tile leave the MMA's critical
+// path, for 2.5 extra HBM bytes per weight per call, which the GEMM's 2 R
+// flops per weight repay well before this token count.  Measured on the
+// 14B layer: input-gradient kernel 1154-1165 vs 966-969 TFLOP/s, step
+// 923-925 vs 901-905 TFLOP/s under the power cap.  The forward, whose
+// in-GEMM decode writes TMEM rather than shared memory, gained ~3% per
+// kernel but lost it to the lower clock under the power cap (step 908-910),
+// so it keeps the in-GEMM decode (QLORA_TC_PRE_FWD=1 switches it over).
+constexpr int64_t kPreMinTokens = 2048;
+
+#ifndef QLORA_TC_PRE_FWD
+#define QLORA_TC_PRE_FWD 0
+#endif
+bool tc_pre(bool dx, const TcPlan& pl, int64_t R) {
+  return (dx || QLORA_TC_PRE_FWD) && pl.bn == 256 && pl.splits == 1 && R >= kPreMinTokens;
+}
+
+size_t wbuf_bytes(const WView& w) { return align_up((size_t)w.O * (size_t)w.I * 2, 256); }
+
 // Workspace: U_pad / V_pad bf16 [R x 64], the adapter weight operand bf16
-// (fwd: [O x 64]; dX: [64 x I]), split-K partials.
+// (fwd: [O x 64]; dX: [64 x I]), split-K partials, and (from kPreMinTokens
+// tokens) the bf16 copy of the decoded weight [O x I].
 size_t tc_fwd_ws(const WView& w, int64_t R) {
   const TcPlan pl = tc_plan(w.O, w.I / kBK, R);
   return align_up((size_t)R * 128, 256) + align_up((size_t)w.O * 128, 256) +
-         partial_bytes(pl, R, w.O);
+         partial_bytes(pl, R, w.O) + (tc_pre(false, pl, R) ? wbuf_bytes(w) : 0);
 }
 
 size_t tc_dx_ws(const WView& w, int64_t R) {
   const TcPlan pl = tc_plan(w.I, w.O / kBK, R);
   return align_up((size_t)R * 128, 256) + align_up((size_t)w.I * 128, 256) +
-         partial_bytes(pl, R, w.I);
+         partial_bytes(pl, R, w.I) + (tc_pre(true, pl, R) ? wbuf_bytes(w) : 0);
+}
+
+namespace {
+
+// Decode inputs of the weight (the same for both directions).
+void fill_weight_params(const WView& w, TcParams& p) {
+  p.C = (uint32_t)(w.group < 1 ? 1 : w.group);
+  p.c_shift = ((p.C & (p.C - 1)) == 0) ? __builtin_ctz(p.C) : -1;
+  p.qcodes = w.qcodes;
+  p.t = w.t;
+  p.mu = w.mu;
+  p.sb = w.fmt == QLORA_FMT_NF4_FP32SCALE ? w.scale : nullptr;
+  p.asc = w.fmt == QLORA_FMT_AFFINE ? w.scale : nullptr;
+  p.abi = w.fmt == QLORA_FMT_AFFINE ? w.bias : nullptr;
+  p.g_shift = w.block == 128 ? 2 : w.block == 64 ? 1 : 0;
+  p.pbits = w.bits;
+}
+
+// The bf16 weight copy of the tensor-core workspace.
+uint16_t* wbuf_of(void* tcws, int64_t R, int64_t Mw, const TcPlan& pl) {
+  return (uint16_t*)((char*)tcws + align_up((size_t)R * 128, 256) + align_up((size_t)Mw * 128, 256) +
+                     partial_bytes(pl, R, Mw));
+}
+
+}  // namespace
+
+cudaError_t tc_prepare(bool dx, const WView& w, int64_t R, void* tcws, cudaStream_t st) {
+  const int64_t Mw = dx ? w.I : w.O;
+  const TcPlan pl = dx ? tc_plan(w.I, w.O / kBK, R) : tc_plan(w.O, w.I / kBK, R);
+  if (!tc_pre(dx, pl, R)) return cudaSuccess;
+  TcParams p = {};
+  fill_weight_params(w, p);
+  const int64_t nb = w.O * w.I / kBK;
+  uint4* out = (uint4*)wbuf_of(tcws, R, Mw, pl);
+  const unsigned grid = (unsigned)((nb + 255) / 256);
+  if (w.fmt == QLORA_FMT_AFFINE) {
+    if (w.bits == 8)
+      expand_bf16_kernel<3><<<grid, 256, 0, st>>>(p, w.codes, nb, out);
+    else
+      expand_bf16_kernel<2><<<grid, 256, 0, st>>>(p, w.codes, nb, out);
+  } else if (w.fmt == QLORA_FMT_NF4_FP32SCALE) {
+    expand_bf16_kernel<1><<<grid, 256, 0, st>>>(p, w.codes, nb, out);
+  } else {
+    expand_bf16_kernel<0><<<grid, 256, 0, st>>>(p, w.codes, nb, out);
+  }
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float* U,
@@ -1075,9 +1210,14 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   const uint32_t bn = (uint32_t)pl.bn;
   // X as {64 columns, R rows, I/64 K steps}; codes as {32 bytes, O rows, I/64 K steps}
   const uint32_t g = (uint32_t)tma_group(pl.bn);
+  const bool pre = tc_pre(false, pl, R);
+  // pre-decoded: the bf16 weight as {64 columns, O rows, I/64 K steps}, 16 KB boxes
   if (!make_map3(&m_act, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, (uint64_t)R, (uint64_t)(I / 64),
                  (uint64_t)I * 2, 128, 64, bn, g, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !(w.bits == 8
+      !(pre ? make_map3(&m_pk, wbuf_of(tcws, R, O, pl), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64,
+                        (uint64_t)O, (uint64_t)(I / 64), (uint64_t)I * 2, 128, 64, 128, 1,
+                        CU_TENSOR_MAP_SWIZZLE_128B)
+      : w.bits == 8
             ? make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 64, (uint64_t)O,
                         (uint64_t)(I / 64), (uint64_t)I, 64, 64, 128, g, CU_TENSOR_MAP_SWIZZLE_64B)
             : make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 32, (uint64_t)O,
@@ -1094,16 +1234,8 @@ cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float*
   p.kb_per_split = pl.kb_per_split;
   p.r_slices = (r + 15) / 16;
   p.rank = r;
-  p.C = (uint32_t)(w.group < 1 ? 1 : w.group);
-  p.c_shift = ((p.C & (p.C - 1)) == 0) ? __builtin_ctz(p.C) : -1;
-  p.qcodes = w.qcodes;
-  p.t = w.t;
-  p.mu = w.mu;
-  p.sb = w.fmt == QLORA_FMT_NF4_FP32SCALE ? w.scale : nullptr;
-  p.asc = w.fmt == QLORA_FMT_AFFINE ? w.scale : nullptr;
-  p.abi = w.fmt == QLORA_FMT_AFFINE ? w.bias : nullptr;
-  p.g_shift = w.block == 128 ? 2 : w.block == 64 ? 1 : 0;
-  p.pbits = w.bits;
+  fill_weight_params(w, p);
+  p.pre = pre ? 1 : 0;
   p.partial = pl.splits > 1;
   p.out = pl.splits > 1 ? (void*)part : Y;
   p.err = hdr;
@@ -1135,9 +1267,15 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   const uint32_t bn = (uint32_t)pl.bn;
   // dY as {64 columns, R rows, O/64 K steps}; codes as {I/2 bytes, 64 rows, O/64 K steps}
   const uint32_t g = (uint32_t)tma_group(pl.bn);
+  const bool pre = tc_pre(true, pl, R);
+  // pre-decoded: the bf16 weight as {I columns, 64 rows, O/64 K steps}, two
+  // 64 x 64 boxes per step (the MN-major W^T tile)
   if (!make_map3(&m_act, dY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, (uint64_t)R, (uint64_t)(O / 64),
                  (uint64_t)O * 2, 128, 64, bn, g, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !(w.bits == 8
+      !(pre ? make_map3(&m_pk, wbuf_of(tcws, R, I, pl), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        (uint64_t)I, 64, (uint64_t)(O / 64), (uint64_t)I * 2, (uint64_t)64 * I * 2,
+                        64, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B)
+      : w.bits == 8
             ? make_map3(&m_pk, w.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)I, 64,
                         (uint64_t)(O / 64), (uint64_t)I, (uint64_t)64 * I, 128, 64, g,
                         CU_TENSOR_MAP_SWIZZLE_128B)
@@ -1155,16 +1293,8 @@ cudaError_t launch_tc_dx(const WView& w, const void* dY, int64_t R, const float*
   p.kb_per_split = pl.kb_per_split;
   p.r_slices = (r + 15) / 16;
   p.rank = r;
-  p.C = (uint32_t)(w.group < 1 ? 1 : w.group);
-  p.c_shift = ((p.C & (p.C - 1)) == 0) ? __builtin_ctz(p.C) : -1;
-  p.qcodes = w.qcodes;
-  p.t = w.t;
-  p.mu = w.mu;
-  p.sb = w.fmt == QLORA_FMT_NF4_FP32SCALE ? w.scale : nullptr;
-  p.asc = w.fmt == QLORA_FMT_AFFINE ? w.scale : nullptr;
-  p.abi = w.fmt == QLORA_FMT_AFFINE ? w.bias : nullptr;
-  p.g_shift = w.block == 128 ? 2 : w.block == 64 ? 1 : 0;
-  p.pbits = w.bits;
+  fill_weight_params(w, p);
+  p.pre = pre ? 1 : 0;
   p.partial = pl.splits > 1;
   p.out = pl.splits > 1 ? (void*)part : dX;
   p.err = hdr;

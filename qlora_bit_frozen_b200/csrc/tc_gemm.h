@@ -33,6 +33,12 @@ inline uint16_t* tc_w_pad(void* tcws, int64_t R) {
   return (uint16_t*)((char*)tcws + (((size_t)R * 128 + 255) / 256) * 256);
 }
 
+// From 2048 tokens (256-token tiles, no K split) the input gradient decodes
+// the weight to a bf16 copy in the workspace once per call and the GEMM
+// reads that copy: this launches the decode (nothing otherwise).  Call it
+// before the rowdot launch that precedes launch_tc_fwd / launch_tc_dx.
+cudaError_t tc_prepare(bool dx, const WView& w, int64_t R, void* tcws, cudaStream_t st);
+
 // Y = X W_hat^T + s U B^T  (bf16 in/out, fp32 accumulation in TMEM).
 cudaError_t launch_tc_fwd(const WView& w, const void* X, int64_t R, const float* U,
                           const float* B, int32_t r, float s, void* Y, void* tcws,

@@ -224,7 +224,9 @@ def _smallr_splits(dx, O, I, R, sms=148):
 def test_tensor_core_plan_through_workspace_sizes(lib, O, I, R):
     """The bf16 workspace exceeds the fp32 one by exactly the tensor-core
     region: the padded U/V copy (R x 64 bf16), the adapter weight operand
-    (rows x 64 bf16) and, when K is split, one fp32 partial per split; at
+    (rows x 64 bf16), when K is split one fp32 partial per split, for the
+    input gradient from 2048 tokens on 256-token tiles the bf16 copy of the
+    decoded weight; at
     1..16 tokens also the few-token path's split partials.  This checks the
     host planners (split count, no empty split) without a GPU; the planners
     see 148 SMs here (no device)."""
@@ -232,11 +234,14 @@ def test_tensor_core_plan_through_workspace_sizes(lib, O, I, R):
     P = ctypes.byref(w)
     for op, Mw, KB in ((0, O, I // 64), (1, I, O // 64)):
         extra = lib.qlora_linear_workspace_bytes(P, R, 8, op, 1) - lib.qlora_linear_workspace_bytes(P, R, 8, op, 0)
-        _, splits = _planned_splits(Mw, KB, R)
+        bn, splits = _planned_splits(Mw, KB, R)
         part = _a256(splits * R * Mw * 4) if splits > 1 else 0
+        # input gradient from 2048 tokens on 256-token tiles without a K
+        # split: the bf16 copy of the decoded weight
+        wbuf = _a256(O * I * 2) if (op == 1 and bn == 256 and splits == 1 and R >= 2048) else 0
         srs = _smallr_splits(op == 1, O, I, R)
         sr = _a256(srs * R * (I if op == 1 else O) * 4) if srs > 1 else 0
-        assert extra == _a256(R * 128) + _a256(Mw * 128) + part + sr, (op, splits, srs)
+        assert extra == _a256(R * 128) + _a256(Mw * 128) + part + wbuf + sr, (op, splits, srs)
         per = -(-KB // splits)
         assert 1 <= splits <= max(1, KB) and (splits - 1) * per < KB <= splits * per
 

@@ -258,10 +258,11 @@ def test_bf16_identity_input_recovers_affine_weight_bitwise(bits, G):
 @pytest.mark.parametrize("fmt,bits,G", [("nf4", 4, 64), ("nf4_fp32scale", 4, 64), ("affine", 4, 32),
                                         ("affine", 8, 128)])
 def test_bf16_identity_input_pre_decoded_bitwise(fmt, bits, G):
-    """From 2048 tokens on 256-token tiles the weight is decoded to bf16 once
-    per call and the GEMM reads that copy: X = I (4096 tokens, W 1024 x 4096)
-    gives Y = bf16(W_hat)^T and dY = I (4096 tokens, W 4096 x 1024) gives
-    dX = bf16(W_hat), bit for bit, for every weight format."""
+    """From 2048 tokens on 256-token tiles the input gradient decodes the
+    weight to bf16 once per call and the GEMM reads that copy: dY = I (4096
+    tokens, W 4096 x 1024) gives dX = bf16(W_hat) bit for bit, for every
+    weight format; X = I (4096 tokens, W 1024 x 4096) checks the forward at
+    the same size (Y = bf16(W_hat)^T)."""
     def quant(W):
         if fmt == "nf4":
             return q.qlora_quantize_nf4(to_dev_f32(W)), oracle.quantize_nf4(W)
