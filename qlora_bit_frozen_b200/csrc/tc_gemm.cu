@@ -496,8 +496,25 @@ __global__ void __launch_bounds__(Cfg<DX, BN, wf_bits(WF)>::kThreads,
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kBM;
-  const int64_t n0 = (int64_t)blockIdx.y * BN;
+  // Tile order: CTAs go in groups of up to kGroupM weight tiles, sweeping
+  // every token tile of the group before the next group starts, so that a
+  // wave's weight slabs and token tiles both stay in L2 (with the plain
+  // order every wave re-read the whole weight; for a bf16 weight copy larger
+  // than L2 that came from DRAM every time).
+  int mt, nt;
+  {
+    constexpr int kGroupM = 16;
+    const int MT = (int)gridDim.x, NT = (int)gridDim.y;
+    const int lin = (int)blockIdx.y * MT + (int)blockIdx.x;
+    const int per_group = kGroupM * NT;
+    const int first = (lin / per_group) * kGroupM;
+    const int gsz = min(MT - first, kGroupM);
+    const int r = lin % per_group;
+    mt = first + r % gsz;
+    nt = r / gsz;
+  }
+  const int m0 = mt * kBM;
+  const int64_t n0 = (int64_t)nt * BN;
   const int split = blockIdx.z;
   const int kb_lo = split * p.kb_per_split;
   const int kb_hi = min(p.KB, kb_lo + p.kb_per_split);
