@@ -271,7 +271,15 @@ qlora_status qlora_adam_step(float* params, const float* grads, float* m, float*
 #define QLORA_OP_FWD 0
 #define QLORA_OP_BWD 1
 
-/* HOST.  Workspace bytes of qlora_linear_fwd (op 0) or qlora_linear_bwd (op 1). */
+/*
+ * HOST.  Workspace bytes of qlora_linear_fwd (op 0) or qlora_linear_bwd
+ * (op 1) for this weight, token count R, rank r and compute mode.  Besides
+ * small per-call scratch (status header, tickets, U / V, split partials),
+ * the bf16 backward from 2048 tokens on includes a bf16 copy of the decoded
+ * weight (2 O I bytes): the input gradient decodes the weight into it once
+ * per call and its GEMM reads it there.  The workspace is scratch for one
+ * call at a time; the weight itself stays packed.
+ */
 size_t qlora_linear_workspace_bytes(const qlora_weight* w, int64_t R, int32_t r, int32_t op,
                                     int32_t compute);
 
