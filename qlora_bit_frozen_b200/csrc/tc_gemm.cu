@@ -4,14 +4,19 @@
 // Input    dX = dY W_hat + s V A         backward"; "QLoRA on Mac",
 // gradient                               "Design / Q-LoRA layer")
 //
-// The frozen weight never exists as a floating-point matrix in HBM: packed
-// 4-bit codes arrive in shared memory by TMA, decoder warps turn each
+// Packed codes arrive in shared memory by TMA, decoder warps turn each
 // 64-weight block into bf16 in registers -- NF4: codebook level times the
 // block scale (double-quantized, rebuilt from q_b, t_g and mu, or the
-// legacy fp32 absmax); affine 4-bit: scale * code + bias of the code's group
-// ("LoRA vs QLoRA on Apple Silicon", "Method") -- and write it where the
-// tensor core reads it (TMEM rows, or 128-byte-swizzled shared-memory rows),
-// and tcgen05.mma accumulates in TMEM.
+// legacy fp32 absmax); affine 4/8-bit: scale * code + bias of the code's
+// group ("LoRA vs QLoRA on Apple Silicon", "Method") -- and write it where
+// the tensor core reads it (TMEM rows, or 128-byte-swizzled shared-memory
+// rows), and tcgen05.mma accumulates in TMEM.  The one exception: the input
+// gradient from 2048 tokens on 256-token tiles decodes the weight once per
+// call (expand_bf16_kernel, the same decode) into a bf16 copy in the
+// call's workspace and reads that by TMA ("QLoRA: Fine-Tuning Under Memory
+// Constraints", "Separate representation from arithmetic": fused or
+// temporary dequantized tensors are the implementation's choice); the
+// weight itself stays packed.
 //
 // Orientation: the decoded weight tile is the MMA "A" operand (M = 128
 // weight-side rows: output features in the forward, input features in the
@@ -29,6 +34,9 @@
 // along the rank, and its B operand is bf16 U or V, all loaded by TMA once
 // the launch that computed them has finished (programmatic dependent
 // launch: the K loop before it overlaps that launch).
+//
+// Tiles are taken in groups of up to 16 weight tiles, every token tile of
+// a group before the next, so a wave's operands stay in L2.
 //
 // Warp roles: warp 0 TMA producer, warp 1 TMEM allocator and MMA issuer,
 // then the decoders in groups of four warps (a whole 64-weight row per
