@@ -511,15 +511,15 @@ __global__ void __launch_bounds__(Cfg<DX, BN, wf_bits(WF)>::kThreads,
   // than L2 that came from DRAM every time).
   int mt, nt;
   {
-    constexpr int kGroupM = 16;
-    const int MT = (int)gridDim.x, NT = (int)gridDim.y;
-    const int lin = (int)blockIdx.y * MT + (int)blockIdx.x;
-    const int per_group = kGroupM * NT;
-    const int first = (lin / per_group) * kGroupM;
-    const int gsz = min(MT - first, kGroupM);
-    const int r = lin % per_group;
-    mt = first + r % gsz;
-    nt = r / gsz;
+    constexpr int64_t kGroupM = 16;
+    const int64_t MT = gridDim.x, NT = gridDim.y;
+    const int64_t lin = (int64_t)blockIdx.y * MT + blockIdx.x;
+    const int64_t per_group = kGroupM * NT;
+    const int64_t first = (lin / per_group) * kGroupM;
+    const int64_t gsz = MT - first < kGroupM ? MT - first : kGroupM;
+    const int64_t r = lin % per_group;
+    mt = (int)(first + r % gsz);
+    nt = (int)(r / gsz);
   }
   const int m0 = mt * kBM;
   const int64_t n0 = (int64_t)nt * BN;

@@ -49,8 +49,13 @@ def test_gpus_flag_starts_one_rank_per_gpu():
     """--gpus 2 outside torchrun re-launches itself with torch.distributed.run:
     two ranks start, each sees its own RANK / LOCAL_RANK and WORLD_SIZE 2."""
     env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
-    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--print-ranks"],
-                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    # The launcher picks its rendezvous port by binding port 0 and releasing
+    # it; another process can take the port in between, so one retry.
+    for attempt in range(2):
+        out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--print-ranks"],
+                             cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+        if out.returncode == 0:
+            break
     assert out.returncode == 0, out.stderr[-2000:]
     ranks = sorted((json.loads(l)["rank"], json.loads(l)["local_rank"], json.loads(l)["world"])
                    for l in out.stdout.splitlines() if l.startswith("{"))
