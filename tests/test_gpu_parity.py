@@ -325,6 +325,16 @@ def test_bf16_small_row_sweep_nf4(name, R):
     _check(_run_layer(wl, 0, want=("Y", "dX")), TOL["bf16"])
 
 
+@pytest.mark.parametrize("R", [9, 16])
+def test_bf16_few_token_gemv_where_tiles_do_not_apply(R):
+    """W 2048 x 1088 (I % 128 = 64: no tensor-core tiles) at 9 and 16 tokens:
+    the few-token kernels with two 8-token MMA tiles, forward and dX,
+    against the oracle (Y, U, dX; dA and dB by the side products)."""
+    wl = synth.workload("qwen3_0.6b_attn_qv", R=R)
+    wl.linears = [synth.Linear("odd_i", 2048, 1088)]
+    _check(_run_layer(wl, 0), TOL["bf16"])
+
+
 @pytest.mark.parametrize("name", ["bw_sweep_4096", "bw_sweep_12288"])
 @pytest.mark.parametrize("R", [1, 16, 128])
 @pytest.mark.parametrize("bits,G", [(4, 32), (4, 64), (4, 128), (8, 32), (8, 64), (8, 128)])
