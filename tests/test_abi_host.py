@@ -220,7 +220,8 @@ def _smallr_splits(dx, O, I, R, sms=148):
 
 @pytest.mark.parametrize("O,I,R", [(12288, 4096, 1), (12288, 4096, 16), (4096, 4096, 1), (4096, 4096, 16),
                                    (4096, 4096, 128), (2048, 1024, 4096), (1024, 1024, 4096),
-                                   (12288, 4096, 8192), (5120, 17408, 16384), (128, 128, 3)])
+                                   (12288, 4096, 8192), (5120, 17408, 16384), (128, 128, 3),
+                                   (2048, 2048, 2047), (2048, 2048, 2048)])
 def test_tensor_core_plan_through_workspace_sizes(lib, O, I, R):
     """The bf16 workspace exceeds the fp32 one by exactly the tensor-core
     region: the padded U/V copy (R x 64 bf16), the adapter weight operand
